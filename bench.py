@@ -1,0 +1,421 @@
+#!/usr/bin/env python
+"""Benchmark of the orthonormalized-update optimizer step on B200.
+
+Workload (one "step"): a Llama-3-8B-shaped parameter set -- 32 layers x
+{q, o 4096x4096; k, v 1024x4096; gate, up 14336x4096; down 4096x14336}, 224
+matrices, 6,979,321,856 parameters -- with bf16 gradients N(0, 0.01^2) plus a
+rank-32 spike, fp32 momentum and bf16 weights.  One step is the whole hot
+path through the library's C ABI:
+
+  dion_momentum_update (error-feedback buffer B = M + G, float64 row keys)
+  dion3_select_rows    (top 1/8 rows by row norm, gather + scale, M[S] = mu B[S])
+  gram_ns_orthogonalize(5 iterations, restart after 3, bf16 / tf32 tensor cores)
+  apply_update         (W[S] -= lr * scale * O)
+
+Prints one JSON line (rank 0).  ``--impl reference`` times the float64 CPU
+oracle on a bounded sample of the same workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "optimizer-step ms (8B-shaped param set) & Gram-NS TFLOP/s vs BF16 peak, 1×B200"
+RHO = 0.125
+MU = 0.95
+LR = 0.02
+ITERS = 5
+RESTART_AFTER = (3,)
+# tf32 / bf16 dense tensor throughput ratio (nominal 1.1 / 2.25 PFLOP/s)
+TF32_RATIO = 1.1 / 2.25
+
+
+def _args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--layers", type=int, default=32)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-sample-layers", type=int, default=1)
+    return ap.parse_args()
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d["bf16_tflops_sustained"]),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0,
+                "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def gram_ns_flops(k: int, n: int, iters: int = ITERS, restarts=RESTART_AFTER):
+    """Algorithmic flops of Gram NS on a k x n block (k <= n after
+    orientation), split into bf16 (k x n products) and tf32 (k x k symmetric
+    products).  Symmetric outputs count the upper triangle only."""
+    if k > n:
+        k, n = n, k
+    syrk = k * (k + 1) * n           # X X^T, triangle
+    qx = 2 * k * k * n               # Q X
+    sym = k * k * (k + 1)            # symmetric k x k product, triangle
+    bf, tf = syrk, 0
+    q_identity = True
+    for t in range(1, iters + 1):
+        tf += sym                    # A^2 inside H
+        if not q_identity:
+            tf += sym                # H Q
+        q_identity = False
+        if t == iters:
+            break
+        if t in restarts:
+            bf += qx + syrk
+            q_identity = True
+        else:
+            tf += 2 * sym            # H (H A)
+    bf += qx
+    return bf, tf
+
+
+def _workload_shapes(layers):
+    from orthonormalized_update_optimizers_b200 import synth
+    return synth.llama8b_shapes(layers)
+
+
+# ----------------------------------------------------------------- reference
+
+def run_reference(args):
+    """Time the float64 oracle, as it stands, on a bounded sample: W warm-up
+    repetitions on one small matrix, then K timed repetitions of the layer
+    sample, each scaled to the full parameter set."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    for _ in range(args.warmup):
+        _oracle_sample(args, n_matrices=1, first=1)  # k projection, 1024 x 4096
+    per_step = [cpu_baseline(args)["value"] for _ in range(args.steps)]
+    ms = statistics.median(per_step)
+    line = cpu_baseline.last
+    line = dict(line, value=round(ms, 3))
+    out = {
+        "impl": "reference", "metric": METRIC, "value": round(ms, 3),
+        "unit": "ms", "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms, 3),
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic",
+        "config": _config(args.layers),
+        "cpu_baseline": line,
+        "e2e": {"value": round(ms, 3), "unit": "ms", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(out), flush=True)
+
+
+def _oracle_sample(args, n_matrices, first=0):
+    """Seconds the oracle's Dion3 step takes on matrices first..first+n-1 of
+    the workload (inputs from the shared seeded generator, on the host)."""
+    import numpy as np
+    import torch
+    from orthonormalized_update_optimizers_b200 import synth
+    from oracle import dion3 as odion3
+
+    shapes = _workload_shapes(args.layers)
+    t_total = 0.0
+    for i in range(first, first + n_matrices):
+        _, m, n = shapes[i]
+        G = synth.lowrank_plus_noise(m, n, 32, 0.01, synth.seed_for(3, i),
+                                     torch.bfloat16, "cpu")
+        G64 = G.float().numpy().astype(np.float64)
+        M = np.zeros((m, n), dtype=np.float32)
+        W = synth.gaussian((m, n), synth.seed_for(3, 1000 + i), 0.02,
+                           torch.bfloat16, "cpu").float().numpy().astype(np.float64)
+        t0 = time.perf_counter()
+        odion3.dion3_step(M, G64, W, MU, RHO, LR, 1.0, iters=ITERS,
+                          restart_after=RESTART_AFTER)
+        t_total += time.perf_counter() - t0
+    return t_total
+
+
+def cpu_baseline(args):
+    """Oracle Dion3 step on the first `cpu_sample_layers` layers' matrices
+    (same generator, same seeds), scaled to the full parameter set by the
+    number of matrices.  Returns the cpu_baseline object."""
+    shapes = _workload_shapes(args.layers)
+    n_sample = 7 * args.cpu_sample_layers
+    t_total = _oracle_sample(args, n_sample)
+    scale = len(shapes) / n_sample
+    ms = t_total * 1e3 * scale
+    cores = len(os.sched_getaffinity(0))
+    line = {"value": round(ms, 3), "unit": "ms", "cores": cores, "kind": "oracle",
+            "sample": f"float64 NumPy oracle Dion3 step on the {n_sample} matrices of "
+                      f"layer(s) 0..{args.cpu_sample_layers - 1}, measured {t_total:.2f} s, "
+                      f"extrapolated x{scale:g} to all {len(shapes)} matrices",
+            "extrapolated": scale != 1.0}
+    cpu_baseline.last = line
+    return line
+
+
+def _config(layers):
+    shapes = _workload_shapes(layers)
+    params = sum(m * n for _, m, n in shapes)
+    return {"workload": f"Llama-3-8B-shaped optimizer step ({layers} layers, {len(shapes)} "
+                        "matrices): Dion3 rho=1/8 with error feedback + Gram Newton-Schulz "
+                        "(5 iterations, restart after 3), bf16 gradients N(0,0.01^2)+rank-32 "
+                        "spike, fp32 momentum, bf16 weights",
+            "params": params, "matrices": len(shapes), "rho": RHO, "mu": MU,
+            "l2": "inputs larger than L2 (about 56 GB resident per step)",
+            "parallelism": "replicas (one independent step per GPU)"}
+
+
+# ----------------------------------------------------------------------- ours
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200", "-i", str(self.index)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def run_ours(args):
+    import numpy as np
+    import torch
+    import orthonormalized_update_optimizers_b200 as ouo
+    from orthonormalized_update_optimizers_b200 import synth
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    dev = torch.device("cuda", local)
+
+    shapes = _workload_shapes(args.layers)
+    Gs, Ms, Ws = [], [], []
+    for i, (_, m, n) in enumerate(shapes):
+        Gs.append(synth.lowrank_plus_noise(m, n, 32, 0.01, synth.seed_for(3, i),
+                                           torch.bfloat16, dev))
+        Ms.append(torch.zeros(m, n, dtype=torch.float32, device=dev))
+        Ws.append(synth.gaussian((m, n), synth.seed_for(3, 1000 + i), 0.02,
+                                 torch.bfloat16, dev))
+    ks = [ouo.dion3_num_selected(m, RHO) for _, m, _ in shapes]
+    keys = torch.empty(sum(m for _, m, _ in shapes), dtype=torch.float64, device=dev)
+    idx = torch.empty(sum(ks), dtype=torch.int32, device=dev)
+    X0 = [torch.empty(k, n, dtype=torch.bfloat16, device=dev) for k, (_, _, n) in zip(ks, shapes)]
+    O = [torch.empty_like(x) for x in X0]
+    scale = torch.empty(len(shapes), dtype=torch.float32, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    Mb, Gb, Wb = ouo.MatBatch(Ms), ouo.MatBatch(Gs), ouo.MatBatch(Ws)
+    Xb, Ob = ouo.MatBatch(X0), ouo.MatBatch(O)
+    params = ouo.ns_params(iters=ITERS, restart_after=RESTART_AFTER, normalize=False)
+    ws = torch.empty(ouo.gram_ns_workspace_bytes(Xb, params), dtype=torch.uint8, device=dev)
+    # Muon-style per-matrix update scale sqrt(max(1, rows / cols))
+    scales = [math.sqrt(max(1.0, m / n)) for _, m, n in shapes]
+
+    def step():
+        ouo.dion_momentum_update(Mb, Gb, MU, "accum", keys)
+        ouo.dion3_select_rows(Mb, keys, RHO, idx, Xb, scale, ef=True, mu=MU)
+        ouo.gram_ns_orthogonalize(Xb, Ob, params, workspace=ws, status=status)
+        ouo.apply_update(Wb, Ob, LR, idx=idx, scale=scales)
+
+    def barrier():
+        torch.cuda.synchronize()
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    def max_over_ranks(x):
+        if dist is None:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    for _ in range(args.warmup):
+        step()
+    barrier()
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    n0 = ouo.launch_count()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        step()
+    e1.record()
+    barrier()
+    launches = ouo.launch_count() - n0
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps)
+    # --- the Gram-NS stage alone (dominant tensor-core kernels)
+    g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    g0.record()
+    for _ in range(args.steps):
+        ouo.gram_ns_orthogonalize(Xb, Ob, params, workspace=ws, status=status)
+    g1.record()
+    barrier()
+    gram_ms = max_over_ranks(g0.elapsed_time(g1) / args.steps)
+    # --- the momentum kernel alone (HBM-bound)
+    m0, m1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    m0.record()
+    for _ in range(args.steps):
+        ouo.dion_momentum_update(Mb, Gb, MU, "accum", keys)
+    m1.record()
+    barrier()
+    mom_ms = max_over_ranks(m0.elapsed_time(m1) / args.steps)
+    clocks = sampler.stop()
+    st = int(status.item())
+
+    peaks = _peaks()
+    bf = tf = 0
+    for k, (_, m, n) in zip(ks, shapes):
+        b_, t_ = gram_ns_flops(k, n)
+        bf += b_
+        tf += t_
+    flops = bf + tf
+    tflops = flops / (gram_ms * 1e-3) / 1e12
+    # effective peak of the bf16 / tf32 mix (each at its own dtype's peak)
+    p_bf = peaks["bf16_tflops"]
+    p_tf = p_bf * TF32_RATIO
+    peak_eff = flops / (bf / p_bf + tf / p_tf)
+    elems = sum(m * n for _, m, n in shapes)
+    rows = keys.numel()
+    mom_bytes = elems * (4 + 2 + 4) + rows * 8   # read M, G; write M; write keys
+    mom_gbs = mom_bytes / (mom_ms * 1e-3) / 1e9
+
+    result = {
+        "metric": METRIC, "value": round(ms, 4), "unit": "ms", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic", "config": _config(args.layers),
+        "gram_ns": {"ms": round(gram_ms, 4), "tflops": round(tflops, 2),
+                    "flops_bf16": bf, "flops_tf32": tf,
+                    "counting": "symmetric products count the upper triangle"},
+        "roofline": {"bound": "tensor", "kernel": "gram_ns_orthogonalize (tcgen05 GEMMs)",
+                     "achieved": round(tflops, 2), "peak": round(peak_eff, 1),
+                     "unit": "TFLOP/s", "frac": round(tflops / peak_eff, 4),
+                     "traffic": None,
+                     "peak_note": f"bf16 {p_bf} ({peaks['source']}, burst) and tf32 = bf16 x "
+                                  f"{TF32_RATIO:.3f} (nominal ratio), weighted by flops"},
+        "roofline_hbm": {"bound": "hbm", "kernel": "momentum_kernel",
+                         "achieved": round(mom_gbs, 1), "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": round(mom_gbs / peaks["hbm_gbs"], 4),
+                         "traffic": None, "ms": round(mom_ms, 4)},
+        "gpu_launches": int(launches),
+        "device_status": st,
+    }
+    if clocks:
+        result["clocks"] = clocks
+
+    if not args.no_e2e:
+        result["e2e"] = e2e_measure(args, step, Gs, idx, scale, dev, barrier, max_over_ranks)
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(args)
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def e2e_measure(args, step, Gs, idx, scale, dev, barrier, max_over_ranks):
+    """Same step through the public API with the gradients arriving from
+    pinned host memory each step and the step's result (kept-row indices and
+    per-matrix scales) read back to the host."""
+    import torch
+    total = sum(g.numel() for g in Gs)
+    host = torch.empty(total, dtype=torch.bfloat16, pin_memory=True)
+    views, off = [], 0
+    for g in Gs:
+        v = host[off:off + g.numel()].view(g.shape)
+        v.copy_(g)
+        views.append(v)
+        off += g.numel()
+    idx_h = torch.empty(idx.shape, dtype=idx.dtype, pin_memory=True)
+    sc_h = torch.empty(scale.shape, dtype=scale.dtype, pin_memory=True)
+    steps = max(1, min(args.steps, 5))
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        for g, v in zip(Gs, views):
+            g.copy_(v, non_blocking=True)
+        step()
+        idx_h.copy_(idx, non_blocking=True)
+        sc_h.copy_(scale, non_blocking=True)
+    e1.record()
+    barrier()
+    ms = max_over_ranks(e0.elapsed_time(e1) / steps)
+    return {"value": round(ms, 3), "unit": "ms", "steps": steps,
+            "h2d_bytes_per_step": total * 2,
+            "d2h_bytes_per_step": idx.numel() * 4 + scale.numel() * 4}
+
+
+def main():
+    args = _args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,216 @@
+"""PyTorch-facing binding of liborthoupd.so: argument marshalling only.
+
+Each function turns lists of 2-D CUDA tensors into ``ouo_mat`` arrays, picks
+the current CUDA stream, calls the C entry point of the same name and raises
+``OuoError`` on a nonzero return.  Every step of the optimizer runs inside the
+library's kernels; there is no fallback.  Workspaces default to a torch
+allocation made here (the library itself never allocates).
+"""
+from __future__ import annotations
+
+import ctypes
+from typing import Iterable, Optional, Sequence
+
+import torch
+
+from . import _lib as L
+from ._lib import OuoError  # noqa: F401  (re-exported)
+
+__all__ = [
+    "MatBatch", "ns_params", "dion_params", "dion_momentum_update",
+    "dion3_num_selected", "dion3_select_rows", "ns_workspace_bytes",
+    "ns_orthogonalize", "gram_ns_workspace_bytes", "gram_ns_orthogonalize",
+    "apply_update", "dion_workspace_bytes", "dion_lowrank_step", "version",
+    "launch_count",
+]
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return L.OUO_F32
+    if t.dtype == torch.bfloat16:
+        return L.OUO_BF16
+    raise TypeError(f"unsupported dtype {t.dtype} (float32 or bfloat16)")
+
+
+class MatBatch:
+    """A list of 2-D row-major CUDA tensors described once as an ouo_mat
+    array, so repeated calls do not rebuild it."""
+
+    def __init__(self, tensors: Iterable[torch.Tensor]):
+        self.tensors = list(tensors)
+        self.n = len(self.tensors)
+        self.arr = (L.OuoMat * max(self.n, 1))()
+        codes = set()
+        for i, t in enumerate(self.tensors):
+            if t.dim() != 2 or (t.shape[1] > 1 and t.stride(1) != 1):
+                raise ValueError("every matrix must be 2-D with unit column stride")
+            if not t.is_cuda:
+                raise ValueError("every matrix must be a CUDA tensor")
+            self.arr[i] = L.OuoMat(t.data_ptr(), t.shape[0], t.shape[1],
+                                   max(t.stride(0), t.shape[1]))
+            codes.add(_dtype_code(t))
+        if len(codes) > 1:
+            raise TypeError("a batch must have one dtype")
+        self.dtype = codes.pop() if codes else L.OUO_F32
+
+    @property
+    def device(self):
+        return self.tensors[0].device if self.tensors else torch.device("cuda")
+
+
+def _batch(x) -> MatBatch:
+    if isinstance(x, MatBatch):
+        return x
+    if isinstance(x, torch.Tensor):
+        return MatBatch([x])
+    return MatBatch(x)
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def version() -> int:
+    return L.lib().ouo_version()
+
+
+def launch_count() -> int:
+    """Kernels the library has enqueued in this process so far."""
+    return int(L.lib().ouo_launch_count())
+
+
+def ns_params(a=None, b=None, c=None, iters=None, safety=None, eps=None,
+              normalize=None, precision="bf16", restart_after=None) -> L.NsParams:
+    """ouo_ns_params with the library defaults, overridden where given."""
+    p = L.NsParams()
+    L.lib().ouo_ns_default(ctypes.byref(p))
+    for name, val in (("a", a), ("b", b), ("c", c), ("iters", iters),
+                      ("safety", safety), ("eps", eps)):
+        if val is not None:
+            setattr(p, name, val)
+    if normalize is not None:
+        p.normalize = int(bool(normalize))
+    p.precision = {"bf16": L.OUO_PREC_BF16, "fp32": L.OUO_PREC_FP32}[precision]
+    if restart_after is not None:
+        ra = list(restart_after)
+        if len(ra) > L.OUO_MAX_RESTARTS:
+            raise ValueError("too many restarts")
+        p.n_restart = len(ra)
+        for i, t in enumerate(ra):
+            p.restart_after[i] = int(t)
+    return p
+
+
+def dion_params(rank=None, mu=None, beta=None, lr=None, wd=None,
+                norm_mode="colnorm", eps=None) -> L.DionParams:
+    p = L.DionParams()
+    L.lib().ouo_dion_default(ctypes.byref(p))
+    for name, val in (("rank", rank), ("mu", mu), ("beta", beta), ("lr", lr),
+                      ("wd", wd), ("eps", eps)):
+        if val is not None:
+            setattr(p, name, val)
+    p.norm_mode = {"colnorm": L.OUO_DION_COLNORM, "qr": L.OUO_DION_QR}[norm_mode]
+    return p
+
+
+def dion_momentum_update(M, G, mu: float, mode: str = "ema",
+                         row_sqnorm: Optional[torch.Tensor] = None,
+                         stream=None) -> None:
+    Mb, Gb = _batch(M), _batch(G)
+    code = {"ema": L.OUO_MOMENTUM_EMA, "accum": L.OUO_MOMENTUM_ACCUM}[mode]
+    L.check("dion_momentum_update", L.lib().dion_momentum_update(
+        Mb.arr, Gb.arr, Mb.n, Gb.dtype, mu, code, _ptr(row_sqnorm),
+        _stream(stream)))
+
+
+def dion3_num_selected(rows: int, rho: float) -> int:
+    return int(L.lib().dion3_num_selected(rows, rho))
+
+
+def dion3_select_rows(B, row_sqnorm: torch.Tensor, rho: float,
+                      idx: torch.Tensor, X0, x0_scale: torch.Tensor,
+                      ef: bool = True, mu: float = 0.95, eps: float = 1e-7,
+                      stream=None) -> None:
+    Bb, Xb = _batch(B), _batch(X0)
+    L.check("dion3_select_rows", L.lib().dion3_select_rows(
+        Bb.arr, _ptr(row_sqnorm), Bb.n, rho,
+        L.OUO_EF_ROWS if ef else L.OUO_EF_NONE, mu, eps, _ptr(idx), Xb.arr,
+        Xb.dtype, _ptr(x0_scale), _stream(stream)))
+
+
+def ns_workspace_bytes(X, params=None) -> int:
+    Xb = _batch(X)
+    p = params or ns_params()
+    return int(L.lib().ns_workspace_bytes(Xb.arr, Xb.n, ctypes.byref(p)))
+
+
+def gram_ns_workspace_bytes(X, params=None) -> int:
+    Xb = _batch(X)
+    p = params or ns_params()
+    return int(L.lib().gram_ns_workspace_bytes(Xb.arr, Xb.n, ctypes.byref(p)))
+
+
+def _workspace(nbytes: int, device, given: Optional[torch.Tensor]):
+    if given is not None:
+        return given
+    return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+
+
+def _run_ns(fname, wsfn, X, O, params, workspace, status, stream):
+    Xb, Ob = _batch(X), _batch(O)
+    p = params or ns_params()
+    need = wsfn(Xb, p)
+    ws = _workspace(need, Xb.device, workspace)
+    fn = getattr(L.lib(), fname)
+    L.check(fname, fn(Xb.arr, Xb.dtype, Ob.arr, Ob.dtype, Xb.n, ctypes.byref(p),
+                      ctypes.c_void_p(ws.data_ptr()), ws.numel(), _ptr(status),
+                      _stream(stream)))
+
+
+def ns_orthogonalize(X, O, params=None, workspace=None, status=None,
+                     stream=None) -> None:
+    _run_ns("ns_orthogonalize", ns_workspace_bytes, X, O, params, workspace,
+            status, stream)
+
+
+def gram_ns_orthogonalize(X, O, params=None, workspace=None, status=None,
+                          stream=None) -> None:
+    _run_ns("gram_ns_orthogonalize", gram_ns_workspace_bytes, X, O, params,
+            workspace, status, stream)
+
+
+def apply_update(W, O, lr: float, idx: Optional[torch.Tensor] = None,
+                 scale: Optional[Sequence[float]] = None, wd: float = 0.0,
+                 stream=None) -> None:
+    Wb, Ob = _batch(W), _batch(O)
+    sc = None
+    if scale is not None:
+        sc = (ctypes.c_float * Wb.n)(*[float(s) for s in scale])
+    L.check("apply_update", L.lib().apply_update(
+        Wb.arr, Wb.dtype, Ob.arr, Ob.dtype, _ptr(idx), Wb.n, lr, sc, wd,
+        _stream(stream)))
+
+
+def dion_workspace_bytes(M, params) -> int:
+    Mb = _batch(M)
+    return int(L.lib().dion_workspace_bytes(Mb.arr, Mb.n, ctypes.byref(params)))
+
+
+def dion_lowrank_step(M, G, Q_state, W, params, scale=None, workspace=None,
+                      status=None, stream=None) -> None:
+    Mb, Gb, Qb, Wb = _batch(M), _batch(G), _batch(Q_state), _batch(W)
+    need = L.lib().dion_workspace_bytes(Mb.arr, Mb.n, ctypes.byref(params))
+    ws = _workspace(need, Mb.device, workspace)
+    sc = None
+    if scale is not None:
+        sc = (ctypes.c_float * Mb.n)(*[float(s) for s in scale])
+    L.check("dion_lowrank_step", L.lib().dion_lowrank_step(
+        Mb.arr, Gb.arr, Gb.dtype, Qb.arr, Wb.arr, Wb.dtype, Mb.n,
+        ctypes.byref(params), sc, ctypes.c_void_p(ws.data_ptr()), ws.numel(),
+        _ptr(status), _stream(stream)))

@@ -1,0 +1,351 @@
+// Host orchestration of standard and Gram Newton-Schulz over a batch.
+//
+// Sources: "Dion3: Full-Stack Orthogonal Updates", Abstract (Muon's
+// cubic-time Newton-Schulz; Gram Newton-Schulz lowers its FLOP cost);
+// "Dion3：全栈正交更新", 核心洞察 / 核心模块 (iterate on the symmetric Gram
+// matrix; restarts and safety factors keep it stable) and 局限 (restarts fix
+// spurious negative eigenvalues and eigenvector drift; fp16 / bf16 need
+// care).
+//
+// Per group of equal-shape matrices (k x n after orientation, k <= n):
+//   prep   X0 = X / (||X||_F + eps) into workspace (transposed if needed)
+//   Gram:  A = X0 X0^T;  for t: H = a'I + b'A + c'A^2;  Q <- H Q  (Q = H on
+//          the first iteration of a segment);  restart: X0 <- Q X0,
+//          A = X0 X0^T;  otherwise A <- H (H A);  finally O = Q X0.
+//   Std:   for t: A = X X^T;  B = b'A + c'A^2;  X <- a'X + B X.
+//
+// Precision (OUO_PREC_BF16): products with an n-long contraction or output
+// (X X^T, Q X, B X) take bf16 operands; the k x k products (A^2, H Q, H A,
+// H T) take tf32 operands, stored already rounded to tf32; every
+// accumulation is fp32 in TMEM.  Rounding A itself to bf16 measurably breaks
+// the 2e-2 accuracy bound on 512 x 4096 inputs; tf32 keeps it below 1e-2.
+// OUO_PREC_FP32 runs every product in fp32 on CUDA cores.
+#include <algorithm>
+#include <cmath>
+
+#include "internal.h"
+
+namespace ouo {
+namespace {
+
+struct Coeffs {
+  float a, b, c;
+};
+
+Coeffs scaled(const ouo_ns_params& p) {
+  double s = p.safety;
+  Coeffs c;
+  c.a = (float)((double)p.a / s);
+  c.b = (float)((double)p.b / (s * s * s));
+  c.c = (float)((double)p.c / (s * s * s * s * s));
+  return c;
+}
+
+struct Oriented {
+  int64_t k, n;
+  bool transpose;
+};
+
+Oriented orient(const Group& g) {
+  Oriented o;
+  o.transpose = g.rows > g.cols;
+  o.k = o.transpose ? g.cols : g.rows;
+  o.n = o.transpose ? g.rows : g.cols;
+  return o;
+}
+
+struct GroupWs {
+  Buf x0, x1, y;       // k x n: current / alternate X, final output
+  Buf kk[3];           // k x k fp32 (A, H/Q rotation)
+  Buf A, T;            // k x k fp32
+  Buf qbf;             // k x k bf16 copy of Q (bf16 path)
+  Buf bm;              // standard NS: b'A + c'A^2 (bf16 or fp32)
+  double* scratch;     // rows doubles per matrix + one float per matrix
+};
+
+GroupWs carve(Arena& ar, const Group& g, const Oriented& o, bool gram,
+              int precision, int o_dtype) {
+  GroupWs w;
+  const int64_t nb = (int64_t)g.members.size();
+  const bool bf = precision == OUO_PREC_BF16;
+  const int xd = bf ? OUO_BF16 : OUO_F32;
+  w.x0 = ar.take(xd, nb, o.k, o.n);
+  w.x1 = ar.take(xd, nb, o.k, o.n);
+  w.y = ar.take(bf ? o_dtype : OUO_F32, nb, o.k, o.n);
+  w.A = ar.take(OUO_F32, nb, o.k, o.k);
+  if (gram) {
+    for (int i = 0; i < 3; ++i) w.kk[i] = ar.take(OUO_F32, nb, o.k, o.k);
+    w.T = ar.take(OUO_F32, nb, o.k, o.k);
+    if (bf) w.qbf = ar.take(OUO_BF16, nb, o.k, o.k);
+  } else {
+    w.bm = ar.take(bf ? OUO_BF16 : OUO_F32, nb, o.k, o.k);
+  }
+  // float64 row sums (rows of the caller's matrix) + float scales
+  Buf s = ar.take(OUO_F32, 1, 1, nb * g.rows * 2 + nb);
+  w.scratch = reinterpret_cast<double*>(s.p);
+  return w;
+}
+
+int run_gemm(const GemmDesc& d, bool bf, cudaStream_t s, int* status) {
+  return bf ? gemm_umma(d, s, status) : gemm_simt(d, s);
+}
+
+GemmDesc syrk(const Buf& X, const Buf& out, bool bf) {
+  GemmDesc d;
+  d.M = d.N = X.rows;
+  d.K = X.cols;
+  d.nb = X.nb;
+  d.A = X;
+  d.B = X;
+  d.tri = true;
+  d.out_f32 = out;
+  d.has_f32 = true;
+  d.round_tf32 = bf;
+  return d;
+}
+
+// out = alpha * L R + beta * C0 + gamma * I for commuting symmetric k x k L, R
+GemmDesc symprod(const Buf& L, const Buf& R, float alpha, const Buf* C0,
+                 float beta, float gamma, bool bf) {
+  GemmDesc d;
+  d.M = d.N = d.K = L.rows;
+  d.nb = L.nb;
+  d.A = L;
+  d.B = R;
+  d.alpha = alpha;
+  if (C0) {
+    d.C0 = *C0;
+    d.has_c0 = true;
+    d.beta = beta;
+  }
+  d.gamma = gamma;
+  d.tri = true;
+  d.round_tf32 = bf;
+  return d;
+}
+
+// out = alpha * L X + beta * C0, L k x k (K-major), X k x n (MN-major)
+GemmDesc apply_left(const Buf& L, const Buf& X, const Buf& out, float alpha,
+                    const Buf* C0, float beta) {
+  GemmDesc d;
+  d.M = L.rows;
+  d.N = X.cols;
+  d.K = L.cols;
+  d.nb = L.nb;
+  d.A = L;
+  d.B = X;
+  d.b_mn = 1;
+  d.alpha = alpha;
+  if (C0) {
+    d.C0 = *C0;
+    d.has_c0 = true;
+    d.beta = beta;
+  }
+  if (out.dtype == OUO_BF16) {
+    d.out_bf16 = out;
+    d.has_bf16 = true;
+  } else {
+    d.out_f32 = out;
+    d.has_f32 = true;
+  }
+  return d;
+}
+
+bool is_restart(const ouo_ns_params& p, int t) {
+  for (int i = 0; i < p.n_restart; ++i)
+    if (p.restart_after[i] == t) return true;
+  return false;
+}
+
+// Index among {0, 1, 2} equal to neither a nor b (a and b may be equal or -1).
+int free_idx(int a, int b) {
+  for (int i = 0; i < 3; ++i)
+    if (i != a && i != b) return i;
+  return -1;
+}
+
+// Gram Newton-Schulz on one group; the result (k x n) is left in w.y.
+int gram_group(const ouo_ns_params& p, GroupWs& w, cudaStream_t s,
+               int* status) {
+  const bool bf = p.precision == OUO_PREC_BF16;
+  const Coeffs c = scaled(p);
+  Buf* X = &w.x0;
+  Buf* Xalt = &w.x1;
+  OUO_TRY(run_gemm(syrk(*X, w.A, bf), bf, s, status));
+  int q = -1;  // buffer holding Q; -1 while Q = I
+  for (int t = 1; t <= p.iters; ++t) {
+    const bool last = t == p.iters;
+    const bool restart = !last && is_restart(p, t);
+    const bool need_qbf = bf && (last || restart);
+    const int h = free_idx(q, -1);
+    // H = c' A A + b' A + a' I
+    GemmDesc dh = symprod(w.A, w.A, c.c, &w.A, c.b, c.a, bf);
+    dh.out_f32 = w.kk[h];
+    dh.has_f32 = true;
+    if (q < 0 && need_qbf) {
+      dh.out_bf16 = w.qbf;
+      dh.has_bf16 = true;
+    }
+    OUO_TRY(run_gemm(dh, bf, s, status));
+    if (q < 0) {
+      q = h;  // Q = H I
+    } else {
+      const int nq = free_idx(q, h);
+      GemmDesc dq = symprod(w.kk[h], w.kk[q], 1.f, nullptr, 0.f, 0.f, bf);
+      dq.out_f32 = w.kk[nq];
+      dq.has_f32 = true;
+      if (need_qbf) {
+        dq.out_bf16 = w.qbf;
+        dq.has_bf16 = true;
+      }
+      OUO_TRY(run_gemm(dq, bf, s, status));
+      q = nq;
+    }
+    if (last) break;
+    if (restart) {
+      const Buf& Qop = bf ? w.qbf : w.kk[q];
+      OUO_TRY(run_gemm(apply_left(Qop, *X, *Xalt, 1.f, nullptr, 0.f), bf, s,
+                       status));
+      std::swap(X, Xalt);
+      OUO_TRY(run_gemm(syrk(*X, w.A, bf), bf, s, status));
+      q = -1;
+    } else {
+      // A <- H (H A)
+      GemmDesc dt = symprod(w.kk[h], w.A, 1.f, nullptr, 0.f, 0.f, bf);
+      dt.out_f32 = w.T;
+      dt.has_f32 = true;
+      OUO_TRY(run_gemm(dt, bf, s, status));
+      GemmDesc da = symprod(w.kk[h], w.T, 1.f, nullptr, 0.f, 0.f, bf);
+      da.out_f32 = w.A;
+      da.has_f32 = true;
+      OUO_TRY(run_gemm(da, bf, s, status));
+    }
+  }
+  if (q < 0) {
+    // no iteration: the output is X0 itself
+    OUO_TRY(convert_buf(*X, w.y, s));
+  } else {
+    const Buf& Qop = bf ? w.qbf : w.kk[q];
+    OUO_TRY(run_gemm(apply_left(Qop, *X, w.y, 1.f, nullptr, 0.f), bf, s, status));
+  }
+  return OUO_OK;
+}
+
+// Standard quintic Newton-Schulz on one group; result in w.y.
+int std_group(const ouo_ns_params& p, GroupWs& w, cudaStream_t s, int* status) {
+  const bool bf = p.precision == OUO_PREC_BF16;
+  const Coeffs c = scaled(p);
+  Buf* X = &w.x0;
+  Buf* Xalt = &w.x1;
+  for (int t = 1; t <= p.iters; ++t) {
+    OUO_TRY(run_gemm(syrk(*X, w.A, bf), bf, s, status));
+    // B = c' A A + b' A
+    GemmDesc db = symprod(w.A, w.A, c.c, &w.A, c.b, 0.f, bf);
+    if (w.bm.dtype == OUO_BF16) {
+      db.out_bf16 = w.bm;
+      db.has_bf16 = true;
+    } else {
+      db.out_f32 = w.bm;
+      db.has_f32 = true;
+    }
+    db.round_tf32 = false;
+    OUO_TRY(run_gemm(db, bf, s, status));
+    // X <- a' X + B X   (the last iteration writes the output buffer)
+    const Buf& dst = t == p.iters ? w.y : *Xalt;
+    OUO_TRY(run_gemm(apply_left(w.bm, *X, dst, 1.f, X, c.a), bf, s, status));
+    std::swap(X, Xalt);
+  }
+  if (p.iters == 0) OUO_TRY(convert_buf(*X, w.y, s));
+  return OUO_OK;
+}
+
+int validate_params(const ouo_ns_params* p) {
+  if (!p) return set_error(OUO_ERR_INVALID_ARG, "NULL ns params");
+  if (p->iters < 0 || p->iters > 1000)
+    return set_error(OUO_ERR_INVALID_ARG, "iters %d out of range", p->iters);
+  if (!(p->safety >= 1.0f) || !std::isfinite(p->safety))
+    return set_error(OUO_ERR_INVALID_ARG, "safety must be >= 1");
+  if (!(p->eps >= 0.0f))
+    return set_error(OUO_ERR_INVALID_ARG, "eps must be >= 0");
+  if (p->precision != OUO_PREC_BF16 && p->precision != OUO_PREC_FP32)
+    return set_error(OUO_ERR_INVALID_ARG, "unknown precision %d", p->precision);
+  if (p->n_restart < 0 || p->n_restart > OUO_MAX_RESTARTS)
+    return set_error(OUO_ERR_INVALID_ARG, "n_restart out of range");
+  if (!std::isfinite(p->a) || !std::isfinite(p->b) || !std::isfinite(p->c))
+    return set_error(OUO_ERR_INVALID_ARG, "non-finite coefficients");
+  return OUO_OK;
+}
+
+size_t plan_bytes(const ouo_mat* X, int nmat, const ouo_ns_params* p,
+                  bool gram, int o_dtype) {
+  Arena ar{nullptr, 0, 0, true};
+  for (const Group& g : group_by_shape(X, nmat))
+    carve(ar, g, orient(g), gram, p->precision, o_dtype);
+  return ar.used + 256;
+}
+
+int run_ns(const ouo_mat* X, int x_dtype, const ouo_mat* O, int o_dtype,
+           int nmat, const ouo_ns_params* p, void* ws, size_t ws_bytes,
+           int* dev_status, void* stream, bool gram) {
+  clear_error();
+  if (nmat < 0 || nmat > OUO_MAX_BATCH)
+    return set_error(OUO_ERR_INVALID_ARG, "nmat %d out of range", nmat);
+  OUO_TRY(validate_params(p));
+  if (nmat == 0) return OUO_OK;
+  OUO_TRY(validate_mats(X, nmat, x_dtype, "X"));
+  OUO_TRY(validate_mats(O, nmat, o_dtype, "O"));
+  OUO_TRY(validate_same_shapes(X, O, nmat, "X", "O"));
+  if (dev_status && ((uintptr_t)dev_status % 4))
+    return set_error(OUO_ERR_INVALID_ARG, "dev_status misaligned");
+  const size_t need = plan_bytes(X, nmat, p, gram, o_dtype);
+  if (!ws || ws_bytes < need)
+    return set_error(OUO_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given",
+                     need, ws_bytes);
+  if ((uintptr_t)ws % 256)
+    return set_error(OUO_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  OUO_TRY(require_sm100());
+  cudaStream_t s = (cudaStream_t)stream;
+  Arena ar{reinterpret_cast<char*>(ws), ws_bytes, 0, false};
+  for (const Group& g : group_by_shape(X, nmat)) {
+    const Oriented o = orient(g);
+    GroupWs w = carve(ar, g, o, gram, p->precision, o_dtype);
+    OUO_TRY(ns_prep(X, x_dtype, g, o.transpose, p->normalize != 0, p->eps, w.x0,
+                    w.scratch, s));
+    if (gram) OUO_TRY(gram_group(*p, w, s, dev_status));
+    else OUO_TRY(std_group(*p, w, s, dev_status));
+    OUO_TRY(ns_writeout(w.y, O, o_dtype, g, o.transpose, s));
+  }
+  return OUO_OK;
+}
+
+}  // namespace
+}  // namespace ouo
+
+extern "C" size_t ns_workspace_bytes(const ouo_mat* X, int nmat,
+                                     const ouo_ns_params* p) {
+  if (!X || !p || nmat <= 0) return 0;
+  return ouo::plan_bytes(X, nmat, p, false, OUO_F32);
+}
+
+extern "C" size_t gram_ns_workspace_bytes(const ouo_mat* X, int nmat,
+                                          const ouo_ns_params* p) {
+  if (!X || !p || nmat <= 0) return 0;
+  return ouo::plan_bytes(X, nmat, p, true, OUO_F32);
+}
+
+extern "C" int ns_orthogonalize(const ouo_mat* X, int x_dtype, const ouo_mat* O,
+                                int o_dtype, int nmat, const ouo_ns_params* p,
+                                void* ws, size_t ws_bytes, int* dev_status,
+                                void* stream) {
+  return ouo::run_ns(X, x_dtype, O, o_dtype, nmat, p, ws, ws_bytes, dev_status,
+                     stream, false);
+}
+
+extern "C" int gram_ns_orthogonalize(const ouo_mat* X, int x_dtype,
+                                     const ouo_mat* O, int o_dtype, int nmat,
+                                     const ouo_ns_params* p, void* ws,
+                                     size_t ws_bytes, int* dev_status,
+                                     void* stream) {
+  return ouo::run_ns(X, x_dtype, O, o_dtype, nmat, p, ws, ws_bytes, dev_status,
+                     stream, true);
+}
