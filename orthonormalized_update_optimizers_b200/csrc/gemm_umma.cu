@@ -33,9 +33,17 @@
 namespace ouo {
 namespace {
 
-constexpr int kThreads = 192;
+constexpr int kEpiWarps = 8;                 // two per TMEM lane quarter
+constexpr int kThreads = 64 + 32 * kEpiWarps;  // producer, MMA, epilogue
 constexpr uint32_t kTileM = 128;
 constexpr uint32_t kRowBytes = 128;  // one swizzle row: K bytes per stage
+// Epilogue staging: a 32 x 32 fp32 chunk per warp, 16-byte groups XOR-
+// swizzled by row so that row-wise and column-wise accesses are both free
+// of bank conflicts.
+__device__ __forceinline__ int stg_idx(int row, int col) {
+  return row * 32 + ((((col >> 2) ^ row) & 7) << 2) + (col & 3) +
+         ((col >> 5) << 5);
+}
 
 struct UmmaArgs {
   CUtensorMap tmA;
@@ -61,8 +69,10 @@ struct Cfg {
   static constexpr uint32_t kStageBytes = kABytes + kBBytes;
   static constexpr int kStages = BN == 256 ? 4 : 6;
   static constexpr uint32_t kTmemCols = 2 * BN;
+  // per epilogue warp: a 32 x 32 fp32 staging buffer
+  static constexpr uint32_t kEpiBytes = kEpiWarps * 32 * 32 * 4;
   static constexpr size_t kSmem =
-      1024 + (size_t)kStages * kStageBytes + 256;  // align pad + ring + bars
+      1024 + (size_t)kStages * kStageBytes + 256 + kEpiBytes;
 };
 
 // First column tile of row tile i that reaches the diagonal.
@@ -98,6 +108,35 @@ __device__ __forceinline__ void store_out(const UmmaArgs& a, int64_t b,
   if (a.has_bf16) a.Ob[b * a.sob + i * a.ldob + j] = f32_to_bf16(v);
 }
 
+// Stores 4 consecutive elements (row, col .. col+3); element t only when
+// bit t of `mask` is set.  Full masks use one 16-byte (fp32) or 8-byte
+// (bf16) store: workspace rows are 16-byte aligned and col is a multiple of 4.
+__device__ __forceinline__ void store4(const UmmaArgs& a, int64_t b,
+                                       int64_t row, int64_t col, float4 w,
+                                       uint32_t mask) {
+  if (mask == 0xFu) {
+    if (a.has_f32) {
+      float4 o = w;
+      if (a.round_tf32) {
+        o.x = round_tf32(o.x); o.y = round_tf32(o.y);
+        o.z = round_tf32(o.z); o.w = round_tf32(o.w);
+      }
+      *reinterpret_cast<float4*>(a.Of + b * a.sof + row * a.ldof + col) = o;
+    }
+    if (a.has_bf16) {
+      uint2 u;
+      u.x = pack_bf16x2(w.x, w.y);
+      u.y = pack_bf16x2(w.z, w.w);
+      *reinterpret_cast<uint2*>(a.Ob + b * a.sob + row * a.ldob + col) = u;
+    }
+    return;
+  }
+  const float e[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+  for (int t = 0; t < 4; ++t)
+    if (mask & (1u << t)) store_out(a, b, row, col + t, e[t]);
+}
+
 __device__ __forceinline__ float load_c0(const UmmaArgs& a, int64_t b,
                                          int64_t i, int64_t j) {
   const int64_t off = b * a.sc0 + i * a.ldc0 + j;
@@ -126,6 +165,8 @@ umma_gemm_kernel(const __grid_constant__ UmmaArgs a) {
   uint64_t* drain = tempty + 2;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  float* epi_smem =
+      reinterpret_cast<float*>(smem + C::kStages * C::kStageBytes + 256);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -136,7 +177,7 @@ umma_gemm_kernel(const __grid_constant__ UmmaArgs a) {
     }
     for (int s = 0; s < 2; ++s) {
       ptx::mbar_init(&tfull[s], 1);
-      ptx::mbar_init(&tempty[s], 4);  // one arrival per epilogue warp
+      ptx::mbar_init(&tempty[s], kEpiWarps);  // one arrival per epilogue warp
     }
     ptx::mbar_init(drain, 1);
     *abort_flag = 0;
@@ -263,23 +304,94 @@ umma_gemm_kernel(const __grid_constant__ UmmaArgs a) {
         break;
       }
       ptx::tc_fence_after();
-      const int64_t gi = ti * kTileM + q * 32 + lane;
+      // This warp owns tile rows q*32 .. q*32+31 (TMEM lanes) and one half
+      // of the columns; each chunk is 32 rows x 32 columns.  Values are
+      // finished with row = lane (where the symmetric C0 read (j, i) is
+      // coalesced), staged in shared memory, and written back with 16-byte
+      // stores: 8 lanes per 128-byte row, 4 rows per instruction, for the
+      // direct tile (i, j) and, for symmetric outputs, the mirrored tile
+      // (j, i).  Chunks entirely below the diagonal of a symmetric output
+      // are skipped; chunks fully inside and above it store without masks.
+      const int64_t row_base = ti * kTileM + q * 32;
+      const int64_t gi = row_base + lane;
+      float* stg = epi_smem + (warp - 2) * (32 * 32);
+      const int sub_r = lane >> 3, sub_c = 4 * (lane & 7);
+      const uint32_t half = (uint32_t)((warp - 2) >> 2);
 #pragma unroll 1
-      for (uint32_t c0 = 0; c0 < (uint32_t)BN; c0 += 32) {
+      for (uint32_t c0 = half * (BN / 2); c0 < (half + 1) * (BN / 2); c0 += 32) {
+        const int64_t gj0 = tj * BN + c0;
+        if (a.tri && gj0 + 31 < row_base) continue;  // below the diagonal
+        if (row_base >= a.M || gj0 >= a.N) continue;  // outside the output
+        const bool full_chunk = row_base + 32 <= a.M && gj0 + 32 <= a.N &&
+                                (!a.tri || gj0 >= row_base + 31);
         float v[32];
         ptx::tmem_ld32(tmem_base + ((q * 32u) << 16) + buf * BN + c0, v);
-        const int64_t gj0 = tj * BN + c0;
-        if (gi < a.M) {
+        if (a.tri) {
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
             const int64_t gj = gj0 + j;
-            if (gj >= a.N || (a.tri && gj < gi)) continue;
             float r = a.alpha * v[j];
-            if (a.has_c0) r += a.beta * (a.tri ? load_c0(a, b, gj, gi) : load_c0(a, b, gi, gj));
+            if (a.has_c0 && (full_chunk || (gi < a.M && gj < a.N && gj >= gi)))
+              r += a.beta * load_c0(a, b, gj, gi);
             if (gi == gj) r += a.gamma;
-            store_out(a, b, gi, gj, r);
-            if (a.tri && gi != gj) store_out(a, b, gj, gi, r);
+            v[j] = r;
           }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] *= a.alpha;
+        }
+        // direct tile: stage row-major [row][col]
+#pragma unroll
+        for (int j = 0; j < 32; j += 4)
+          *reinterpret_cast<float4*>(stg + stg_idx(lane, j)) =
+              make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+        __syncwarp();
+#pragma unroll 2
+        for (int it = 0; it < 8; ++it) {
+          const int rr = it * 4 + sub_r;
+          const int64_t gr = row_base + rr, gc = gj0 + sub_c;
+          float4 w = *reinterpret_cast<const float4*>(stg + stg_idx(rr, sub_c));
+          uint32_t mask = 0xFu;
+          if (!full_chunk) {
+            mask = 0;
+#pragma unroll
+            for (int t = 0; t < 4; ++t)
+              if (gr < a.M && gc + t < a.N && (!a.tri || gc + t >= gr)) mask |= 1u << t;
+          }
+          if (!a.tri && mask && (a.has_c0 || a.gamma != 0.f)) {
+            float e[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+              if (!(mask & (1u << t))) continue;
+              if (a.has_c0) e[t] += a.beta * load_c0(a, b, gr, gc + t);
+              if (gr == gc + t) e[t] += a.gamma;
+            }
+            w = make_float4(e[0], e[1], e[2], e[3]);
+          }
+          if (mask) store4(a, b, gr, gc, w, mask);
+        }
+        __syncwarp();
+        if (a.tri) {
+          // mirrored tile: stage transposed [col][row], store row gj
+#pragma unroll
+          for (int j = 0; j < 32; ++j) stg[stg_idx(j, lane)] = v[j];
+          __syncwarp();
+#pragma unroll 2
+          for (int it = 0; it < 8; ++it) {
+            const int rr = it * 4 + sub_r;           // source column offset
+            const int64_t dst_r = gj0 + rr;          // = source column gj
+            const int64_t dst_c = row_base + sub_c;  // = source rows gi
+            float4 w = *reinterpret_cast<const float4*>(stg + stg_idx(rr, sub_c));
+            uint32_t mask = 0xFu;
+            if (!full_chunk) {
+              mask = 0;
+#pragma unroll
+              for (int t = 0; t < 4; ++t)
+                if (dst_c + t < a.M && dst_r < a.N && dst_r >= dst_c + t) mask |= 1u << t;
+            }
+            if (mask) store4(a, b, dst_r, dst_c, w, mask);
+          }
+          __syncwarp();
         }
       }
       ptx::tc_fence_before();
