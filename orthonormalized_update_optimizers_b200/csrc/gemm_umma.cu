@@ -45,21 +45,36 @@ __device__ __forceinline__ int stg_idx(int row, int col) {
          ((col >> 5) << 5);
 }
 
-struct UmmaArgs {
+// One segment of a launch: a batch range [b0, b0 + nb) of one group of
+// equal-shape matrices, with its own operand maps, sizes and outputs.
+struct Segment {
   CUtensorMap tmA;
   CUtensorMap tmB;
-  int64_t M, N, K, nb;
-  int64_t tiles_m, tiles_n, tiles_per_mat, total_tiles;
-  int tri;
-  float alpha, beta, gamma;
-  int has_c0, c0_bf16, has_f32, round_tf32, has_bf16;
+  int64_t M, N, K;
+  int64_t nb, b0;
+  int64_t tiles_n, tiles_per_mat, tile_start;  // tile_start: first tile id
   const void* C0;
   int64_t ldc0, sc0;
   float* Of;
   int64_t ldof, sof;
   uint16_t* Ob;
   int64_t ldob, sob;
+  int direct;  // outputs go to dptr[dbase + b]
+  int dbase;
+};
+
+constexpr int kMaxSeg = 6;
+
+struct UmmaArgs {
+  Segment seg[kMaxSeg];
+  int nseg;
+  int64_t total_tiles;
+  int tri;
+  float alpha, beta, gamma;
+  int has_c0, c0_bf16, has_f32, round_tf32, has_bf16;
   int* status;
+  void* dptr[kChunk];
+  int64_t dld[kChunk];
 };
 
 template <int BN>
@@ -80,68 +95,126 @@ __device__ __forceinline__ int64_t tri_jmin(int64_t i, int BN) {
   return (i * (int64_t)kTileM) / BN;
 }
 
-__device__ __forceinline__ void decode_tile(const UmmaArgs& a, int BN,
-                                            int64_t tile, int64_t* b,
-                                            int64_t* ti, int64_t* tj) {
-  *b = tile / a.tiles_per_mat;
-  int64_t t = tile - *b * a.tiles_per_mat;
+// Launch-wide tile id -> (segment, matrix within the segment, tile row,
+// tile column).
+__device__ __forceinline__ int decode_tile(const UmmaArgs& a, int BN,
+                                           int64_t tile, int64_t* b,
+                                           int64_t* ti, int64_t* tj) {
+  int g = 0;
+  while (g + 1 < a.nseg && tile >= a.seg[g + 1].tile_start) ++g;
+  const Segment& sg = a.seg[g];
+  int64_t t = tile - sg.tile_start;
+  *b = t / sg.tiles_per_mat;
+  t -= *b * sg.tiles_per_mat;
   if (!a.tri) {
-    *ti = t / a.tiles_n;
-    *tj = t - *ti * a.tiles_n;
-    return;
+    *ti = t / sg.tiles_n;
+    *tj = t - *ti * sg.tiles_n;
+    return g;
   }
   int64_t i = 0;
   while (true) {
-    int64_t cnt = a.tiles_n - tri_jmin(i, BN);
+    int64_t cnt = sg.tiles_n - tri_jmin(i, BN);
     if (t < cnt) break;
     t -= cnt;
     ++i;
   }
   *ti = i;
   *tj = tri_jmin(i, BN) + t;
+  return g;
 }
 
-__device__ __forceinline__ void store_out(const UmmaArgs& a, int64_t b,
-                                          int64_t i, int64_t j, float v) {
-  if (a.has_f32)
-    a.Of[b * a.sof + i * a.ldof + j] = a.round_tf32 ? round_tf32(v) : v;
-  if (a.has_bf16) a.Ob[b * a.sob + i * a.ldob + j] = f32_to_bf16(v);
+// Output element addresses: workspace batch [b0 + b] or a caller matrix.
+__device__ __forceinline__ float* out_f32_at(const UmmaArgs& a,
+                                             const Segment& sg, int64_t b,
+                                             int64_t i, int64_t j) {
+  return sg.direct
+      ? reinterpret_cast<float*>(a.dptr[sg.dbase + b]) + i * a.dld[sg.dbase + b] + j
+      : sg.Of + (sg.b0 + b) * sg.sof + i * sg.ldof + j;
+}
+__device__ __forceinline__ uint16_t* out_bf16_at(const UmmaArgs& a,
+                                                 const Segment& sg, int64_t b,
+                                                 int64_t i, int64_t j) {
+  return sg.direct
+      ? reinterpret_cast<uint16_t*>(a.dptr[sg.dbase + b]) + i * a.dld[sg.dbase + b] + j
+      : sg.Ob + (sg.b0 + b) * sg.sob + i * sg.ldob + j;
+}
+
+// Output bases of one matrix of a segment (workspace or caller memory).
+struct TileOut {
+  float* f;
+  uint16_t* h;
+  int64_t ldf, ldh;
+};
+
+__device__ __forceinline__ TileOut tile_out(const UmmaArgs& a,
+                                            const Segment& sg, int64_t b) {
+  TileOut o;
+  o.f = a.has_f32 ? out_f32_at(a, sg, b, 0, 0) : nullptr;
+  o.h = a.has_bf16 ? out_bf16_at(a, sg, b, 0, 0) : nullptr;
+  o.ldf = sg.direct ? a.dld[sg.dbase + b] : sg.ldof;
+  o.ldh = sg.direct ? a.dld[sg.dbase + b] : sg.ldob;
+  return o;
+}
+
+__device__ __forceinline__ void store_elem(const UmmaArgs& a, const TileOut& o,
+                                           int64_t i, int64_t j, float v) {
+  if (a.has_f32) o.f[i * o.ldf + j] = a.round_tf32 ? round_tf32(v) : v;
+  if (a.has_bf16) o.h[i * o.ldh + j] = f32_to_bf16(v);
 }
 
 // Stores 4 consecutive elements (row, col .. col+3); element t only when
 // bit t of `mask` is set.  Full masks use one 16-byte (fp32) or 8-byte
-// (bf16) store: workspace rows are 16-byte aligned and col is a multiple of 4.
-__device__ __forceinline__ void store4(const UmmaArgs& a, int64_t b,
-                                       int64_t row, int64_t col, float4 w,
-                                       uint32_t mask) {
+// (bf16) store: output rows are 16-byte aligned and col is a multiple of 4.
+__device__ __forceinline__ void store4t(const UmmaArgs& a, const TileOut& o,
+                                        int64_t row, int64_t col, float4 w,
+                                        uint32_t mask) {
   if (mask == 0xFu) {
     if (a.has_f32) {
-      float4 o = w;
+      float4 v = w;
       if (a.round_tf32) {
-        o.x = round_tf32(o.x); o.y = round_tf32(o.y);
-        o.z = round_tf32(o.z); o.w = round_tf32(o.w);
+        v.x = round_tf32(v.x); v.y = round_tf32(v.y);
+        v.z = round_tf32(v.z); v.w = round_tf32(v.w);
       }
-      *reinterpret_cast<float4*>(a.Of + b * a.sof + row * a.ldof + col) = o;
+      *reinterpret_cast<float4*>(o.f + row * o.ldf + col) = v;
     }
     if (a.has_bf16) {
       uint2 u;
       u.x = pack_bf16x2(w.x, w.y);
       u.y = pack_bf16x2(w.z, w.w);
-      *reinterpret_cast<uint2*>(a.Ob + b * a.sob + row * a.ldob + col) = u;
+      *reinterpret_cast<uint2*>(o.h + row * o.ldh + col) = u;
     }
     return;
   }
   const float e[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
   for (int t = 0; t < 4; ++t)
-    if (mask & (1u << t)) store_out(a, b, row, col + t, e[t]);
+    if (mask & (1u << t)) store_elem(a, o, row, col + t, e[t]);
 }
 
-__device__ __forceinline__ float load_c0(const UmmaArgs& a, int64_t b,
-                                         int64_t i, int64_t j) {
-  const int64_t off = b * a.sc0 + i * a.ldc0 + j;
-  return a.c0_bf16 ? bf16_to_f32(reinterpret_cast<const uint16_t*>(a.C0)[off])
-                   : reinterpret_cast<const float*>(a.C0)[off];
+__device__ __forceinline__ float load_c0(const Segment& sg, int64_t b,
+                                         int64_t i, int64_t j, int bf16) {
+  const int64_t off = (sg.b0 + b) * sg.sc0 + i * sg.ldc0 + j;
+  return bf16 ? bf16_to_f32(reinterpret_cast<const uint16_t*>(sg.C0)[off])
+              : reinterpret_cast<const float*>(sg.C0)[off];
+}
+
+// Four consecutive C0 elements (i, j .. j+3); workspace rows are 16-byte
+// aligned and j is a multiple of 4.
+__device__ __forceinline__ void load_c0x4(const Segment& sg, int64_t b,
+                                          int64_t i, int64_t j, float e[4],
+                                          int bf16) {
+  const int64_t off = (sg.b0 + b) * sg.sc0 + i * sg.ldc0 + j;
+  if (bf16) {
+    uint2 u = *reinterpret_cast<const uint2*>(
+        reinterpret_cast<const uint16_t*>(sg.C0) + off);
+    e[0] = __uint_as_float(u.x << 16);
+    e[1] = __uint_as_float(u.x & 0xffff0000u);
+    e[2] = __uint_as_float(u.y << 16);
+    e[3] = __uint_as_float(u.y & 0xffff0000u);
+  } else {
+    float4 f = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(sg.C0) + off);
+    e[0] = f.x; e[1] = f.y; e[2] = f.z; e[3] = f.w;
+  }
 }
 
 template <int BN, int FMT /*1 bf16, 2 tf32*/, int B_MN>
@@ -182,8 +255,10 @@ umma_gemm_kernel(const __grid_constant__ UmmaArgs a) {
     ptx::mbar_init(drain, 1);
     *abort_flag = 0;
     ptx::fence_barrier_init();
-    ptx::prefetch_tmap(&a.tmA);
-    ptx::prefetch_tmap(&a.tmB);
+    for (int g = 0; g < a.nseg; ++g) {
+      ptx::prefetch_tmap(&a.seg[g].tmA);
+      ptx::prefetch_tmap(&a.seg[g].tmB);
+    }
   }
   if (warp == 1) {
     ptx::tmem_alloc(tmem_holder, C::kTmemCols);
@@ -193,7 +268,6 @@ umma_gemm_kernel(const __grid_constant__ UmmaArgs a) {
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
-  const int64_t nk = (a.K + kBK - 1) / kBK;
 
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------------------ producer
@@ -203,7 +277,10 @@ umma_gemm_kernel(const __grid_constant__ UmmaArgs a) {
     for (int64_t tile = blockIdx.x; ok && tile < a.total_tiles;
          tile += gridDim.x) {
       int64_t b, ti, tj;
-      decode_tile(a, BN, tile, &b, &ti, &tj);
+      const int g = decode_tile(a, BN, tile, &b, &ti, &tj);
+      const Segment& sg = a.seg[g];
+      const int64_t nk = (sg.K + kBK - 1) / kBK;
+      const int32_t z = (int32_t)(sg.b0 + b);
       for (int64_t kb = 0; kb < nk; ++kb) {
         if (!ptx::mbar_wait(&empty[stage], phase ^ 1, abort_flag)) {
           ok = false;
@@ -212,17 +289,17 @@ umma_gemm_kernel(const __grid_constant__ UmmaArgs a) {
         ptx::mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
         uint8_t* sa = smem + stage * C::kStageBytes;
         uint8_t* sb = sa + C::kABytes;
-        ptx::tma_load_3d(sa, &a.tmA, &full[stage], (int32_t)(kb * kBK),
-                         (int32_t)(ti * kTileM), (int32_t)b);
+        ptx::tma_load_3d(sa, &sg.tmA, &full[stage], (int32_t)(kb * kBK),
+                         (int32_t)(ti * kTileM), z);
         if (!B_MN) {
-          ptx::tma_load_3d(sb, &a.tmB, &full[stage], (int32_t)(kb * kBK),
-                           (int32_t)(tj * BN), (int32_t)b);
+          ptx::tma_load_3d(sb, &sg.tmB, &full[stage], (int32_t)(kb * kBK),
+                           (int32_t)(tj * BN), z);
         } else {
 #pragma unroll
           for (uint32_t c = 0; c < (uint32_t)BN / kChunkCols; ++c)
-            ptx::tma_load_3d(sb + c * kChunkBytes, &a.tmB, &full[stage],
+            ptx::tma_load_3d(sb + c * kChunkBytes, &sg.tmB, &full[stage],
                              (int32_t)(tj * BN + c * kChunkCols),
-                             (int32_t)(kb * kBK), (int32_t)b);
+                             (int32_t)(kb * kBK), z);
         }
         ++issued;
         if (++stage == (uint32_t)C::kStages) { stage = 0; phase ^= 1; }
@@ -231,10 +308,8 @@ umma_gemm_kernel(const __grid_constant__ UmmaArgs a) {
     if (!ok) {
       *abort_flag = 1;
       report_status(a.status, OUO_STATUS_TIMEOUT);
-    }
-    // Loads still in flight complete on their own; before the CTA exits,
-    // wait (bounded) for the last fill of every stage to land.
-    if (!ok) {
+      // Loads still in flight complete on their own; before the CTA exits,
+      // wait (bounded) for the last fill of every stage to land.
       for (int s = 0; s < C::kStages; ++s) {
         const int64_t fills = issued / C::kStages + (s < issued % C::kStages ? 1 : 0);
         if (fills > 0)
@@ -248,6 +323,9 @@ umma_gemm_kernel(const __grid_constant__ UmmaArgs a) {
     int64_t local = 0;
     for (int64_t tile = blockIdx.x; ok && tile < a.total_tiles;
          tile += gridDim.x, ++local) {
+      int64_t b, ti, tj;
+      const int g = decode_tile(a, BN, tile, &b, &ti, &tj);
+      const int64_t nk = (a.seg[g].K + kBK - 1) / kBK;
       const uint32_t buf = (uint32_t)(local & 1);
       const uint32_t tphase = (uint32_t)((local >> 1) & 1);
       if (!ptx::mbar_wait(&tempty[buf], tphase ^ 1, abort_flag)) {
@@ -295,12 +373,19 @@ umma_gemm_kernel(const __grid_constant__ UmmaArgs a) {
     for (int64_t tile = blockIdx.x; tile < a.total_tiles;
          tile += gridDim.x, ++local) {
       int64_t b, ti, tj;
-      decode_tile(a, BN, tile, &b, &ti, &tj);
+      const int g = decode_tile(a, BN, tile, &b, &ti, &tj);
+      const Segment& sg = a.seg[g];
       const uint32_t buf = (uint32_t)(local & 1);
       const uint32_t tphase = (uint32_t)((local >> 1) & 1);
-      if (!ptx::mbar_wait(&tfull[buf], tphase, abort_flag)) {
-        *abort_flag = 1;
-        report_status(a.status, OUO_STATUS_TIMEOUT);
+      // one lane polls the barrier; the warp follows through __syncwarp
+      int ok = 1;
+      if (lane == 0) ok = ptx::mbar_wait(&tfull[buf], tphase, abort_flag) ? 1 : 0;
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) {
+        if (lane == 0) {
+          *abort_flag = 1;
+          report_status(a.status, OUO_STATUS_TIMEOUT);
+        }
         break;
       }
       ptx::tc_fence_after();
@@ -316,25 +401,38 @@ umma_gemm_kernel(const __grid_constant__ UmmaArgs a) {
       const int64_t gi = row_base + lane;
       float* stg = epi_smem + (warp - 2) * (32 * 32);
       const int sub_r = lane >> 3, sub_c = 4 * (lane & 7);
+      const TileOut to = tile_out(a, sg, b);
       const uint32_t half = (uint32_t)((warp - 2) >> 2);
 #pragma unroll 1
       for (uint32_t c0 = half * (BN / 2); c0 < (half + 1) * (BN / 2); c0 += 32) {
         const int64_t gj0 = tj * BN + c0;
         if (a.tri && gj0 + 31 < row_base) continue;  // below the diagonal
-        if (row_base >= a.M || gj0 >= a.N) continue;  // outside the output
-        const bool full_chunk = row_base + 32 <= a.M && gj0 + 32 <= a.N &&
+        if (row_base >= sg.M || gj0 >= sg.N) continue;  // outside the output
+        const bool full_chunk = row_base + 32 <= sg.M && gj0 + 32 <= sg.N &&
                                 (!a.tri || gj0 >= row_base + 31);
         float v[32];
         ptx::tmem_ld32(tmem_base + ((q * 32u) << 16) + buf * BN + c0, v);
         if (a.tri) {
+          if (a.has_c0) {
+            // 32 independent loads (clamped into the matrix, so they can be
+            // issued together), used only where the element is kept
+            const int64_t gic = gi < sg.M ? gi : sg.M - 1;
+            float c0v[32];
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const int64_t gj = gj0 + j;
-            float r = a.alpha * v[j];
-            if (a.has_c0 && (full_chunk || (gi < a.M && gj < a.N && gj >= gi)))
-              r += a.beta * load_c0(a, b, gj, gi);
-            if (gi == gj) r += a.gamma;
-            v[j] = r;
+            for (int j = 0; j < 32; ++j) {
+              const int64_t gjc = gj0 + j < sg.N ? gj0 + j : sg.N - 1;
+              c0v[j] = load_c0(sg, b, gjc, gic, a.c0_bf16);
+            }
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = a.alpha * v[j] + a.beta * c0v[j];
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] *= a.alpha;
+          }
+          if (gi >= gj0 && gi < gj0 + 32) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (gi == gj0 + j) v[j] += a.gamma;
           }
         } else {
 #pragma unroll
@@ -356,19 +454,31 @@ umma_gemm_kernel(const __grid_constant__ UmmaArgs a) {
             mask = 0;
 #pragma unroll
             for (int t = 0; t < 4; ++t)
-              if (gr < a.M && gc + t < a.N && (!a.tri || gc + t >= gr)) mask |= 1u << t;
+              if (gr < sg.M && gc + t < sg.N && (!a.tri || gc + t >= gr)) mask |= 1u << t;
           }
-          if (!a.tri && mask && (a.has_c0 || a.gamma != 0.f)) {
-            float e[4] = {w.x, w.y, w.z, w.w};
+          if (!a.tri && mask) {
+            if (a.has_c0) {
+              float e[4];
+              if (mask == 0xFu) {
+                load_c0x4(sg, b, gr, gc, e, a.c0_bf16);
+              } else {
 #pragma unroll
-            for (int t = 0; t < 4; ++t) {
-              if (!(mask & (1u << t))) continue;
-              if (a.has_c0) e[t] += a.beta * load_c0(a, b, gr, gc + t);
-              if (gr == gc + t) e[t] += a.gamma;
+                for (int t = 0; t < 4; ++t)
+                  e[t] = (mask & (1u << t)) ? load_c0(sg, b, gr, gc + t, a.c0_bf16) : 0.f;
+              }
+              w.x += a.beta * e[0];
+              w.y += a.beta * e[1];
+              w.z += a.beta * e[2];
+              w.w += a.beta * e[3];
             }
-            w = make_float4(e[0], e[1], e[2], e[3]);
+            if (a.gamma != 0.f && gr >= gc && gr < gc + 4) {
+              if (gr == gc) w.x += a.gamma;
+              if (gr == gc + 1) w.y += a.gamma;
+              if (gr == gc + 2) w.z += a.gamma;
+              if (gr == gc + 3) w.w += a.gamma;
+            }
           }
-          if (mask) store4(a, b, gr, gc, w, mask);
+          if (mask) store4t(a, to, gr, gc, w, mask);
         }
         __syncwarp();
         if (a.tri) {
@@ -387,9 +497,9 @@ umma_gemm_kernel(const __grid_constant__ UmmaArgs a) {
               mask = 0;
 #pragma unroll
               for (int t = 0; t < 4; ++t)
-                if (dst_c + t < a.M && dst_r < a.N && dst_r >= dst_c + t) mask |= 1u << t;
+                if (dst_c + t < sg.M && dst_r < sg.N && dst_r >= dst_c + t) mask |= 1u << t;
             }
-            if (mask) store4(a, b, dst_r, dst_c, w, mask);
+            if (mask) store4t(a, to, dst_r, dst_c, w, mask);
           }
           __syncwarp();
         }
@@ -454,24 +564,19 @@ int make_map(CUtensorMap* map, const Buf& t, uint32_t box_cols,
   return OUO_OK;
 }
 
+int64_t tiles_per_matrix(const GemmDesc& g, int BN) {
+  const int64_t tm = ceil_div(g.M, kTileM), tn = ceil_div(g.N, BN);
+  if (!g.tri) return tm * tn;
+  int64_t cnt = 0;
+  for (int64_t i = 0; i < tm; ++i) cnt += tn - (i * (int64_t)kTileM) / BN;
+  return cnt;
+}
+
 template <int BN, int FMT, int B_MN>
-int launch(const GemmDesc& g, UmmaArgs& a, cudaStream_t stream) {
+int launch(const std::vector<GemmDesc>& gs, cudaStream_t stream, int* status) {
   using C = Cfg<BN>;
   constexpr uint32_t es = FMT == 1 ? 2 : 4;
   constexpr uint32_t bk = kRowBytes / es;
-  OUO_TRY(make_map(&a.tmA, g.A, bk, kTileM));
-  if (!B_MN) OUO_TRY(make_map(&a.tmB, g.B, bk, BN));
-  else OUO_TRY(make_map(&a.tmB, g.B, kRowBytes / es, bk));
-  a.tiles_m = ceil_div(g.M, kTileM);
-  a.tiles_n = ceil_div(g.N, BN);
-  if (g.tri) {
-    int64_t cnt = 0;
-    for (int64_t i = 0; i < a.tiles_m; ++i) cnt += a.tiles_n - (i * (int64_t)kTileM) / BN;
-    a.tiles_per_mat = cnt;
-  } else {
-    a.tiles_per_mat = a.tiles_m * a.tiles_n;
-  }
-  a.total_tiles = a.tiles_per_mat * g.nb;
   auto kern = umma_gemm_kernel<BN, FMT, B_MN>;
   static bool configured[64] = {false};
   int dev = 0;
@@ -481,44 +586,111 @@ int launch(const GemmDesc& g, UmmaArgs& a, cudaStream_t stream) {
         kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::kSmem));
     if (dev >= 0 && dev < 64) configured[dev] = true;
   }
-  int64_t grid = a.total_tiles < num_sms() ? a.total_tiles : num_sms();
-  if (grid < 1) return OUO_OK;
-  kern<<<(unsigned)grid, kThreads, C::kSmem, stream>>>(a);
-  OUO_CHECK_LAUNCH();
-  return OUO_OK;
+  const GemmDesc& g0 = gs[0];
+  UmmaArgs a;
+  memset(&a, 0, sizeof(a));
+  a.tri = g0.tri;
+  a.alpha = g0.alpha; a.beta = g0.beta; a.gamma = g0.gamma;
+  a.has_c0 = g0.has_c0;
+  a.c0_bf16 = g0.has_c0 && g0.C0.dtype == OUO_BF16;
+  a.has_f32 = g0.has_f32; a.round_tf32 = g0.round_tf32;
+  a.has_bf16 = g0.has_bf16;
+  a.status = status;
+  if (!g0.direct.empty()) {
+    a.has_f32 = g0.direct_dtype == OUO_F32;
+    a.has_bf16 = g0.direct_dtype == OUO_BF16;
+    a.round_tf32 = 0;
+  }
+  int ndirect = 0;
+  auto flush = [&]() -> int {
+    if (a.nseg == 0) return OUO_OK;
+    a.total_tiles = 0;
+    for (int s = 0; s < a.nseg; ++s) {
+      a.seg[s].tile_start = a.total_tiles;
+      a.total_tiles += a.seg[s].tiles_per_mat * a.seg[s].nb;
+    }
+    int64_t grid = a.total_tiles < num_sms() ? a.total_tiles : num_sms();
+    if (grid >= 1) {
+      kern<<<(unsigned)grid, kThreads, C::kSmem, stream>>>(a);
+      OUO_CHECK_LAUNCH();
+    }
+    a.nseg = 0;
+    ndirect = 0;
+    return OUO_OK;
+  };
+  for (const GemmDesc& g : gs) {
+    if (g.M < 1 || g.N < 1 || g.K < 1 || g.nb < 1) continue;
+    Segment proto;
+    memset(&proto, 0, sizeof(proto));
+    OUO_TRY(make_map(&proto.tmA, g.A, bk, kTileM));
+    if (!B_MN) OUO_TRY(make_map(&proto.tmB, g.B, bk, BN));
+    else OUO_TRY(make_map(&proto.tmB, g.B, kRowBytes / es, bk));
+    proto.M = g.M; proto.N = g.N; proto.K = g.K;
+    proto.tiles_n = ceil_div(g.N, BN);
+    proto.tiles_per_mat = tiles_per_matrix(g, BN);
+    proto.C0 = g.has_c0 ? g.C0.p : nullptr;
+    proto.ldc0 = g.C0.ld; proto.sc0 = g.C0.stride;
+    proto.Of = g.has_f32 ? reinterpret_cast<float*>(g.out_f32.p) : nullptr;
+    proto.ldof = g.out_f32.ld; proto.sof = g.out_f32.stride;
+    proto.Ob = g.has_bf16 ? reinterpret_cast<uint16_t*>(g.out_bf16.p) : nullptr;
+    proto.ldob = g.out_bf16.ld; proto.sob = g.out_bf16.stride;
+    proto.direct = g.direct.empty() ? 0 : 1;
+    int64_t b0 = 0;
+    while (b0 < g.nb) {
+      if (a.nseg == kMaxSeg || (proto.direct && ndirect == kChunk)) OUO_TRY(flush());
+      int64_t nb = g.nb - b0;
+      if (proto.direct && nb > kChunk - ndirect) nb = kChunk - ndirect;
+      Segment& sg = a.seg[a.nseg++];
+      sg = proto;
+      sg.b0 = b0;
+      sg.nb = nb;
+      if (proto.direct) {
+        sg.dbase = ndirect;
+        for (int64_t i = 0; i < nb; ++i) {
+          a.dptr[ndirect + i] = g.direct[b0 + i].p;
+          a.dld[ndirect + i] = g.direct[b0 + i].ld;
+        }
+        ndirect += (int)nb;
+      }
+      b0 += nb;
+    }
+  }
+  return flush();
 }
 
 }  // namespace
 
-int gemm_umma(const GemmDesc& g, cudaStream_t stream, int* status) {
-  if (g.A.dtype != g.B.dtype)
-    return set_error(OUO_ERR_UNSUPPORTED, "tensor-core GEMM needs equal operand types");
-  if (g.tri && (g.M != g.N || g.b_mn))
-    return set_error(OUO_ERR_INVALID_ARG, "symmetric GEMM needs M == N, K-major B");
-  if (g.M < 1 || g.N < 1 || g.K < 1 || g.nb < 1) return OUO_OK;
-  UmmaArgs a;
-  memset(&a, 0, sizeof(a));
-  a.M = g.M; a.N = g.N; a.K = g.K; a.nb = g.nb;
-  a.tri = g.tri;
-  a.alpha = g.alpha; a.beta = g.beta; a.gamma = g.gamma;
-  a.has_c0 = g.has_c0;
-  a.c0_bf16 = g.has_c0 && g.C0.dtype == OUO_BF16;
-  a.C0 = g.has_c0 ? g.C0.p : nullptr;
-  a.ldc0 = g.C0.ld; a.sc0 = g.C0.stride;
-  a.has_f32 = g.has_f32; a.round_tf32 = g.round_tf32;
-  a.Of = g.has_f32 ? reinterpret_cast<float*>(g.out_f32.p) : nullptr;
-  a.ldof = g.out_f32.ld; a.sof = g.out_f32.stride;
-  a.has_bf16 = g.has_bf16;
-  a.Ob = g.has_bf16 ? reinterpret_cast<uint16_t*>(g.out_bf16.p) : nullptr;
-  a.ldob = g.out_bf16.ld; a.sob = g.out_bf16.stride;
-  a.status = status;
-  const bool wide = g.N > 128;
-  if (g.A.dtype == OUO_BF16) {
-    if (g.b_mn) return wide ? launch<256, 1, 1>(g, a, stream) : launch<128, 1, 1>(g, a, stream);
-    return wide ? launch<256, 1, 0>(g, a, stream) : launch<128, 1, 0>(g, a, stream);
+int gemm_umma_grouped(const std::vector<GemmDesc>& gs, cudaStream_t stream,
+                      int* status) {
+  if (gs.empty()) return OUO_OK;
+  const GemmDesc& g0 = gs[0];
+  bool wide = false;
+  for (const GemmDesc& g : gs) {
+    if (g.A.dtype != g.B.dtype || g.A.dtype != g0.A.dtype)
+      return set_error(OUO_ERR_UNSUPPORTED, "tensor-core GEMM needs equal operand types");
+    if (g.tri != g0.tri || g.b_mn != g0.b_mn || g.has_c0 != g0.has_c0 ||
+        g.has_f32 != g0.has_f32 || g.has_bf16 != g0.has_bf16 ||
+        g.round_tf32 != g0.round_tf32 || g.direct.empty() != g0.direct.empty() ||
+        g.alpha != g0.alpha || g.beta != g0.beta || g.gamma != g0.gamma ||
+        (g.has_c0 && g.C0.dtype != g0.C0.dtype) ||
+        (!g.direct.empty() && g.direct_dtype != g0.direct_dtype))
+      return set_error(OUO_ERR_INVALID_ARG, "grouped GEMM descriptors differ");
+    if (g.tri && (g.M != g.N || g.b_mn))
+      return set_error(OUO_ERR_INVALID_ARG, "symmetric GEMM needs M == N, K-major B");
+    if (!g.direct.empty() && (int64_t)g.direct.size() != g.nb)
+      return set_error(OUO_ERR_INVALID_ARG, "direct output table size mismatch");
+    wide = wide || g.N > 128;
   }
-  if (g.b_mn) return wide ? launch<256, 2, 1>(g, a, stream) : launch<128, 2, 1>(g, a, stream);
-  return wide ? launch<256, 2, 0>(g, a, stream) : launch<128, 2, 0>(g, a, stream);
+  if (g0.A.dtype == OUO_BF16) {
+    if (g0.b_mn) return wide ? launch<256, 1, 1>(gs, stream, status) : launch<128, 1, 1>(gs, stream, status);
+    return wide ? launch<256, 1, 0>(gs, stream, status) : launch<128, 1, 0>(gs, stream, status);
+  }
+  if (g0.b_mn) return wide ? launch<256, 2, 1>(gs, stream, status) : launch<128, 2, 1>(gs, stream, status);
+  return wide ? launch<256, 2, 0>(gs, stream, status) : launch<128, 2, 0>(gs, stream, status);
+}
+
+int gemm_umma(const GemmDesc& g, cudaStream_t stream, int* status) {
+  return gemm_umma_grouped(std::vector<GemmDesc>{g}, stream, status);
 }
 
 }  // namespace ouo

@@ -78,11 +78,21 @@ struct GemmDesc {
   Buf out_bf16;
   bool has_bf16 = false;
   bool tri = false;
+  // When non-empty, matrix b of the batch is written to direct[b] (caller
+  // memory, element type direct_dtype, rows 16-byte aligned) instead of to
+  // out_f32 / out_bf16.  Tensor-core path only.
+  std::vector<MatRef> direct;
+  int direct_dtype = OUO_BF16;
 };
 
 // Tensor-core GEMM (tcgen05 / TMEM / TMA).  A and B are both bf16
 // (kind::f16) or both fp32 read as tf32 (kind::tf32).
 int gemm_umma(const GemmDesc& g, cudaStream_t stream, int* status);
+// Several equal-kind GEMMs (same operand types, majorness, symmetry,
+// epilogue coefficients and output kinds; any sizes) in as few launches as
+// possible: one persistent launch covers up to 6 batch segments.
+int gemm_umma_grouped(const std::vector<GemmDesc>& gs, cudaStream_t stream,
+                      int* status);
 // CUDA-core fp32 GEMM for the fp32 precision path.
 int gemm_simt(const GemmDesc& g, cudaStream_t stream);
 

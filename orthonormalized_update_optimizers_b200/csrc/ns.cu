@@ -164,14 +164,52 @@ int free_idx(int a, int b) {
   return -1;
 }
 
-// Gram Newton-Schulz on one group; the result (k x n) is left in w.y.
-int gram_group(const ouo_ns_params& p, GroupWs& w, cudaStream_t s,
-               int* status) {
+// One stage of the iteration over all groups: a single grouped tensor-core
+// launch (bf16 path) or one CUDA-core GEMM per group (fp32 path).
+int run_stage(const std::vector<GemmDesc>& ds, bool bf, cudaStream_t s,
+              int* status) {
+  if (bf) return gemm_umma_grouped(ds, s, status);
+  for (const GemmDesc& d : ds) OUO_TRY(gemm_simt(d, s));
+  return OUO_OK;
+}
+
+// The final product: groups writing to caller memory and groups writing to
+// workspace differ in output kind, so they go in separate grouped launches.
+int run_final(const std::vector<GemmDesc>& ds, bool bf, cudaStream_t s,
+              int* status) {
+  if (!bf) return run_stage(ds, bf, s, status);
+  std::vector<GemmDesc> dir, ws;
+  for (const GemmDesc& d : ds) (d.direct.empty() ? ws : dir).push_back(d);
+  if (!dir.empty()) OUO_TRY(gemm_umma_grouped(dir, s, status));
+  if (!ws.empty()) OUO_TRY(gemm_umma_grouped(ws, s, status));
+  return OUO_OK;
+}
+
+struct Plan {
+  std::vector<GroupWs> ws;
+  std::vector<std::vector<MatRef>> direct;  // per group; empty = write-out
+  int o_dtype;
+};
+
+// Attaches the caller's output table (if any) to the final product of group i.
+void final_output(GemmDesc& d, const Plan& pl, size_t i, bool bf) {
+  if (bf && !pl.direct[i].empty()) {
+    d.direct = pl.direct[i];
+    d.direct_dtype = pl.o_dtype;
+  }
+}
+
+// Gram Newton-Schulz, all groups in lockstep (they share the schedule).
+int gram_all(const ouo_ns_params& p, Plan& pl, cudaStream_t s, int* status) {
   const bool bf = p.precision == OUO_PREC_BF16;
   const Coeffs c = scaled(p);
-  Buf* X = &w.x0;
-  Buf* Xalt = &w.x1;
-  OUO_TRY(run_gemm(syrk(*X, w.A, bf), bf, s, status));
+  const size_t ng = pl.ws.size();
+  int xi = 0;  // current X is x0 (0) or x1 (1)
+  auto Xc = [&](GroupWs& w) -> Buf& { return xi ? w.x1 : w.x0; };
+  auto Xa = [&](GroupWs& w) -> Buf& { return xi ? w.x0 : w.x1; };
+  std::vector<GemmDesc> ds(ng);
+  for (size_t i = 0; i < ng; ++i) ds[i] = syrk(Xc(pl.ws[i]), pl.ws[i].A, bf);
+  OUO_TRY(run_stage(ds, bf, s, status));
   int q = -1;  // buffer holding Q; -1 while Q = I
   for (int t = 1; t <= p.iters; ++t) {
     const bool last = t == p.iters;
@@ -179,83 +217,123 @@ int gram_group(const ouo_ns_params& p, GroupWs& w, cudaStream_t s,
     const bool need_qbf = bf && (last || restart);
     const int h = free_idx(q, -1);
     // H = c' A A + b' A + a' I
-    GemmDesc dh = symprod(w.A, w.A, c.c, &w.A, c.b, c.a, bf);
-    dh.out_f32 = w.kk[h];
-    dh.has_f32 = true;
-    if (q < 0 && need_qbf) {
-      dh.out_bf16 = w.qbf;
-      dh.has_bf16 = true;
+    for (size_t i = 0; i < ng; ++i) {
+      GroupWs& w = pl.ws[i];
+      ds[i] = symprod(w.A, w.A, c.c, &w.A, c.b, c.a, bf);
+      ds[i].out_f32 = w.kk[h];
+      ds[i].has_f32 = true;
+      if (q < 0 && need_qbf) {
+        ds[i].out_bf16 = w.qbf;
+        ds[i].has_bf16 = true;
+      }
     }
-    OUO_TRY(run_gemm(dh, bf, s, status));
+    OUO_TRY(run_stage(ds, bf, s, status));
     if (q < 0) {
       q = h;  // Q = H I
     } else {
       const int nq = free_idx(q, h);
-      GemmDesc dq = symprod(w.kk[h], w.kk[q], 1.f, nullptr, 0.f, 0.f, bf);
-      dq.out_f32 = w.kk[nq];
-      dq.has_f32 = true;
-      if (need_qbf) {
-        dq.out_bf16 = w.qbf;
-        dq.has_bf16 = true;
+      for (size_t i = 0; i < ng; ++i) {
+        GroupWs& w = pl.ws[i];
+        ds[i] = symprod(w.kk[h], w.kk[q], 1.f, nullptr, 0.f, 0.f, bf);
+        ds[i].out_f32 = w.kk[nq];
+        ds[i].has_f32 = true;
+        if (need_qbf) {
+          ds[i].out_bf16 = w.qbf;
+          ds[i].has_bf16 = true;
+        }
       }
-      OUO_TRY(run_gemm(dq, bf, s, status));
+      OUO_TRY(run_stage(ds, bf, s, status));
       q = nq;
     }
     if (last) break;
     if (restart) {
-      const Buf& Qop = bf ? w.qbf : w.kk[q];
-      OUO_TRY(run_gemm(apply_left(Qop, *X, *Xalt, 1.f, nullptr, 0.f), bf, s,
-                       status));
-      std::swap(X, Xalt);
-      OUO_TRY(run_gemm(syrk(*X, w.A, bf), bf, s, status));
+      for (size_t i = 0; i < ng; ++i) {
+        GroupWs& w = pl.ws[i];
+        ds[i] = apply_left(bf ? w.qbf : w.kk[q], Xc(w), Xa(w), 1.f, nullptr, 0.f);
+      }
+      OUO_TRY(run_stage(ds, bf, s, status));
+      xi ^= 1;
+      for (size_t i = 0; i < ng; ++i) ds[i] = syrk(Xc(pl.ws[i]), pl.ws[i].A, bf);
+      OUO_TRY(run_stage(ds, bf, s, status));
       q = -1;
     } else {
       // A <- H (H A)
-      GemmDesc dt = symprod(w.kk[h], w.A, 1.f, nullptr, 0.f, 0.f, bf);
-      dt.out_f32 = w.T;
-      dt.has_f32 = true;
-      OUO_TRY(run_gemm(dt, bf, s, status));
-      GemmDesc da = symprod(w.kk[h], w.T, 1.f, nullptr, 0.f, 0.f, bf);
-      da.out_f32 = w.A;
-      da.has_f32 = true;
-      OUO_TRY(run_gemm(da, bf, s, status));
+      for (size_t i = 0; i < ng; ++i) {
+        GroupWs& w = pl.ws[i];
+        ds[i] = symprod(w.kk[h], w.A, 1.f, nullptr, 0.f, 0.f, bf);
+        ds[i].out_f32 = w.T;
+        ds[i].has_f32 = true;
+      }
+      OUO_TRY(run_stage(ds, bf, s, status));
+      for (size_t i = 0; i < ng; ++i) {
+        GroupWs& w = pl.ws[i];
+        ds[i] = symprod(w.kk[h], w.T, 1.f, nullptr, 0.f, 0.f, bf);
+        ds[i].out_f32 = w.A;
+        ds[i].has_f32 = true;
+      }
+      OUO_TRY(run_stage(ds, bf, s, status));
     }
   }
   if (q < 0) {
     // no iteration: the output is X0 itself
-    OUO_TRY(convert_buf(*X, w.y, s));
+    for (size_t i = 0; i < ng; ++i) {
+      OUO_TRY(convert_buf(Xc(pl.ws[i]), pl.ws[i].y, s));
+      pl.direct[i].clear();
+    }
   } else {
-    const Buf& Qop = bf ? w.qbf : w.kk[q];
-    OUO_TRY(run_gemm(apply_left(Qop, *X, w.y, 1.f, nullptr, 0.f), bf, s, status));
+    for (size_t i = 0; i < ng; ++i) {
+      GroupWs& w = pl.ws[i];
+      ds[i] = apply_left(bf ? w.qbf : w.kk[q], Xc(w), w.y, 1.f, nullptr, 0.f);
+      final_output(ds[i], pl, i, bf);
+    }
+    OUO_TRY(run_final(ds, bf, s, status));
   }
   return OUO_OK;
 }
 
-// Standard quintic Newton-Schulz on one group; result in w.y.
-int std_group(const ouo_ns_params& p, GroupWs& w, cudaStream_t s, int* status) {
+// Standard quintic Newton-Schulz, all groups in lockstep.
+int std_all(const ouo_ns_params& p, Plan& pl, cudaStream_t s, int* status) {
   const bool bf = p.precision == OUO_PREC_BF16;
   const Coeffs c = scaled(p);
-  Buf* X = &w.x0;
-  Buf* Xalt = &w.x1;
+  const size_t ng = pl.ws.size();
+  int xi = 0;
+  auto Xc = [&](GroupWs& w) -> Buf& { return xi ? w.x1 : w.x0; };
+  auto Xa = [&](GroupWs& w) -> Buf& { return xi ? w.x0 : w.x1; };
+  std::vector<GemmDesc> ds(ng);
   for (int t = 1; t <= p.iters; ++t) {
-    OUO_TRY(run_gemm(syrk(*X, w.A, bf), bf, s, status));
+    for (size_t i = 0; i < ng; ++i) ds[i] = syrk(Xc(pl.ws[i]), pl.ws[i].A, bf);
+    OUO_TRY(run_stage(ds, bf, s, status));
     // B = c' A A + b' A
-    GemmDesc db = symprod(w.A, w.A, c.c, &w.A, c.b, 0.f, bf);
-    if (w.bm.dtype == OUO_BF16) {
-      db.out_bf16 = w.bm;
-      db.has_bf16 = true;
-    } else {
-      db.out_f32 = w.bm;
-      db.has_f32 = true;
+    for (size_t i = 0; i < ng; ++i) {
+      GroupWs& w = pl.ws[i];
+      ds[i] = symprod(w.A, w.A, c.c, &w.A, c.b, 0.f, bf);
+      ds[i].round_tf32 = false;
+      if (w.bm.dtype == OUO_BF16) {
+        ds[i].out_bf16 = w.bm;
+        ds[i].has_bf16 = true;
+      } else {
+        ds[i].out_f32 = w.bm;
+        ds[i].has_f32 = true;
+      }
     }
-    db.round_tf32 = false;
-    OUO_TRY(run_gemm(db, bf, s, status));
-    // X <- a' X + B X   (the last iteration writes the output buffer)
-    const Buf& dst = t == p.iters ? w.y : *Xalt;
-    OUO_TRY(run_gemm(apply_left(w.bm, *X, dst, 1.f, X, c.a), bf, s, status));
-    std::swap(X, Xalt);
+    OUO_TRY(run_stage(ds, bf, s, status));
+    // X <- a' X + B X   (the last iteration writes the output)
+    const bool last = t == p.iters;
+    for (size_t i = 0; i < ng; ++i) {
+      GroupWs& w = pl.ws[i];
+      Buf& X = Xc(w);
+      ds[i] = apply_left(w.bm, X, last ? w.y : Xa(w), 1.f, &X, c.a);
+      if (last) final_output(ds[i], pl, i, bf);
+    }
+    OUO_TRY(last ? run_final(ds, bf, s, status) : run_stage(ds, bf, s, status));
+    xi ^= 1;
   }
-  if (p.iters == 0) OUO_TRY(convert_buf(*X, w.y, s));
+  if (p.iters == 0) {
+    for (size_t i = 0; i < ng; ++i) {
+      OUO_TRY(convert_buf(Xc(pl.ws[i]), pl.ws[i].y, s));
+      pl.direct[i].clear();
+    }
+  }
   return OUO_OK;
 }
 
@@ -306,15 +384,28 @@ int run_ns(const ouo_mat* X, int x_dtype, const ouo_mat* O, int o_dtype,
   OUO_TRY(require_sm100());
   cudaStream_t s = (cudaStream_t)stream;
   Arena ar{reinterpret_cast<char*>(ws), ws_bytes, 0, false};
-  for (const Group& g : group_by_shape(X, nmat)) {
+  const std::vector<Group> groups = group_by_shape(X, nmat);
+  Plan pl;
+  pl.o_dtype = o_dtype;
+  for (const Group& g : groups) {
     const Oriented o = orient(g);
-    GroupWs w = carve(ar, g, o, gram, p->precision, o_dtype);
-    OUO_TRY(ns_prep(X, x_dtype, g, o.transpose, p->normalize != 0, p->eps, w.x0,
-                    w.scratch, s));
-    if (gram) OUO_TRY(gram_group(*p, w, s, dev_status));
-    else OUO_TRY(std_group(*p, w, s, dev_status));
-    OUO_TRY(ns_writeout(w.y, O, o_dtype, g, o.transpose, s));
+    pl.ws.push_back(carve(ar, g, o, gram, p->precision, o_dtype));
+    OUO_TRY(ns_prep(X, x_dtype, g, o.transpose, p->normalize != 0, p->eps,
+                    pl.ws.back().x0, pl.ws.back().scratch, s));
+    // The last product writes straight into the caller's O when the layout
+    // allows (no transposition, 16-byte aligned rows, tensor-core path).
+    std::vector<MatRef> direct;
+    bool can_direct = p->precision == OUO_PREC_BF16 && !o.transpose;
+    for (int m : g.members) can_direct = can_direct && vec16(O[m], o_dtype);
+    if (can_direct)
+      for (int m : g.members) direct.push_back(MatRef{O[m].ptr, O[m].ld});
+    pl.direct.push_back(direct);
   }
+  if (gram) OUO_TRY(gram_all(*p, pl, s, dev_status));
+  else OUO_TRY(std_all(*p, pl, s, dev_status));
+  for (size_t i = 0; i < groups.size(); ++i)
+    if (pl.direct[i].empty())
+      OUO_TRY(ns_writeout(pl.ws[i].y, O, o_dtype, groups[i], orient(groups[i]).transpose, s));
   return OUO_OK;
 }
 

@@ -160,6 +160,83 @@ copy_kernel(const __grid_constant__ CopyArgs a) {
   }
 }
 
+struct RowCopyArgs {
+  int nmat;
+  int src_bf16, dst_bf16;
+  int to_caller;       // 0: caller -> workspace, 1: workspace -> caller
+  const float* scale;  // per matrix of the launch, or NULL
+  int64_t rows, cols;
+  void* C[kChunk];
+  int64_t ldc[kChunk];
+  uint8_t vec[kChunk];  // caller rows start on 16-byte boundaries
+  char* wbase;
+  int64_t wld, wstride;
+};
+
+__device__ __forceinline__ void load4v(const char* p, int bf16, float v[4]) {
+  if (bf16) {
+    uint2 u = *reinterpret_cast<const uint2*>(p);
+    v[0] = __uint_as_float(u.x << 16);
+    v[1] = __uint_as_float(u.x & 0xffff0000u);
+    v[2] = __uint_as_float(u.y << 16);
+    v[3] = __uint_as_float(u.y & 0xffff0000u);
+  } else {
+    float4 f = *reinterpret_cast<const float4*>(p);
+    v[0] = f.x; v[1] = f.y; v[2] = f.z; v[3] = f.w;
+  }
+}
+
+__device__ __forceinline__ void store4v(char* p, int bf16, const float v[4]) {
+  if (bf16) {
+    uint2 u;
+    u.x = pack_bf16x2(v[0], v[1]);
+    u.y = pack_bf16x2(v[2], v[3]);
+    *reinterpret_cast<uint2*>(p) = u;
+  } else {
+    *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+  }
+}
+
+// Row-to-row copy without transposition: one warp per row, 4 elements per
+// lane per step with 8- or 16-byte accesses where the caller rows allow.
+__global__ void __launch_bounds__(256)
+rowcopy_kernel(const __grid_constant__ RowCopyArgs a) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  const int64_t total = a.rows * a.nmat;
+  const int ses = a.src_bf16 ? 2 : 4, des = a.dst_bf16 ? 2 : 4;
+  for (int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+       row < total; row += warps) {
+    const int64_t b = row / a.rows, r = row - b * a.rows;
+    const float s = a.scale ? a.scale[b] : 1.0f;
+    const char* src;
+    char* dst;
+    if (a.to_caller) {
+      src = a.wbase + ((size_t)b * a.wstride + (size_t)r * a.wld) * ses;
+      dst = reinterpret_cast<char*>(a.C[b]) + (size_t)r * a.ldc[b] * des;
+    } else {
+      src = reinterpret_cast<const char*>(a.C[b]) + (size_t)r * a.ldc[b] * ses;
+      dst = a.wbase + ((size_t)b * a.wstride + (size_t)r * a.wld) * des;
+    }
+    const int64_t n4 = a.vec[b] ? (a.cols >> 2) : 0;
+    for (int64_t q = lane; q < n4; q += 32) {
+      float v[4];
+      load4v(src + 4 * q * ses, a.src_bf16, v);
+      v[0] *= s; v[1] *= s; v[2] *= s; v[3] *= s;
+      store4v(dst + 4 * q * des, a.dst_bf16, v);
+    }
+    for (int64_t c = 4 * n4 + lane; c < a.cols; c += 32)
+      st_elem(dst, c, a.dst_bf16, ld_elem(src, c, a.src_bf16) * s);
+  }
+}
+
+unsigned rows_grid(int64_t rows) {
+  int64_t blocks = ceil_div(rows, 8);
+  int64_t cap = (int64_t)num_sms() * 8;
+  if (blocks > cap) blocks = cap;
+  return (unsigned)(blocks < 1 ? 1 : blocks);
+}
+
 dim3 copy_grid(int64_t rows, int64_t cols, int nmat) {
   int64_t tr = ceil_div(rows, 32), tc = ceil_div(cols, 32);
   int64_t want = (int64_t)num_sms() * 8;
@@ -229,6 +306,28 @@ int ns_prep(const ouo_mat* X, int x_dtype, const Group& grp, bool transpose,
                                               grp.rows, eps, scales + c0);
       OUO_CHECK_LAUNCH();
     }
+    if (!transpose) {
+      RowCopyArgs ra;
+      ra.nmat = cn;
+      ra.src_bf16 = x_dtype == OUO_BF16;
+      ra.dst_bf16 = x0.dtype == OUO_BF16;
+      ra.to_caller = 0;
+      ra.scale = normalize ? scales + c0 : nullptr;
+      ra.rows = grp.rows;
+      ra.cols = grp.cols;
+      for (int i = 0; i < cn; ++i) {
+        const ouo_mat& m = X[grp.members[c0 + i]];
+        ra.C[i] = m.ptr;
+        ra.ldc[i] = m.ld;
+        ra.vec[i] = vec16(m, x_dtype);
+      }
+      ra.wbase = x0.p + (size_t)c0 * x0.stride * elem_size(x0.dtype);
+      ra.wld = x0.ld;
+      ra.wstride = x0.stride;
+      rowcopy_kernel<<<rows_grid(grp.rows * cn), 256, 0, stream>>>(ra);
+      OUO_CHECK_LAUNCH();
+      continue;
+    }
     CopyArgs ca;
     ca.nmat = cn;
     ca.src_bf16 = x_dtype == OUO_BF16;
@@ -257,6 +356,28 @@ int ns_writeout(const Buf& y, const ouo_mat* O, int o_dtype, const Group& grp,
   const int nb = (int)grp.members.size();
   for (int c0 = 0; c0 < nb; c0 += kChunk) {
     int cn = nb - c0 < kChunk ? nb - c0 : kChunk;
+    if (!transpose) {
+      RowCopyArgs ra;
+      ra.nmat = cn;
+      ra.src_bf16 = y.dtype == OUO_BF16;
+      ra.dst_bf16 = o_dtype == OUO_BF16;
+      ra.to_caller = 1;
+      ra.scale = nullptr;
+      ra.rows = grp.rows;
+      ra.cols = grp.cols;
+      for (int i = 0; i < cn; ++i) {
+        const ouo_mat& m = O[grp.members[c0 + i]];
+        ra.C[i] = m.ptr;
+        ra.ldc[i] = m.ld;
+        ra.vec[i] = vec16(m, o_dtype);
+      }
+      ra.wbase = y.p + (size_t)c0 * y.stride * elem_size(y.dtype);
+      ra.wld = y.ld;
+      ra.wstride = y.stride;
+      rowcopy_kernel<<<rows_grid(grp.rows * cn), 256, 0, stream>>>(ra);
+      OUO_CHECK_LAUNCH();
+      continue;
+    }
     CopyArgs ca;
     ca.nmat = cn;
     ca.src_bf16 = y.dtype == OUO_BF16;
