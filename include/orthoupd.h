@@ -89,6 +89,8 @@ extern "C" {
 
 #define OUO_MAX_BATCH 4096
 #define OUO_MAX_RESTARTS 8
+/* size of the fixed scratch array of gram_ns_orthogonalize_noalloc (64 MiB) */
+#define OUO_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
 
 typedef struct ouo_mat {
   void* ptr;     /* device pointer to element (0, 0)                        */
@@ -217,6 +219,33 @@ int gram_ns_orthogonalize(const ouo_mat* X, int x_dtype, const ouo_mat* O,
                           int o_dtype, int nmat, const ouo_ns_params* p,
                           void* ws, size_t ws_bytes, int* dev_status,
                           void* stream);
+
+/*
+ * gram_ns_orthogonalize_noalloc -- gram_ns_orthogonalize for callers that
+ * cannot allocate device memory (no counterpart on the pages: it is a
+ * service of this library).  Such callers include plugins running inside a
+ * host framework whose own pool owns all device memory, and latency-critical
+ * paths that must not pay cudaMalloc's implicit synchronization; they cannot
+ * provide the workspace gram_ns_orthogonalize needs.
+ *
+ * Same arguments and results as gram_ns_orthogonalize minus the workspace:
+ * the library uses a fixed scratch array of OUO_NOALLOC_SCRATCH_BYTES bytes
+ * in its own device image instead, and allocates nothing (no cudaMalloc, no
+ * allocating library routine).  Every GPU that loads this part of the
+ * library holds the array until the process exits.
+ *   - A batch whose gram_ns_workspace_bytes() exceeds the array is refused
+ *     with OUO_ERR_WORKSPACE before anything is launched.
+ *   - The first call on each device (with that device current) looks up the
+ *     array's device address; make that first call before any stream
+ *     capture.
+ *   - Every call shares the array; calls whose kernels overlap on the GPU
+ *     (e.g. on two unordered streams) race on it.  Each call overwrites what
+ *     it reads, so no state carries over between calls.
+ */
+int gram_ns_orthogonalize_noalloc(const ouo_mat* X, int x_dtype,
+                                  const ouo_mat* O, int o_dtype, int nmat,
+                                  const ouo_ns_params* p, int* dev_status,
+                                  void* stream);
 
 /*
  * apply_update -- the weight update that ends the step ([D3s] 输入输出流程:

@@ -27,14 +27,15 @@ OUO_DION_QR = 1
 OUO_STATUS_TIMEOUT = 1
 OUO_STATUS_BREAKDOWN = 2
 OUO_MAX_RESTARTS = 8
+OUO_NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024
 
 # every symbol the header declares
 EXPORTED = (
     "ouo_version", "ouo_last_error", "ouo_launch_count", "ouo_ns_default", "ouo_dion_default",
     "dion_momentum_update", "dion3_num_selected", "dion3_select_rows",
     "ns_workspace_bytes", "ns_orthogonalize", "gram_ns_workspace_bytes",
-    "gram_ns_orthogonalize", "apply_update", "dion_workspace_bytes",
-    "dion_lowrank_step",
+    "gram_ns_orthogonalize", "gram_ns_orthogonalize_noalloc", "apply_update",
+    "dion_workspace_bytes", "dion_lowrank_step",
 )
 
 
@@ -90,6 +91,7 @@ _PROTOS = {
     "ns_orthogonalize": (_I, [_MP, _I, _MP, _I, _I, _NP, _P, _SZ, _P, _P]),
     "gram_ns_workspace_bytes": (_SZ, [_MP, _I, _NP]),
     "gram_ns_orthogonalize": (_I, [_MP, _I, _MP, _I, _I, _NP, _P, _SZ, _P, _P]),
+    "gram_ns_orthogonalize_noalloc": (_I, [_MP, _I, _MP, _I, _I, _NP, _P, _P]),
     "apply_update": (_I, [_MP, _I, _MP, _I, _P, _I, _F, _P, _F, _P]),
     "dion_workspace_bytes": (_SZ, [_MP, _I, _DP]),
     "dion_lowrank_step": (_I, [_MP, _MP, _I, _MP, _MP, _I, _I, _DP, _P, _P, _SZ,

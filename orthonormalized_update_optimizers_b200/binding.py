@@ -20,6 +20,7 @@ __all__ = [
     "MatBatch", "ns_params", "dion_params", "dion_momentum_update",
     "dion3_num_selected", "dion3_select_rows", "ns_workspace_bytes",
     "ns_orthogonalize", "gram_ns_workspace_bytes", "gram_ns_orthogonalize",
+    "gram_ns_orthogonalize_noalloc",
     "apply_update", "dion_workspace_bytes", "dion_lowrank_step", "version",
     "launch_count",
 ]
@@ -183,6 +184,18 @@ def gram_ns_orthogonalize(X, O, params=None, workspace=None, status=None,
                           stream=None) -> None:
     _run_ns("gram_ns_orthogonalize", gram_ns_workspace_bytes, X, O, params,
             workspace, status, stream)
+
+
+def gram_ns_orthogonalize_noalloc(X, O, params=None, status=None,
+                                  stream=None) -> None:
+    """gram_ns_orthogonalize without a workspace, for callers that cannot
+    allocate device memory: the library's fixed scratch array (shared by all
+    calls; calls that overlap on the GPU race) stands in for it."""
+    Xb, Ob = _batch(X), _batch(O)
+    p = params or ns_params()
+    L.check("gram_ns_orthogonalize_noalloc", L.lib().gram_ns_orthogonalize_noalloc(
+        Xb.arr, Xb.dtype, Ob.arr, Ob.dtype, Xb.n, ctypes.byref(p), _ptr(status),
+        _stream(stream)))
 
 
 def apply_update(W, O, lr: float, idx: Optional[torch.Tensor] = None,
