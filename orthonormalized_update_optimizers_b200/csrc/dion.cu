@@ -1,10 +1,402 @@
-// Dion / Orth-Dion low-rank step (placeholder until its kernels land).
+// Dion / Orth-Dion low-rank step.
+//
+// Source: "Orth-Dion: Eliminating Geometric Mismatch in Distributed Low-Rank
+// Spectral Optimization" -- Problem Statement (rank-r factors from a single
+// power-iteration step per optimizer step), The Geometric Insight (Dion's
+// column normalization of the right factor), Orth-Dion (QR of the right
+// factor instead, same power iteration and residual buffer), Theoretical
+// Contributions (error-feedback coefficient beta); "Dion: The Distributed
+// Orthonormal Update Revolution Is Here", Technical details.
+//
+// Per matrix (B is the momentum buffer after B = M + G, m x n fp32):
+//   Pt = Qt B^T                      (r x m; Qt = Q_prev^T is the state)
+//   Pt <- rows orthonormalized       (CholeskyQR2: P = orth(B Q_prev))
+//   Rt = Pt B                        (r x n; R = B^T P)
+//   Qt_new = rows of Rt normalized   (Dion)  or  rows orthonormalized (Orth-Dion)
+//   M <- beta B - (beta - mu) P Rt   (residual buffer / error feedback)
+//   W <- (1 - lr wd) W - lr s P Qt_new
+//   state <- Qt_new
+// Working in the transposed layouts keeps every large product on the
+// tcgen05 GEMM (tf32 operands, fp32 accumulation) with K-major A.  The
+// orthonormalization works on r x L row blocks X: S = X X^T in fp32 (split
+// over L, partial sums added in float64 in a fixed order), S = L L^T by a
+// one-CTA Cholesky, L inverted in place, X <- L^-1 X (rows orthonormal; the
+// implied R = L^T has a positive diagonal, the unique QR).  Two passes
+// (CholeskyQR2).  A failed pivot retries with the shift of shifted
+// CholeskyQR (11 (L r + r (r + 1)) u ||X||_F^2); a second failure sets
+// OUO_STATUS_BREAKDOWN.
+#include <cmath>
+
 #include "internal.h"
+
+namespace ouo {
+namespace {
+
+// --------------------------------------------------------------- Gram S
+constexpr int kGT = 32;  // Gram tile
+
+struct GramArgs {
+  const float* X;
+  int64_t ld;
+  int r;
+  int64_t L, chunk;
+  float* part;  // [splits][r][r]
+  int tiles;    // ceil(r / 32)
+};
+
+// grid.x: upper tile pairs (ti <= tj), grid.y: split of the L range.
+__global__ void __launch_bounds__(256) gram_partial_kernel(const GramArgs a) {
+  __shared__ float xi[kGT][kGT + 1];
+  __shared__ float xj[kGT][kGT + 1];
+  int t = blockIdx.x, ti = 0;
+  while (t >= a.tiles - ti) { t -= a.tiles - ti; ++ti; }
+  const int tj = ti + t;
+  const int64_t l0 = (int64_t)blockIdx.y * a.chunk;
+  const int64_t l1 = l0 + a.chunk < a.L ? l0 + a.chunk : a.L;
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int64_t k0 = l0; k0 < l1; k0 += kGT) {
+    for (int e = threadIdx.x; e < kGT * kGT; e += 256) {
+      const int rr = e >> 5, kk = e & 31;
+      const int64_t k = k0 + kk;
+      const int ri = ti * kGT + rr, rj = tj * kGT + rr;
+      xi[kk][rr] = (ri < a.r && k < l1) ? a.X[ri * a.ld + k] : 0.f;
+      xj[kk][rr] = (rj < a.r && k < l1) ? a.X[rj * a.ld + k] : 0.f;
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int kk = 0; kk < kGT; ++kk) {
+      const float bj = xj[kk][tx];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) acc[u] = __fmaf_rn(xi[kk][ty + 8 * u], bj, acc[u]);
+    }
+    __syncthreads();
+  }
+  float* part = a.part + (size_t)blockIdx.y * a.r * a.r;
+  const int j = tj * kGT + tx;
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int i = ti * kGT + ty + 8 * u;
+    if (i < a.r && j < a.r) {
+      part[(size_t)i * a.r + j] = acc[u];
+      part[(size_t)j * a.r + i] = acc[u];
+    }
+  }
+}
+
+// ---------------------------------------------------- Cholesky + inverse
+// One CTA.  S is summed from the partials in float64 (fixed order) and kept
+// as a packed lower triangle (fp32) in `tri` (shared or global memory).
+// Cholesky S = L L^T in place, then L^-1 in place, then written as a full
+// lower-triangular r x r row-major fp32 matrix.
+__device__ __forceinline__ int tri_at(int i, int j) {  // j <= i
+  return i * (i + 1) / 2 + j;
+}
+
+struct CholArgs {
+  const float* part;
+  int splits;
+  int r;
+  int64_t L;        // length of the rows of X (for the shift)
+  float* tri_glob;  // packed scratch when the triangle does not fit in smem
+  float* Linv;      // r x r out, row pitch ldl
+  int64_t ldl;
+  int* status;
+  int use_smem;
+};
+
+__device__ void chol_load(const CholArgs& a, float* tri, float shift) {
+  const int n = a.r * (a.r + 1) / 2;
+  for (int e = threadIdx.x; e < n; e += blockDim.x) {
+    // invert e -> (i, j), j <= i
+    int i = (int)((sqrtf(8.f * (float)e + 1.f) - 1.f) * 0.5f);
+    while (tri_at(i + 1, 0) <= e) ++i;
+    while (tri_at(i, 0) > e) --i;
+    const int j = e - tri_at(i, 0);
+    double s = 0.0;
+    for (int p = 0; p < a.splits; ++p)
+      s += (double)a.part[(size_t)p * a.r * a.r + (size_t)i * a.r + j];
+    if (i == j) s += (double)shift;
+    tri[e] = (float)s;
+  }
+  __syncthreads();
+}
+
+// Right-looking Cholesky in place; returns false if a pivot is not positive.
+__device__ bool chol_factor(const CholArgs& a, float* tri, int* s_fail) {
+  const int r = a.r;
+  if (threadIdx.x == 0) *s_fail = 0;
+  __syncthreads();
+  for (int k = 0; k < r; ++k) {
+    const float piv = tri[tri_at(k, k)];
+    if (!(piv > 0.f) || !isfinite(piv)) {
+      if (threadIdx.x == 0) *s_fail = 1;
+      __syncthreads();
+      return false;
+    }
+    const float d = sqrtf(piv);
+    const float inv = 1.0f / d;
+    __syncthreads();
+    if (threadIdx.x == 0) tri[tri_at(k, k)] = d;
+    for (int i = k + 1 + threadIdx.x; i < r; i += blockDim.x) tri[tri_at(i, k)] *= inv;
+    __syncthreads();
+    // trailing update S[i][j] -= L[i][k] L[j][k], k < j <= i
+    const int m = r - k - 1;
+    const int cnt = m * (m + 1) / 2;
+    for (int e = threadIdx.x; e < cnt; e += blockDim.x) {
+      int ii = (int)((sqrtf(8.f * (float)e + 1.f) - 1.f) * 0.5f);
+      while ((ii + 1) * (ii + 2) / 2 <= e) ++ii;
+      while (ii * (ii + 1) / 2 > e) --ii;
+      const int jj = e - ii * (ii + 1) / 2;
+      const int i = k + 1 + ii, j = k + 1 + jj;
+      tri[tri_at(i, j)] -= tri[tri_at(i, k)] * tri[tri_at(j, k)];
+    }
+    __syncthreads();
+  }
+  return true;
+}
+
+// In-place inverse of the packed lower-triangular L (column j from the
+// last to the first: L^-1[j+1:, j] = -L^-1[j+1:, j+1:] L[j+1:, j] / L[j][j]).
+__device__ void tri_invert(const CholArgs& a, float* tri, float* tmp) {
+  const int r = a.r;
+  for (int j = r - 1; j >= 0; --j) {
+    const float djj = 1.0f / tri[tri_at(j, j)];
+    // tmp = L[j+1:, j] (original column)
+    for (int i = j + 1 + threadIdx.x; i < r; i += blockDim.x) tmp[i] = tri[tri_at(i, j)];
+    __syncthreads();
+    for (int i = j + 1 + threadIdx.x; i < r; i += blockDim.x) {
+      float s = 0.f;
+      for (int k = j + 1; k <= i; ++k) s = __fmaf_rn(tri[tri_at(i, k)], tmp[k], s);
+      tri[tri_at(i, j)] = -s * djj;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) tri[tri_at(j, j)] = djj;
+    __syncthreads();
+  }
+}
+
+__global__ void __launch_bounds__(1024) chol_inv_kernel(const CholArgs a) {
+  extern __shared__ float sm[];
+  __shared__ int s_fail;
+  const int r = a.r;
+  float* tri = a.use_smem ? sm : a.tri_glob;
+  float* tmp = a.use_smem ? sm + r * (r + 1) / 2 : a.tri_glob + r * (r + 1) / 2;
+  chol_load(a, tri, 0.f);
+  if (!chol_factor(a, tri, &s_fail)) {
+    // shifted CholeskyQR: 11 (L r + r (r + 1)) u ||X||_F^2, ||X||_F^2 = tr S
+    __shared__ float s_trace;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      double tr = 0.0;
+      for (int i = 0; i < r; ++i)
+        for (int p = 0; p < a.splits; ++p)
+          tr += (double)a.part[(size_t)p * r * r + (size_t)i * r + i];
+      const double u = 5.9604644775390625e-8;  // 2^-24
+      s_trace = (float)(11.0 * ((double)a.L * r + (double)r * (r + 1)) * u * tr);
+    }
+    __syncthreads();
+    chol_load(a, tri, s_trace > 0.f ? s_trace : 1e-30f);
+    if (!chol_factor(a, tri, &s_fail)) {
+      if (threadIdx.x == 0) report_status(a.status, OUO_STATUS_BREAKDOWN);
+      // keep going with unit pivots where the factorization failed
+      __syncthreads();
+      for (int e = threadIdx.x; e < r * (r + 1) / 2; e += blockDim.x) tri[e] = 0.f;
+      __syncthreads();
+      for (int i = threadIdx.x; i < r; i += blockDim.x) tri[tri_at(i, i)] = 1.f;
+      __syncthreads();
+    }
+  }
+  tri_invert(a, tri, tmp);
+  for (int e = threadIdx.x; e < r * r; e += blockDim.x) {
+    const int i = e / r, j = e - (e / r) * r;
+    a.Linv[(int64_t)i * a.ldl + j] = j <= i ? tri[tri_at(i, j)] : 0.f;
+  }
+}
+
+// ------------------------------------------------------ row normalization
+// Q[c][:] = R[c][:] / (||R[c][:]||_2 + eps); one block per row, float64
+// sum of squares in a fixed order.
+__global__ void __launch_bounds__(256)
+rownorm_kernel(const float* R, int64_t ldr, float* Q, int64_t ldq, int64_t n,
+               float eps) {
+  __shared__ double part[8];
+  const int64_t c = blockIdx.x;
+  const float* row = R + c * ldr;
+  double acc = 0.0;
+  for (int64_t j = threadIdx.x; j < n; j += blockDim.x) acc += (double)row[j] * row[j];
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = acc;
+  __syncthreads();
+  double tot = 0.0;
+  for (int w = 0; w < 8; ++w) tot += part[w];
+  const float inv = (float)(1.0 / (sqrt(tot) + (double)eps));
+  for (int64_t j = threadIdx.x; j < n; j += blockDim.x) Q[c * ldq + j] = row[j] * inv;
+}
+
+// --------------------------------------------------------------- helpers
+__global__ void transpose_kernel(const float* src, int64_t lds, float* dst,
+                                 int64_t ldd, int64_t rows, int64_t cols) {
+  __shared__ float t[32][33];
+  const int64_t r0 = (int64_t)blockIdx.y * 32, c0 = (int64_t)blockIdx.x * 32;
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;  // 32 x 8
+  for (int y = ty; y < 32; y += 8) {
+    const int64_t r = r0 + y, c = c0 + tx;
+    t[y][tx] = (r < rows && c < cols) ? src[r * lds + c] : 0.f;
+  }
+  __syncthreads();
+  for (int y = ty; y < 32; y += 8) {
+    const int64_t r = c0 + y, c = r0 + tx;  // dst is cols x rows
+    if (r < cols && c < rows) dst[r * ldd + c] = t[tx][y];
+  }
+}
+
+__global__ void copy2d_kernel(const float* src, int64_t lds, float* dst,
+                              int64_t ldd, int64_t rows, int64_t cols) {
+  const int64_t total = rows * cols;
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total;
+       e += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t r = e / cols, c = e - (e / cols) * cols;
+    dst[r * ldd + c] = src[r * lds + c];
+  }
+}
+
+unsigned grid_1d(int64_t n, int per_block) {
+  int64_t b = ceil_div(n, per_block);
+  int64_t cap = (int64_t)num_sms() * 8;
+  if (b > cap) b = cap;
+  return (unsigned)(b < 1 ? 1 : b);
+}
+
+// Largest packed triangle (plus r floats) the one-CTA kernel keeps in
+// shared memory.
+size_t chol_smem_bytes(int r) { return ((size_t)r * (r + 1) / 2 + r) * sizeof(float); }
+constexpr size_t kCholSmemMax = 200 * 1024;
+
+int gram_splits(int r, int64_t L) {
+  const int tiles = (int)ceil_div(r, kGT);
+  const int pairs = tiles * (tiles + 1) / 2;
+  int64_t want = ceil_div((int64_t)num_sms() * 4, pairs);
+  int64_t maxs = ceil_div(L, 256);  // at least 256 columns per split
+  if (want > maxs) want = maxs;
+  if (want < 1) want = 1;
+  if (want > 64) want = 64;
+  return (int)want;
+}
+
+struct DionWs {
+  Buf Pa, Pb;   // r x m
+  Buf P;        // m x r
+  Buf Ra, Rb;   // r x n
+  Buf part;     // [64][r][r]
+  Buf Linv;     // r x r
+  Buf tri;      // packed triangle + r (global fallback)
+};
+
+DionWs carve_dion(Arena& ar, int64_t m, int64_t n, int r) {
+  DionWs w;
+  w.Pa = ar.take(OUO_F32, 1, r, m);
+  w.Pb = ar.take(OUO_F32, 1, r, m);
+  w.P = ar.take(OUO_F32, 1, m, r);
+  w.Ra = ar.take(OUO_F32, 1, r, n);
+  w.Rb = ar.take(OUO_F32, 1, r, n);
+  w.part = ar.take(OUO_F32, 64, r, r);
+  w.Linv = ar.take(OUO_F32, 1, r, r);
+  w.tri = ar.take(OUO_F32, 1, 1, (int64_t)r * (r + 1) / 2 + r);
+  return w;
+}
+
+Buf caller_buf(const ouo_mat& m, int dtype) {
+  Buf b;
+  b.p = reinterpret_cast<char*>(m.ptr);
+  b.dtype = dtype;
+  b.rows = m.rows;
+  b.cols = m.cols;
+  b.ld = m.ld;
+  b.stride = m.rows * m.ld;
+  b.nb = 1;
+  return b;
+}
+
+// Rows of X (r x L, workspace) made orthonormal into Y: two CholeskyQR
+// passes (X -> tmp -> Y); X is clobbered.
+int orth_rows(Buf X, Buf tmp, Buf Y, const DionWs& w, cudaStream_t s,
+              int* status) {
+  const int r = (int)X.rows;
+  const int64_t L = X.cols;
+  Buf src = X;
+  for (int pass = 0; pass < 2; ++pass) {
+    Buf dst = pass == 0 ? tmp : Y;
+    GramArgs ga;
+    ga.X = reinterpret_cast<const float*>(src.p);
+    ga.ld = src.ld;
+    ga.r = r;
+    ga.L = L;
+    const int splits = gram_splits(r, L);
+    ga.chunk = ceil_div(ceil_div(L, splits), kGT) * kGT;
+    const int used = (int)ceil_div(L, ga.chunk);
+    ga.part = reinterpret_cast<float*>(w.part.p);
+    ga.tiles = (int)ceil_div(r, kGT);
+    dim3 grid((unsigned)(ga.tiles * (ga.tiles + 1) / 2), (unsigned)used);
+    gram_partial_kernel<<<grid, 256, 0, s>>>(ga);
+    OUO_CHECK_LAUNCH();
+    CholArgs ca;
+    ca.part = ga.part;
+    ca.splits = used;
+    ca.r = r;
+    ca.L = L;
+    ca.tri_glob = reinterpret_cast<float*>(w.tri.p);
+    ca.Linv = reinterpret_cast<float*>(w.Linv.p);
+    ca.ldl = w.Linv.ld;
+    ca.status = status;
+    const size_t smem = chol_smem_bytes(r);
+    ca.use_smem = smem <= kCholSmemMax;
+    if (ca.use_smem) {
+      OUO_CHECK_CUDA(cudaFuncSetAttribute(chol_inv_kernel,
+                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          (int)kCholSmemMax));
+    }
+    chol_inv_kernel<<<1, 1024, ca.use_smem ? smem : 0, s>>>(ca);
+    OUO_CHECK_LAUNCH();
+    // dst = Linv src
+    GemmDesc d;
+    d.M = r;
+    d.N = L;
+    d.K = r;
+    d.nb = 1;
+    d.A = w.Linv;
+    d.B = src;
+    d.b_mn = 1;
+    d.out_f32 = dst;
+    d.has_f32 = true;
+    OUO_TRY(gemm_simt(d, s));
+    src = dst;
+  }
+  return OUO_OK;
+}
+
+int validate_dion(const ouo_dion_params* p) {
+  if (!p) return set_error(OUO_ERR_INVALID_ARG, "NULL dion params");
+  if (p->norm_mode != OUO_DION_COLNORM && p->norm_mode != OUO_DION_QR)
+    return set_error(OUO_ERR_INVALID_ARG, "unknown norm_mode %d", p->norm_mode);
+  if (!(p->eps >= 0.f)) return set_error(OUO_ERR_INVALID_ARG, "eps must be >= 0");
+  return OUO_OK;
+}
+
+size_t dion_plan_bytes(const ouo_mat* M, int nmat, const ouo_dion_params* p) {
+  Arena ar{nullptr, 0, 0, true};
+  for (int i = 0; i < nmat; ++i) carve_dion(ar, M[i].rows, M[i].cols, p->rank);
+  return ar.used + 256;
+}
+
+}  // namespace
+}  // namespace ouo
 
 extern "C" size_t dion_workspace_bytes(const ouo_mat* M, int nmat,
                                        const ouo_dion_params* p) {
-  (void)M; (void)nmat; (void)p;
-  return 0;
+  if (!M || !p || nmat <= 0 || p->rank < 1) return 0;
+  return ouo::dion_plan_bytes(M, nmat, p);
 }
 
 extern "C" int dion_lowrank_step(const ouo_mat* M, const ouo_mat* G,
@@ -13,8 +405,130 @@ extern "C" int dion_lowrank_step(const ouo_mat* M, const ouo_mat* G,
                                  const ouo_dion_params* p, const float* scale,
                                  void* ws, size_t ws_bytes, int* dev_status,
                                  void* stream) {
-  (void)M; (void)G; (void)g_dtype; (void)Q_state; (void)W; (void)w_dtype;
-  (void)nmat; (void)p; (void)scale; (void)ws; (void)ws_bytes;
-  (void)dev_status; (void)stream;
-  return ouo::set_error(OUO_ERR_UNSUPPORTED, "dion_lowrank_step: not built yet");
+  using namespace ouo;
+  clear_error();
+  if (nmat < 0 || nmat > OUO_MAX_BATCH)
+    return set_error(OUO_ERR_INVALID_ARG, "nmat %d out of range", nmat);
+  OUO_TRY(validate_dion(p));
+  if (nmat == 0) return OUO_OK;
+  OUO_TRY(validate_mats(M, nmat, OUO_F32, "M"));
+  OUO_TRY(validate_mats(G, nmat, g_dtype, "G"));
+  OUO_TRY(validate_mats(Q_state, nmat, OUO_F32, "Q_state"));
+  OUO_TRY(validate_mats(W, nmat, w_dtype, "W"));
+  OUO_TRY(validate_same_shapes(M, G, nmat, "M", "G"));
+  OUO_TRY(validate_same_shapes(M, W, nmat, "M", "W"));
+  const int r = p->rank;
+  for (int i = 0; i < nmat; ++i) {
+    if (r < 1 || r > M[i].rows || r > M[i].cols)
+      return set_error(OUO_ERR_INVALID_ARG, "rank %d outside [1, min(rows, cols)] for M[%d]",
+                       r, i);
+    if (Q_state[i].rows != r || Q_state[i].cols != M[i].cols)
+      return set_error(OUO_ERR_INVALID_ARG,
+                       "Q_state[%d] must be r x cols (%d x %lld, the transposed factor)",
+                       i, r, (long long)M[i].cols);
+    if (!vec16(M[i], OUO_F32) || !vec16(Q_state[i], OUO_F32) || !vec16(W[i], w_dtype))
+      return set_error(OUO_ERR_INVALID_ARG,
+                       "dion_lowrank_step needs M, Q_state and W rows on 16-byte "
+                       "boundaries (matrix %d)", i);
+  }
+  if (dev_status && ((uintptr_t)dev_status % 4))
+    return set_error(OUO_ERR_INVALID_ARG, "dev_status misaligned");
+  const size_t need = dion_plan_bytes(M, nmat, p);
+  if (!ws || ws_bytes < need)
+    return set_error(OUO_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given",
+                     need, ws_bytes);
+  if ((uintptr_t)ws % 256)
+    return set_error(OUO_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  OUO_TRY(require_sm100());
+  cudaStream_t s = (cudaStream_t)stream;
+  // B = M + G for the whole batch
+  OUO_TRY(dion_momentum_update(M, G, nmat, g_dtype, p->mu, OUO_MOMENTUM_ACCUM,
+                               nullptr, stream));
+  Arena ar{reinterpret_cast<char*>(ws), ws_bytes, 0, false};
+  const float mu = p->mu, beta = p->beta;
+  for (int i = 0; i < nmat; ++i) {
+    const int64_t m = M[i].rows, n = M[i].cols;
+    DionWs w = carve_dion(ar, m, n, r);
+    const Buf Bm = caller_buf(M[i], OUO_F32);
+    const Buf Qt = caller_buf(Q_state[i], OUO_F32);
+    // Pt = Qt B^T  (r x m)
+    {
+      GemmDesc d;
+      d.M = r; d.N = m; d.K = n; d.nb = 1;
+      d.A = Qt;
+      d.B = Bm;
+      d.out_f32 = w.Pa;
+      d.has_f32 = true;
+      OUO_TRY(gemm_umma(d, s, dev_status));
+    }
+    // rows of Pt orthonormal (P = orth(B Q_prev)) -> Pa
+    OUO_TRY(orth_rows(w.Pa, w.Pb, w.Pa, w, s, dev_status));
+    // Rt = Pt B  (r x n)
+    {
+      GemmDesc d;
+      d.M = r; d.N = n; d.K = m; d.nb = 1;
+      d.A = w.Pa;
+      d.B = Bm;
+      d.b_mn = 1;
+      d.out_f32 = w.Ra;
+      d.has_f32 = true;
+      OUO_TRY(gemm_umma(d, s, dev_status));
+    }
+    // P = Pt^T (m x r), the K-major left operand of the updates
+    {
+      dim3 grid((unsigned)ceil_div(m, 32), (unsigned)ceil_div(r, 32));
+      transpose_kernel<<<grid, 256, 0, s>>>(reinterpret_cast<const float*>(w.Pa.p),
+                                            w.Pa.ld, reinterpret_cast<float*>(w.P.p),
+                                            w.P.ld, r, m);
+      OUO_CHECK_LAUNCH();
+    }
+    // M <- beta B - (beta - mu) P Rt   (in place over B)
+    {
+      GemmDesc d;
+      d.M = m; d.N = n; d.K = r; d.nb = 1;
+      d.A = w.P;
+      d.B = w.Ra;
+      d.b_mn = 1;
+      d.alpha = -(beta - mu);
+      d.beta = beta;
+      d.has_c0 = true;
+      d.direct = {MatRef{M[i].ptr, M[i].ld}};
+      d.direct_dtype = OUO_F32;
+      d.c0_from_out = true;
+      OUO_TRY(gemm_umma(d, s, dev_status));
+    }
+    // Qt_new: rows of Rt normalized (Dion) or orthonormalized (Orth-Dion) -> Rb
+    Buf Qn = w.Rb;
+    if (p->norm_mode == OUO_DION_COLNORM) {
+      rownorm_kernel<<<r, 256, 0, s>>>(reinterpret_cast<const float*>(w.Ra.p), w.Ra.ld,
+                                       reinterpret_cast<float*>(w.Rb.p), w.Rb.ld, n,
+                                       p->eps);
+      OUO_CHECK_LAUNCH();
+    } else {
+      OUO_TRY(orth_rows(w.Ra, w.Rb, w.Ra, w, s, dev_status));
+      Qn = w.Ra;
+    }
+    // W <- (1 - lr wd) W - lr s P Qt_new
+    {
+      const float sc = scale ? scale[i] : 1.0f;
+      GemmDesc d;
+      d.M = m; d.N = n; d.K = r; d.nb = 1;
+      d.A = w.P;
+      d.B = Qn;
+      d.b_mn = 1;
+      d.alpha = -p->lr * sc;
+      d.beta = 1.0f - p->lr * p->wd;
+      d.has_c0 = true;
+      d.direct = {MatRef{W[i].ptr, W[i].ld}};
+      d.direct_dtype = w_dtype;
+      d.c0_from_out = true;
+      OUO_TRY(gemm_umma(d, s, dev_status));
+    }
+    // state <- Qt_new
+    copy2d_kernel<<<grid_1d((int64_t)r * n, 256), 256, 0, s>>>(
+        reinterpret_cast<const float*>(Qn.p), Qn.ld,
+        reinterpret_cast<float*>(Q_state[i].ptr), Q_state[i].ld, r, n);
+    OUO_CHECK_LAUNCH();
+  }
+  return OUO_OK;
 }

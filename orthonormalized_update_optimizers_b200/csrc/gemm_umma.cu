@@ -72,6 +72,7 @@ struct UmmaArgs {
   int tri;
   float alpha, beta, gamma;
   int has_c0, c0_bf16, has_f32, round_tf32, has_bf16;
+  int c0_out;  // C0 is read from the (direct) output itself
   int* status;
   void* dptr[kChunk];
   int64_t dld[kChunk];
@@ -189,6 +190,26 @@ __device__ __forceinline__ void store4t(const UmmaArgs& a, const TileOut& o,
 #pragma unroll
   for (int t = 0; t < 4; ++t)
     if (mask & (1u << t)) store_elem(a, o, row, col + t, e[t]);
+}
+
+// In-place updates read their C0 from the output location.
+__device__ __forceinline__ float load_out1(const UmmaArgs& a, const TileOut& o,
+                                           int64_t i, int64_t j) {
+  return a.has_f32 ? o.f[i * o.ldf + j] : bf16_to_f32(o.h[i * o.ldh + j]);
+}
+
+__device__ __forceinline__ void load_out4(const UmmaArgs& a, const TileOut& o,
+                                          int64_t i, int64_t j, float e[4]) {
+  if (a.has_f32) {
+    float4 f = *reinterpret_cast<const float4*>(o.f + i * o.ldf + j);
+    e[0] = f.x; e[1] = f.y; e[2] = f.z; e[3] = f.w;
+  } else {
+    uint2 u = *reinterpret_cast<const uint2*>(o.h + i * o.ldh + j);
+    e[0] = __uint_as_float(u.x << 16);
+    e[1] = __uint_as_float(u.x & 0xffff0000u);
+    e[2] = __uint_as_float(u.y << 16);
+    e[3] = __uint_as_float(u.y & 0xffff0000u);
+  }
 }
 
 __device__ __forceinline__ float load_c0(const Segment& sg, int64_t b,
@@ -345,9 +366,12 @@ umma_gemm_kernel(const __grid_constant__ UmmaArgs a) {
 #pragma unroll
         for (uint32_t kk = 0; kk < kBK / kInstK; ++kk) {
           const uint64_t ad = ptx::smem_desc_sw128(sa + kk * 32, 16, 1024);
+          // MN-major tf32 takes the 32-byte-atom swizzle (4-row groups)
           const uint64_t bd =
-              B_MN ? ptx::smem_desc_sw128(sb + kk * kInstK * kRowBytes,
-                                          kChunkBytes, 1024)
+              B_MN ? (FMT == 2 ? ptx::smem_desc_sw128_32b(sb + kk * kInstK * kRowBytes,
+                                                          kChunkBytes, 512)
+                               : ptx::smem_desc_sw128(sb + kk * kInstK * kRowBytes,
+                                                      kChunkBytes, 1024))
                    : ptx::smem_desc_sw128(sb + kk * 32, 16, 1024);
           const uint32_t acc = (kb > 0 || kk > 0) ? 1u : 0u;
           if (FMT == 1) ptx::mma_bf16(d, ad, bd, kIdesc, acc);
@@ -459,7 +483,15 @@ umma_gemm_kernel(const __grid_constant__ UmmaArgs a) {
           if (!a.tri && mask) {
             if (a.has_c0) {
               float e[4];
-              if (mask == 0xFu) {
+              if (a.c0_out) {
+                if (mask == 0xFu) {
+                  load_out4(a, to, gr, gc, e);
+                } else {
+#pragma unroll
+                  for (int t = 0; t < 4; ++t)
+                    e[t] = (mask & (1u << t)) ? load_out1(a, to, gr, gc + t) : 0.f;
+                }
+              } else if (mask == 0xFu) {
                 load_c0x4(sg, b, gr, gc, e, a.c0_bf16);
               } else {
 #pragma unroll
@@ -540,9 +572,11 @@ EncodeTiledFn encode_fn() {
 }
 
 // 3-D map over a workspace batch [nb][rows][ld]: dims (cols, rows, nb), box
-// (box_cols, box_rows, 1), 128-byte swizzle, zero fill out of bounds.
+// (box_cols, box_rows, 1), 128-byte swizzle (16-byte atoms, or 32-byte
+// atoms for MN-major tf32 operands), zero fill out of bounds.
 int make_map(CUtensorMap* map, const Buf& t, uint32_t box_cols,
-             uint32_t box_rows) {
+             uint32_t box_rows,
+             CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
   EncodeTiledFn fn = encode_fn();
   if (!fn)
     return set_error(OUO_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
@@ -556,7 +590,7 @@ int make_map(CUtensorMap* map, const Buf& t, uint32_t box_cols,
                   t.dtype == OUO_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
                                       : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
                   3, t.p, dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS)
@@ -600,6 +634,8 @@ int launch(const std::vector<GemmDesc>& gs, cudaStream_t stream, int* status) {
     a.has_f32 = g0.direct_dtype == OUO_F32;
     a.has_bf16 = g0.direct_dtype == OUO_BF16;
     a.round_tf32 = 0;
+    a.c0_out = g0.c0_from_out ? 1 : 0;
+    if (a.c0_out) a.has_c0 = 1;
   }
   int ndirect = 0;
   auto flush = [&]() -> int {
@@ -624,11 +660,13 @@ int launch(const std::vector<GemmDesc>& gs, cudaStream_t stream, int* status) {
     memset(&proto, 0, sizeof(proto));
     OUO_TRY(make_map(&proto.tmA, g.A, bk, kTileM));
     if (!B_MN) OUO_TRY(make_map(&proto.tmB, g.B, bk, BN));
-    else OUO_TRY(make_map(&proto.tmB, g.B, kRowBytes / es, bk));
+    else OUO_TRY(make_map(&proto.tmB, g.B, kRowBytes / es, bk,
+                          FMT == 2 ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B
+                                   : CU_TENSOR_MAP_SWIZZLE_128B));
     proto.M = g.M; proto.N = g.N; proto.K = g.K;
     proto.tiles_n = ceil_div(g.N, BN);
     proto.tiles_per_mat = tiles_per_matrix(g, BN);
-    proto.C0 = g.has_c0 ? g.C0.p : nullptr;
+    proto.C0 = (g.has_c0 && !g.c0_from_out) ? g.C0.p : nullptr;
     proto.ldc0 = g.C0.ld; proto.sc0 = g.C0.stride;
     proto.Of = g.has_f32 ? reinterpret_cast<float*>(g.out_f32.p) : nullptr;
     proto.ldof = g.out_f32.ld; proto.sof = g.out_f32.stride;
@@ -671,6 +709,7 @@ int gemm_umma_grouped(const std::vector<GemmDesc>& gs, cudaStream_t stream,
     if (g.tri != g0.tri || g.b_mn != g0.b_mn || g.has_c0 != g0.has_c0 ||
         g.has_f32 != g0.has_f32 || g.has_bf16 != g0.has_bf16 ||
         g.round_tf32 != g0.round_tf32 || g.direct.empty() != g0.direct.empty() ||
+        g.c0_from_out != g0.c0_from_out ||
         g.alpha != g0.alpha || g.beta != g0.beta || g.gamma != g0.gamma ||
         (g.has_c0 && g.C0.dtype != g0.C0.dtype) ||
         (!g.direct.empty() && g.direct_dtype != g0.direct_dtype))
@@ -679,6 +718,8 @@ int gemm_umma_grouped(const std::vector<GemmDesc>& gs, cudaStream_t stream,
       return set_error(OUO_ERR_INVALID_ARG, "symmetric GEMM needs M == N, K-major B");
     if (!g.direct.empty() && (int64_t)g.direct.size() != g.nb)
       return set_error(OUO_ERR_INVALID_ARG, "direct output table size mismatch");
+    if (g.c0_from_out && (g.direct.empty() || g.tri))
+      return set_error(OUO_ERR_INVALID_ARG, "in-place C0 needs direct, non-symmetric outputs");
     wide = wide || g.N > 128;
   }
   if (g0.A.dtype == OUO_BF16) {

@@ -83,6 +83,9 @@ struct GemmDesc {
   // out_f32 / out_bf16.  Tensor-core path only.
   std::vector<MatRef> direct;
   int direct_dtype = OUO_BF16;
+  // With direct outputs: C0 is the output matrix itself (in-place update
+  // out = alpha * A op(B) + beta * out).  Non-symmetric outputs only.
+  bool c0_from_out = false;
 };
 
 // Tensor-core GEMM (tcgen05 / TMEM / TMA).  A and B are both bf16

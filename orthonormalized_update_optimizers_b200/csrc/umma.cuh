@@ -188,6 +188,20 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr,
   return d;
 }
 
+// Same, for MN-major 32-bit operands: 128-byte swizzle with 32-byte atoms
+// (layout type 1), K rows grouped by 4 (sbo = distance between 4-row groups).
+__device__ __forceinline__ uint64_t smem_desc_sw128_32b(uint32_t saddr,
+                                                        uint32_t lbo,
+                                                        uint32_t sbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1 << 46;  // descriptor version for sm_100
+  d |= (uint64_t)1 << 61;  // 128-byte swizzle, 32-byte atoms
+  return d;
+}
+
 // Instruction descriptor: fp32 accumulator, A and B of `fmt` (1 = bf16,
 // 2 = tf32), A K-major, B K-major or MN-major, M = 128, N = n.
 __host__ __device__ constexpr uint32_t instr_desc(uint32_t fmt, uint32_t b_mn,
