@@ -132,6 +132,19 @@ const char* ouo_last_error(void);
 /* Number of kernels this library has enqueued in this process, all devices
  * and threads together (monotonic; for accounting in benchmarks). */
 unsigned long long ouo_launch_count(void);
+
+/* Kernel timing for benchmarks.  ouo_timing_enable(1) creates a pool of CUDA
+ * events (on the current device) and from then on brackets every
+ * tensor-core GEMM launch with two events on its stream, recording the
+ * launch's kind and algorithmic flops (2 M N K per matrix; symmetric
+ * outputs M (M + 1) K, the upper triangle).  ouo_timing_enable(0) drops the
+ * records and the pool.  At most 4096 launches are recorded.
+ * ouo_timing_read(kind, ...) waits for the recorded events and returns the
+ * number of launches, their summed device time (ms) and summed flops for
+ * one kind (-1 = all): kind = (symmetric ? 4 : 0) + (tf32 ? 2 : 0) +
+ * (B operand MN-major ? 1 : 0). */
+int ouo_timing_enable(int on);
+int ouo_timing_read(int kind, int* launches, double* total_ms, double* flops);
 void ouo_ns_default(ouo_ns_params* p);
 void ouo_dion_default(ouo_dion_params* p);
 

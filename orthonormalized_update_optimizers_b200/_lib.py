@@ -31,7 +31,8 @@ OUO_NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024
 
 # every symbol the header declares
 EXPORTED = (
-    "ouo_version", "ouo_last_error", "ouo_launch_count", "ouo_ns_default", "ouo_dion_default",
+    "ouo_version", "ouo_last_error", "ouo_launch_count", "ouo_timing_enable",
+    "ouo_timing_read", "ouo_ns_default", "ouo_dion_default",
     "dion_momentum_update", "dion3_num_selected", "dion3_select_rows",
     "ns_workspace_bytes", "ns_orthogonalize", "gram_ns_workspace_bytes",
     "gram_ns_orthogonalize", "gram_ns_orthogonalize_noalloc", "apply_update",
@@ -82,6 +83,10 @@ _PROTOS = {
     "ouo_version": (_I, []),
     "ouo_last_error": (ctypes.c_char_p, []),
     "ouo_launch_count": (ctypes.c_ulonglong, []),
+    "ouo_timing_enable": (_I, [_I]),
+    "ouo_timing_read": (_I, [_I, ctypes.POINTER(ctypes.c_int),
+                             ctypes.POINTER(ctypes.c_double),
+                             ctypes.POINTER(ctypes.c_double)]),
     "ouo_ns_default": (None, [_NP]),
     "ouo_dion_default": (None, [_DP]),
     "dion_momentum_update": (_I, [_MP, _MP, _I, _I, _F, _I, _P, _P]),

@@ -22,7 +22,7 @@ __all__ = [
     "ns_orthogonalize", "gram_ns_workspace_bytes", "gram_ns_orthogonalize",
     "gram_ns_orthogonalize_noalloc",
     "apply_update", "dion_workspace_bytes", "dion_lowrank_step", "version",
-    "launch_count",
+    "launch_count", "timing_enable", "timing_read",
 ]
 
 
@@ -84,6 +84,22 @@ def version() -> int:
 def launch_count() -> int:
     """Kernels the library has enqueued in this process so far."""
     return int(L.lib().ouo_launch_count())
+
+
+def timing_enable(on: bool = True) -> None:
+    """Start (or stop and clear) event timing of tensor-core GEMM launches."""
+    L.check("ouo_timing_enable", L.lib().ouo_timing_enable(1 if on else 0))
+
+
+def timing_read(kind: int = -1):
+    """(launches, total_ms, flops) of the recorded GEMM launches of one kind
+    ((symmetric ? 4 : 0) + (tf32 ? 2 : 0) + (MN-major B ? 1 : 0); -1 = all)."""
+    n = ctypes.c_int(0)
+    ms = ctypes.c_double(0.0)
+    fl = ctypes.c_double(0.0)
+    L.check("ouo_timing_read", L.lib().ouo_timing_read(kind, ctypes.byref(n),
+                                                      ctypes.byref(ms), ctypes.byref(fl)))
+    return n.value, ms.value, fl.value
 
 
 def ns_params(a=None, b=None, c=None, iters=None, safety=None, eps=None,

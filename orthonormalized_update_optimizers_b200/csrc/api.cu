@@ -147,6 +147,16 @@ int ouo_version(void) { return OUO_VERSION; }
 
 const char* ouo_last_error(void) { return ouo::g_last_error; }
 
+int ouo_timing_enable(int on) {
+  ouo::clear_error();
+  return ouo::gemm_timing_enable(on);
+}
+
+int ouo_timing_read(int kind, int* launches, double* total_ms, double* flops) {
+  ouo::clear_error();
+  return ouo::gemm_timing_read(kind, launches, total_ms, flops);
+}
+
 unsigned long long ouo_launch_count(void) {
   return ouo::g_launches.load(std::memory_order_relaxed);
 }

@@ -550,6 +550,32 @@ umma_gemm_kernel(const __grid_constant__ UmmaArgs a) {
 
 // ------------------------------------------------------------------- host
 
+// ------------------------------------------------ per-launch timing (opt-in)
+// While enabled, every launch of the tensor-core GEMM is bracketed by two
+// CUDA events on its stream and its algorithmic flops (symmetric outputs:
+// the upper triangle only) are recorded per kernel kind.  Events come from a
+// pool created when timing is switched on.
+constexpr int kTimingKinds = 8;  // (tri ? 4 : 0) + (tf32 ? 2 : 0) + b_mn
+constexpr int kTimingMax = 4096;
+struct TimingRec {
+  cudaEvent_t e0, e1;
+  int kind;
+  double flops;
+};
+std::mutex g_tmu;
+bool g_timing = false;
+std::vector<TimingRec> g_recs;
+std::vector<cudaEvent_t> g_pool;
+size_t g_next = 0;
+
+int timing_record_begin(cudaStream_t s, TimingRec* r) {
+  if (g_next + 2 > g_pool.size()) return 0;
+  r->e0 = g_pool[g_next++];
+  r->e1 = g_pool[g_next++];
+  cudaEventRecord(r->e0, s);
+  return 1;
+}
+
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   void*, const cuuint64_t*, const cuuint64_t*,
                                   const cuuint32_t*, const cuuint32_t*,
@@ -647,8 +673,27 @@ int launch(const std::vector<GemmDesc>& gs, cudaStream_t stream, int* status) {
     }
     int64_t grid = a.total_tiles < num_sms() ? a.total_tiles : num_sms();
     if (grid >= 1) {
+      TimingRec rec;
+      bool timed = false;
+      if (g_timing) {
+        std::lock_guard<std::mutex> lock(g_tmu);
+        timed = timing_record_begin(stream, &rec) != 0;
+      }
       kern<<<(unsigned)grid, kThreads, C::kSmem, stream>>>(a);
       OUO_CHECK_LAUNCH();
+      if (timed) {
+        cudaEventRecord(rec.e1, stream);
+        rec.kind = (a.tri ? 4 : 0) + (FMT == 2 ? 2 : 0) + B_MN;
+        rec.flops = 0.0;
+        for (int sgi = 0; sgi < a.nseg; ++sgi) {
+          const Segment& sg = a.seg[sgi];
+          const double per = a.tri ? (double)sg.M * (double)(sg.M + 1) * (double)sg.K
+                                   : 2.0 * (double)sg.M * (double)sg.N * (double)sg.K;
+          rec.flops += per * (double)sg.nb;
+        }
+        std::lock_guard<std::mutex> lock(g_tmu);
+        g_recs.push_back(rec);
+      }
     }
     a.nseg = 0;
     ndirect = 0;
@@ -697,6 +742,42 @@ int launch(const std::vector<GemmDesc>& gs, cudaStream_t stream, int* status) {
 }
 
 }  // namespace
+
+int gemm_timing_enable(int on) {
+  std::lock_guard<std::mutex> lock(g_tmu);
+  for (cudaEvent_t e : g_pool) cudaEventDestroy(e);
+  g_pool.clear();
+  g_recs.clear();
+  g_next = 0;
+  g_timing = false;
+  if (!on) return OUO_OK;
+  for (int i = 0; i < 2 * kTimingMax; ++i) {
+    cudaEvent_t e;
+    OUO_CHECK_CUDA(cudaEventCreate(&e));
+    g_pool.push_back(e);
+  }
+  g_timing = true;
+  return OUO_OK;
+}
+
+int gemm_timing_read(int kind, int* launches, double* total_ms, double* flops) {
+  std::lock_guard<std::mutex> lock(g_tmu);
+  int n = 0;
+  double ms = 0.0, fl = 0.0;
+  for (const TimingRec& r : g_recs) {
+    if (kind >= 0 && r.kind != kind) continue;
+    OUO_CHECK_CUDA(cudaEventSynchronize(r.e1));
+    float t = 0.f;
+    OUO_CHECK_CUDA(cudaEventElapsedTime(&t, r.e0, r.e1));
+    ++n;
+    ms += t;
+    fl += r.flops;
+  }
+  if (launches) *launches = n;
+  if (total_ms) *total_ms = ms;
+  if (flops) *flops = fl;
+  return OUO_OK;
+}
 
 int gemm_umma_grouped(const std::vector<GemmDesc>& gs, cudaStream_t stream,
                       int* status) {

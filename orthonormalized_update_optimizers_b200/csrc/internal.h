@@ -96,6 +96,9 @@ int gemm_umma(const GemmDesc& g, cudaStream_t stream, int* status);
 // possible: one persistent launch covers up to 6 batch segments.
 int gemm_umma_grouped(const std::vector<GemmDesc>& gs, cudaStream_t stream,
                       int* status);
+// Opt-in event timing of tensor-core GEMM launches (see ouo_timing_enable).
+int gemm_timing_enable(int on);
+int gemm_timing_read(int kind, int* launches, double* total_ms, double* flops);
 // CUDA-core fp32 GEMM for the fp32 precision path.
 int gemm_simt(const GemmDesc& g, cudaStream_t stream);
 
