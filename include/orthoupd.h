@@ -145,6 +145,14 @@ unsigned long long ouo_launch_count(void);
  * (B operand MN-major ? 1 : 0). */
 int ouo_timing_enable(int on);
 int ouo_timing_read(int kind, int* launches, double* total_ms, double* flops);
+
+/* Test hook for the failure path of the bounded device waits: launches one
+ * block that waits on an mbarrier nothing ever completes, gives up after
+ * limit_ns (at most 1 s) and ORs OUO_STATUS_TIMEOUT into *dev_status, the
+ * way a stalled GEMM pipeline reports.  Nothing faults or hangs; the
+ * context stays usable. */
+int ouo_debug_wait_timeout(int* dev_status, unsigned long long limit_ns,
+                           void* stream);
 void ouo_ns_default(ouo_ns_params* p);
 void ouo_dion_default(ouo_dion_params* p);
 

@@ -32,7 +32,7 @@ OUO_NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024
 # every symbol the header declares
 EXPORTED = (
     "ouo_version", "ouo_last_error", "ouo_launch_count", "ouo_timing_enable",
-    "ouo_timing_read", "ouo_ns_default", "ouo_dion_default",
+    "ouo_timing_read", "ouo_debug_wait_timeout", "ouo_ns_default", "ouo_dion_default",
     "dion_momentum_update", "dion3_num_selected", "dion3_select_rows",
     "ns_workspace_bytes", "ns_orthogonalize", "gram_ns_workspace_bytes",
     "gram_ns_orthogonalize", "gram_ns_orthogonalize_noalloc", "apply_update",
@@ -84,6 +84,7 @@ _PROTOS = {
     "ouo_last_error": (ctypes.c_char_p, []),
     "ouo_launch_count": (ctypes.c_ulonglong, []),
     "ouo_timing_enable": (_I, [_I]),
+    "ouo_debug_wait_timeout": (_I, [_P, ctypes.c_ulonglong, _P]),
     "ouo_timing_read": (_I, [_I, ctypes.POINTER(ctypes.c_int),
                              ctypes.POINTER(ctypes.c_double),
                              ctypes.POINTER(ctypes.c_double)]),

@@ -8,6 +8,7 @@
 #include <utility>
 
 #include "internal.h"
+#include "umma.cuh"
 
 namespace ouo {
 
@@ -139,9 +140,39 @@ Buf Arena::take(int dtype, int64_t nb, int64_t rows, int64_t cols) {
   return b;
 }
 
+namespace {
+
+// Waits on an mbarrier that nothing arrives on, bounded by limit_ns, then
+// reports OUO_STATUS_TIMEOUT: the same bounded wait the GEMM pipeline uses,
+// made to run out on purpose.
+__global__ void wait_timeout_kernel(int* status, unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(&bar, 1);
+    ptx::fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && !ptx::mbar_wait_timed(&bar, 0, limit_ns))
+    report_status(status, OUO_STATUS_TIMEOUT);
+}
+
+}  // namespace
 }  // namespace ouo
 
 extern "C" {
+
+int ouo_debug_wait_timeout(int* dev_status, unsigned long long limit_ns,
+                           void* stream) {
+  ouo::clear_error();
+  if (!dev_status)
+    return ouo::set_error(OUO_ERR_INVALID_ARG, "dev_status is required");
+  if (limit_ns > 1000000000ull)
+    return ouo::set_error(OUO_ERR_INVALID_ARG, "limit above 1 s");
+  OUO_TRY(ouo::require_sm100());
+  ouo::wait_timeout_kernel<<<1, 32, 0, (cudaStream_t)stream>>>(dev_status, limit_ns);
+  OUO_CHECK_LAUNCH();
+  return OUO_OK;
+}
 
 int ouo_version(void) { return OUO_VERSION; }
 
