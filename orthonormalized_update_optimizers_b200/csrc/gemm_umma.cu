@@ -37,6 +37,12 @@ constexpr int kEpiWarps = 8;                 // two per TMEM lane quarter
 constexpr int kThreads = 64 + 32 * kEpiWarps;  // producer, MMA, epilogue
 constexpr uint32_t kTileM = 128;
 constexpr uint32_t kRowBytes = 128;  // one swizzle row: K bytes per stage
+// bf16 staging for TMA stores: 64-byte rows, 16-byte chunks XOR (row / 2) % 4
+// (the 64-byte swizzle pattern).
+__device__ __forceinline__ int stg16_idx(int row, int col) {
+  return row * 32 + ((((col >> 3) ^ (row >> 1)) & 3) << 3) + (col & 7);
+}
+
 // Epilogue staging: a 32 x 32 fp32 chunk per warp, 16-byte groups XOR-
 // swizzled by row so that row-wise and column-wise accesses are both free
 // of bank conflicts.
@@ -50,6 +56,7 @@ __device__ __forceinline__ int stg_idx(int row, int col) {
 struct Segment {
   CUtensorMap tmA;
   CUtensorMap tmB;
+  CUtensorMap tmC;  // workspace output (TMA-store epilogue)
   int64_t M, N, K;
   int64_t nb, b0;
   int64_t tiles_n, tiles_per_mat, tile_start;  // tile_start: first tile id
@@ -73,6 +80,7 @@ struct UmmaArgs {
   float alpha, beta, gamma;
   int has_c0, c0_bf16, has_f32, round_tf32, has_bf16;
   int c0_out;  // C0 is read from the (direct) output itself
+  int tma_out;  // single workspace output written by TMA stores
   int* status;
   void* dptr[kChunk];
   int64_t dld[kChunk];
@@ -252,15 +260,17 @@ umma_gemm_kernel(const __grid_constant__ UmmaArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kStages * C::kStageBytes);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kStages * C::kStageBytes +
+                                               C::kEpiBytes);
   uint64_t* empty = full + C::kStages;
   uint64_t* tfull = empty + C::kStages;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
-  float* epi_smem =
-      reinterpret_cast<float*>(smem + C::kStages * C::kStageBytes + 256);
+  // per-warp 4 KB staging buffers, 1024-byte aligned (the TMA swizzle
+  // patterns are computed from absolute shared-memory address bits)
+  float* epi_smem = reinterpret_cast<float*>(smem + C::kStages * C::kStageBytes);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -413,6 +423,119 @@ umma_gemm_kernel(const __grid_constant__ UmmaArgs a) {
         break;
       }
       ptx::tc_fence_after();
+      if (a.tma_out) {
+        // Finished values (row = lane) are staged in the TMA's swizzled box
+        // layout (fp32: 128-byte rows, 16-byte chunks XOR row % 8; bf16:
+        // 64-byte rows, chunks XOR (row / 2) % 4) and written by one lane
+        // with a bulk tensor store; rows and columns past the matrix are
+        // clipped by the TMA.  Symmetric outputs: the mirrored box (j, i)
+        // is a second store from a transposed staging; a chunk on the
+        // diagonal is made symmetric in place and stored once.
+        const int64_t row_base = ti * kTileM + q * 32;
+        const int64_t gi = row_base + lane;
+        float* stg = epi_smem + (warp - 2) * (32 * 32);
+        uint16_t* stg16 = reinterpret_cast<uint16_t*>(stg);
+        const uint32_t half = (uint32_t)((warp - 2) >> 2);
+        const int32_t z = (int32_t)(sg.b0 + b);
+        const bool obf = a.has_bf16 != 0;
+#pragma unroll 1
+        for (uint32_t c0 = half * (BN / 2); c0 < (half + 1) * (BN / 2); c0 += 32) {
+          const int64_t gj0 = tj * BN + c0;
+          if (a.tri && gj0 + 31 < row_base) continue;  // below the diagonal
+          if (row_base >= sg.M || gj0 >= sg.N) continue;
+          float v[32];
+          ptx::tmem_ld32(tmem_base + ((q * 32u) << 16) + buf * BN + c0, v);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] *= a.alpha;
+          if (a.has_c0) {
+            float c0v[32];
+            if (a.tri) {
+              const int64_t gic = gi < sg.M ? gi : sg.M - 1;
+#pragma unroll
+              for (int j = 0; j < 32; ++j) {
+                const int64_t gjc = gj0 + j < sg.N ? gj0 + j : sg.N - 1;
+                c0v[j] = load_c0(sg, b, gjc, gic, a.c0_bf16);
+              }
+            } else if (gi < sg.M && gj0 + 32 <= sg.N) {
+#pragma unroll
+              for (int j = 0; j < 32; j += 4) load_c0x4(sg, b, gi, gj0 + j, c0v + j, a.c0_bf16);
+            } else {
+              const int64_t gic = gi < sg.M ? gi : sg.M - 1;
+#pragma unroll
+              for (int j = 0; j < 32; ++j) {
+                const int64_t gjc = gj0 + j < sg.N ? gj0 + j : sg.N - 1;
+                c0v[j] = load_c0(sg, b, gic, gjc, a.c0_bf16);
+              }
+            }
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] += a.beta * c0v[j];
+          }
+          if (gi >= gj0 && gi < gj0 + 32) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (gi == gj0 + j) v[j] += a.gamma;
+          }
+          if (a.round_tf32 && !obf) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = round_tf32(v[j]);
+          }
+          const bool diag = a.tri && gj0 == row_base;
+          // the previous store from this buffer must have read it
+          if (lane == 0) ptx::bulk_wait_read0();
+          __syncwarp();
+          if (!obf) {
+#pragma unroll
+            for (int j = 0; j < 32; j += 4)
+              *reinterpret_cast<float4*>(stg + stg_idx(lane, j)) =
+                  make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+          } else {
+#pragma unroll
+            for (int qq = 0; qq < 4; ++qq) {
+              uint4 u;
+              u.x = pack_bf16x2(v[8 * qq + 0], v[8 * qq + 1]);
+              u.y = pack_bf16x2(v[8 * qq + 2], v[8 * qq + 3]);
+              u.z = pack_bf16x2(v[8 * qq + 4], v[8 * qq + 5]);
+              u.w = pack_bf16x2(v[8 * qq + 6], v[8 * qq + 7]);
+              *reinterpret_cast<uint4*>(stg16 + stg16_idx(lane, 8 * qq)) = u;
+            }
+          }
+          if (diag) {
+            // lower triangle of the chunk := its upper triangle, transposed
+            __syncwarp();
+            for (int j = 0; j < lane; ++j) {
+              if (!obf) stg[stg_idx(lane, j)] = stg[stg_idx(j, lane)];
+              else stg16[stg16_idx(lane, j)] = stg16[stg16_idx(j, lane)];
+            }
+          }
+          ptx::fence_async_shared();
+          __syncwarp();
+          if (lane == 0) {
+            ptx::tma_store_3d(&sg.tmC, stg, (int32_t)gj0, (int32_t)row_base, z);
+            ptx::bulk_commit();
+          }
+          if (a.tri && !diag) {
+            if (lane == 0) ptx::bulk_wait_read0();
+            __syncwarp();
+            if (!obf) {
+#pragma unroll
+              for (int j = 0; j < 32; ++j) stg[stg_idx(j, lane)] = v[j];
+            } else {
+#pragma unroll
+              for (int j = 0; j < 32; ++j) stg16[stg16_idx(j, lane)] = f32_to_bf16(v[j]);
+            }
+            ptx::fence_async_shared();
+            __syncwarp();
+            if (lane == 0) {
+              ptx::tma_store_3d(&sg.tmC, stg, (int32_t)row_base, (int32_t)gj0, z);
+              ptx::bulk_commit();
+            }
+          }
+        }
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&tempty[buf]);
+        continue;
+      }
       // This warp owns tile rows q*32 .. q*32+31 (TMEM lanes) and one half
       // of the columns; each chunk is 32 rows x 32 columns.  Values are
       // finished with row = lane (where the symmetric C0 read (j, i) is
@@ -540,6 +663,9 @@ umma_gemm_kernel(const __grid_constant__ UmmaArgs a) {
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(&tempty[buf]);
     }
+    // bulk stores complete before the CTA (and its shared memory) goes away
+    if (lane == 0) ptx::bulk_wait0();
+    __syncwarp();
   }
   __syncthreads();
   if (warp == 1) {
@@ -663,6 +789,8 @@ int launch(const std::vector<GemmDesc>& gs, cudaStream_t stream, int* status) {
     a.c0_out = g0.c0_from_out ? 1 : 0;
     if (a.c0_out) a.has_c0 = 1;
   }
+  // single workspace output: TMA-store epilogue
+  a.tma_out = (g0.direct.empty() && (g0.has_f32 != g0.has_bf16)) ? 1 : 0;
   int ndirect = 0;
   auto flush = [&]() -> int {
     if (a.nseg == 0) return OUO_OK;
@@ -718,6 +846,11 @@ int launch(const std::vector<GemmDesc>& gs, cudaStream_t stream, int* status) {
     proto.Ob = g.has_bf16 ? reinterpret_cast<uint16_t*>(g.out_bf16.p) : nullptr;
     proto.ldob = g.out_bf16.ld; proto.sob = g.out_bf16.stride;
     proto.direct = g.direct.empty() ? 0 : 1;
+    if (a.tma_out) {
+      const Buf& ob = g.has_f32 ? g.out_f32 : g.out_bf16;
+      OUO_TRY(make_map(&proto.tmC, ob, 32, 32,
+                       g.has_f32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B));
+    }
     int64_t b0 = 0;
     while (b0 < g.nb) {
       if (a.nseg == kMaxSeg || (proto.direct && ndirect == kChunk)) OUO_TRY(flush());
