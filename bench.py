@@ -53,6 +53,10 @@ def _args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-layers", type=int, default=1)
+    ap.add_argument("--sweep", action="store_true",
+                    help="shape sweep instead of the step: standard vs Gram NS over "
+                         "m in 512..8192, n/m in 1, 4, 16; Dion / Orth-Dion over rank "
+                         "64..1024 on 4096x4096 (one JSON line)")
     return ap.parse_args()
 
 
@@ -123,6 +127,15 @@ def gram_ns_flops(k: int, n: int, iters: int = ITERS, restarts=RESTART_AFTER):
             tf += 2 * sym            # H (H A)
     bf += qx
     return bf, tf
+
+
+def std_ns_flops(k: int, n: int, iters: int = ITERS):
+    """Algorithmic flops of the standard quintic iteration on a k x n block
+    (k <= n after orientation): per iteration the triangle of X X^T, the
+    triangle of the symmetric b A + c A^2, and the dense a X + B X."""
+    if k > n:
+        k, n = n, k
+    return iters * (k * (k + 1) * n + k * k * (k + 1) + 2 * k * k * n)
 
 
 def _workload_shapes(layers):
@@ -292,8 +305,9 @@ def run_ours(args):
     ks = [ouo.dion3_num_selected(m, RHO) for _, m, _ in shapes]
     keys = torch.empty(sum(m for _, m, _ in shapes), dtype=torch.float64, device=dev)
     idx = torch.empty(sum(ks), dtype=torch.int32, device=dev)
-    X0 = [torch.empty(k, n, dtype=torch.bfloat16, device=dev) for k, (_, _, n) in zip(ks, shapes)]
-    O = [torch.empty_like(x) for x in X0]
+    kn = [(k, n) for k, (_, _, n) in zip(ks, shapes)]
+    X0 = ouo.batch_empty(kn, torch.bfloat16, dev)
+    O = ouo.batch_empty(kn, torch.bfloat16, dev)
     scale = torch.empty(len(shapes), dtype=torch.float32, device=dev)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
     Mb, Gb, Wb = ouo.MatBatch(Ms), ouo.MatBatch(Gs), ouo.MatBatch(Ws)
@@ -486,8 +500,91 @@ def e2e_measure(args, step, Gs, idx, scale, dev, barrier, max_over_ranks):
             "d2h_bytes_per_step": idx.numel() * 4 + scale.numel() * 4}
 
 
+def run_sweep(args):
+    """Standard vs Gram Newton-Schulz over square-to-wide shapes (bf16
+    low-rank(64) + noise inputs, normalization on, one batch per shape sized
+    to about 2^29 elements), and Dion / Orth-Dion steps on one 4096 x 4096
+    matrix over the rank.  Device time per call with CUDA events after
+    warm-up; prints one JSON line."""
+    import torch
+
+    import orthonormalized_update_optimizers_b200 as ouo
+    from orthonormalized_update_optimizers_b200 import synth
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    K, W = max(args.steps, 1), max(args.warmup, 3)
+
+    def timed(fn):
+        for _ in range(W):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(K):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / K
+
+    sampler = ClockSampler(0)
+    sampler.start()
+    ns_rows = []
+    for m in (512, 1024, 2048, 4096, 8192):
+        for ratio in (1, 4, 16):
+            n = m * ratio
+            nb = max(1, min(64, (1 << 29) // (m * n)))
+            X = [synth.lowrank_plus_noise(m, n, 64, 0.02, synth.seed_for(4, 100 * i + ratio),
+                                          torch.bfloat16, dev) for i in range(nb)]
+            O = [torch.empty_like(x) for x in X]
+            Xb, Ob = ouo.MatBatch(X), ouo.MatBatch(O)
+            row = {"m": m, "n": n, "batch": nb}
+            for name, fn_name, flops in (("standard", "ns_orthogonalize", std_ns_flops(m, n)),
+                                         ("gram", "gram_ns_orthogonalize", sum(gram_ns_flops(m, n)))):
+                params = ouo.ns_params()
+                wsb = getattr(ouo, fn_name.replace("orthogonalize", "workspace_bytes"))(Xb, params)
+                ws = torch.empty(wsb, dtype=torch.uint8, device=dev)
+                fn = getattr(ouo, fn_name)
+                ms = timed(lambda: fn(Xb, Ob, params, workspace=ws))
+                row[name] = {"ms": round(ms, 4), "tflops": round(nb * flops / ms / 1e9, 1),
+                             "us_per_matrix": round(ms * 1e3 / nb, 2)}
+                del ws
+            row["gram_speedup"] = round(row["standard"]["ms"] / row["gram"]["ms"], 3)
+            ns_rows.append(row)
+            del X, O, Xb, Ob
+            torch.cuda.empty_cache()
+
+    dion_rows = []
+    m = n = 4096
+    G = synth.lowrank_plus_noise(m, n, 64, 0.02, synth.seed_for(4, 7), torch.bfloat16, dev)
+    for r in (64, 128, 256, 512, 1024):
+        for mode in ("colnorm", "qr"):
+            M = torch.zeros(m, n, dtype=torch.float32, device=dev)
+            Wt = torch.zeros(m, n, dtype=torch.bfloat16, device=dev)
+            q = torch.linalg.qr(synth.dion_q0(n, r, 1).to(dev))[0]
+            Qt = q.T.contiguous()
+            p = ouo.dion_params(rank=r, norm_mode=mode)
+            ws = torch.empty(ouo.dion_workspace_bytes([M], p), dtype=torch.uint8, device=dev)
+            status = torch.zeros(1, dtype=torch.int32, device=dev)
+            ms = timed(lambda: ouo.dion_lowrank_step([M], [G], [Qt], [Wt], p,
+                                                      workspace=ws, status=status))
+            gemm = 8 * m * n * r
+            dion_rows.append({"r": r, "mode": mode, "ms": round(ms, 4),
+                              "gemm_tflops": round(gemm / ms / 1e9, 1),
+                              "status": int(status.item())})
+            del M, Wt, Qt, ws
+    clocks = sampler.stop()
+    print(json.dumps({"mode": "sweep", "unit": "ms per call (device time)", "steps": K,
+                      "warmup": W, "dtype": "bf16 (k x k products tf32; Dion tf32)",
+                      "data": "synthetic low-rank(64) + N(0, 0.02^2) noise",
+                      "ns": ns_rows, "dion": dion_rows, "clocks": clocks}), flush=True)
+
+
 def main():
     args = _args()
+    if args.sweep:
+        run_sweep(args)
+        return
     if args.impl == "reference":
         run_reference(args)
     else:

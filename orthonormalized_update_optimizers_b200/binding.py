@@ -22,7 +22,7 @@ __all__ = [
     "ns_orthogonalize", "gram_ns_workspace_bytes", "gram_ns_orthogonalize",
     "gram_ns_orthogonalize_noalloc",
     "apply_update", "dion_workspace_bytes", "dion_lowrank_step", "version",
-    "launch_count", "timing_enable", "timing_read",
+    "launch_count", "timing_enable", "timing_read", "batch_empty",
 ]
 
 
@@ -58,6 +58,27 @@ class MatBatch:
     @property
     def device(self):
         return self.tensors[0].device if self.tensors else torch.device("cuda")
+
+
+def batch_empty(shapes: Sequence[Sequence[int]], dtype=torch.bfloat16,
+                device=None) -> list:
+    """Uninitialised matrices, one per (rows, cols) in ``shapes``, carved so
+    that all matrices of one shape are consecutive slices of one contiguous
+    [count, rows, cols] block, in the order they appear.  A Newton-Schulz
+    input batch laid out this way (one uniform stride per shape) is read in
+    place instead of being copied into the workspace first."""
+    order = {}
+    for s in shapes:
+        order.setdefault((int(s[0]), int(s[1])), []).append(None)
+    blocks = {key: torch.empty((len(v), key[0], key[1]), dtype=dtype, device=device)
+              for key, v in order.items()}
+    used = {key: 0 for key in order}
+    out = []
+    for s in shapes:
+        key = (int(s[0]), int(s[1]))
+        out.append(blocks[key][used[key]])
+        used[key] += 1
+    return out
 
 
 def _batch(x) -> MatBatch:

@@ -337,6 +337,55 @@ int std_all(const ouo_ns_params& p, Plan& pl, cudaStream_t s, int* status) {
   return OUO_OK;
 }
 
+// True when a group's matrices can serve directly as the (read-only) X0
+// operand of Gram NS: no
+// normalization, no transposition, the arithmetic's own element type, rows
+// on 16-byte boundaries, matrices equally spaced in memory (a batched
+// [nb][rows][ld] block with a 16-byte multiple stride), and no output of the
+// call overlapping the block (X0 is read again by later stages).
+bool caller_x0(const ouo_mat* X, int x_dtype, const ouo_mat* O, int o_dtype,
+               int nmat, const Group& g, const Oriented& o,
+               const ouo_ns_params& p, bool gram, Buf* out) {
+  const int want = p.precision == OUO_PREC_BF16 ? OUO_BF16 : OUO_F32;
+  if (p.normalize || o.transpose || x_dtype != want) return false;
+  // Standard NS and a second Gram restart write into the X0 buffer; only a
+  // Gram schedule with at most one restart leaves it read-only.
+  if (!gram) return false;
+  int restarts = 0;
+  for (int t = 1; t < p.iters; ++t) restarts += is_restart(p, t) ? 1 : 0;
+  if (restarts > 1) return false;
+  const size_t es = elem_size(x_dtype);
+  const ouo_mat& f = X[g.members[0]];
+  for (int m : g.members)
+    if (!vec16(X[m], x_dtype) || X[m].ld != f.ld) return false;
+  int64_t stride_b = 0;
+  if (g.members.size() > 1) {
+    stride_b = (int64_t)((const char*)X[g.members[1]].ptr - (const char*)f.ptr);
+    if (stride_b <= 0 || stride_b % 16 || stride_b < f.rows * f.ld * (int64_t)es)
+      return false;
+    for (size_t i = 1; i < g.members.size(); ++i)
+      if ((const char*)X[g.members[i]].ptr - (const char*)f.ptr != (int64_t)i * stride_b)
+        return false;
+  }
+  const char* lo = (const char*)f.ptr;
+  const char* hi = (const char*)X[g.members.back()].ptr + f.rows * f.ld * es;
+  for (int i = 0; i < nmat; ++i) {
+    const char* olo = (const char*)O[i].ptr;
+    const char* ohi = olo + O[i].rows * O[i].ld * elem_size(o_dtype);
+    if (olo < hi && lo < ohi) return false;
+  }
+  Buf b;
+  b.p = const_cast<char*>(lo);
+  b.dtype = x_dtype;
+  b.rows = f.rows;
+  b.cols = f.cols;
+  b.ld = f.ld;
+  b.stride = g.members.size() > 1 ? stride_b / (int64_t)es : f.rows * f.ld;
+  b.nb = (int64_t)g.members.size();
+  *out = b;
+  return true;
+}
+
 int validate_params(const ouo_ns_params* p) {
   if (!p) return set_error(OUO_ERR_INVALID_ARG, "NULL ns params");
   if (p->iters < 0 || p->iters > 1000)
@@ -390,8 +439,14 @@ int run_ns(const ouo_mat* X, int x_dtype, const ouo_mat* O, int o_dtype,
   for (const Group& g : groups) {
     const Oriented o = orient(g);
     pl.ws.push_back(carve(ar, g, o, gram, p->precision, o_dtype));
-    OUO_TRY(ns_prep(X, x_dtype, g, o.transpose, p->normalize != 0, p->eps,
-                    pl.ws.back().x0, pl.ws.back().scratch, s));
+    Buf direct_x0;
+    if (caller_x0(X, x_dtype, O, o_dtype, nmat, g, o, *p, gram, &direct_x0)) {
+      // the caller's batch already is the layout X0 needs: read it in place
+      pl.ws.back().x0 = direct_x0;
+    } else {
+      OUO_TRY(ns_prep(X, x_dtype, g, o.transpose, p->normalize != 0, p->eps,
+                      pl.ws.back().x0, pl.ws.back().scratch, s));
+    }
     // The last product writes straight into the caller's O when the layout
     // allows (no transposition, 16-byte aligned rows, tensor-core path).
     std::vector<MatRef> direct;

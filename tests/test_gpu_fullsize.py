@@ -166,3 +166,54 @@ def test_bounded_wait_reports_timeout_and_context_survives():
     torch.cuda.synchronize()
     assert st2.item() == 0
     assert rel_fro(to64(O), ons.gram_newton_schulz(to64(X), 5)) <= TOL_BF16
+
+
+# Shape sweep (square to 16x wide, bf16 low-rank(64) + noise), standard and
+# Gram NS with normalization on.  Sizes the oracle finishes in seconds are
+# checked matrix by matrix; the largest shapes by the identity both iterations
+# satisfy in exact arithmetic (Gram NS computes the standard iteration's
+# polynomial), within twice the per-path tolerance.
+SWEEP_ORACLE = [(512, 512), (512, 8192), (1024, 1024), (1024, 16384), (2048, 2048),
+                (2048, 8192), (1024, 4096)]
+SWEEP_LARGE = [(4096, 16384), (8192, 8192), (4096, 65536), (8192, 131072)]
+
+
+@pytest.mark.parametrize("shape", SWEEP_ORACLE)
+def test_shape_sweep_against_oracle(shape):
+    m, n = shape
+    nb = 3
+    Xs = ouo.batch_empty([shape] * nb, torch.bfloat16, DEV)
+    for i, x in enumerate(Xs):
+        x.copy_(synth.lowrank_plus_noise(m, n, 64, 0.02, synth.seed_for(4, 100 * i + n // m),
+                                         torch.bfloat16, DEV))
+    Os = [torch.empty_like(x) for x in Xs]
+    Og = [torch.empty_like(x) for x in Xs]
+    ouo.ns_orthogonalize(Xs, Os, ouo.ns_params())
+    ouo.gram_ns_orthogonalize(Xs, Og, ouo.ns_params())
+    torch.cuda.synchronize()
+    for i in (0, nb - 1):
+        X64 = to64(Xs[i])
+        assert rel_fro(to64(Os[i]), ons.newton_schulz(X64, 5)) <= TOL_BF16
+        assert rel_fro(to64(Og[i]), ons.gram_newton_schulz(X64, 5, restart_after=(3,))) <= TOL_BF16
+
+
+@pytest.mark.parametrize("shape", SWEEP_LARGE)
+def test_shape_sweep_large_gram_equals_standard(shape):
+    m, n = shape
+    X = synth.lowrank_plus_noise(m, n, 64, 0.02, synth.seed_for(4, n // m), torch.bfloat16, DEV)
+    Os, Og = torch.empty_like(X), torch.empty_like(X)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    ouo.ns_orthogonalize([X], [Os], ouo.ns_params(), status=status)
+    ouo.gram_ns_orthogonalize([X], [Og], ouo.ns_params(), status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    d = (Os.float() - Og.float()).norm() / Os.float().norm()
+    assert torch.isfinite(Og.float()).all()
+    assert d.item() <= 2 * TOL_BF16
+    # the output is neither vanishing nor blown up: ||O||_F^2 / m is the mean
+    # of the squared output singular values, each at most 1.2024^2 (the upper
+    # edge of the quintic's band), and most of them are near one here
+    ms = (Og.float().norm() ** 2 / m).item()
+    assert 0.3 <= ms <= 1.2024 ** 2
+    del X, Os, Og
+    torch.cuda.empty_cache()

@@ -134,3 +134,75 @@ def test_correctness_matrix_256x1024_against_svd():
                 assert np.abs(off).max() <= 1e-4
                 sv = np.diag(D)
                 assert sv.min() >= 0.68 and sv.max() <= 1.2025
+
+
+@pytest.mark.parametrize("precision", ["bf16", "fp32"])
+@pytest.mark.parametrize("restarts", [(3,), (), (1, 3)])
+def test_gram_contiguous_batch_read_in_place(precision, restarts):
+    # A batch carved by batch_empty (one uniform stride per shape) is read in
+    # place when normalization is off; the result must equal, bit for bit, the
+    # same batch given as separate tensors (which goes through the copy), and
+    # the inputs must be left untouched.  Two restarts force the copy path.
+    dtype = torch.bfloat16 if precision == "bf16" else torch.float32
+    shapes = [(128, 512), (64, 1000), (128, 512), (300, 128), (64, 1000), (128, 512)]
+    src = [_inputs(s, dtype, 40 + i) for i, s in enumerate(shapes)]
+    src = [(x.float() / x.float().norm()).to(dtype) for x in src]  # normalization is off
+    Xc = ouo.batch_empty(shapes, dtype, DEV)
+    for x, s in zip(Xc, src):
+        x.copy_(s)
+    Xs = [s.clone() for s in src]
+    p = ouo.ns_params(precision=precision, normalize=False, restart_after=restarts)
+    Oc = [torch.empty_like(x) for x in Xc]
+    Os = [torch.empty_like(x) for x in Xs]
+    ouo.gram_ns_orthogonalize(Xc, Oc, p)
+    ouo.gram_ns_orthogonalize(Xs, Os, p)
+    torch.cuda.synchronize()
+    for a, b, x, s in zip(Oc, Os, Xc, src):
+        assert torch.equal(a, b)
+        assert torch.equal(x, s)
+    for i in (0, 3):
+        ref = _oracle(to64(src[i]), True, restarts=restarts, normalize=False)
+        tol = TOL_BF16 if precision == "bf16" else TOL_FP32
+        assert rel_fro(to64(Oc[i]), ref) <= tol
+
+
+def test_gram_contiguous_batch_output_over_input():
+    # O written over its own input block (full aliasing): the in-place read is
+    # refused, the copy path runs, and the result equals the separate-output run.
+    shapes = [(128, 512)] * 4
+    Xc = ouo.batch_empty(shapes, torch.bfloat16, DEV)
+    for i, x in enumerate(Xc):
+        y = _inputs((128, 512), torch.float32, 60 + i)
+        x.copy_(y / y.norm())
+    ref = [torch.empty_like(x) for x in Xc]
+    p = ouo.ns_params(normalize=False)
+    ouo.gram_ns_orthogonalize(Xc, ref, p)
+    ouo.gram_ns_orthogonalize(Xc, Xc, p)
+    torch.cuda.synchronize()
+    for a, b in zip(Xc, ref):
+        assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("gram", [True, False])
+def test_single_cta_and_cta_pair_tiles_agree(gram, monkeypatch):
+    # Matrices taller than 128 rows run on CTA-pair tiles (256 x 256) by
+    # default; OUO_CTA_PAIR=0 selects single-CTA 128 x 256 tiles.  Both must
+    # meet the oracle and agree with each other within half the bf16
+    # tolerance.
+    shapes = [(300, 1000), (512, 2048), (1792, 4096), (256, 256)]
+    Xs = [_inputs(s, torch.bfloat16, 70 + i) for i, s in enumerate(shapes)]
+    p = ouo.ns_params()
+    fn = ouo.gram_ns_orthogonalize if gram else ouo.ns_orthogonalize
+    outs = {}
+    for mode in ("1", "0"):
+        monkeypatch.setenv("OUO_CTA_PAIR", mode)
+        Os = [torch.empty_like(x) for x in Xs]
+        fn(Xs, Os, p)
+        torch.cuda.synchronize()
+        outs[mode] = Os
+    for i, x in enumerate(Xs):
+        if i < 2:
+            ref = _oracle(to64(x), gram)
+            assert rel_fro(to64(outs["1"][i]), ref) <= TOL_BF16
+            assert rel_fro(to64(outs["0"][i]), ref) <= TOL_BF16
+        assert rel_fro(to64(outs["1"][i]), to64(outs["0"][i])) <= 1e-2
