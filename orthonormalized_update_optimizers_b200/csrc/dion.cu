@@ -20,7 +20,8 @@
 // tcgen05 GEMM (tf32 operands, fp32 accumulation) with K-major A.  The
 // orthonormalization works on r x L row blocks X: S = X X^T in fp32 (split
 // over L, partial sums added in float64 in a fixed order), S = L L^T by a
-// one-CTA Cholesky, L inverted in place, X <- L^-1 X (rows orthonormal; the
+// one-CTA Cholesky (r <= 128) or the blocked cooperative Cholesky of chol.cu
+// (wider ranks), L inverted, X <- L^-1 X (rows orthonormal; the
 // implied R = L^T has a positive diagonal, the unique QR).  Two passes
 // (CholeskyQR2).  A failed pivot retries with the shift of shifted
 // CholeskyQR (11 (L r + r (r + 1)) u ||X||_F^2); a second failure sets
@@ -85,8 +86,9 @@ __global__ void __launch_bounds__(256) gram_partial_kernel(const GramArgs a) {
 }
 
 // ---------------------------------------------------- Cholesky + inverse
-// One CTA.  S is summed from the partials in float64 (fixed order) and kept
-// as a packed lower triangle (fp32) in `tri` (shared or global memory).
+// One CTA, ranks up to 128 (larger ones use the blocked kernel in chol.cu).
+// S is summed from the partials in float64 (fixed order) and kept as a
+// packed lower triangle (fp32) in shared memory.
 // Cholesky S = L L^T in place, then L^-1 in place, then written as a full
 // lower-triangular r x r row-major fp32 matrix.
 __device__ __forceinline__ int tri_at(int i, int j) {  // j <= i
@@ -98,11 +100,9 @@ struct CholArgs {
   int splits;
   int r;
   int64_t L;        // length of the rows of X (for the shift)
-  float* tri_glob;  // packed scratch when the triangle does not fit in smem
   float* Linv;      // r x r out, row pitch ldl
   int64_t ldl;
   int* status;
-  int use_smem;
 };
 
 __device__ void chol_load(const CholArgs& a, float* tri, float shift) {
@@ -180,8 +180,8 @@ __global__ void __launch_bounds__(1024) chol_inv_kernel(const CholArgs a) {
   extern __shared__ float sm[];
   __shared__ int s_fail;
   const int r = a.r;
-  float* tri = a.use_smem ? sm : a.tri_glob;
-  float* tmp = a.use_smem ? sm + r * (r + 1) / 2 : a.tri_glob + r * (r + 1) / 2;
+  float* tri = sm;
+  float* tmp = sm + r * (r + 1) / 2;
   chol_load(a, tri, 0.f);
   if (!chol_factor(a, tri, &s_fail)) {
     // shifted CholeskyQR: 11 (L r + r (r + 1)) u ||X||_F^2, ||X||_F^2 = tr S
@@ -269,10 +269,9 @@ unsigned grid_1d(int64_t n, int per_block) {
   return (unsigned)(b < 1 ? 1 : b);
 }
 
-// Largest packed triangle (plus r floats) the one-CTA kernel keeps in
-// shared memory.
+// Packed triangle (plus r floats) the one-CTA kernel keeps in shared
+// memory: at most 33 KB for the ranks it serves (r <= 128).
 size_t chol_smem_bytes(int r) { return ((size_t)r * (r + 1) / 2 + r) * sizeof(float); }
-constexpr size_t kCholSmemMax = 200 * 1024;
 
 int gram_splits(int r, int64_t L) {
   const int tiles = (int)ceil_div(r, kGT);
@@ -290,9 +289,15 @@ struct DionWs {
   Buf P;        // m x r
   Buf Ra, Rb;   // r x n
   Buf part;     // [64][r][r]
-  Buf Linv;     // r x r
-  Buf tri;      // packed triangle + r (global fallback)
+  Buf Linv;     // R x R (R = r rounded up to 32)
+  Buf S;        // R x R (blocked Cholesky)
+  Buf ctl;      // barrier counter and flags of the blocked Cholesky
 };
+
+// Ranks above this use the blocked multi-CTA Cholesky; the one-CTA kernel
+// keeps smaller ones (their triangle fits in its shared memory).
+constexpr int kBlockedCholMinRank = 129;
+int64_t padded_rank(int r) { return ceil_div(r, 32) * 32; }
 
 DionWs carve_dion(Arena& ar, int64_t m, int64_t n, int r) {
   DionWs w;
@@ -302,8 +307,10 @@ DionWs carve_dion(Arena& ar, int64_t m, int64_t n, int r) {
   w.Ra = ar.take(OUO_F32, 1, r, n);
   w.Rb = ar.take(OUO_F32, 1, r, n);
   w.part = ar.take(OUO_F32, 64, r, r);
-  w.Linv = ar.take(OUO_F32, 1, r, r);
-  w.tri = ar.take(OUO_F32, 1, 1, (int64_t)r * (r + 1) / 2 + r);
+  const int64_t R = padded_rank(r);
+  w.Linv = ar.take(OUO_F32, 1, R, R);
+  w.S = ar.take(OUO_F32, 1, R, R);
+  w.ctl = ar.take(OUO_F32, 1, 1, (int64_t)ceil_div(chol_blocked_ctl_bytes(r), 4));
   return w;
 }
 
@@ -341,24 +348,21 @@ int orth_rows(Buf X, Buf tmp, Buf Y, const DionWs& w, cudaStream_t s,
     dim3 grid((unsigned)(ga.tiles * (ga.tiles + 1) / 2), (unsigned)used);
     gram_partial_kernel<<<grid, 256, 0, s>>>(ga);
     OUO_CHECK_LAUNCH();
-    CholArgs ca;
-    ca.part = ga.part;
-    ca.splits = used;
-    ca.r = r;
-    ca.L = L;
-    ca.tri_glob = reinterpret_cast<float*>(w.tri.p);
-    ca.Linv = reinterpret_cast<float*>(w.Linv.p);
-    ca.ldl = w.Linv.ld;
-    ca.status = status;
-    const size_t smem = chol_smem_bytes(r);
-    ca.use_smem = smem <= kCholSmemMax;
-    if (ca.use_smem) {
-      OUO_CHECK_CUDA(cudaFuncSetAttribute(chol_inv_kernel,
-                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                          (int)kCholSmemMax));
+    if (r >= kBlockedCholMinRank) {
+      OUO_TRY(chol_blocked(ga.part, used, r, L, reinterpret_cast<float*>(w.S.p),
+                           reinterpret_cast<float*>(w.Linv.p), w.ctl.p, status, s));
+    } else {
+      CholArgs ca;
+      ca.part = ga.part;
+      ca.splits = used;
+      ca.r = r;
+      ca.L = L;
+      ca.Linv = reinterpret_cast<float*>(w.Linv.p);
+      ca.ldl = w.Linv.ld;
+      ca.status = status;
+      chol_inv_kernel<<<1, 1024, chol_smem_bytes(r), s>>>(ca);
+      OUO_CHECK_LAUNCH();
     }
-    chol_inv_kernel<<<1, 1024, ca.use_smem ? smem : 0, s>>>(ca);
-    OUO_CHECK_LAUNCH();
     // dst = Linv src
     GemmDesc d;
     d.M = r;

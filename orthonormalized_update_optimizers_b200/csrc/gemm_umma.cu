@@ -22,8 +22,19 @@
 // Tile: 128 (M) x BN (N), K staged 128 bytes per stage (64 bf16 or 32 tf32
 // elements) with the 128-byte swizzle.  A is always K-major.  B is K-major
 // (an N x K buffer) or MN-major (a K x N buffer, e.g. X in Q X).
+//
+// CTA-pair mode (CG = 2, BN = 256): the launch is made of clusters of two
+// CTAs on neighbouring SMs that share one 256 x 256 tile.  Each CTA stages
+// its own 128 rows of A and its own half (128 columns) of B, so an SM moves
+// two thirds of the operand bytes of the single-CTA 128 x 256 tile for the
+// same number of MMA cycles.  The even CTA issues tcgen05.mma.cta_group::2
+// (M = 256) over both CTAs' shared memory; both CTAs' TMA loads complete on
+// the even CTA's stage barrier, MMA completion is multicast to the stage and
+// accumulator barriers of both CTAs (tcgen05.commit multicast), and each CTA
+// drains its own 128 TMEM lanes.  TMA loads never multicast.
 #include <cuda.h>
 
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -86,12 +97,14 @@ struct UmmaArgs {
   int64_t dld[kChunk];
 };
 
-template <int BN>
+template <int BN, int CG>
 struct Cfg {
-  static constexpr uint32_t kABytes = kTileM * kRowBytes;       // 16 KB
-  static constexpr uint32_t kBBytes = (uint32_t)BN * kRowBytes;  // 16/32 KB
+  static constexpr uint32_t kTileRows = kTileM * CG;  // rows of one scheduled tile
+  static constexpr uint32_t kBRows = (uint32_t)BN / CG;  // B rows (N) staged per CTA
+  static constexpr uint32_t kABytes = kTileM * kRowBytes;      // 16 KB
+  static constexpr uint32_t kBBytes = kBRows * kRowBytes;      // 16/32 KB
   static constexpr uint32_t kStageBytes = kABytes + kBBytes;
-  static constexpr int kStages = BN == 256 ? 4 : 6;
+  static constexpr int kStages = CG == 2 ? 6 : (BN == 256 ? 4 : 6);
   static constexpr uint32_t kTmemCols = 2 * BN;
   // per epilogue warp: a 32 x 32 fp32 staging buffer
   static constexpr uint32_t kEpiBytes = kEpiWarps * 32 * 32 * 4;
@@ -99,14 +112,15 @@ struct Cfg {
       1024 + (size_t)kStages * kStageBytes + 256 + kEpiBytes;
 };
 
-// First column tile of row tile i that reaches the diagonal.
-__device__ __forceinline__ int64_t tri_jmin(int64_t i, int BN) {
-  return (i * (int64_t)kTileM) / BN;
+// First column tile of row tile i (tiles of TR rows) that reaches the
+// diagonal.
+__host__ __device__ __forceinline__ int64_t tri_jmin(int64_t i, int BN, int TR) {
+  return (i * (int64_t)TR) / BN;
 }
 
 // Launch-wide tile id -> (segment, matrix within the segment, tile row,
 // tile column).
-__device__ __forceinline__ int decode_tile(const UmmaArgs& a, int BN,
+__device__ __forceinline__ int decode_tile(const UmmaArgs& a, int BN, int TR,
                                            int64_t tile, int64_t* b,
                                            int64_t* ti, int64_t* tj) {
   int g = 0;
@@ -122,13 +136,13 @@ __device__ __forceinline__ int decode_tile(const UmmaArgs& a, int BN,
   }
   int64_t i = 0;
   while (true) {
-    int64_t cnt = sg.tiles_n - tri_jmin(i, BN);
+    int64_t cnt = sg.tiles_n - tri_jmin(i, BN, TR);
     if (t < cnt) break;
     t -= cnt;
     ++i;
   }
   *ti = i;
-  *tj = tri_jmin(i, BN) + t;
+  *tj = tri_jmin(i, BN, TR) + t;
   return g;
 }
 
@@ -246,16 +260,17 @@ __device__ __forceinline__ void load_c0x4(const Segment& sg, int64_t b,
   }
 }
 
-template <int BN, int FMT /*1 bf16, 2 tf32*/, int B_MN>
+template <int BN, int FMT /*1 bf16, 2 tf32*/, int B_MN, int CG /*CTAs per tile*/>
 __global__ void __launch_bounds__(kThreads, 1)
 umma_gemm_kernel(const __grid_constant__ UmmaArgs a) {
-  using C = Cfg<BN>;
+  using C = Cfg<BN, CG>;
+  constexpr int TR = (int)C::kTileRows;
   constexpr uint32_t kEs = FMT == 1 ? 2 : 4;           // element bytes
   constexpr uint32_t kBK = kRowBytes / kEs;            // K elements per stage
   constexpr uint32_t kInstK = 32 / kEs;                // K per MMA (32 bytes)
   constexpr uint32_t kChunkCols = kRowBytes / kEs;     // MN-major chunk width
   constexpr uint32_t kChunkBytes = kBK * kRowBytes;    // one MN-major chunk
-  constexpr uint32_t kIdesc = ptx::instr_desc(FMT, B_MN, BN);
+  constexpr uint32_t kIdesc = ptx::instr_desc(FMT, B_MN, BN, kTileM * CG);
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -273,6 +288,10 @@ umma_gemm_kernel(const __grid_constant__ UmmaArgs a) {
   float* epi_smem = reinterpret_cast<float*>(smem + C::kStages * C::kStageBytes);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // CTA pair: rank 0 issues the MMAs and owns the stage and accumulator-free
+  // barriers both CTAs signal; a scheduled tile is shared by the pair.
+  const uint32_t rank = CG == 2 ? ptx::cluster_ctarank() : 0u;
+  const int64_t tile0 = blockIdx.x / CG, tile_step = gridDim.x / CG;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
@@ -281,7 +300,7 @@ umma_gemm_kernel(const __grid_constant__ UmmaArgs a) {
     }
     for (int s = 0; s < 2; ++s) {
       ptx::mbar_init(&tfull[s], 1);
-      ptx::mbar_init(&tempty[s], kEpiWarps);  // one arrival per epilogue warp
+      ptx::mbar_init(&tempty[s], kEpiWarps * CG);  // one arrival per epilogue warp
     }
     ptx::mbar_init(drain, 1);
     *abort_flag = 0;
@@ -292,11 +311,18 @@ umma_gemm_kernel(const __grid_constant__ UmmaArgs a) {
     }
   }
   if (warp == 1) {
-    ptx::tmem_alloc(tmem_holder, C::kTmemCols);
-    ptx::tmem_relinquish();
+    if (CG == 2) {
+      ptx::tmem_alloc2(tmem_holder, C::kTmemCols);
+      ptx::tmem_relinquish2();
+    } else {
+      ptx::tmem_alloc(tmem_holder, C::kTmemCols);
+      ptx::tmem_relinquish();
+    }
   }
   ptx::tc_fence_before();
   __syncthreads();
+  // the peer's barriers are initialized before anything signals them
+  if (CG == 2) ptx::cluster_sync();
   ptx::tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
 
@@ -305,32 +331,37 @@ umma_gemm_kernel(const __grid_constant__ UmmaArgs a) {
     uint32_t stage = 0, phase = 0;
     bool ok = true;
     int64_t issued = 0;
-    for (int64_t tile = blockIdx.x; ok && tile < a.total_tiles;
-         tile += gridDim.x) {
+    for (int64_t tile = tile0; ok && tile < a.total_tiles;
+         tile += tile_step) {
       int64_t b, ti, tj;
-      const int g = decode_tile(a, BN, tile, &b, &ti, &tj);
+      const int g = decode_tile(a, BN, TR, tile, &b, &ti, &tj);
       const Segment& sg = a.seg[g];
       const int64_t nk = (sg.K + kBK - 1) / kBK;
       const int32_t z = (int32_t)(sg.b0 + b);
+      const int32_t arow = (int32_t)(ti * TR + rank * kTileM);
+      const int32_t bcol = (int32_t)(tj * BN + rank * C::kBRows);
       for (int64_t kb = 0; kb < nk; ++kb) {
         if (!ptx::mbar_wait(&empty[stage], phase ^ 1, abort_flag)) {
           ok = false;
           break;
         }
-        ptx::mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
+        // the stage barrier of the pair's even CTA counts both CTAs' bytes
+        if (rank == 0) ptx::mbar_arrive_expect_tx(&full[stage], CG * C::kStageBytes);
+        const uint32_t fb = CG == 2 ? ptx::mapa(ptx::smem_u32(&full[stage]), 0) : 0u;
+        auto load = [&](void* dst, const CUtensorMap* m, int32_t c0, int32_t c1) {
+          if (CG == 2) ptx::tma_load_3d_pair(dst, m, fb, c0, c1, z);
+          else ptx::tma_load_3d(dst, m, &full[stage], c0, c1, z);
+        };
         uint8_t* sa = smem + stage * C::kStageBytes;
         uint8_t* sb = sa + C::kABytes;
-        ptx::tma_load_3d(sa, &sg.tmA, &full[stage], (int32_t)(kb * kBK),
-                         (int32_t)(ti * kTileM), z);
+        load(sa, &sg.tmA, (int32_t)(kb * kBK), arow);
         if (!B_MN) {
-          ptx::tma_load_3d(sb, &sg.tmB, &full[stage], (int32_t)(kb * kBK),
-                           (int32_t)(tj * BN), z);
+          load(sb, &sg.tmB, (int32_t)(kb * kBK), bcol);
         } else {
 #pragma unroll
-          for (uint32_t c = 0; c < (uint32_t)BN / kChunkCols; ++c)
-            ptx::tma_load_3d(sb + c * kChunkBytes, &sg.tmB, &full[stage],
-                             (int32_t)(tj * BN + c * kChunkCols),
-                             (int32_t)(kb * kBK), z);
+          for (uint32_t c = 0; c < C::kBRows / kChunkCols; ++c)
+            load(sb + c * kChunkBytes, &sg.tmB, (int32_t)(bcol + c * kChunkCols),
+                 (int32_t)(kb * kBK));
         }
         ++issued;
         if (++stage == (uint32_t)C::kStages) { stage = 0; phase ^= 1; }
@@ -340,22 +371,30 @@ umma_gemm_kernel(const __grid_constant__ UmmaArgs a) {
       *abort_flag = 1;
       report_status(a.status, OUO_STATUS_TIMEOUT);
       // Loads still in flight complete on their own; before the CTA exits,
-      // wait (bounded) for the last fill of every stage to land.
+      // wait (bounded) for the last fill of every stage to land.  The odd
+      // CTA of a pair signals the even CTA's barriers and cannot observe
+      // them: it waits a fixed 2 ms, far longer than a tile load takes.
+      if (CG == 2 && rank != 0) {
+        const uint64_t t0 = globaltimer_ns();
+        while (globaltimer_ns() - t0 < 2000000ull) {
+        }
+        issued = 0;
+      }
       for (int s = 0; s < C::kStages; ++s) {
         const int64_t fills = issued / C::kStages + (s < issued % C::kStages ? 1 : 0);
         if (fills > 0)
           ptx::mbar_wait_timed(&full[s], (uint32_t)((fills - 1) & 1), 100000000ull);
       }
     }
-  } else if (warp == 1 && lane == 0) {
+  } else if (warp == 1 && lane == 0 && rank == 0) {
     // ----------------------------------------------------------- MMA issuer
     uint32_t stage = 0, phase = 0;
     bool ok = true;
     int64_t local = 0;
-    for (int64_t tile = blockIdx.x; ok && tile < a.total_tiles;
-         tile += gridDim.x, ++local) {
+    for (int64_t tile = tile0; ok && tile < a.total_tiles;
+         tile += tile_step, ++local) {
       int64_t b, ti, tj;
-      const int g = decode_tile(a, BN, tile, &b, &ti, &tj);
+      const int g = decode_tile(a, BN, TR, tile, &b, &ti, &tj);
       const int64_t nk = (a.seg[g].K + kBK - 1) / kBK;
       const uint32_t buf = (uint32_t)(local & 1);
       const uint32_t tphase = (uint32_t)((local >> 1) & 1);
@@ -384,30 +423,42 @@ umma_gemm_kernel(const __grid_constant__ UmmaArgs a) {
                                                       kChunkBytes, 1024))
                    : ptx::smem_desc_sw128(sb + kk * 32, 16, 1024);
           const uint32_t acc = (kb > 0 || kk > 0) ? 1u : 0u;
-          if (FMT == 1) ptx::mma_bf16(d, ad, bd, kIdesc, acc);
-          else ptx::mma_tf32(d, ad, bd, kIdesc, acc);
+          if (CG == 2) {
+            if (FMT == 1) ptx::mma2_bf16(d, ad, bd, kIdesc, acc);
+            else ptx::mma2_tf32(d, ad, bd, kIdesc, acc);
+          } else {
+            if (FMT == 1) ptx::mma_bf16(d, ad, bd, kIdesc, acc);
+            else ptx::mma_tf32(d, ad, bd, kIdesc, acc);
+          }
         }
-        ptx::mma_commit(&empty[stage]);
+        // frees the stage in both CTAs of a pair
+        if (CG == 2) ptx::mma2_commit(&empty[stage], 0x3);
+        else ptx::mma_commit(&empty[stage]);
         if (++stage == (uint32_t)C::kStages) { stage = 0; phase ^= 1; }
       }
       if (!ok) break;
-      ptx::mma_commit(&tfull[buf]);
+      if (CG == 2) ptx::mma2_commit(&tfull[buf], 0x3);
+      else ptx::mma_commit(&tfull[buf]);
     }
     if (!ok) {
       *abort_flag = 1;
       report_status(a.status, OUO_STATUS_TIMEOUT);
     }
-    // all MMAs of this thread complete before TMEM is released
-    ptx::mma_commit(drain);
+    // all MMAs of this thread complete before TMEM (of both CTAs of a pair)
+    // is released
+    if (CG == 2) ptx::mma2_commit(drain, 0x1);
+    else ptx::mma_commit(drain);
     ptx::mbar_wait_timed(drain, 0, kWaitLimitNs);
   } else if (warp >= 2) {
     // ------------------------------------------------------------- epilogue
     const uint32_t q = (uint32_t)(warp & 3);  // TMEM lanes 32q .. 32q+31
     int64_t local = 0;
-    for (int64_t tile = blockIdx.x; tile < a.total_tiles;
-         tile += gridDim.x, ++local) {
+    // accumulator-free barrier of the pair's even CTA (cluster address)
+    const uint32_t tempty_lead = CG == 2 ? ptx::mapa(ptx::smem_u32(tempty), 0) : 0u;
+    for (int64_t tile = tile0; tile < a.total_tiles;
+         tile += tile_step, ++local) {
       int64_t b, ti, tj;
-      const int g = decode_tile(a, BN, tile, &b, &ti, &tj);
+      const int g = decode_tile(a, BN, TR, tile, &b, &ti, &tj);
       const Segment& sg = a.seg[g];
       const uint32_t buf = (uint32_t)(local & 1);
       const uint32_t tphase = (uint32_t)((local >> 1) & 1);
@@ -431,7 +482,7 @@ umma_gemm_kernel(const __grid_constant__ UmmaArgs a) {
         // clipped by the TMA.  Symmetric outputs: the mirrored box (j, i)
         // is a second store from a transposed staging; a chunk on the
         // diagonal is made symmetric in place and stored once.
-        const int64_t row_base = ti * kTileM + q * 32;
+        const int64_t row_base = ti * TR + rank * kTileM + q * 32;
         const int64_t gi = row_base + lane;
         float* stg = epi_smem + (warp - 2) * (32 * 32);
         uint16_t* stg16 = reinterpret_cast<uint16_t*>(stg);
@@ -533,7 +584,10 @@ umma_gemm_kernel(const __grid_constant__ UmmaArgs a) {
         }
         ptx::tc_fence_before();
         __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(&tempty[buf]);
+        if (lane == 0) {
+          if (CG == 2) ptx::mbar_arrive_cluster(tempty_lead + buf * 8u);
+          else ptx::mbar_arrive(&tempty[buf]);
+        }
         continue;
       }
       // This warp owns tile rows q*32 .. q*32+31 (TMEM lanes) and one half
@@ -544,7 +598,7 @@ umma_gemm_kernel(const __grid_constant__ UmmaArgs a) {
       // direct tile (i, j) and, for symmetric outputs, the mirrored tile
       // (j, i).  Chunks entirely below the diagonal of a symmetric output
       // are skipped; chunks fully inside and above it store without masks.
-      const int64_t row_base = ti * kTileM + q * 32;
+      const int64_t row_base = ti * TR + rank * kTileM + q * 32;
       const int64_t gi = row_base + lane;
       float* stg = epi_smem + (warp - 2) * (32 * 32);
       const int sub_r = lane >> 3, sub_c = 4 * (lane & 7);
@@ -661,16 +715,26 @@ umma_gemm_kernel(const __grid_constant__ UmmaArgs a) {
       }
       ptx::tc_fence_before();
       __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(&tempty[buf]);
+      if (lane == 0) {
+        if (CG == 2) ptx::mbar_arrive_cluster(tempty_lead + buf * 8u);
+        else ptx::mbar_arrive(&tempty[buf]);
+      }
     }
     // bulk stores complete before the CTA (and its shared memory) goes away
     if (lane == 0) ptx::bulk_wait0();
     __syncwarp();
   }
   __syncthreads();
+  // a pair frees TMEM only after the even CTA's MMAs (which write both
+  // CTAs' TMEM) and both CTAs' epilogues (which signal the even CTA) are done
+  if (CG == 2) {
+    __syncwarp();
+    ptx::cluster_sync();
+  }
   if (warp == 1) {
     ptx::tc_fence_after();
-    ptx::tmem_dealloc(tmem_base, C::kTmemCols);
+    if (CG == 2) ptx::tmem_dealloc2(tmem_base, C::kTmemCols);
+    else ptx::tmem_dealloc(tmem_base, C::kTmemCols);
   }
 }
 
@@ -750,27 +814,64 @@ int make_map(CUtensorMap* map, const Buf& t, uint32_t box_cols,
   return OUO_OK;
 }
 
-int64_t tiles_per_matrix(const GemmDesc& g, int BN) {
-  const int64_t tm = ceil_div(g.M, kTileM), tn = ceil_div(g.N, BN);
+int64_t tiles_per_matrix(const GemmDesc& g, int BN, int TR) {
+  const int64_t tm = ceil_div(g.M, (int64_t)TR), tn = ceil_div(g.N, BN);
   if (!g.tri) return tm * tn;
   int64_t cnt = 0;
-  for (int64_t i = 0; i < tm; ++i) cnt += tn - (i * (int64_t)kTileM) / BN;
+  for (int64_t i = 0; i < tm; ++i) cnt += tn - tri_jmin(i, BN, TR);
   return cnt;
 }
 
-template <int BN, int FMT, int B_MN>
+// Launch configuration of one kernel instance; CTA pairs are clusters of 2.
+cudaLaunchConfig_t launch_cfg(unsigned grid, size_t smem, cudaStream_t stream,
+                              int cg, cudaLaunchAttribute* attr) {
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)cg;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cfg;
+}
+
+template <int BN, int FMT, int B_MN, int CG>
 int launch(const std::vector<GemmDesc>& gs, cudaStream_t stream, int* status) {
-  using C = Cfg<BN>;
+  using C = Cfg<BN, CG>;
+  constexpr int TR = (int)C::kTileRows;
   constexpr uint32_t es = FMT == 1 ? 2 : 4;
   constexpr uint32_t bk = kRowBytes / es;
-  auto kern = umma_gemm_kernel<BN, FMT, B_MN>;
+  auto kern = umma_gemm_kernel<BN, FMT, B_MN, CG>;
+  // per device: shared-memory opt-in done, and how many CTAs (pairs: CTA
+  // pairs) of this kernel can be resident at once -- a persistent grid
+  // larger than that would run its last CTAs after the others finish
   static bool configured[64] = {false};
+  static int resident[64] = {0};
   int dev = 0;
   OUO_CHECK_CUDA(cudaGetDevice(&dev));
-  if (dev < 0 || dev >= 64 || !configured[dev]) {
+  if (dev < 0 || dev >= 64)
+    return set_error(OUO_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+  if (!configured[dev]) {
     OUO_CHECK_CUDA(cudaFuncSetAttribute(
         kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::kSmem));
-    if (dev >= 0 && dev < 64) configured[dev] = true;
+    int n = num_sms();
+    if (CG == 2) {
+      cudaLaunchAttribute attr[1];
+      cudaLaunchConfig_t cfg = launch_cfg(
+          (unsigned)(2 * num_sms()), C::kSmem, stream, CG, attr);
+      int clusters = 0;
+      OUO_CHECK_CUDA(cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg));
+      if (clusters < 1)
+        return set_error(OUO_ERR_UNSUPPORTED, "no CTA pair of the GEMM kernel fits on this device");
+      n = clusters;
+    }
+    resident[dev] = n;
+    configured[dev] = true;
   }
   const GemmDesc& g0 = gs[0];
   UmmaArgs a;
@@ -799,15 +900,23 @@ int launch(const std::vector<GemmDesc>& gs, cudaStream_t stream, int* status) {
       a.seg[s].tile_start = a.total_tiles;
       a.total_tiles += a.seg[s].tiles_per_mat * a.seg[s].nb;
     }
-    int64_t grid = a.total_tiles < num_sms() ? a.total_tiles : num_sms();
-    if (grid >= 1) {
+    // one CTA (or CTA pair) per resident slot, at most one per tile
+    const int64_t slots = a.total_tiles < resident[dev] ? a.total_tiles : resident[dev];
+    if (slots >= 1) {
       TimingRec rec;
       bool timed = false;
       if (g_timing) {
         std::lock_guard<std::mutex> lock(g_tmu);
         timed = timing_record_begin(stream, &rec) != 0;
       }
-      kern<<<(unsigned)grid, kThreads, C::kSmem, stream>>>(a);
+      if (CG == 1) {
+        kern<<<(unsigned)slots, kThreads, C::kSmem, stream>>>(a);
+      } else {
+        cudaLaunchAttribute attr[1];
+        cudaLaunchConfig_t cfg = launch_cfg(
+            (unsigned)(CG * slots), C::kSmem, stream, CG, attr);
+        OUO_CHECK_CUDA(cudaLaunchKernelEx(&cfg, kern, a));
+      }
       OUO_CHECK_LAUNCH();
       if (timed) {
         cudaEventRecord(rec.e1, stream);
@@ -832,13 +941,13 @@ int launch(const std::vector<GemmDesc>& gs, cudaStream_t stream, int* status) {
     Segment proto;
     memset(&proto, 0, sizeof(proto));
     OUO_TRY(make_map(&proto.tmA, g.A, bk, kTileM));
-    if (!B_MN) OUO_TRY(make_map(&proto.tmB, g.B, bk, BN));
+    if (!B_MN) OUO_TRY(make_map(&proto.tmB, g.B, bk, C::kBRows));
     else OUO_TRY(make_map(&proto.tmB, g.B, kRowBytes / es, bk,
                           FMT == 2 ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B
                                    : CU_TENSOR_MAP_SWIZZLE_128B));
     proto.M = g.M; proto.N = g.N; proto.K = g.K;
     proto.tiles_n = ceil_div(g.N, BN);
-    proto.tiles_per_mat = tiles_per_matrix(g, BN);
+    proto.tiles_per_mat = tiles_per_matrix(g, BN, TR);
     proto.C0 = (g.has_c0 && !g.c0_from_out) ? g.C0.p : nullptr;
     proto.ldc0 = g.C0.ld; proto.sc0 = g.C0.stride;
     proto.Of = g.has_f32 ? reinterpret_cast<float*>(g.out_f32.p) : nullptr;
@@ -916,7 +1025,7 @@ int gemm_umma_grouped(const std::vector<GemmDesc>& gs, cudaStream_t stream,
                       int* status) {
   if (gs.empty()) return OUO_OK;
   const GemmDesc& g0 = gs[0];
-  bool wide = false;
+  bool wide = false, tall = false;
   for (const GemmDesc& g : gs) {
     if (g.A.dtype != g.B.dtype || g.A.dtype != g0.A.dtype)
       return set_error(OUO_ERR_UNSUPPORTED, "tensor-core GEMM needs equal operand types");
@@ -935,13 +1044,28 @@ int gemm_umma_grouped(const std::vector<GemmDesc>& gs, cudaStream_t stream,
     if (g.c0_from_out && (g.direct.empty() || g.tri))
       return set_error(OUO_ERR_INVALID_ARG, "in-place C0 needs direct, non-symmetric outputs");
     wide = wide || g.N > 128;
+    tall = tall || g.M > 128;
   }
+  // CTA pairs (256 x 256 tiles) for wide outputs with more than 128 rows and
+  // K-major B.  OUO_CTA_PAIR=0 selects single-CTA 128 x BN tiles throughout;
+  // OUO_CTA_PAIR=2 also puts MN-major B (Q X) on pairs.
+  const char* env = getenv("OUO_CTA_PAIR");
+  const int pair_mode = env && env[0] >= '0' && env[0] <= '2' ? env[0] - '0' : 1;
+  const bool pair = wide && tall && pair_mode > 0 && (!g0.b_mn || pair_mode == 2);
   if (g0.A.dtype == OUO_BF16) {
-    if (g0.b_mn) return wide ? launch<256, 1, 1>(gs, stream, status) : launch<128, 1, 1>(gs, stream, status);
-    return wide ? launch<256, 1, 0>(gs, stream, status) : launch<128, 1, 0>(gs, stream, status);
+    if (g0.b_mn) {
+      if (pair) return launch<256, 1, 1, 2>(gs, stream, status);
+      return wide ? launch<256, 1, 1, 1>(gs, stream, status) : launch<128, 1, 1, 1>(gs, stream, status);
+    }
+    if (pair) return launch<256, 1, 0, 2>(gs, stream, status);
+    return wide ? launch<256, 1, 0, 1>(gs, stream, status) : launch<128, 1, 0, 1>(gs, stream, status);
   }
-  if (g0.b_mn) return wide ? launch<256, 2, 1>(gs, stream, status) : launch<128, 2, 1>(gs, stream, status);
-  return wide ? launch<256, 2, 0>(gs, stream, status) : launch<128, 2, 0>(gs, stream, status);
+  if (g0.b_mn) {
+    if (pair) return launch<256, 2, 1, 2>(gs, stream, status);
+    return wide ? launch<256, 2, 1, 1>(gs, stream, status) : launch<128, 2, 1, 1>(gs, stream, status);
+  }
+  if (pair) return launch<256, 2, 0, 2>(gs, stream, status);
+  return wide ? launch<256, 2, 0, 1>(gs, stream, status) : launch<128, 2, 0, 1>(gs, stream, status);
 }
 
 int gemm_umma(const GemmDesc& g, cudaStream_t stream, int* status) {

@@ -116,6 +116,14 @@ int ns_writeout(const Buf& y, const ouo_mat* O, int o_dtype, const Group& grp,
                 bool transpose, cudaStream_t stream);
 // Fill nb identity matrices (fp32 and / or bf16 copies).
 int fill_identity(const Buf& q, cudaStream_t stream);
+
+// Blocked Cholesky + triangular inverse (chol.cu): S = sum of `splits`
+// partial r x r Gram matrices; writes L^-1 into Linv (R x R, ld R, R = r
+// rounded up to 32).  S is R x R scratch (ld R); ctl is
+// chol_blocked_ctl_bytes(r) bytes of 8-byte aligned scratch.
+size_t chol_blocked_ctl_bytes(int r);
+int chol_blocked(const float* part, int splits, int r, int64_t L, float* S,
+                 float* Linv, void* ctl, int* status, cudaStream_t stream);
 int convert_buf(const Buf& src, const Buf& dst, cudaStream_t stream);
 
 }  // namespace ouo

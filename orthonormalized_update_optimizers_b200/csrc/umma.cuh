@@ -1,6 +1,7 @@
 // Thin wrappers over the sm_100a PTX used by the tensor-core kernels:
-// mbarriers, TMA tiled loads (no multicast), tcgen05 MMA / commit / TMEM
-// allocation and loads, and the shared-memory matrix descriptors.
+// mbarriers, TMA tiled loads (no multicast), cluster addressing, tcgen05
+// MMA / commit / TMEM allocation and loads (single CTA and CTA pair), and the
+// shared-memory matrix descriptors.
 #pragma once
 
 #include <cuda.h>
@@ -87,6 +88,47 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map,
       : "memory");
 }
 
+// TMA load for a CTA pair (cluster of two): the data lands in this CTA's
+// shared memory, completion is signalled on an mbarrier given by its
+// shared::cluster address, which may be in the peer CTA.
+__device__ __forceinline__ void tma_load_3d_pair(void* dst, const CUtensorMap* map,
+                                                 uint32_t bar_cluster, int32_t c0,
+                                                 int32_t c1, int32_t c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.tile.mbarrier::"
+      "complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(c0), "r"(c1),
+      "r"(c2)
+      : "memory");
+}
+
+// ---- clusters
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+// shared::cluster address of the same shared-memory offset in CTA `rank`.
+__device__ __forceinline__ uint32_t mapa(uint32_t saddr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+  return r;
+}
+
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(
+                   bar_cluster)
+               : "memory");
+}
+
+// All threads of every CTA of the cluster.
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile(
+      "barrier.cluster.arrive.release.aligned;\n\t"
+      "barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
 // 3-D tiled TMA store shared -> global (bulk-group completion).  Elements
 // outside the tensor's extent are not written.
 __device__ __forceinline__ void tma_store_3d(const CUtensorMap* map,
@@ -145,6 +187,28 @@ __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
                : "memory");
 }
 
+// CTA-pair forms: one warp of each CTA of the pair allocates (and frees) the
+// same columns in both CTAs' TMEM.
+__device__ __forceinline__ void tmem_alloc2(uint32_t* holder, uint32_t ncols) {
+  asm volatile(
+      "tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+          smem_u32(holder)),
+      "r"(ncols)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_relinquish2() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::
+                   : "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc2(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(
+                   taddr),
+               "r"(ncols)
+               : "memory");
+}
+
 __device__ __forceinline__ void tc_fence_before() {
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
 }
@@ -172,6 +236,39 @@ __device__ __forceinline__ void mma_tf32(uint32_t d, uint64_t adesc,
       "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// CTA-pair MMA (issued by the even CTA of the pair): M = 256 rows, 128 from
+// each CTA's shared memory; B's N columns split in halves the same way; each
+// CTA's TMEM receives its own 128 rows.
+__device__ __forceinline__ void mma2_bf16(uint32_t d, uint64_t adesc,
+                                          uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma2_tf32(uint32_t d, uint64_t adesc,
+                                          uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Arrive on the mbarrier at `bar`'s offset in every CTA of `cta_mask` once
+// all previously issued CTA-pair MMAs of this thread have completed.
+__device__ __forceinline__ void mma2_commit(uint64_t* bar, uint16_t cta_mask) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster."
+      "multicast::cluster.b64 [%0], %1;" ::"r"(smem_u32(bar)),
+      "h"(cta_mask)
       : "memory");
 }
 
@@ -235,11 +332,12 @@ __device__ __forceinline__ uint64_t smem_desc_sw128_32b(uint32_t saddr,
 }
 
 // Instruction descriptor: fp32 accumulator, A and B of `fmt` (1 = bf16,
-// 2 = tf32), A K-major, B K-major or MN-major, M = 128, N = n.
+// 2 = tf32), A K-major, B K-major or MN-major, M = m (128, or 256 for a CTA
+// pair), N = n.
 __host__ __device__ constexpr uint32_t instr_desc(uint32_t fmt, uint32_t b_mn,
-                                                  uint32_t n) {
+                                                  uint32_t n, uint32_t m = 128) {
   return (1u << 4) | (fmt << 7) | (fmt << 10) | (b_mn << 16) |
-         ((n >> 3) << 17) | ((128u >> 4) << 24);
+         ((n >> 3) << 17) | ((m >> 4) << 24);
 }
 
 }  // namespace ptx

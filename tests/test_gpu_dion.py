@@ -81,6 +81,22 @@ def test_dion_4096_rank256_20_steps(mode):
         assert e_m <= TOL_BF16 and e_q <= TOL_BF16 and e_w <= TOL_BF16, (step, errs)
 
 
+@pytest.mark.parametrize("mode", [odion.COLNORM, odion.QR])
+@pytest.mark.parametrize("shape,r,steps", [((1024, 768), 300, 3), ((1536, 1536), 512, 3)])
+def test_dion_wide_ranks(mode, shape, r, steps):
+    # ranks above 128 take the blocked multi-CTA Cholesky (r = 300 is not a
+    # multiple of its 32-wide blocks)
+    errs = _run(*shape, r, mode, steps=steps, seed=r)
+    for e_m, e_q, e_w in errs:
+        assert e_m <= TOL_BF16 and e_q <= TOL_BF16 and e_w <= TOL_BF16, errs
+
+
+def test_orth_dion_rank_1024():
+    errs = _run(2048, 2048, 1024, odion.QR, steps=2, seed=1024)
+    for e_m, e_q, e_w in errs:
+        assert e_m <= TOL_BF16 and e_q <= TOL_BF16 and e_w <= TOL_BF16, errs
+
+
 def test_dion_orthonormal_factors_and_isometry():
     # Orth-Dion's update is a partial isometry: singular values of the
     # applied update P Q^T all equal one (nu_t = 1).

@@ -186,7 +186,8 @@ def test_gram_contiguous_batch_output_over_input():
 @pytest.mark.parametrize("gram", [True, False])
 def test_single_cta_and_cta_pair_tiles_agree(gram, monkeypatch):
     # Matrices taller than 128 rows run on CTA-pair tiles (256 x 256) by
-    # default; OUO_CTA_PAIR=0 selects single-CTA 128 x 256 tiles.  Both must
+    # default (K-major B); OUO_CTA_PAIR=0 selects single-CTA 128 x 256 tiles,
+    # OUO_CTA_PAIR=2 puts the MN-major Q X products on pairs too.  All must
     # meet the oracle and agree with each other within half the bf16
     # tolerance.
     shapes = [(300, 1000), (512, 2048), (1792, 4096), (256, 256)]
@@ -194,7 +195,7 @@ def test_single_cta_and_cta_pair_tiles_agree(gram, monkeypatch):
     p = ouo.ns_params()
     fn = ouo.gram_ns_orthogonalize if gram else ouo.ns_orthogonalize
     outs = {}
-    for mode in ("1", "0"):
+    for mode in ("1", "0", "2"):
         monkeypatch.setenv("OUO_CTA_PAIR", mode)
         Os = [torch.empty_like(x) for x in Xs]
         fn(Xs, Os, p)
@@ -203,6 +204,7 @@ def test_single_cta_and_cta_pair_tiles_agree(gram, monkeypatch):
     for i, x in enumerate(Xs):
         if i < 2:
             ref = _oracle(to64(x), gram)
-            assert rel_fro(to64(outs["1"][i]), ref) <= TOL_BF16
-            assert rel_fro(to64(outs["0"][i]), ref) <= TOL_BF16
+            for mode in outs:
+                assert rel_fro(to64(outs[mode][i]), ref) <= TOL_BF16
         assert rel_fro(to64(outs["1"][i]), to64(outs["0"][i])) <= 1e-2
+        assert rel_fro(to64(outs["2"][i]), to64(outs["0"][i])) <= 1e-2
