@@ -53,6 +53,15 @@ def _args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-layers", type=int, default=1)
+    ap.add_argument("--micro", choices=["gram", "dion"], default=None,
+                    help="one kernel-level case for profiling: Gram NS on --nb blocks "
+                         "of --m x --n bf16, or one Dion / Orth-Dion matrix --m x --n "
+                         "at --rank (--mode colnorm|qr)")
+    ap.add_argument("--nb", type=int, default=32)
+    ap.add_argument("--m", type=int, default=1792)
+    ap.add_argument("--n", type=int, default=4096)
+    ap.add_argument("--rank", type=int, default=256)
+    ap.add_argument("--mode", choices=["colnorm", "qr"], default="qr")
     ap.add_argument("--sweep", action="store_true",
                     help="shape sweep instead of the step: standard vs Gram NS over "
                          "m in 512..8192, n/m in 1, 4, 16; Dion / Orth-Dion over rank "
@@ -580,8 +589,57 @@ def run_sweep(args):
                       "ns": ns_rows, "dion": dion_rows, "clocks": clocks}), flush=True)
 
 
+def run_micro(args):
+    """One kernel-level case (for ncu captures): W warm-up calls, then K
+    calls timed with CUDA events; prints one JSON line."""
+    import torch
+
+    import orthonormalized_update_optimizers_b200 as ouo
+    from orthonormalized_update_optimizers_b200 import synth
+
+    dev = torch.device("cuda", 0)
+    m, n = args.m, args.n
+    if args.micro == "gram":
+        X = [synth.lowrank_plus_noise(m, n, 64, 0.02, synth.seed_for(4, 500 + i),
+                                      torch.bfloat16, dev) for i in range(args.nb)]
+        O = [torch.empty_like(x) for x in X]
+        Xb, Ob = ouo.MatBatch(X), ouo.MatBatch(O)
+        p = ouo.ns_params()
+        ws = torch.empty(ouo.gram_ns_workspace_bytes(Xb, p), dtype=torch.uint8, device=dev)
+        fn = lambda: ouo.gram_ns_orthogonalize(Xb, Ob, p, workspace=ws)  # noqa: E731
+        flops = args.nb * sum(gram_ns_flops(m, n))
+        case = f"Gram NS, {args.nb} x bf16 {m}x{n}"
+    else:
+        r = args.rank
+        G = synth.lowrank_plus_noise(m, n, 64, 0.02, synth.seed_for(4, 7), torch.bfloat16, dev)
+        M = torch.zeros(m, n, dtype=torch.float32, device=dev)
+        W = torch.zeros(m, n, dtype=torch.bfloat16, device=dev)
+        Qt = torch.linalg.qr(synth.dion_q0(n, r, 1).to(dev))[0].T.contiguous()
+        p = ouo.dion_params(rank=r, norm_mode=args.mode)
+        ws = torch.empty(ouo.dion_workspace_bytes([M], p), dtype=torch.uint8, device=dev)
+        fn = lambda: ouo.dion_lowrank_step([M], [G], [Qt], [W], p, workspace=ws)  # noqa: E731
+        flops = 8 * m * n * r
+        case = f"{'Orth-Dion' if args.mode == 'qr' else 'Dion'} step, {m}x{n}, r={r}"
+    for _ in range(max(args.warmup, 1)):
+        fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    print(json.dumps({"mode": "micro", "case": case, "ms": round(ms, 4),
+                      "tflops": round(flops / ms / 1e9, 1), "steps": args.steps,
+                      "warmup": args.warmup}), flush=True)
+
+
 def main():
     args = _args()
+    if args.micro:
+        run_micro(args)
+        return
     if args.sweep:
         run_sweep(args)
         return

@@ -20,13 +20,14 @@
 // tcgen05 GEMM (tf32 operands, fp32 accumulation) with K-major A.  The
 // orthonormalization works on r x L row blocks X: S = X X^T in fp32 (split
 // over L, partial sums added in float64 in a fixed order), S = L L^T by a
-// one-CTA Cholesky (r <= 128) or the blocked cooperative Cholesky of chol.cu
+// one-CTA Cholesky (r <= 64) or the blocked cooperative Cholesky of chol.cu
 // (wider ranks), L inverted, X <- L^-1 X (rows orthonormal; the
 // implied R = L^T has a positive diagonal, the unique QR).  Two passes
 // (CholeskyQR2).  A failed pivot retries with the shift of shifted
 // CholeskyQR (11 (L r + r (r + 1)) u ||X||_F^2); a second failure sets
 // OUO_STATUS_BREAKDOWN.
 #include <cmath>
+#include <cstdlib>
 
 #include "internal.h"
 
@@ -86,7 +87,8 @@ __global__ void __launch_bounds__(256) gram_partial_kernel(const GramArgs a) {
 }
 
 // ---------------------------------------------------- Cholesky + inverse
-// One CTA, ranks up to 128 (larger ones use the blocked kernel in chol.cu).
+// One CTA, ranks up to 128 (by default up to 64; larger ones use the
+// blocked kernel in chol.cu).
 // S is summed from the partials in float64 (fixed order) and kept as a
 // packed lower triangle (fp32) in shared memory.
 // Cholesky S = L L^T in place, then L^-1 in place, then written as a full
@@ -294,9 +296,18 @@ struct DionWs {
   Buf ctl;      // barrier counter and flags of the blocked Cholesky
 };
 
-// Ranks above this use the blocked multi-CTA Cholesky; the one-CTA kernel
-// keeps smaller ones (their triangle fits in its shared memory).
-constexpr int kBlockedCholMinRank = 129;
+// Ranks from this one up use the blocked multi-CTA Cholesky; the one-CTA
+// kernel keeps smaller ones (measured on 4096 x 4096: equal at r = 64, the
+// blocked kernel 8-23% faster per Dion step from r = 96).
+// OUO_CHOL_BLOCKED_MIN_RANK overrides the threshold (1 to 129).
+int blocked_chol_min_rank() {
+  const char* env = getenv("OUO_CHOL_BLOCKED_MIN_RANK");
+  if (env) {
+    const int v = atoi(env);
+    if (v >= 1 && v <= 129) return v;
+  }
+  return 65;
+}
 int64_t padded_rank(int r) { return ceil_div(r, 32) * 32; }
 
 DionWs carve_dion(Arena& ar, int64_t m, int64_t n, int r) {
@@ -348,7 +359,7 @@ int orth_rows(Buf X, Buf tmp, Buf Y, const DionWs& w, cudaStream_t s,
     dim3 grid((unsigned)(ga.tiles * (ga.tiles + 1) / 2), (unsigned)used);
     gram_partial_kernel<<<grid, 256, 0, s>>>(ga);
     OUO_CHECK_LAUNCH();
-    if (r >= kBlockedCholMinRank) {
+    if (r >= blocked_chol_min_rank()) {
       OUO_TRY(chol_blocked(ga.part, used, r, L, reinterpret_cast<float*>(w.S.p),
                            reinterpret_cast<float*>(w.Linv.p), w.ctl.p, status, s));
     } else {

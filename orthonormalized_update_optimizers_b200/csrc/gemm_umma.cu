@@ -104,10 +104,13 @@ struct Cfg {
   static constexpr uint32_t kABytes = kTileM * kRowBytes;      // 16 KB
   static constexpr uint32_t kBBytes = kBRows * kRowBytes;      // 16/32 KB
   static constexpr uint32_t kStageBytes = kABytes + kBBytes;
-  static constexpr int kStages = CG == 2 ? 6 : (BN == 256 ? 4 : 6);
+  static constexpr int kStages = CG == 2 ? 5 : (BN == 256 ? 4 : 6);
+  // epilogue staging buffers per warp: two where shared memory allows, so a
+  // bulk store can still be reading one while the next chunk fills the other
+  static constexpr int kStg = CG == 2 ? 2 : 1;
   static constexpr uint32_t kTmemCols = 2 * BN;
   // per epilogue warp: a 32 x 32 fp32 staging buffer
-  static constexpr uint32_t kEpiBytes = kEpiWarps * 32 * 32 * 4;
+  static constexpr uint32_t kEpiBytes = kEpiWarps * kStg * 32 * 32 * 4;
   static constexpr size_t kSmem =
       1024 + (size_t)kStages * kStageBytes + 256 + kEpiBytes;
 };
@@ -455,6 +458,7 @@ umma_gemm_kernel(const __grid_constant__ UmmaArgs a) {
     int64_t local = 0;
     // accumulator-free barrier of the pair's even CTA (cluster address)
     const uint32_t tempty_lead = CG == 2 ? ptx::mapa(ptx::smem_u32(tempty), 0) : 0u;
+    uint32_t nstores = 0;  // bulk stores issued by this warp
     for (int64_t tile = tile0; tile < a.total_tiles;
          tile += tile_step, ++local) {
       int64_t b, ti, tj;
@@ -484,8 +488,22 @@ umma_gemm_kernel(const __grid_constant__ UmmaArgs a) {
         // diagonal is made symmetric in place and stored once.
         const int64_t row_base = ti * TR + rank * kTileM + q * 32;
         const int64_t gi = row_base + lane;
-        float* stg = epi_smem + (warp - 2) * (32 * 32);
+        float* const stg_base = epi_smem + (warp - 2) * (C::kStg * 32 * 32);
+        float* stg = stg_base;
         uint16_t* stg16 = reinterpret_cast<uint16_t*>(stg);
+        // Stores rotate over the warp's staging buffers; before a buffer is
+        // refilled, the store that last read it must have finished reading
+        // (with two buffers that is every store but the latest one).
+        auto next_stg = [&]() {
+          if (C::kStg == 2) {
+            if (lane == 0) ptx::bulk_wait_read1();
+            stg = stg_base + (nstores & 1u) * (32 * 32);
+          } else {
+            if (lane == 0) ptx::bulk_wait_read0();
+          }
+          stg16 = reinterpret_cast<uint16_t*>(stg);
+          __syncwarp();
+        };
         const uint32_t half = (uint32_t)((warp - 2) >> 2);
         const int32_t z = (int32_t)(sg.b0 + b);
         const bool obf = a.has_bf16 != 0;
@@ -531,9 +549,7 @@ umma_gemm_kernel(const __grid_constant__ UmmaArgs a) {
             for (int j = 0; j < 32; ++j) v[j] = round_tf32(v[j]);
           }
           const bool diag = a.tri && gj0 == row_base;
-          // the previous store from this buffer must have read it
-          if (lane == 0) ptx::bulk_wait_read0();
-          __syncwarp();
+          next_stg();
           if (!obf) {
 #pragma unroll
             for (int j = 0; j < 32; j += 4)
@@ -564,9 +580,9 @@ umma_gemm_kernel(const __grid_constant__ UmmaArgs a) {
             ptx::tma_store_3d(&sg.tmC, stg, (int32_t)gj0, (int32_t)row_base, z);
             ptx::bulk_commit();
           }
+          ++nstores;
           if (a.tri && !diag) {
-            if (lane == 0) ptx::bulk_wait_read0();
-            __syncwarp();
+            next_stg();
             if (!obf) {
 #pragma unroll
               for (int j = 0; j < 32; ++j) stg[stg_idx(j, lane)] = v[j];
@@ -580,6 +596,7 @@ umma_gemm_kernel(const __grid_constant__ UmmaArgs a) {
               ptx::tma_store_3d(&sg.tmC, stg, (int32_t)row_base, (int32_t)gj0, z);
               ptx::bulk_commit();
             }
+            ++nstores;
           }
         }
         ptx::tc_fence_before();
@@ -600,7 +617,7 @@ umma_gemm_kernel(const __grid_constant__ UmmaArgs a) {
       // are skipped; chunks fully inside and above it store without masks.
       const int64_t row_base = ti * TR + rank * kTileM + q * 32;
       const int64_t gi = row_base + lane;
-      float* stg = epi_smem + (warp - 2) * (32 * 32);
+      float* stg = epi_smem + (warp - 2) * (C::kStg * 32 * 32);
       const int sub_r = lane >> 3, sub_c = 4 * (lane & 7);
       const TileOut to = tile_out(a, sg, b);
       const uint32_t half = (uint32_t)((warp - 2) >> 2);
