@@ -171,9 +171,9 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": round(ms, 3),
         "unit": "ms", "n_gpus": args.gpus, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms, 3),
-        "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
+        "higher_is_better": False, "scaling": "strong", "vs_baseline": None,
         "dtype": "f64", "data": "synthetic",
-        "config": _config(args.layers),
+        "config": _config(args.layers, args.gpus),
         "cpu_baseline": line,
         "e2e": {"value": round(ms, 3), "unit": "ms", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
@@ -225,7 +225,7 @@ def cpu_baseline(args):
     return line
 
 
-def _config(layers):
+def _config(layers, world=1):
     shapes = _workload_shapes(layers)
     params = sum(m * n for _, m, n in shapes)
     return {"workload": f"Llama-3-8B-shaped optimizer step ({layers} layers, {len(shapes)} "
@@ -234,7 +234,10 @@ def _config(layers):
                         "spike, fp32 momentum, bf16 weights",
             "params": params, "matrices": len(shapes), "rho": RHO, "mu": MU,
             "l2": "inputs larger than L2 (about 56 GB resident per step)",
-            "parallelism": "replicas (one independent step per GPU)"}
+            "parallelism": "single GPU" if world == 1 else
+                           f"dp{world}: per-matrix partition of the step across {world} GPUs, "
+                           "NCCL all-gather of the kept-row updates, every rank updates "
+                           "all weights"}
 
 
 # ----------------------------------------------------------------------- ours
@@ -290,7 +293,7 @@ def run_ours(args):
     import numpy as np
     import torch
     import orthonormalized_update_optimizers_b200 as ouo
-    from orthonormalized_update_optimizers_b200 import synth
+    from orthonormalized_update_optimizers_b200 import shard, synth
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -304,33 +307,54 @@ def run_ours(args):
     dev = torch.device("cuda", local)
 
     shapes = _workload_shapes(args.layers)
-    Gs, Ms, Ws = [], [], []
-    for i, (_, m, n) in enumerate(shapes):
+    mn = [(m, n) for _, m, n in shapes]
+    # Per-matrix partition: this rank steps its own matrices, the kept-row
+    # updates are all-gathered, every rank updates all its weights.  With one
+    # rank the plan is everything and the exchange is nothing.
+    parts = shard.plan_partition(mn, world, RHO)
+    own = parts[rank]
+    lay = shard.ExchangeLayout(mn, parts, RHO)
+    Gs, Ms = [], []
+    for i in own:
+        m, n = mn[i]
         Gs.append(synth.lowrank_plus_noise(m, n, 32, 0.01, synth.seed_for(3, i),
                                            torch.bfloat16, dev))
         Ms.append(torch.zeros(m, n, dtype=torch.float32, device=dev))
-        Ws.append(synth.gaussian((m, n), synth.seed_for(3, 1000 + i), 0.02,
-                                 torch.bfloat16, dev))
-    ks = [ouo.dion3_num_selected(m, RHO) for _, m, _ in shapes]
-    keys = torch.empty(sum(m for _, m, _ in shapes), dtype=torch.float64, device=dev)
-    idx = torch.empty(sum(ks), dtype=torch.int32, device=dev)
-    kn = [(k, n) for k, (_, _, n) in zip(ks, shapes)]
+    Ws = [synth.gaussian((m, n), synth.seed_for(3, 1000 + i), 0.02, torch.bfloat16, dev)
+          for i, (m, n) in enumerate(mn)]
+    ks = [lay.k[i] for i in own]
+    assert ks == [ouo.dion3_num_selected(mn[i][0], RHO) for i in own]
+    keys = torch.empty(max(1, sum(mn[i][0] for i in own)), dtype=torch.float64, device=dev)
+    payload = torch.empty(max(1, lay.payload_bytes), dtype=torch.uint8, device=dev)
+    gathered = payload if world == 1 else torch.empty(world * lay.payload_bytes,
+                                                      dtype=torch.uint8, device=dev)
+    idx, O = lay.views(payload, rank)  # selection and Gram NS write the payload
+    kn = [(k, mn[i][1]) for k, i in zip(ks, own)]
     X0 = ouo.batch_empty(kn, torch.bfloat16, dev)
-    O = ouo.batch_empty(kn, torch.bfloat16, dev)
-    scale = torch.empty(len(shapes), dtype=torch.float32, device=dev)
+    scale = torch.empty(max(1, len(own)), dtype=torch.float32, device=dev)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
-    Mb, Gb, Wb = ouo.MatBatch(Ms), ouo.MatBatch(Gs), ouo.MatBatch(Ws)
+    Mb, Gb = ouo.MatBatch(Ms), ouo.MatBatch(Gs)
     Xb, Ob = ouo.MatBatch(X0), ouo.MatBatch(O)
     params = ouo.ns_params(iters=ITERS, restart_after=RESTART_AFTER, normalize=False)
-    ws = torch.empty(ouo.gram_ns_workspace_bytes(Xb, params), dtype=torch.uint8, device=dev)
+    ws = torch.empty(max(1, ouo.gram_ns_workspace_bytes(Xb, params) if own else 1),
+                     dtype=torch.uint8, device=dev)
     # Muon-style per-matrix update scale sqrt(max(1, rows / cols))
-    scales = [math.sqrt(max(1.0, m / n)) for _, m, n in shapes]
+    scales = [math.sqrt(max(1.0, m / n)) for m, n in mn]
+    # one weight-update call per source rank, on its segment of the exchange
+    segs = []
+    for r, (gidx, gO) in enumerate(lay.gathered_views(gathered)):
+        if parts[r]:
+            segs.append((ouo.MatBatch([Ws[i] for i in parts[r]]), ouo.MatBatch(gO), gidx,
+                         [scales[i] for i in parts[r]]))
 
     def step():
-        ouo.dion_momentum_update(Mb, Gb, MU, "accum", keys)
-        ouo.dion3_select_rows(Mb, keys, RHO, idx, Xb, scale, ef=True, mu=MU)
-        ouo.gram_ns_orthogonalize(Xb, Ob, params, workspace=ws, status=status)
-        ouo.apply_update(Wb, Ob, LR, idx=idx, scale=scales)
+        if own:
+            ouo.dion_momentum_update(Mb, Gb, MU, "accum", keys)
+            ouo.dion3_select_rows(Mb, keys, RHO, idx, Xb, scale, ef=True, mu=MU)
+            ouo.gram_ns_orthogonalize(Xb, Ob, params, workspace=ws, status=status)
+        shard.all_gather_payload(payload, gathered)
+        for Wb_r, Ob_r, idx_r, sc_r in segs:
+            ouo.apply_update(Wb_r, Ob_r, LR, idx=idx_r, scale=sc_r)
 
     def barrier():
         torch.cuda.synchronize()
@@ -364,7 +388,8 @@ def run_ours(args):
     g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     g0.record()
     for _ in range(args.steps):
-        ouo.gram_ns_orthogonalize(Xb, Ob, params, workspace=ws, status=status)
+        if own:
+            ouo.gram_ns_orthogonalize(Xb, Ob, params, workspace=ws, status=status)
     g1.record()
     barrier()
     gram_ms = max_over_ranks(g0.elapsed_time(g1) / args.steps)
@@ -372,7 +397,8 @@ def run_ours(args):
     m0, m1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     m0.record()
     for _ in range(args.steps):
-        ouo.dion_momentum_update(Mb, Gb, MU, "accum", keys)
+        if own:
+            ouo.dion_momentum_update(Mb, Gb, MU, "accum", keys)
     m1.record()
     barrier()
     mom_ms = max_over_ranks(m0.elapsed_time(m1) / args.steps)
@@ -395,9 +421,11 @@ def run_ours(args):
     st = int(status.item())
 
     peaks = _peaks()
+    # Gram-NS flops of the whole job (all ranks' matrices) over the slowest
+    # rank's Gram-NS time
     bf = tf = 0
-    for k, (_, m, n) in zip(ks, shapes):
-        b_, t_ = gram_ns_flops(k, n)
+    for i, (m, n) in enumerate(mn):
+        b_, t_ = gram_ns_flops(lay.k[i], n)
         bf += b_
         tf += t_
     flops = bf + tf
@@ -406,11 +434,12 @@ def run_ours(args):
     p_bf = peaks["bf16_tflops"]
     p_tf = p_bf * TF32_RATIO
     peak_eff = flops / (bf / p_bf + tf / p_tf)
-    elems = sum(m * n for _, m, n in shapes)
-    rows = keys.numel()
+    # momentum kernel of this rank (its own matrices)
+    elems = sum(mn[i][0] * mn[i][1] for i in own)
+    rows = sum(mn[i][0] for i in own)
     mom_bytes = elems * (4 + 2 + 4) + rows * 8   # read M, G; write M; write keys
-    mom_gbs = mom_bytes / (mom_ms * 1e-3) / 1e9
-    mom_launches = -(-len(shapes) // 128)
+    mom_gbs = mom_bytes / (mom_ms * 1e-3) / 1e9 if mom_ms > 0 else 0.0
+    mom_launches = -(-len(own) // 128)
     # The dominant kernel of the step by device time: a GEMM kind or the
     # momentum kernel.  Kernels timed inside full steps use the sustained
     # dense-bf16 peak (tf32 at the nominal tf32/bf16 ratio).
@@ -440,8 +469,8 @@ def run_ours(args):
     result = {
         "metric": METRIC, "value": round(ms, 4), "unit": "ms", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
-        "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
-        "dtype": "bf16", "data": "synthetic", "config": _config(args.layers),
+        "higher_is_better": False, "scaling": "strong", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic", "config": _config(args.layers, world),
         "gram_ns": {"ms": round(gram_ms, 4), "tflops": round(tflops, 2),
                     "frac_of_peak": round(tflops / peak_eff, 4),
                     "peak_tflops": round(peak_eff, 1),
