@@ -217,3 +217,42 @@ def test_shape_sweep_large_gram_equals_standard(shape):
     assert 0.3 <= ms <= 1.2024 ** 2
     del X, Os, Og
     torch.cuda.empty_cache()
+
+
+def test_chunked_step_equals_whole_step_bitwise():
+    # A matrix's result does not depend on the batch it is stepped in: two
+    # layers stepped as one batch, and as two one-layer chunks through views
+    # of the same row-key / index / X0 / O buffers (the end-to-end schedule of
+    # the benchmark), give bit-identical momentum, indices, O and weights.
+    shapes = synth.llama8b_shapes(2)
+    mn = [(m, n) for _, m, n in shapes]
+    ks = [ouo.dion3_num_selected(m, RHO) for m, _ in mn]
+    res = []
+    for chunked in (False, True):
+        G = [synth.lowrank_plus_noise(m, n, 32, 0.01, synth.seed_for(3, i), torch.bfloat16, DEV)
+             for i, (m, n) in enumerate(mn)]
+        M = [torch.zeros(m, n, device=DEV) for m, n in mn]
+        W = [synth.gaussian((m, n), synth.seed_for(3, 1000 + i), 0.02, torch.bfloat16, DEV)
+             for i, (m, n) in enumerate(mn)]
+        keys = torch.empty(sum(m for m, _ in mn), dtype=torch.float64, device=DEV)
+        idx = torch.empty(sum(ks), dtype=torch.int32, device=DEV)
+        sc = torch.empty(len(mn), dtype=torch.float32, device=DEV)
+        kn = [(k, n) for k, (_, n) in zip(ks, mn)]
+        X0 = ouo.batch_empty(kn, torch.bfloat16, DEV)
+        O = ouo.batch_empty(kn, torch.bfloat16, DEV)
+        p = ouo.ns_params(normalize=False)
+        spans = [(0, 7), (7, 14)] if chunked else [(0, 14)]
+        kp = np.concatenate([[0], np.cumsum(ks)]).astype(int)
+        rp = np.concatenate([[0], np.cumsum([m for m, _ in mn])]).astype(int)
+        for a, b in spans:
+            ouo.dion_momentum_update(M[a:b], G[a:b], MU, "accum", keys[rp[a]:rp[b]])
+            ouo.dion3_select_rows(M[a:b], keys[rp[a]:rp[b]], RHO, idx[kp[a]:kp[b]], X0[a:b],
+                                  sc[a:b], ef=True, mu=MU)
+            ouo.gram_ns_orthogonalize(X0[a:b], O[a:b], p)
+        ouo.apply_update(W, O, LR, idx=idx, scale=[1.0] * len(mn))
+        torch.cuda.synchronize()
+        res.append((M, W, idx.clone(), O))
+    (M1, W1, i1, O1), (M2, W2, i2, O2) = res
+    assert torch.equal(i1, i2)
+    for a, b in zip(M1 + W1 + O1, M2 + W2 + O2):
+        assert torch.equal(a, b)
