@@ -116,7 +116,8 @@ typedef struct ouo_ns_params {
 /* Dion / Orth-Dion parameters.  ouo_dion_default(): rank 256, mu 0.95,
  * beta 1, lr 0.01, wd 0, COLNORM, eps 1e-8. */
 typedef struct ouo_dion_params {
-  int rank;            /* r, 1 <= r <= min(rows, cols)                       */
+  int rank;            /* r, 1 <= r <= min(rows, cols); 0 = per matrix, from
+                          Q_state[i].rows (ragged ranks)                      */
   float mu;            /* momentum / error-feedback factor                    */
   float beta;          /* error-feedback coefficient (1 = Dion's buffer)      */
   float lr;            /* learning rate                                       */
@@ -305,6 +306,43 @@ int dion_lowrank_step(const ouo_mat* M, const ouo_mat* G, int g_dtype,
                       int nmat, const ouo_dion_params* p, const float* scale,
                       void* ws, size_t ws_bytes, int* dev_status,
                       void* stream);
+
+/*
+ * Per-matrix working ranks ([OD] Ada-Orth-Dion: the working rank of every
+ * layer is adjusted to its gradient spectrum).
+ *
+ * Ragged ranks: with p->rank == 0, dion_lowrank_step and
+ * dion_lowrank_step_stats give matrix i the rank r_i = Q_state[i].rows
+ * (1 <= r_i <= min(rows, cols)); a nonzero p->rank must equal every
+ * Q_state[i].rows as before.  dion_workspace_bytes_ranks sizes the
+ * workspace for per-matrix ranks (ranks: host int[nmat]); it returns 0 for
+ * invalid arguments.
+ *
+ * dion_lowrank_step_stats -- dion_lowrank_step that also writes, for every
+ * matrix, the Euclidean norms of the r_i rows of R^T = P^T B (the columns of
+ * R: the power iteration's estimates of B's leading singular values) to
+ * sigma, a device float array of sum_i r_i values, matrix i's after those
+ * of the matrices before it.  sigma == NULL is dion_lowrank_step.
+ *
+ * dion_effective_rank -- per matrix, exp(-sum_j p_j ln p_j) with
+ * p_j = sigma_j^2 / sum_k sigma_k^2: the exponential of the Shannon entropy of
+ * the energy the rank-r_i factors capture, between 1 (one direction holds
+ * all of it) and r_i (evenly spread).  The pages name "a lightweight
+ * entropy-based estimator derived from the power iteration factors" without
+ * defining it; this is that reading (the effective rank of the estimated
+ * spectrum).  sigma: device float[sum r_i] laid out as above; ranks: host
+ * int[nmat]; erank: device float[nmat]; all-zero sigma gives 0.  Float64
+ * sums in a fixed order.  Asynchronous on `stream`.
+ */
+size_t dion_workspace_bytes_ranks(const ouo_mat* M, const int* ranks, int nmat,
+                                  const ouo_dion_params* p);
+int dion_lowrank_step_stats(const ouo_mat* M, const ouo_mat* G, int g_dtype,
+                            const ouo_mat* Q_state, const ouo_mat* W,
+                            int w_dtype, int nmat, const ouo_dion_params* p,
+                            const float* scale, void* ws, size_t ws_bytes,
+                            float* sigma, int* dev_status, void* stream);
+int dion_effective_rank(const float* sigma, const int* ranks, int nmat,
+                        float* erank, void* stream);
 
 #ifdef __cplusplus
 }

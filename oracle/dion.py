@@ -27,6 +27,15 @@ Step (one matrix; readings listed in the design notes):
 
 ColNorm(R)_j = R_j / (||R_j||_2 + eps), eps = 1e-8.
 
+Ada-Orth-Dion ("Ada-Orth-Dion": the working rank of each layer follows an
+entropy-based estimate of its intrinsic dimensionality, derived from the
+power-iteration factors; the pages do not define the estimator).  Reading:
+sigma_j = ||R_j||_2, the power iteration's estimates of B's leading singular
+values, and the estimate is the effective rank exp(H(p)),
+p_j = sigma_j^2 / sum_k sigma_k^2, H the Shannon entropy.  Parity of this
+estimator against the method is unpinned (the pages give no formula); the
+function itself is pinned by its closed forms.
+
 TEST INFRASTRUCTURE: see the package docstring.
 """
 from __future__ import annotations
@@ -120,4 +129,15 @@ def dion_step(M, G, Q_prev, W, mu: float, lr: float, scale: float,
     O = P @ Q_new.T
     W_new = _apply.apply_update(W, O, None, lr, scale, wd)
     return {"M": M_new, "Q": Q_new, "W": W_new, "B": B, "P": P, "R": R,
-            "O": O}
+            "O": O, "sigma": np.linalg.norm(R, axis=0)}
+
+
+def effective_rank(sigma) -> float:
+    """exp(-sum_j p_j ln p_j), p_j = sigma_j^2 / sum_k sigma_k^2 (terms with
+    p_j = 0 contribute 0); 0 when every sigma_j is 0."""
+    s2 = np.asarray(sigma, dtype=np.float64) ** 2
+    tot = s2.sum()
+    if tot <= 0.0:
+        return 0.0
+    p = s2[s2 > 0] / tot
+    return float(np.exp(-np.sum(p * np.log(p))))

@@ -36,7 +36,8 @@ EXPORTED = (
     "dion_momentum_update", "dion3_num_selected", "dion3_select_rows",
     "ns_workspace_bytes", "ns_orthogonalize", "gram_ns_workspace_bytes",
     "gram_ns_orthogonalize", "gram_ns_orthogonalize_noalloc", "apply_update",
-    "dion_workspace_bytes", "dion_lowrank_step",
+    "dion_workspace_bytes", "dion_lowrank_step", "dion_workspace_bytes_ranks",
+    "dion_lowrank_step_stats", "dion_effective_rank",
 )
 
 
@@ -102,6 +103,10 @@ _PROTOS = {
     "dion_workspace_bytes": (_SZ, [_MP, _I, _DP]),
     "dion_lowrank_step": (_I, [_MP, _MP, _I, _MP, _MP, _I, _I, _DP, _P, _P, _SZ,
                                _P, _P]),
+    "dion_workspace_bytes_ranks": (_SZ, [_MP, _P, _I, _DP]),
+    "dion_lowrank_step_stats": (_I, [_MP, _MP, _I, _MP, _MP, _I, _I, _DP, _P, _P, _SZ,
+                                     _P, _P, _P]),
+    "dion_effective_rank": (_I, [_P, _P, _I, _P, _P]),
 }
 
 

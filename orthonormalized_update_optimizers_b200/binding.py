@@ -21,7 +21,8 @@ __all__ = [
     "dion3_num_selected", "dion3_select_rows", "ns_workspace_bytes",
     "ns_orthogonalize", "gram_ns_workspace_bytes", "gram_ns_orthogonalize",
     "gram_ns_orthogonalize_noalloc",
-    "apply_update", "dion_workspace_bytes", "dion_lowrank_step", "version",
+    "apply_update", "dion_workspace_bytes", "dion_lowrank_step", "dion_effective_rank",
+    "version",
     "launch_count", "timing_enable", "timing_read", "batch_empty",
 ]
 
@@ -247,20 +248,58 @@ def apply_update(W, O, lr: float, idx: Optional[torch.Tensor] = None,
         _stream(stream)))
 
 
-def dion_workspace_bytes(M, params) -> int:
+def _ranks(Mb, Qb, params):
+    """Per-matrix ranks: params.rank, or each Q_state's row count when
+    params.rank == 0 (ragged ranks)."""
+    if params.rank:
+        return [int(params.rank)] * Mb.n
+    if Qb is None:
+        raise ValueError("ragged ranks (rank=0) need the Q_state batch")
+    return [int(t.shape[0]) for t in Qb.tensors]
+
+
+def dion_workspace_bytes(M, params, Q_state=None) -> int:
+    """Workspace bytes of dion_lowrank_step; with params.rank == 0 the ranks
+    come from the Q_state batch (one rank per matrix)."""
     Mb = _batch(M)
-    return int(L.lib().dion_workspace_bytes(Mb.arr, Mb.n, ctypes.byref(params)))
+    if params.rank:
+        return int(L.lib().dion_workspace_bytes(Mb.arr, Mb.n, ctypes.byref(params)))
+    Qb = _batch(Q_state) if Q_state is not None else None
+    rk = (ctypes.c_int * max(Mb.n, 1))(*_ranks(Mb, Qb, params))
+    return int(L.lib().dion_workspace_bytes_ranks(Mb.arr, rk, Mb.n, ctypes.byref(params)))
 
 
 def dion_lowrank_step(M, G, Q_state, W, params, scale=None, workspace=None,
-                      status=None, stream=None) -> None:
+                      status=None, stream=None, sigma: Optional[torch.Tensor] = None) -> None:
+    """One Dion / Orth-Dion step per matrix.  params.rank == 0 takes each
+    matrix's rank from its Q_state rows.  With `sigma` (a float32 CUDA
+    tensor of sum(ranks) elements) the step also writes the norms of R's
+    columns, matrix after matrix."""
     Mb, Gb, Qb, Wb = _batch(M), _batch(G), _batch(Q_state), _batch(W)
-    need = L.lib().dion_workspace_bytes(Mb.arr, Mb.n, ctypes.byref(params))
+    need = dion_workspace_bytes(Mb, params, Qb)
     ws = _workspace(need, Mb.device, workspace)
     sc = None
     if scale is not None:
         sc = (ctypes.c_float * Mb.n)(*[float(s) for s in scale])
-    L.check("dion_lowrank_step", L.lib().dion_lowrank_step(
+    if sigma is not None:
+        if sigma.dtype != torch.float32 or not sigma.is_cuda:
+            raise TypeError("sigma must be a float32 CUDA tensor")
+        if sigma.numel() < sum(_ranks(Mb, Qb, params)):
+            raise ValueError("sigma needs sum(ranks) elements")
+    L.check("dion_lowrank_step", L.lib().dion_lowrank_step_stats(
         Mb.arr, Gb.arr, Gb.dtype, Qb.arr, Wb.arr, Wb.dtype, Mb.n,
         ctypes.byref(params), sc, ctypes.c_void_p(ws.data_ptr()), ws.numel(),
-        _ptr(status), _stream(stream)))
+        _ptr(sigma), _ptr(status), _stream(stream)))
+
+
+def dion_effective_rank(sigma: torch.Tensor, ranks: Sequence[int],
+                        erank: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Per matrix exp(Shannon entropy of sigma_j^2 / sum sigma^2), from the
+    sigma that dion_lowrank_step writes; returns a float32 CUDA tensor."""
+    n = len(ranks)
+    if erank is None:
+        erank = torch.empty(max(n, 1), dtype=torch.float32, device=sigma.device)
+    rk = (ctypes.c_int * max(n, 1))(*[int(r) for r in ranks])
+    L.check("dion_effective_rank", L.lib().dion_effective_rank(
+        _ptr(sigma), rk, n, _ptr(erank), _stream(stream)))
+    return erank

@@ -237,6 +237,63 @@ rownorm_kernel(const float* R, int64_t ldr, float* Q, int64_t ldq, int64_t n,
   for (int64_t j = threadIdx.x; j < n; j += blockDim.x) Q[c * ldq + j] = row[j] * inv;
 }
 
+// sigma[c] = ||R[c][:]||_2 (float64 sum of squares in a fixed order).
+__global__ void __launch_bounds__(256)
+rownorm_only_kernel(const float* R, int64_t ldr, int64_t n, float* sigma) {
+  __shared__ double part[8];
+  const int64_t c = blockIdx.x;
+  const float* row = R + c * ldr;
+  double acc = 0.0;
+  for (int64_t j = threadIdx.x; j < n; j += blockDim.x) acc += (double)row[j] * row[j];
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = acc;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double tot = 0.0;
+    for (int w = 0; w < 8; ++w) tot += part[w];
+    sigma[c] = (float)sqrt(tot);
+  }
+}
+
+// One block per matrix: exp(-sum p ln p), p_j = sigma_j^2 / sum sigma^2.
+struct ERankArgs {
+  const float* sigma;
+  int64_t off[kChunk + 1];
+  float* erank;
+};
+
+__global__ void __launch_bounds__(256) erank_kernel(const ERankArgs a) {
+  __shared__ double red[256];
+  const int i = blockIdx.x;
+  const float* s = a.sigma + a.off[i];
+  const int64_t r = a.off[i + 1] - a.off[i];
+  double e = 0.0;
+  for (int64_t j = threadIdx.x; j < r; j += blockDim.x) e += (double)s[j] * s[j];
+  red[threadIdx.x] = e;
+  __syncthreads();
+  for (int w = 128; w > 0; w >>= 1) {
+    if (threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
+    __syncthreads();
+  }
+  const double tot = red[0];
+  __syncthreads();
+  double h = 0.0;
+  if (tot > 0.0) {
+    for (int64_t j = threadIdx.x; j < r; j += blockDim.x) {
+      const double pj = (double)s[j] * s[j] / tot;
+      if (pj > 0.0) h -= pj * log(pj);
+    }
+  }
+  red[threadIdx.x] = h;
+  __syncthreads();
+  for (int w = 128; w > 0; w >>= 1) {
+    if (threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) a.erank[i] = tot > 0.0 ? (float)exp(red[0]) : 0.f;
+}
+
 // --------------------------------------------------------------- helpers
 __global__ void transpose_kernel(const float* src, int64_t lds, float* dst,
                                  int64_t ldd, int64_t rows, int64_t cols) {
@@ -399,9 +456,9 @@ int validate_dion(const ouo_dion_params* p) {
   return OUO_OK;
 }
 
-size_t dion_plan_bytes(const ouo_mat* M, int nmat, const ouo_dion_params* p) {
+size_t dion_plan_bytes(const ouo_mat* M, int nmat, const int* ranks) {
   Arena ar{nullptr, 0, 0, true};
-  for (int i = 0; i < nmat; ++i) carve_dion(ar, M[i].rows, M[i].cols, p->rank);
+  for (int i = 0; i < nmat; ++i) carve_dion(ar, M[i].rows, M[i].cols, ranks[i]);
   return ar.used + 256;
 }
 
@@ -410,8 +467,17 @@ size_t dion_plan_bytes(const ouo_mat* M, int nmat, const ouo_dion_params* p) {
 
 extern "C" size_t dion_workspace_bytes(const ouo_mat* M, int nmat,
                                        const ouo_dion_params* p) {
-  if (!M || !p || nmat <= 0 || p->rank < 1) return 0;
-  return ouo::dion_plan_bytes(M, nmat, p);
+  if (!M || !p || nmat <= 0 || nmat > OUO_MAX_BATCH || p->rank < 1) return 0;
+  std::vector<int> ranks((size_t)nmat, p->rank);
+  return ouo::dion_plan_bytes(M, nmat, ranks.data());
+}
+
+extern "C" size_t dion_workspace_bytes_ranks(const ouo_mat* M, const int* ranks,
+                                             int nmat, const ouo_dion_params* p) {
+  if (!M || !ranks || !p || nmat <= 0 || nmat > OUO_MAX_BATCH) return 0;
+  for (int i = 0; i < nmat; ++i)
+    if (ranks[i] < 1) return 0;
+  return ouo::dion_plan_bytes(M, nmat, ranks);
 }
 
 extern "C" int dion_lowrank_step(const ouo_mat* M, const ouo_mat* G,
@@ -420,6 +486,16 @@ extern "C" int dion_lowrank_step(const ouo_mat* M, const ouo_mat* G,
                                  const ouo_dion_params* p, const float* scale,
                                  void* ws, size_t ws_bytes, int* dev_status,
                                  void* stream) {
+  return dion_lowrank_step_stats(M, G, g_dtype, Q_state, W, w_dtype, nmat, p, scale,
+                                 ws, ws_bytes, nullptr, dev_status, stream);
+}
+
+extern "C" int dion_lowrank_step_stats(const ouo_mat* M, const ouo_mat* G,
+                                       int g_dtype, const ouo_mat* Q_state,
+                                       const ouo_mat* W, int w_dtype, int nmat,
+                                       const ouo_dion_params* p, const float* scale,
+                                       void* ws, size_t ws_bytes, float* sigma,
+                                       int* dev_status, void* stream) {
   using namespace ouo;
   clear_error();
   if (nmat < 0 || nmat > OUO_MAX_BATCH)
@@ -432,8 +508,12 @@ extern "C" int dion_lowrank_step(const ouo_mat* M, const ouo_mat* G,
   OUO_TRY(validate_mats(W, nmat, w_dtype, "W"));
   OUO_TRY(validate_same_shapes(M, G, nmat, "M", "G"));
   OUO_TRY(validate_same_shapes(M, W, nmat, "M", "W"));
-  const int r = p->rank;
+  if (p->rank < 0) return set_error(OUO_ERR_INVALID_ARG, "rank %d < 0", p->rank);
+  // per-matrix ranks: p->rank, or Q_state[i].rows when p->rank == 0
+  std::vector<int> ranks((size_t)nmat);
   for (int i = 0; i < nmat; ++i) {
+    const int r = p->rank ? p->rank : (int)Q_state[i].rows;
+    ranks[i] = r;
     if (r < 1 || r > M[i].rows || r > M[i].cols)
       return set_error(OUO_ERR_INVALID_ARG, "rank %d outside [1, min(rows, cols)] for M[%d]",
                        r, i);
@@ -448,7 +528,9 @@ extern "C" int dion_lowrank_step(const ouo_mat* M, const ouo_mat* G,
   }
   if (dev_status && ((uintptr_t)dev_status % 4))
     return set_error(OUO_ERR_INVALID_ARG, "dev_status misaligned");
-  const size_t need = dion_plan_bytes(M, nmat, p);
+  if (sigma && ((uintptr_t)sigma % 4))
+    return set_error(OUO_ERR_INVALID_ARG, "sigma misaligned");
+  const size_t need = dion_plan_bytes(M, nmat, ranks.data());
   if (!ws || ws_bytes < need)
     return set_error(OUO_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given",
                      need, ws_bytes);
@@ -461,8 +543,10 @@ extern "C" int dion_lowrank_step(const ouo_mat* M, const ouo_mat* G,
                                nullptr, stream));
   Arena ar{reinterpret_cast<char*>(ws), ws_bytes, 0, false};
   const float mu = p->mu, beta = p->beta;
+  int64_t sig_off = 0;
   for (int i = 0; i < nmat; ++i) {
     const int64_t m = M[i].rows, n = M[i].cols;
+    const int r = ranks[i];
     DionWs w = carve_dion(ar, m, n, r);
     const Buf Bm = caller_buf(M[i], OUO_F32);
     const Buf Qt = caller_buf(Q_state[i], OUO_F32);
@@ -489,6 +573,13 @@ extern "C" int dion_lowrank_step(const ouo_mat* M, const ouo_mat* G,
       d.has_f32 = true;
       OUO_TRY(gemm_umma(d, s, dev_status));
     }
+    // the power iteration's singular-value estimates: ||rows of Rt||
+    if (sigma) {
+      rownorm_only_kernel<<<r, 256, 0, s>>>(reinterpret_cast<const float*>(w.Ra.p), w.Ra.ld,
+                                            n, sigma + sig_off);
+      OUO_CHECK_LAUNCH();
+    }
+    sig_off += r;
     // P = Pt^T (m x r), the K-major left operand of the updates
     {
       dim3 grid((unsigned)ceil_div(m, 32), (unsigned)ceil_div(r, 32));
@@ -544,6 +635,36 @@ extern "C" int dion_lowrank_step(const ouo_mat* M, const ouo_mat* G,
         reinterpret_cast<const float*>(Qn.p), Qn.ld,
         reinterpret_cast<float*>(Q_state[i].ptr), Q_state[i].ld, r, n);
     OUO_CHECK_LAUNCH();
+  }
+  return OUO_OK;
+}
+
+extern "C" int dion_effective_rank(const float* sigma, const int* ranks, int nmat,
+                                   float* erank, void* stream) {
+  using namespace ouo;
+  clear_error();
+  if (nmat < 0 || nmat > OUO_MAX_BATCH)
+    return set_error(OUO_ERR_INVALID_ARG, "nmat %d out of range", nmat);
+  if (nmat == 0) return OUO_OK;
+  if (!sigma || !ranks || !erank)
+    return set_error(OUO_ERR_INVALID_ARG, "NULL sigma, ranks or erank");
+  if ((uintptr_t)sigma % 4 || (uintptr_t)erank % 4)
+    return set_error(OUO_ERR_INVALID_ARG, "sigma / erank misaligned");
+  for (int i = 0; i < nmat; ++i)
+    if (ranks[i] < 1) return set_error(OUO_ERR_INVALID_ARG, "ranks[%d] < 1", i);
+  OUO_TRY(require_sm100());
+  cudaStream_t s = (cudaStream_t)stream;
+  int64_t base = 0;
+  for (int c0 = 0; c0 < nmat; c0 += kChunk) {
+    const int cn = nmat - c0 < kChunk ? nmat - c0 : kChunk;
+    ERankArgs a;
+    a.sigma = sigma + base;
+    a.erank = erank + c0;
+    a.off[0] = 0;
+    for (int i = 0; i < cn; ++i) a.off[i + 1] = a.off[i] + ranks[c0 + i];
+    erank_kernel<<<cn, 256, 0, s>>>(a);
+    OUO_CHECK_LAUNCH();
+    base += a.off[cn];
   }
   return OUO_OK;
 }

@@ -112,3 +112,80 @@ def test_dion_orthonormal_factors_and_isometry():
     assert np.max(np.abs(q @ q.T - np.eye(r))) <= 1e-4
     sv = np.linalg.svd(-to64(W), compute_uv=False)
     assert np.max(np.abs(sv[:r] - 1.0)) <= 1e-3 and np.max(sv[r:]) <= 1e-3
+
+
+# ---- per-matrix working ranks (Ada-Orth-Dion) ----------------------------
+def _state(shapes, ranks, seed=0):
+    G = [synth.lowrank_plus_noise(m, n, min(64, m, n), 0.02, seed + i, torch.bfloat16, DEV)
+         for i, (m, n) in enumerate(shapes)]
+    W = [synth.gaussian((m, n), seed + 50 + i, 0.02, torch.float32, DEV)
+         for i, (m, n) in enumerate(shapes)]
+    Q = [torch.tensor(_q0(n, r, seed + 100 + i).T.copy(), device=DEV)
+         for i, ((m, n), r) in enumerate(zip(shapes, ranks))]
+    M = [torch.zeros(m, n, device=DEV) for m, n in shapes]
+    return M, G, Q, W
+
+
+@pytest.mark.parametrize("mode", ["colnorm", "qr"])
+def test_ragged_ranks_equal_separate_calls(mode):
+    # rank 0 = every matrix's rank from its Q_state rows; one ragged call must
+    # give, bit for bit, what one call per matrix gives (ranks on both sides
+    # of the one-CTA / blocked Cholesky threshold)
+    shapes = [(256, 384), (512, 256), (300, 700), (640, 512)]
+    ranks = [16, 48, 96, 300]
+    M1, G, Q1, W1 = _state(shapes, ranks)
+    M2, _, Q2, W2 = _state(shapes, ranks)
+    sig1 = torch.empty(sum(ranks), device=DEV)
+    sig2 = torch.empty(sum(ranks), device=DEV)
+    p0 = ouo.dion_params(rank=0, norm_mode=mode)
+    st = torch.zeros(1, dtype=torch.int32, device=DEV)
+    for _ in range(2):
+        ouo.dion_lowrank_step(M1, G, Q1, W1, p0, scale=[1.0, 2.0, 1.0, 0.5], status=st, sigma=sig1)
+        off = 0
+        for i, r in enumerate(ranks):
+            pi = ouo.dion_params(rank=r, norm_mode=mode)
+            ouo.dion_lowrank_step([M2[i]], [G[i]], [Q2[i]], [W2[i]], pi,
+                                  scale=[[1.0, 2.0, 1.0, 0.5][i]], status=st,
+                                  sigma=sig2[off:off + r])
+            off += r
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    for a, b in zip(M1 + Q1 + W1, M2 + Q2 + W2):
+        assert torch.equal(a, b)
+    assert torch.equal(sig1, sig2)
+
+
+@pytest.mark.parametrize("mode", [odion.COLNORM, odion.QR])
+def test_sigma_and_effective_rank_against_oracle(mode):
+    m, n, r = 512, 768, 64
+    G = synth.lowrank_plus_noise(m, n, 24, 0.02, 31, torch.bfloat16, DEV)
+    M = torch.zeros(m, n, device=DEV)
+    W = torch.zeros(m, n, device=DEV)
+    q0 = _q0(n, r, 3)
+    Qt = torch.tensor(q0.T.copy(), device=DEV)
+    sig = torch.empty(r, device=DEV)
+    p = ouo.dion_params(rank=r, norm_mode="qr" if mode == odion.QR else "colnorm")
+    Mr, Qr = np.zeros((m, n), np.float32), q0.astype(np.float64)
+    for _ in range(3):
+        ouo.dion_lowrank_step([M], [G], [Qt], [W], p, sigma=sig)
+        er = ouo.dion_effective_rank(sig, [r])
+        torch.cuda.synchronize()
+        ref = odion.dion_step(Mr, to64(G), Qr, np.zeros((m, n)), 0.95, 0.01, 1.0, mode)
+        Mr, Qr = ref["M"], ref["Q"]
+        s_gpu = sig.double().cpu().numpy()
+        assert rel_fro(s_gpu, ref["sigma"]) <= TOL_BF16
+        # the kernel's entropy matches the oracle's formula on the same sigma
+        assert abs(er.item() - odion.effective_rank(s_gpu)) <= 1e-5 * odion.effective_rank(s_gpu)
+        assert abs(er.item() - odion.effective_rank(ref["sigma"])) <= TOL_BF16 * r
+        assert 1.0 <= er.item() <= r
+
+
+def test_effective_rank_closed_forms_on_device():
+    ranks = [37, 3, 4, 5]
+    sig = torch.cat([torch.ones(37), torch.tensor([0.0, 3.0, 0.0]),
+                     torch.tensor([2.0, 2.0, 0.0, 0.0]), torch.zeros(5)]).to(DEV)
+    er = ouo.dion_effective_rank(sig, ranks).cpu().numpy()
+    assert er[0] == pytest.approx(37.0, rel=1e-6)
+    assert er[1] == pytest.approx(1.0, rel=1e-6)
+    assert er[2] == pytest.approx(2.0, rel=1e-6)
+    assert er[3] == 0.0

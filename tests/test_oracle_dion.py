@@ -114,3 +114,35 @@ def test_single_step_shapes_and_dtypes():
     assert d["M"].dtype == np.float32 and d["M"].shape == (33, 70)
     assert d["Q"].shape == (70, 5) and d["P"].shape == (33, 5)
     assert np.max(np.abs(np.linalg.norm(d["Q"], axis=0) - 1)) <= 1e-7
+
+
+# ---- Ada-Orth-Dion's effective-rank estimate (closed forms)
+def test_effective_rank_closed_forms():
+    assert dion.effective_rank(np.ones(37)) == pytest.approx(37.0, rel=1e-12)
+    assert dion.effective_rank(np.array([0.0, 3.0, 0.0])) == pytest.approx(1.0, abs=1e-12)
+    assert dion.effective_rank(np.array([2.0, 2.0, 0.0, 0.0])) == pytest.approx(2.0, rel=1e-12)
+    assert dion.effective_rank(np.zeros(5)) == 0.0
+    # energy split 3/4, 1/4: exp(-(3/4 ln 3/4 + 1/4 ln 1/4)) = 4 / 3^(3/4)
+    assert dion.effective_rank(np.array([np.sqrt(3.0), 1.0])) == pytest.approx(
+        4.0 / 3.0 ** 0.75, rel=1e-12)
+    # scale and order invariance, and 1 <= erank <= r
+    s = np.random.default_rng(4).random(50)
+    e = dion.effective_rank(s)
+    assert dion.effective_rank(7.5 * s[::-1]) == pytest.approx(e, rel=1e-12)
+    assert 1.0 <= e <= 50.0
+
+
+def test_effective_rank_of_a_dion_step_tracks_the_spectrum():
+    # B = U diag(s) V^T with s = (1, ..., 1, 0, ...): a full-rank warm start
+    # captures the spectrum, so the estimate equals the number of ones.
+    rng = np.random.default_rng(6)
+    m, n, r, k = 64, 48, 16, 6
+    U = np.linalg.qr(rng.standard_normal((m, m)))[0][:, :n]
+    V = np.linalg.qr(rng.standard_normal((n, n)))[0]
+    s = np.zeros(n)
+    s[:k] = 1.0
+    B = (U * s) @ V.T
+    Q0 = dion.orth(np.hstack([V[:, :k], rng.standard_normal((n, r - k))]))
+    out = dion.dion_step(np.zeros((m, n)), B, Q0, np.zeros((m, n)), 0.95, 0.1, 1.0,
+                          dion.QR, state_dtype=None)
+    assert dion.effective_rank(out["sigma"]) == pytest.approx(float(k), rel=1e-9)
