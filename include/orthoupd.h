@@ -344,6 +344,57 @@ int dion_lowrank_step_stats(const ouo_mat* M, const ouo_mat* G, int g_dtype,
 int dion_effective_rank(const float* sigma, const int* ranks, int nmat,
                         float* erank, void* stream);
 
+/*
+ * Row-sharded Dion / Orth-Dion step: the power iteration with the rows of
+ * every matrix spread over ranks, the form Dion takes when weights are
+ * sharded ([OD] Problem Statement: Dion's communication is the rank-r
+ * factors; [D1] Technical details).  Each rank holds a block of rows of M, G
+ * and W of each matrix (m_i local rows, any split) and a full copy of
+ * Q_state.  A step is four calls on one workspace; after each of the first
+ * three the caller sums the float buffer `red` over the ranks in place (an
+ * all-reduce) before the next call:
+ *   dion_shard_project  B = M + G; P^T = Q^T B^T (r x m_i); red = P^T P.
+ *   dion_shard_orth1    red = sum of P^T P: P^T <- L^-1 P^T (CholeskyQR);
+ *                       red = P^T P.
+ *   dion_shard_orth2    red = sum: P^T <- L^-1 P^T; red = P^T B (r x n).
+ *   dion_shard_update   red = sum = R^T: Q_new^T = ColNorm or orth of the rows
+ *                       of R^T; M <- beta B - (beta - mu) P R^T;
+ *                       W <- (1 - lr wd) W - lr scale P Q_new^T;
+ *                       Q_state <- Q_new^T.
+ * With one rank (nothing summed) the four calls compute what
+ * dion_lowrank_step computes, bit for bit (except for the trace behind a
+ * shifted CholeskyQR retry).
+ * red: device float[dion_shard_red_floats(...)]; matrix i's block follows
+ * those of the matrices before it (256-byte aligned), r_i x r_i packed for
+ * P^T P and r_i x n_i (row pitch n_i rounded up to 4) for P^T B.
+ * rows_total: host int64[nmat], every matrix's global row count (the
+ * shifted-CholeskyQR retry uses it).  ws: dion_shard_workspace_bytes(...)
+ * bytes, the same buffer for the four calls of a step (P^T lives in it
+ * between them).  Ranks as in dion_lowrank_step: p->rank, or 0 for
+ * Q_state[i].rows.  The size queries return 0 for invalid arguments.
+ */
+size_t dion_shard_workspace_bytes(const ouo_mat* M, const ouo_mat* Q_state,
+                                  int nmat, const ouo_dion_params* p);
+size_t dion_shard_red_floats(const ouo_mat* M, const ouo_mat* Q_state, int nmat,
+                             const ouo_dion_params* p);
+int dion_shard_project(const ouo_mat* M, const ouo_mat* G, int g_dtype,
+                       const ouo_mat* Q_state, int nmat,
+                       const ouo_dion_params* p, void* ws, size_t ws_bytes,
+                       float* red, int* dev_status, void* stream);
+int dion_shard_orth1(const ouo_mat* M, const ouo_mat* Q_state, int nmat,
+                     const ouo_dion_params* p, const int64_t* rows_total,
+                     void* ws, size_t ws_bytes, float* red, int* dev_status,
+                     void* stream);
+int dion_shard_orth2(const ouo_mat* M, const ouo_mat* Q_state, int nmat,
+                     const ouo_dion_params* p, const int64_t* rows_total,
+                     void* ws, size_t ws_bytes, float* red, int* dev_status,
+                     void* stream);
+int dion_shard_update(const ouo_mat* M, const ouo_mat* Q_state,
+                      const ouo_mat* W, int w_dtype, int nmat,
+                      const ouo_dion_params* p, const float* scale, void* ws,
+                      size_t ws_bytes, float* red, int* dev_status,
+                      void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -37,7 +37,9 @@ EXPORTED = (
     "ns_workspace_bytes", "ns_orthogonalize", "gram_ns_workspace_bytes",
     "gram_ns_orthogonalize", "gram_ns_orthogonalize_noalloc", "apply_update",
     "dion_workspace_bytes", "dion_lowrank_step", "dion_workspace_bytes_ranks",
-    "dion_lowrank_step_stats", "dion_effective_rank",
+    "dion_lowrank_step_stats", "dion_effective_rank", "dion_shard_workspace_bytes",
+    "dion_shard_red_floats", "dion_shard_project", "dion_shard_orth1", "dion_shard_orth2",
+    "dion_shard_update",
 )
 
 
@@ -107,6 +109,12 @@ _PROTOS = {
     "dion_lowrank_step_stats": (_I, [_MP, _MP, _I, _MP, _MP, _I, _I, _DP, _P, _P, _SZ,
                                      _P, _P, _P]),
     "dion_effective_rank": (_I, [_P, _P, _I, _P, _P]),
+    "dion_shard_workspace_bytes": (_SZ, [_MP, _MP, _I, _DP]),
+    "dion_shard_red_floats": (_SZ, [_MP, _MP, _I, _DP]),
+    "dion_shard_project": (_I, [_MP, _MP, _I, _MP, _I, _DP, _P, _SZ, _P, _P, _P]),
+    "dion_shard_orth1": (_I, [_MP, _MP, _I, _DP, _P, _P, _SZ, _P, _P, _P]),
+    "dion_shard_orth2": (_I, [_MP, _MP, _I, _DP, _P, _P, _SZ, _P, _P, _P]),
+    "dion_shard_update": (_I, [_MP, _MP, _MP, _I, _I, _DP, _P, _P, _SZ, _P, _P, _P]),
 }
 
 

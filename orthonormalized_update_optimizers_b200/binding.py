@@ -22,7 +22,7 @@ __all__ = [
     "ns_orthogonalize", "gram_ns_workspace_bytes", "gram_ns_orthogonalize",
     "gram_ns_orthogonalize_noalloc",
     "apply_update", "dion_workspace_bytes", "dion_lowrank_step", "dion_effective_rank",
-    "version",
+    "DionShardStep", "version",
     "launch_count", "timing_enable", "timing_read", "batch_empty",
 ]
 
@@ -303,3 +303,65 @@ def dion_effective_rank(sigma: torch.Tensor, ranks: Sequence[int],
     L.check("dion_effective_rank", L.lib().dion_effective_rank(
         _ptr(sigma), rk, n, _ptr(erank), _stream(stream)))
     return erank
+
+
+class DionShardStep:
+    """The row-sharded Dion / Orth-Dion step of one rank: its row blocks of
+    M, G, W for every matrix and a full copy of each Q_state.  The four
+    library calls run in order; `allreduce(red)` must sum the float32 CUDA
+    tensor `red` over the ranks in place (e.g. torch.distributed.all_reduce)
+    and is called between them.  `rows_total` are the matrices' global row
+    counts."""
+
+    def __init__(self, M, G, Q_state, W, params, rows_total: Sequence[int], scale=None):
+        self.Mb, self.Gb, self.Qb, self.Wb = _batch(M), _batch(G), _batch(Q_state), _batch(W)
+        self.p = params
+        n = self.Mb.n
+        if len(rows_total) != n:
+            raise ValueError("rows_total needs one entry per matrix")
+        self.rows = (ctypes.c_int64 * max(n, 1))(*[int(x) for x in rows_total])
+        self.scale = None if scale is None else (ctypes.c_float * n)(*[float(x) for x in scale])
+        lib = L.lib()
+        wsb = lib.dion_shard_workspace_bytes(self.Mb.arr, self.Qb.arr, n, ctypes.byref(params))
+        rf = lib.dion_shard_red_floats(self.Mb.arr, self.Qb.arr, n, ctypes.byref(params))
+        if n and (wsb == 0 or rf == 0):
+            raise ValueError("invalid sharded Dion batch")
+        dev = self.Mb.device
+        self.ws = torch.empty(max(wsb, 256), dtype=torch.uint8, device=dev)
+        self.red = torch.empty(max(rf, 64), dtype=torch.float32, device=dev)
+
+    def _args(self, status, stream):
+        return (ctypes.byref(self.p), ctypes.c_void_p(self.ws.data_ptr()), self.ws.numel(),
+                _ptr(self.red), _ptr(status), _stream(stream))
+
+    def project(self, status=None, stream=None) -> None:
+        pp, ws, wn, red, st, s = self._args(status, stream)
+        L.check("dion_shard_project", L.lib().dion_shard_project(
+            self.Mb.arr, self.Gb.arr, self.Gb.dtype, self.Qb.arr, self.Mb.n, pp, ws, wn,
+            red, st, s))
+
+    def orth1(self, status=None, stream=None) -> None:
+        pp, ws, wn, red, st, s = self._args(status, stream)
+        L.check("dion_shard_orth1", L.lib().dion_shard_orth1(
+            self.Mb.arr, self.Qb.arr, self.Mb.n, pp, self.rows, ws, wn, red, st, s))
+
+    def orth2(self, status=None, stream=None) -> None:
+        pp, ws, wn, red, st, s = self._args(status, stream)
+        L.check("dion_shard_orth2", L.lib().dion_shard_orth2(
+            self.Mb.arr, self.Qb.arr, self.Mb.n, pp, self.rows, ws, wn, red, st, s))
+
+    def update(self, status=None, stream=None) -> None:
+        pp, ws, wn, red, st, s = self._args(status, stream)
+        L.check("dion_shard_update", L.lib().dion_shard_update(
+            self.Mb.arr, self.Qb.arr, self.Wb.arr, self.Wb.dtype, self.Mb.n, pp, self.scale,
+            ws, wn, red, st, s))
+
+    def __call__(self, allreduce, status=None, stream=None) -> None:
+        """One step: the four calls with allreduce(self.red) between them."""
+        self.project(status, stream)
+        allreduce(self.red)
+        self.orth1(status, stream)
+        allreduce(self.red)
+        self.orth2(status, stream)
+        allreduce(self.red)
+        self.update(status, stream)

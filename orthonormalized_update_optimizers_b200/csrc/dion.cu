@@ -394,55 +394,77 @@ Buf caller_buf(const ouo_mat& m, int dtype) {
   return b;
 }
 
+// Partial Gram matrices of the rows of X (r x L) into w.part: returns the
+// number of partials written (their float64 sum is X X^T).
+int gram_parts(const Buf& X, const DionWs& w, cudaStream_t s, int* used) {
+  const int r = (int)X.rows;
+  const int64_t L = X.cols;
+  GramArgs ga;
+  ga.X = reinterpret_cast<const float*>(X.p);
+  ga.ld = X.ld;
+  ga.r = r;
+  ga.L = L;
+  const int splits = gram_splits(r, L);
+  ga.chunk = ceil_div(ceil_div(L, splits), kGT) * kGT;
+  *used = (int)ceil_div(L, ga.chunk);
+  ga.part = reinterpret_cast<float*>(w.part.p);
+  ga.tiles = (int)ceil_div(r, kGT);
+  dim3 grid((unsigned)(ga.tiles * (ga.tiles + 1) / 2), (unsigned)*used);
+  gram_partial_kernel<<<grid, 256, 0, s>>>(ga);
+  OUO_CHECK_LAUNCH();
+  return OUO_OK;
+}
+
+// w.Linv = L^-1 where L L^T = sum of `splits` r x r partials at `part`
+// (L_rows: the rows' length, for the shifted retry).
+int cholesky_inverse(const float* part, int splits, int r, int64_t L_rows,
+                     const DionWs& w, int* status, cudaStream_t s) {
+  if (r >= blocked_chol_min_rank()) {
+    OUO_TRY(chol_blocked(part, splits, r, L_rows, reinterpret_cast<float*>(w.S.p),
+                         reinterpret_cast<float*>(w.Linv.p), w.ctl.p, status, s));
+  } else {
+    CholArgs ca;
+    ca.part = part;
+    ca.splits = splits;
+    ca.r = r;
+    ca.L = L_rows;
+    ca.Linv = reinterpret_cast<float*>(w.Linv.p);
+    ca.ldl = w.Linv.ld;
+    ca.status = status;
+    chol_inv_kernel<<<1, 1024, chol_smem_bytes(r), s>>>(ca);
+    OUO_CHECK_LAUNCH();
+  }
+  return OUO_OK;
+}
+
+// dst = Linv src (r x L, fp32 SIMT)
+int apply_linv(const DionWs& w, int r, const Buf& src, const Buf& dst, cudaStream_t s) {
+  GemmDesc d;
+  d.M = r;
+  d.N = src.cols;
+  d.K = r;
+  d.nb = 1;
+  d.A = w.Linv;
+  d.B = src;
+  d.b_mn = 1;
+  d.out_f32 = dst;
+  d.has_f32 = true;
+  return gemm_simt(d, s);
+}
+
 // Rows of X (r x L, workspace) made orthonormal into Y: two CholeskyQR
 // passes (X -> tmp -> Y); X is clobbered.
 int orth_rows(Buf X, Buf tmp, Buf Y, const DionWs& w, cudaStream_t s,
               int* status) {
   const int r = (int)X.rows;
-  const int64_t L = X.cols;
   Buf src = X;
   for (int pass = 0; pass < 2; ++pass) {
     Buf dst = pass == 0 ? tmp : Y;
-    GramArgs ga;
-    ga.X = reinterpret_cast<const float*>(src.p);
-    ga.ld = src.ld;
-    ga.r = r;
-    ga.L = L;
-    const int splits = gram_splits(r, L);
-    ga.chunk = ceil_div(ceil_div(L, splits), kGT) * kGT;
-    const int used = (int)ceil_div(L, ga.chunk);
-    ga.part = reinterpret_cast<float*>(w.part.p);
-    ga.tiles = (int)ceil_div(r, kGT);
-    dim3 grid((unsigned)(ga.tiles * (ga.tiles + 1) / 2), (unsigned)used);
-    gram_partial_kernel<<<grid, 256, 0, s>>>(ga);
-    OUO_CHECK_LAUNCH();
-    if (r >= blocked_chol_min_rank()) {
-      OUO_TRY(chol_blocked(ga.part, used, r, L, reinterpret_cast<float*>(w.S.p),
-                           reinterpret_cast<float*>(w.Linv.p), w.ctl.p, status, s));
-    } else {
-      CholArgs ca;
-      ca.part = ga.part;
-      ca.splits = used;
-      ca.r = r;
-      ca.L = L;
-      ca.Linv = reinterpret_cast<float*>(w.Linv.p);
-      ca.ldl = w.Linv.ld;
-      ca.status = status;
-      chol_inv_kernel<<<1, 1024, chol_smem_bytes(r), s>>>(ca);
-      OUO_CHECK_LAUNCH();
-    }
-    // dst = Linv src
-    GemmDesc d;
-    d.M = r;
-    d.N = L;
-    d.K = r;
-    d.nb = 1;
-    d.A = w.Linv;
-    d.B = src;
-    d.b_mn = 1;
-    d.out_f32 = dst;
-    d.has_f32 = true;
-    OUO_TRY(gemm_simt(d, s));
+    int used = 0;
+    OUO_TRY(gram_parts(src, w, s, &used));
+    OUO_TRY(cholesky_inverse(reinterpret_cast<const float*>(w.part.p), used, r, src.cols,
+                             w, status, s));
+    OUO_TRY(apply_linv(w, r, src, dst, s));
     src = dst;
   }
   return OUO_OK;
@@ -665,6 +687,300 @@ extern "C" int dion_effective_rank(const float* sigma, const int* ranks, int nma
     erank_kernel<<<cn, 256, 0, s>>>(a);
     OUO_CHECK_LAUNCH();
     base += a.off[cn];
+  }
+  return OUO_OK;
+}
+
+// ------------------------------------------------------ row-sharded step
+// The power iteration with the rows of every matrix spread over ranks: the
+// r x r Gram matrices of P^T and the r x n product P^T B are the only
+// quantities summed across ranks (by the caller, between the calls below);
+// everything else is local to a rank's rows, and the right factor is
+// formed redundantly on every rank.
+namespace ouo {
+namespace {
+
+// out[e] = sum_p part[p][e] in float64, fixed order (the reduction the
+// Cholesky kernels apply to their partials), rounded to fp32.
+__global__ void sum_parts_kernel(const float* part, int splits, int64_t n, float* out) {
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n;
+       e += (int64_t)gridDim.x * blockDim.x) {
+    double s = 0.0;
+    for (int q = 0; q < splits; ++q) s += (double)part[(size_t)q * n + e];
+    out[e] = (float)s;
+  }
+}
+
+int64_t pitch4(int64_t n) { return ceil_div(n, 4) * 4; }
+
+// floats of matrix i's block of `red` (256-byte multiple)
+int64_t red_block(int r, int64_t n) {
+  const int64_t f = (int64_t)r * r > (int64_t)r * pitch4(n) ? (int64_t)r * r : (int64_t)r * pitch4(n);
+  return ceil_div(f, 64) * 64;
+}
+
+// Ranks of the batch (p->rank, or Q_state rows with p->rank == 0) and the
+// shared shape checks of every sharded call.
+int shard_ranks(const ouo_mat* M, const ouo_mat* Q_state, int nmat,
+                const ouo_dion_params* p, std::vector<int>& ranks) {
+  OUO_TRY(validate_dion(p));
+  if (p->rank < 0) return set_error(OUO_ERR_INVALID_ARG, "rank %d < 0", p->rank);
+  OUO_TRY(validate_mats(M, nmat, OUO_F32, "M"));
+  OUO_TRY(validate_mats(Q_state, nmat, OUO_F32, "Q_state"));
+  ranks.assign((size_t)nmat, 0);
+  for (int i = 0; i < nmat; ++i) {
+    const int r = p->rank ? p->rank : (int)Q_state[i].rows;
+    ranks[i] = r;
+    if (r < 1 || r > M[i].cols)
+      return set_error(OUO_ERR_INVALID_ARG, "rank %d outside [1, cols] for M[%d]", r, i);
+    if (Q_state[i].rows != r || Q_state[i].cols != M[i].cols)
+      return set_error(OUO_ERR_INVALID_ARG, "Q_state[%d] must be r x cols", i);
+    if (!vec16(M[i], OUO_F32) || !vec16(Q_state[i], OUO_F32))
+      return set_error(OUO_ERR_INVALID_ARG,
+                       "sharded Dion needs M and Q_state rows on 16-byte boundaries (%d)", i);
+  }
+  return OUO_OK;
+}
+
+int shard_common(const ouo_mat* M, const ouo_mat* Q_state, int nmat,
+                 const ouo_dion_params* p, void* ws, size_t ws_bytes, float* red,
+                 int* dev_status, std::vector<int>& ranks) {
+  OUO_TRY(shard_ranks(M, Q_state, nmat, p, ranks));
+  if (dev_status && ((uintptr_t)dev_status % 4))
+    return set_error(OUO_ERR_INVALID_ARG, "dev_status misaligned");
+  if (!red || ((uintptr_t)red % 256))
+    return set_error(OUO_ERR_INVALID_ARG, "red must be a 256-byte aligned device buffer");
+  const size_t need = dion_plan_bytes(M, nmat, ranks.data());
+  if (!ws || ws_bytes < need)
+    return set_error(OUO_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given",
+                     need, ws_bytes);
+  if ((uintptr_t)ws % 256)
+    return set_error(OUO_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  return require_sm100();
+}
+
+int sum_parts(const DionWs& w, int used, int r, float* out, cudaStream_t s) {
+  const int64_t n = (int64_t)r * r;
+  sum_parts_kernel<<<grid_1d(n, 256), 256, 0, s>>>(reinterpret_cast<const float*>(w.part.p),
+                                                   used, n, out);
+  OUO_CHECK_LAUNCH();
+  return OUO_OK;
+}
+
+}  // namespace
+}  // namespace ouo
+
+extern "C" size_t dion_shard_workspace_bytes(const ouo_mat* M, const ouo_mat* Q_state,
+                                             int nmat, const ouo_dion_params* p) {
+  if (!M || !Q_state || !p || nmat <= 0 || nmat > OUO_MAX_BATCH || p->rank < 0) return 0;
+  std::vector<int> ranks((size_t)nmat);
+  for (int i = 0; i < nmat; ++i) {
+    ranks[i] = p->rank ? p->rank : (int)Q_state[i].rows;
+    if (ranks[i] < 1) return 0;
+  }
+  return ouo::dion_plan_bytes(M, nmat, ranks.data());
+}
+
+extern "C" size_t dion_shard_red_floats(const ouo_mat* M, const ouo_mat* Q_state, int nmat,
+                                        const ouo_dion_params* p) {
+  if (!M || !Q_state || !p || nmat <= 0 || nmat > OUO_MAX_BATCH || p->rank < 0) return 0;
+  size_t f = 0;
+  for (int i = 0; i < nmat; ++i) {
+    const int r = p->rank ? p->rank : (int)Q_state[i].rows;
+    if (r < 1) return 0;
+    f += (size_t)ouo::red_block(r, M[i].cols);
+  }
+  return f;
+}
+
+extern "C" int dion_shard_project(const ouo_mat* M, const ouo_mat* G, int g_dtype,
+                                  const ouo_mat* Q_state, int nmat,
+                                  const ouo_dion_params* p, void* ws, size_t ws_bytes,
+                                  float* red, int* dev_status, void* stream) {
+  using namespace ouo;
+  clear_error();
+  if (nmat < 0 || nmat > OUO_MAX_BATCH)
+    return set_error(OUO_ERR_INVALID_ARG, "nmat %d out of range", nmat);
+  if (nmat == 0) return OUO_OK;
+  std::vector<int> ranks;
+  OUO_TRY(shard_common(M, Q_state, nmat, p, ws, ws_bytes, red, dev_status, ranks));
+  OUO_TRY(validate_mats(G, nmat, g_dtype, "G"));
+  OUO_TRY(validate_same_shapes(M, G, nmat, "M", "G"));
+  cudaStream_t s = (cudaStream_t)stream;
+  OUO_TRY(dion_momentum_update(M, G, nmat, g_dtype, p->mu, OUO_MOMENTUM_ACCUM, nullptr,
+                               stream));
+  Arena ar{reinterpret_cast<char*>(ws), ws_bytes, 0, false};
+  int64_t off = 0;
+  for (int i = 0; i < nmat; ++i) {
+    const int r = ranks[i];
+    const int64_t m = M[i].rows, n = M[i].cols;
+    DionWs w = carve_dion(ar, m, n, r);
+    GemmDesc d;  // P^T = Q^T B^T (r x m local)
+    d.M = r; d.N = m; d.K = n; d.nb = 1;
+    d.A = caller_buf(Q_state[i], OUO_F32);
+    d.B = caller_buf(M[i], OUO_F32);
+    d.out_f32 = w.Pa;
+    d.has_f32 = true;
+    OUO_TRY(gemm_umma(d, s, dev_status));
+    int used = 0;
+    OUO_TRY(gram_parts(w.Pa, w, s, &used));
+    OUO_TRY(sum_parts(w, used, r, red + off, s));
+    off += red_block(r, n);
+  }
+  return OUO_OK;
+}
+
+namespace ouo {
+namespace {
+// orth1 (second = false) and orth2 (second = true)
+int shard_orth(const ouo_mat* M, const ouo_mat* Q_state, int nmat,
+               const ouo_dion_params* p, const int64_t* rows_total, void* ws,
+               size_t ws_bytes, float* red, int* dev_status, void* stream, bool second) {
+  clear_error();
+  if (nmat < 0 || nmat > OUO_MAX_BATCH)
+    return set_error(OUO_ERR_INVALID_ARG, "nmat %d out of range", nmat);
+  if (nmat == 0) return OUO_OK;
+  if (!rows_total) return set_error(OUO_ERR_INVALID_ARG, "NULL rows_total");
+  std::vector<int> ranks;
+  OUO_TRY(shard_common(M, Q_state, nmat, p, ws, ws_bytes, red, dev_status, ranks));
+  for (int i = 0; i < nmat; ++i)
+    if (rows_total[i] < ranks[i] || rows_total[i] < M[i].rows)
+      return set_error(OUO_ERR_INVALID_ARG, "rows_total[%d] smaller than rank or local rows", i);
+  cudaStream_t s = (cudaStream_t)stream;
+  Arena ar{reinterpret_cast<char*>(ws), ws_bytes, 0, false};
+  int64_t off = 0;
+  for (int i = 0; i < nmat; ++i) {
+    const int r = ranks[i];
+    const int64_t m = M[i].rows, n = M[i].cols;
+    DionWs w = carve_dion(ar, m, n, r);
+    OUO_TRY(cholesky_inverse(red + off, 1, r, rows_total[i], w, dev_status, s));
+    if (!second) {
+      OUO_TRY(apply_linv(w, r, w.Pa, w.Pb, s));
+      int used = 0;
+      OUO_TRY(gram_parts(w.Pb, w, s, &used));
+      OUO_TRY(sum_parts(w, used, r, red + off, s));
+    } else {
+      OUO_TRY(apply_linv(w, r, w.Pb, w.Pa, s));
+      Buf rt;  // P^T B (r x n) into the exchange buffer
+      rt.p = reinterpret_cast<char*>(red + off);
+      rt.dtype = OUO_F32;
+      rt.rows = r;
+      rt.cols = n;
+      rt.ld = pitch4(n);
+      rt.stride = rt.rows * rt.ld;
+      rt.nb = 1;
+      GemmDesc d;
+      d.M = r; d.N = n; d.K = m; d.nb = 1;
+      d.A = w.Pa;
+      d.B = caller_buf(M[i], OUO_F32);
+      d.b_mn = 1;
+      d.out_f32 = rt;
+      d.has_f32 = true;
+      OUO_TRY(gemm_umma(d, s, dev_status));
+    }
+    off += red_block(r, n);
+  }
+  return OUO_OK;
+}
+}  // namespace
+}  // namespace ouo
+
+extern "C" int dion_shard_orth1(const ouo_mat* M, const ouo_mat* Q_state, int nmat,
+                                const ouo_dion_params* p, const int64_t* rows_total,
+                                void* ws, size_t ws_bytes, float* red, int* dev_status,
+                                void* stream) {
+  return ouo::shard_orth(M, Q_state, nmat, p, rows_total, ws, ws_bytes, red, dev_status,
+                         stream, false);
+}
+
+extern "C" int dion_shard_orth2(const ouo_mat* M, const ouo_mat* Q_state, int nmat,
+                                const ouo_dion_params* p, const int64_t* rows_total,
+                                void* ws, size_t ws_bytes, float* red, int* dev_status,
+                                void* stream) {
+  return ouo::shard_orth(M, Q_state, nmat, p, rows_total, ws, ws_bytes, red, dev_status,
+                         stream, true);
+}
+
+extern "C" int dion_shard_update(const ouo_mat* M, const ouo_mat* Q_state,
+                                 const ouo_mat* W, int w_dtype, int nmat,
+                                 const ouo_dion_params* p, const float* scale, void* ws,
+                                 size_t ws_bytes, float* red, int* dev_status,
+                                 void* stream) {
+  using namespace ouo;
+  clear_error();
+  if (nmat < 0 || nmat > OUO_MAX_BATCH)
+    return set_error(OUO_ERR_INVALID_ARG, "nmat %d out of range", nmat);
+  if (nmat == 0) return OUO_OK;
+  std::vector<int> ranks;
+  OUO_TRY(shard_common(M, Q_state, nmat, p, ws, ws_bytes, red, dev_status, ranks));
+  OUO_TRY(validate_mats(W, nmat, w_dtype, "W"));
+  OUO_TRY(validate_same_shapes(M, W, nmat, "M", "W"));
+  for (int i = 0; i < nmat; ++i)
+    if (!vec16(W[i], w_dtype))
+      return set_error(OUO_ERR_INVALID_ARG, "W rows must be on 16-byte boundaries (%d)", i);
+  cudaStream_t s = (cudaStream_t)stream;
+  Arena ar{reinterpret_cast<char*>(ws), ws_bytes, 0, false};
+  const float mu = p->mu, beta = p->beta;
+  int64_t off = 0;
+  for (int i = 0; i < nmat; ++i) {
+    const int r = ranks[i];
+    const int64_t m = M[i].rows, n = M[i].cols;
+    DionWs w = carve_dion(ar, m, n, r);
+    // R^T (summed over ranks) into the workspace
+    copy2d_kernel<<<grid_1d((int64_t)r * n, 256), 256, 0, s>>>(
+        red + off, pitch4(n), reinterpret_cast<float*>(w.Ra.p), w.Ra.ld, r, n);
+    OUO_CHECK_LAUNCH();
+    {
+      dim3 grid((unsigned)ceil_div(m, 32), (unsigned)ceil_div(r, 32));
+      transpose_kernel<<<grid, 256, 0, s>>>(reinterpret_cast<const float*>(w.Pa.p),
+                                            w.Pa.ld, reinterpret_cast<float*>(w.P.p),
+                                            w.P.ld, r, m);
+      OUO_CHECK_LAUNCH();
+    }
+    {  // M <- beta B - (beta - mu) P R^T (local rows)
+      GemmDesc d;
+      d.M = m; d.N = n; d.K = r; d.nb = 1;
+      d.A = w.P;
+      d.B = w.Ra;
+      d.b_mn = 1;
+      d.alpha = -(beta - mu);
+      d.beta = beta;
+      d.has_c0 = true;
+      d.direct = {MatRef{M[i].ptr, M[i].ld}};
+      d.direct_dtype = OUO_F32;
+      d.c0_from_out = true;
+      OUO_TRY(gemm_umma(d, s, dev_status));
+    }
+    Buf Qn = w.Rb;
+    if (p->norm_mode == OUO_DION_COLNORM) {
+      rownorm_kernel<<<r, 256, 0, s>>>(reinterpret_cast<const float*>(w.Ra.p), w.Ra.ld,
+                                       reinterpret_cast<float*>(w.Rb.p), w.Rb.ld, n,
+                                       p->eps);
+      OUO_CHECK_LAUNCH();
+    } else {
+      OUO_TRY(orth_rows(w.Ra, w.Rb, w.Ra, w, s, dev_status));
+      Qn = w.Ra;
+    }
+    {  // W <- (1 - lr wd) W - lr s P Q_new^T (local rows)
+      const float sc = scale ? scale[i] : 1.0f;
+      GemmDesc d;
+      d.M = m; d.N = n; d.K = r; d.nb = 1;
+      d.A = w.P;
+      d.B = Qn;
+      d.b_mn = 1;
+      d.alpha = -p->lr * sc;
+      d.beta = 1.0f - p->lr * p->wd;
+      d.has_c0 = true;
+      d.direct = {MatRef{W[i].ptr, W[i].ld}};
+      d.direct_dtype = w_dtype;
+      d.c0_from_out = true;
+      OUO_TRY(gemm_umma(d, s, dev_status));
+    }
+    copy2d_kernel<<<grid_1d((int64_t)r * n, 256), 256, 0, s>>>(
+        reinterpret_cast<const float*>(Qn.p), Qn.ld,
+        reinterpret_cast<float*>(Q_state[i].ptr), Q_state[i].ld, r, n);
+    OUO_CHECK_LAUNCH();
+    off += red_block(r, n);
   }
   return OUO_OK;
 }

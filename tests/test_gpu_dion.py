@@ -189,3 +189,69 @@ def test_effective_rank_closed_forms_on_device():
     assert er[1] == pytest.approx(1.0, rel=1e-6)
     assert er[2] == pytest.approx(2.0, rel=1e-6)
     assert er[3] == 0.0
+
+
+# ---- row-sharded step (the power iteration with rows spread over ranks) ---
+def _full_state(m, n, r, seed, w_dtype=torch.float32):
+    G = synth.lowrank_plus_noise(m, n, min(64, m, n), 0.02, seed, torch.bfloat16, DEV)
+    W = synth.gaussian((m, n), seed + 7, 0.02, w_dtype, DEV)
+    Q = torch.tensor(_q0(n, r, seed + 3).T.copy(), device=DEV)
+    return torch.zeros(m, n, device=DEV), G, Q, W
+
+
+@pytest.mark.parametrize("mode", ["colnorm", "qr"])
+@pytest.mark.parametrize("r", [32, 128])
+def test_shard_one_rank_is_the_unsharded_step(mode, r):
+    m, n = 640, 512
+    M1, G, Q1, W1 = _full_state(m, n, r, 11)
+    M2, _, Q2, W2 = M1.clone(), None, Q1.clone(), W1.clone()
+    p = ouo.dion_params(rank=r, norm_mode=mode, lr=0.05)
+    step = ouo.DionShardStep([M2], [G], [Q2], [W2], p, rows_total=[m], scale=[1.5])
+    st = torch.zeros(1, dtype=torch.int32, device=DEV)
+    for _ in range(2):
+        ouo.dion_lowrank_step([M1], [G], [Q1], [W1], p, scale=[1.5], status=st)
+        step(lambda red: None, status=st)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    for a, b in ((M1, M2), (Q1, Q2), (W1, W2)):
+        assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("mode", [odion.COLNORM, odion.QR])
+@pytest.mark.parametrize("splits", [(300, 340), (100, 260, 280)])
+def test_shard_emulated_ranks_match_the_unsharded_step(mode, splits):
+    # Ranks emulated in one process: each row block runs the four calls, and
+    # between calls the blocks' partial sums are added (in rank order) and
+    # handed back to every block -- what an all-reduce does.
+    m, n, r = sum(splits), 512, 96
+    name = "qr" if mode == odion.QR else "colnorm"
+    M, G, Q, W = _full_state(m, n, r, 21)
+    Mr, Wr = M.clone(), W.clone()
+    W0 = to64(W)
+    Qs = [Q.clone() for _ in splits]
+    p = ouo.dion_params(rank=r, norm_mode=name, lr=0.05)
+    bounds = np.concatenate([[0], np.cumsum(splits)]).astype(int)
+    steps = [ouo.DionShardStep([Mr[a:b]], [G[a:b]], [Qs[k]], [Wr[a:b]], p, rows_total=[m])
+             for k, (a, b) in enumerate(zip(bounds[:-1], bounds[1:]))]
+    st = torch.zeros(1, dtype=torch.int32, device=DEV)
+    Mo, Qo, Wo = np.zeros((m, n), np.float32), _q0(n, r, 24).astype(np.float64), to64(W)
+    for _ in range(2):
+        for phase in ("project", "orth1", "orth2", "update"):
+            for s_ in steps:
+                getattr(s_, phase)(status=st)
+            if phase != "update":
+                tot = steps[0].red.clone()
+                for s_ in steps[1:]:
+                    tot += s_.red
+                for s_ in steps:
+                    s_.red.copy_(tot)
+        ouo.dion_lowrank_step([M], [G], [Q], [W], p, status=st)
+        ref = odion.dion_step(Mo, to64(G), Qo, Wo, 0.95, 0.05, 1.0, mode)
+        Mo, Qo, Wo = ref["M"], ref["Q"], ref["W"]
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    for Qk in Qs[1:]:
+        assert torch.equal(Qk, Qs[0])  # every rank forms the same right factor
+    assert rel_fro(to64(Mr), to64(M)) <= 1e-2 and rel_fro(to64(Mr), Mo) <= TOL_BF16
+    assert rel_fro(to64(Qs[0]), to64(Q)) <= 1e-2 and rel_fro(to64(Qs[0]).T, Qo) <= TOL_BF16
+    assert rel_fro(to64(Wr) - W0, to64(W) - W0) <= 1e-2

@@ -135,3 +135,100 @@ def test_gloo_exchange_reproduces_the_single_process_step(world):
             ref = oapply.apply_update(W, O16, res["idx"], LR, _scale(m, n))
             for r in range(world):
                 assert np.array_equal(got[r][str(i)], ref), (i, r)
+
+
+# ---- row-sharded Dion step: the orchestration over gloo ranks -------------
+from oracle import dion as odion  # noqa: E402
+from orthonormalized_update_optimizers_b200.binding import DionShardStep  # noqa: E402
+
+
+class _Float64Phases:
+    """Test-side float64 stand-in for one rank's four library calls (the
+    same decomposition: Gram matrices and P^T B are the only summed parts),
+    so DionShardStep's orchestration can run over real gloo ranks."""
+
+    def __init__(self, M, G, Qt, W, mu, lr, beta, mode, rows_total):
+        self.M, self.G, self.Qt, self.W = M, G, Qt, W
+        # the oracle takes mu and beta as the fp32 values the library receives
+        self.mu, self.beta = float(np.float32(mu)), float(np.float32(beta))
+        self.lr, self.mode = lr, mode
+        self.r, self.n = Qt.shape
+        self.red = torch.zeros(max(self.r * self.r, self.r * self.n), dtype=torch.float64)
+
+    def _put(self, a):
+        self.red.zero_()
+        self.red[:a.size] = torch.from_numpy(np.ascontiguousarray(a).ravel())
+
+    def _get(self, shape):
+        return self.red[:shape[0] * shape[1]].numpy().reshape(shape).copy()
+
+    def _chol_apply(self, Pt):
+        S = self._get((self.r, self.r))
+        Lc = np.linalg.cholesky(S)
+        return np.linalg.solve(Lc, Pt)
+
+    def project(self, status=None, stream=None):
+        self.B = self.M + self.G
+        self.Pt = self.Qt @ self.B.T
+        self._put(self.Pt @ self.Pt.T)
+
+    def orth1(self, status=None, stream=None):
+        self.Pt = self._chol_apply(self.Pt)
+        self._put(self.Pt @ self.Pt.T)
+
+    def orth2(self, status=None, stream=None):
+        self.Pt = self._chol_apply(self.Pt)
+        self._put(self.Pt @ self.B)
+
+    def update(self, status=None, stream=None):
+        Rt = self._get((self.r, self.n))
+        P = self.Pt.T
+        self.M = self.beta * self.B - (self.beta - self.mu) * (P @ Rt)
+        if self.mode == odion.QR:
+            Qn = odion.orth(Rt.T).T
+        else:
+            Qn = (odion.colnorm(Rt.T)).T
+        self.W = self.W - self.lr * (P @ Qn)
+        self.Qt = Qn
+
+
+def _shard_worker(rank, world, port, out_dir, mode):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        m, n, r = 90, 40, 6
+        rng = np.random.default_rng(5)
+        G = rng.standard_normal((m, n))
+        W = rng.standard_normal((m, n)) * 0.1
+        Q0 = odion.orth(rng.standard_normal((n, r)))
+        rows = np.array_split(np.arange(m), world)[rank]
+        ph = _Float64Phases(np.zeros((len(rows), n)), G[rows], Q0.T.copy(), W[rows],
+                            0.95, 0.1, 1.0, mode, m)
+        for _ in range(2):
+            DionShardStep.__call__(ph, lambda t: dist.all_reduce(t))
+        np.savez(os.path.join(out_dir, f"rank{rank}.npz"), M=ph.M, W=ph.W, Q=ph.Qt, rows=rows)
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("mode", [odion.COLNORM, odion.QR])
+def test_gloo_row_sharded_dion_matches_the_unsharded_oracle(mode):
+    world = 3
+    with tempfile.TemporaryDirectory() as d:
+        mp.spawn(_shard_worker, args=(world, _free_port(), d, mode), nprocs=world, join=True)
+        m, n, r = 90, 40, 6
+        rng = np.random.default_rng(5)
+        G = rng.standard_normal((m, n))
+        W = rng.standard_normal((m, n)) * 0.1
+        Q = odion.orth(rng.standard_normal((n, r)))
+        M = np.zeros((m, n))
+        for _ in range(2):
+            ref = odion.dion_step(M, G, Q, W, 0.95, 0.1, 1.0, mode, state_dtype=None)
+            M, Q, W = ref["M"], ref["Q"], ref["W"]
+        for k in range(world):
+            got = np.load(os.path.join(d, f"rank{k}.npz"))
+            rows = got["rows"]
+            assert np.allclose(got["M"], M[rows], rtol=0, atol=1e-9)
+            assert np.allclose(got["W"], W[rows], rtol=0, atol=1e-9)
+            assert np.allclose(got["Q"], Q.T, rtol=0, atol=1e-9)
