@@ -433,6 +433,23 @@ def run_ours(args):
     m1.record()
     barrier()
     mom_ms = max_over_ranks(m0.elapsed_time(m1) / args.steps)
+    # --- row selection + gather, and the weight update (HBM-bound), alone
+    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s0.record()
+    for _ in range(args.steps):
+        if own:
+            ouo.dion3_select_rows(Mb, keys, RHO, idx, Xb, scale, ef=True, mu=MU)
+    s1.record()
+    barrier()
+    sel_ms = max_over_ranks(s0.elapsed_time(s1) / args.steps)
+    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a0.record()
+    for _ in range(args.steps):
+        for Wb_r, Ob_r, idx_r, sc_r in segs:
+            ouo.apply_update(Wb_r, Ob_r, LR, idx=idx_r, scale=sc_r)
+    a1.record()
+    barrier()
+    app_ms = max_over_ranks(a0.elapsed_time(a1) / args.steps)
     # --- per-launch timing of every tensor-core GEMM launch of full steps
     # (CUDA events recorded by the library around each launch, on its stream)
     ouo.timing_enable(True)
@@ -465,6 +482,7 @@ def run_ours(args):
     p_bf = peaks["bf16_tflops"]
     p_tf = p_bf * TF32_RATIO
     peak_eff = flops / (bf / p_bf + tf / p_tf)
+    all_kn = [(lay.k[i], mn[i][1]) for i in range(len(mn))]
     # momentum kernel of this rank (its own matrices)
     elems = sum(mn[i][0] * mn[i][1] for i in own)
     rows = sum(mn[i][0] for i in own)
@@ -517,7 +535,9 @@ def run_ours(args):
                          "traffic": traffic.get("momentum_kernel"),
                          "ms_per_step": round(mom_ms, 4),
                          "launches_per_step": mom_launches},
+        "matrices_per_s": round(len(mn) / (ms * 1e-3), 1),
         "kernels": kinds,
+        "elementwise": _elementwise(sel_ms, app_ms, own, all_kn, lay, peaks),
         "gpu_launches": int(launches),
         "device_status": st,
     }
@@ -535,6 +555,24 @@ def run_ours(args):
     if dist is not None:
         dist.barrier()
         dist.destroy_process_group()
+
+
+def _elementwise(sel_ms, app_ms, own, all_kn, lay, peaks):
+    """HBM figures of the selection + gather and weight-update kernels:
+    gather reads B[S] (fp32) and writes X0 (bf16) and M[S] (fp32), 10 bytes
+    per kept element; the update reads and writes W[S] (bf16) and reads O
+    (bf16), 6 bytes per kept element (every rank updates all matrices)."""
+    kept_own = sum(all_kn[i][0] * all_kn[i][1] for i in own)
+    kept_all = sum(k * n for k, n in all_kn)
+    out = {}
+    for name, ms, nbytes in (("select_gather", sel_ms, 10 * kept_own),
+                             ("apply_update", app_ms, 6 * kept_all)):
+        gbs = nbytes / (ms * 1e-3) / 1e9 if ms > 0 else 0.0
+        out[name] = {"ms_per_step": round(ms, 4), "bytes_per_step": nbytes,
+                     "achieved_gbs": round(gbs, 1),
+                     "frac_of_measured_hbm": round(gbs / peaks["hbm_gbs"], 4),
+                     "frac_of_8tbs": round(gbs / 8000.0, 4)}
+    return out
 
 
 def e2e_measure(args, chunks, step_chunk, exchange_and_update, idx, scale, barrier,
@@ -626,6 +664,13 @@ def run_sweep(args):
         torch.cuda.synchronize()
         return e0.elapsed_time(e1) / K
 
+    peaks = _peaks()
+    p_bf = peaks["bf16_tflops"]
+    p_tf = p_bf * TF32_RATIO
+
+    def peak_for(bf, tf):
+        return (bf + tf) / (bf / p_bf + tf / p_tf)
+
     sampler = ClockSampler(0)
     sampler.start()
     ns_rows = []
@@ -638,14 +683,22 @@ def run_sweep(args):
             O = [torch.empty_like(x) for x in X]
             Xb, Ob = ouo.MatBatch(X), ouo.MatBatch(O)
             row = {"m": m, "n": n, "batch": nb}
-            for name, fn_name, flops in (("standard", "ns_orthogonalize", std_ns_flops(m, n)),
-                                         ("gram", "gram_ns_orthogonalize", sum(gram_ns_flops(m, n)))):
+            kk = min(m, n)
+            std_tf = ITERS * kk * kk * (kk + 1)
+            std_bf = std_ns_flops(m, n) - std_tf
+            gbf, gtf = gram_ns_flops(m, n)
+            for name, fn_name, flops, pk in (
+                    ("standard", "ns_orthogonalize", std_bf + std_tf, peak_for(std_bf, std_tf)),
+                    ("gram", "gram_ns_orthogonalize", gbf + gtf, peak_for(gbf, gtf))):
                 params = ouo.ns_params()
                 wsb = getattr(ouo, fn_name.replace("orthogonalize", "workspace_bytes"))(Xb, params)
                 ws = torch.empty(wsb, dtype=torch.uint8, device=dev)
                 fn = getattr(ouo, fn_name)
                 ms = timed(lambda: fn(Xb, Ob, params, workspace=ws))
-                row[name] = {"ms": round(ms, 4), "tflops": round(nb * flops / ms / 1e9, 1),
+                tfl = nb * flops / ms / 1e9
+                row[name] = {"ms": round(ms, 4), "tflops": round(tfl, 1),
+                             "frac_of_peak": round(tfl / pk, 4),
+                             "matrices_per_s": round(nb / (ms * 1e-3), 1),
                              "us_per_matrix": round(ms * 1e3 / nb, 2)}
                 del ws
             row["gram_speedup"] = round(row["standard"]["ms"] / row["gram"]["ms"], 3)
@@ -674,6 +727,9 @@ def run_sweep(args):
             del M, Wt, Qt, ws
     clocks = sampler.stop()
     print(json.dumps({"mode": "sweep", "unit": "ms per call (device time)", "steps": K,
+                      "peak_note": f"frac_of_peak: against bf16 {p_bf} TFLOP/s ({peaks['source']}, "
+                                   f"burst) and tf32 = bf16 x {TF32_RATIO:.3f}, weighted by each "
+                                   "point's bf16 / tf32 flops",
                       "warmup": W, "dtype": "bf16 (k x k products tf32; Dion tf32)",
                       "data": "synthetic low-rank(64) + N(0, 0.02^2) noise",
                       "ns": ns_rows, "dion": dion_rows, "clocks": clocks}), flush=True)

@@ -79,6 +79,7 @@ struct Segment {
   int64_t ldob, sob;
   int direct;  // outputs go to dptr[dbase + b]
   int dbase;
+  int b4d;  // MN-major B: tmB is 4-D, one TMA load brings every chunk of a stage
 };
 
 constexpr int kMaxSeg = 6;
@@ -360,6 +361,11 @@ umma_gemm_kernel(const __grid_constant__ UmmaArgs a) {
         load(sa, &sg.tmA, (int32_t)(kb * kBK), arow);
         if (!B_MN) {
           load(sb, &sg.tmB, (int32_t)(kb * kBK), bcol);
+        } else if (CG == 1 && sg.b4d) {
+          // (chunk column, K row, chunk, matrix): the chunks land back to
+          // back, the layout the per-chunk loads produce
+          ptx::tma_load_4d(sb, &sg.tmB, &full[stage], 0, (int32_t)(kb * kBK),
+                           (int32_t)(bcol / kChunkCols), z);
         } else {
 #pragma unroll
           for (uint32_t c = 0; c < C::kBRows / kChunkCols; ++c)
@@ -831,6 +837,34 @@ int make_map(CUtensorMap* map, const Buf& t, uint32_t box_cols,
   return OUO_OK;
 }
 
+// 4-D map of an MN-major operand whose columns split into whole chunks:
+// dims (chunk columns, rows, chunk index, matrix), the chunk index striding
+// by one chunk's bytes.  A box of `nchunks` chunks is one TMA load that
+// fills consecutive chunk tiles in shared memory.
+int make_map4(CUtensorMap* map, const Buf& t, uint32_t chunk_cols, uint32_t box_rows,
+              uint32_t nchunks, CUtensorMapSwizzle swz) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn)
+    return set_error(OUO_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  const size_t es = elem_size(t.dtype);
+  cuuint64_t dims[4] = {(cuuint64_t)chunk_cols, (cuuint64_t)t.rows,
+                        (cuuint64_t)(t.cols / chunk_cols), (cuuint64_t)t.nb};
+  cuuint64_t strides[3] = {(cuuint64_t)(t.ld * es), (cuuint64_t)(chunk_cols * es),
+                           (cuuint64_t)(t.stride * es)};
+  cuuint32_t box[4] = {chunk_cols, box_rows, nchunks, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(map,
+                  t.dtype == OUO_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                      : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                  4, t.p, dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return set_error(OUO_ERR_CUDA, "cuTensorMapEncodeTiled (4-D) failed (%d)", (int)r);
+  return OUO_OK;
+}
+
 int64_t tiles_per_matrix(const GemmDesc& g, int BN, int TR) {
   const int64_t tm = ceil_div(g.M, (int64_t)TR), tn = ceil_div(g.N, BN);
   if (!g.tri) return tm * tn;
@@ -958,11 +992,20 @@ int launch(const std::vector<GemmDesc>& gs, cudaStream_t stream, int* status) {
     Segment proto;
     memset(&proto, 0, sizeof(proto));
     OUO_TRY(make_map(&proto.tmA, g.A, bk, kTileM));
+    const CUtensorMapSwizzle mn_swz =
+        FMT == 2 ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B : CU_TENSOR_MAP_SWIZZLE_128B;
+    // one 4-D load per stage when the columns split into whole chunks (a
+    // partial last chunk would be zero-filled whole by the chunk dimension)
+    // (OUO_TMA_4D=0 keeps the per-chunk loads)
+    const char* env4 = getenv("OUO_TMA_4D");
+    const bool b4d = B_MN && CG == 1 && g.N % (kRowBytes / es) == 0 &&
+                     !(env4 && env4[0] == '0');
     if (!B_MN) OUO_TRY(make_map(&proto.tmB, g.B, bk, C::kBRows));
-    else OUO_TRY(make_map(&proto.tmB, g.B, kRowBytes / es, bk,
-                          FMT == 2 ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B
-                                   : CU_TENSOR_MAP_SWIZZLE_128B));
+    else if (b4d) OUO_TRY(make_map4(&proto.tmB, g.B, kRowBytes / es, bk,
+                                    C::kBRows / (kRowBytes / es), mn_swz));
+    else OUO_TRY(make_map(&proto.tmB, g.B, kRowBytes / es, bk, mn_swz));
     proto.M = g.M; proto.N = g.N; proto.K = g.K;
+    proto.b4d = b4d ? 1 : 0;
     proto.tiles_n = ceil_div(g.N, BN);
     proto.tiles_per_mat = tiles_per_matrix(g, BN, TR);
     proto.C0 = (g.has_c0 && !g.c0_from_out) ? g.C0.p : nullptr;

@@ -176,7 +176,24 @@ gather_kernel(const __grid_constant__ GatherArgs a) {
     const int64_t n4 = a.vec[lo] ? (n >> 2) : 0;
     if (a.x0_bf16) {
       uint16_t* x = reinterpret_cast<uint16_t*>(a.X0[lo]) + j * a.ldx[lo];
-      for (int64_t q = lane; q < n4; q += 32) {
+      int64_t q = lane;
+      // four 16-byte vectors in flight per lane
+      for (; q + 96 < n4; q += 128) {
+        float4 v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) v[u] = *reinterpret_cast<const float4*>(b + 4 * (q + 32 * u));
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          uint2 o;
+          o.x = pack_bf16x2(v[u].x * s, v[u].y * s);
+          o.y = pack_bf16x2(v[u].z * s, v[u].w * s);
+          *reinterpret_cast<uint2*>(x + 4 * (q + 32 * u)) = o;
+          if (a.ef)
+            *reinterpret_cast<float4*>(b + 4 * (q + 32 * u)) =
+                make_float4(a.mu * v[u].x, a.mu * v[u].y, a.mu * v[u].z, a.mu * v[u].w);
+        }
+      }
+      for (; q < n4; q += 32) {
         float4 v = *reinterpret_cast<const float4*>(b + 4 * q);
         uint2 o;
         o.x = pack_bf16x2(v.x * s, v.y * s);
@@ -194,7 +211,21 @@ gather_kernel(const __grid_constant__ GatherArgs a) {
       }
     } else {
       float* x = reinterpret_cast<float*>(a.X0[lo]) + j * a.ldx[lo];
-      for (int64_t q = lane; q < n4; q += 32) {
+      int64_t q = lane;
+      for (; q + 96 < n4; q += 128) {
+        float4 v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) v[u] = *reinterpret_cast<const float4*>(b + 4 * (q + 32 * u));
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          *reinterpret_cast<float4*>(x + 4 * (q + 32 * u)) =
+              make_float4(v[u].x * s, v[u].y * s, v[u].z * s, v[u].w * s);
+          if (a.ef)
+            *reinterpret_cast<float4*>(b + 4 * (q + 32 * u)) =
+                make_float4(a.mu * v[u].x, a.mu * v[u].y, a.mu * v[u].z, a.mu * v[u].w);
+        }
+      }
+      for (; q < n4; q += 32) {
         float4 v = *reinterpret_cast<const float4*>(b + 4 * q);
         *reinterpret_cast<float4*>(x + 4 * q) =
             make_float4(v.x * s, v.y * s, v.z * s, v.w * s);
@@ -285,7 +316,23 @@ apply_kernel(const __grid_constant__ ApplyArgs a) {
     char* w = reinterpret_cast<char*>(a.W[lo]) + r * a.ldw[lo] * (a.w_bf16 ? 2 : 4);
     const char* o = reinterpret_cast<const char*>(a.O[lo]) + j * a.ldo[lo] * (a.o_bf16 ? 2 : 4);
     const int64_t n4 = a.vec[lo] ? (n >> 2) : 0;
-    for (int64_t q = lane; q < n4; q += 32) {
+    int64_t q = lane;
+    // four vectors of W and of O in flight per lane
+    for (; q + 96 < n4; q += 128) {
+      float wv[4][4], ov[4][4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        load4(w, 4 * (q + 32 * u), a.w_bf16, wv[u]);
+        load4(o, 4 * (q + 32 * u), a.o_bf16, ov[u]);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+#pragma unroll
+        for (int t = 0; t < 4; ++t) wv[u][t] = __fmaf_rn(-lrs, ov[u][t], a.decay * wv[u][t]);
+        store4(w, 4 * (q + 32 * u), a.w_bf16, wv[u]);
+      }
+    }
+    for (; q < n4; q += 32) {
       float wv[4], ov[4];
       load4(w, 4 * q, a.w_bf16, wv);
       load4(o, 4 * q, a.o_bf16, ov);
