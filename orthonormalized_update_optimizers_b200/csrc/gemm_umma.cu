@@ -80,6 +80,12 @@ struct Segment {
   int direct;  // outputs go to dptr[dbase + b]
   int dbase;
   int b4d;  // MN-major B: tmB is 4-D, one TMA load brings every chunk of a stage
+  // upper-stored symmetric operands: maps of the same matrices read with
+  // rows and columns exchanged (MN-major tiles; 4-D when the matrix splits
+  // into whole 32-column chunks, else one 3-D load per chunk)
+  CUtensorMap tmAt;
+  CUtensorMap tmBt;
+  int t4d;
 };
 
 constexpr int kMaxSeg = 6;
@@ -92,6 +98,7 @@ struct UmmaArgs {
   float alpha, beta, gamma;
   int has_c0, c0_bf16, has_f32, round_tf32, has_bf16;
   int c0_out;  // C0 is read from the (direct) output itself
+  int a_sym, b_sym, c0_upper, sym_half;  // upper-stored symmetric matrices
   int tma_out;  // single workspace output written by TMA stores
   int* status;
   void* dptr[kChunk];
@@ -287,6 +294,8 @@ umma_gemm_kernel(const __grid_constant__ UmmaArgs a) {
   uint64_t* drain = tempty + 2;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  // per stage: bit 0 = A tile MN-major (transposed block), bit 1 = B tile
+  volatile uint32_t* stage_fmt = reinterpret_cast<volatile uint32_t*>(tmem_holder + 2);
   // per-warp 4 KB staging buffers, 1024-byte aligned (the TMA swizzle
   // patterns are computed from absolute shared-memory address bits)
   float* epi_smem = reinterpret_cast<float*>(smem + C::kStages * C::kStageBytes);
@@ -349,6 +358,13 @@ umma_gemm_kernel(const __grid_constant__ UmmaArgs a) {
           ok = false;
           break;
         }
+        // Upper-stored symmetric operands: a K stage left of the tile's block
+        // diagonal (256-wide blocks, pair tiles) comes from the transposed
+        // block.  Both CTAs of a pair take the same decision.
+        const int64_t cblk = (kb * (int64_t)kBK) / 256;
+        const bool at = CG == 2 && a.a_sym && cblk < ti;
+        const bool bt = CG == 2 && a.b_sym && cblk < tj;
+        if (rank == 0) stage_fmt[stage] = (at ? 1u : 0u) | (bt ? 2u : 0u);
         // the stage barrier of the pair's even CTA counts both CTAs' bytes
         if (rank == 0) ptx::mbar_arrive_expect_tx(&full[stage], CG * C::kStageBytes);
         const uint32_t fb = CG == 2 ? ptx::mapa(ptx::smem_u32(&full[stage]), 0) : 0u;
@@ -358,8 +374,24 @@ umma_gemm_kernel(const __grid_constant__ UmmaArgs a) {
         };
         uint8_t* sa = smem + stage * C::kStageBytes;
         uint8_t* sb = sa + C::kABytes;
-        load(sa, &sg.tmA, (int32_t)(kb * kBK), arow);
-        if (!B_MN) {
+        // transposed tile: rows = this K stage, columns = the tile's 128
+        // rows (M or N), as 32-column MN-major chunks
+        auto load_t = [&](uint8_t* dst, const CUtensorMap* m, int32_t col0) {
+          if (CG == 2) {
+            if (sg.t4d) {
+              ptx::tma_load_4d_pair(dst, m, fb, 0, (int32_t)(kb * kBK), col0 / 32, z);
+            } else {
+#pragma unroll
+              for (uint32_t c = 0; c < kTileM / 32; ++c)
+                load(dst + c * kChunkBytes, m, col0 + (int32_t)(c * 32), (int32_t)(kb * kBK));
+            }
+          }
+        };
+        if (at) load_t(sa, &sg.tmAt, arow);
+        else load(sa, &sg.tmA, (int32_t)(kb * kBK), arow);
+        if (bt) {
+          load_t(sb, &sg.tmBt, bcol);
+        } else if (!B_MN) {
           load(sb, &sg.tmB, (int32_t)(kb * kBK), bcol);
         } else if (CG == 1 && sg.b4d) {
           // (chunk column, K row, chunk, matrix): the chunks land back to
@@ -421,23 +453,29 @@ umma_gemm_kernel(const __grid_constant__ UmmaArgs a) {
         ptx::tc_fence_after();
         const uint32_t sa = ptx::smem_u32(smem + stage * C::kStageBytes);
         const uint32_t sb = sa + C::kABytes;
+        const uint32_t fmt = stage_fmt[stage];
+        const bool a_mn = (fmt & 1u) != 0;
+        const bool b_mn = B_MN || (fmt & 2u) != 0;
+        const uint32_t idesc = kIdesc | (a_mn ? (1u << 15) : 0u) | (b_mn ? (1u << 16) : 0u);
+        // MN-major tiles: chunks of one 128-byte row across kBK K rows; tf32
+        // takes the 32-byte-atom swizzle (4-row groups)
+        auto mn_desc = [&](uint32_t base, uint32_t kk) {
+          return FMT == 2 ? ptx::smem_desc_sw128_32b(base + kk * kInstK * kRowBytes,
+                                                     kChunkBytes, 512)
+                          : ptx::smem_desc_sw128(base + kk * kInstK * kRowBytes,
+                                                 kChunkBytes, 1024);
+        };
 #pragma unroll
         for (uint32_t kk = 0; kk < kBK / kInstK; ++kk) {
-          const uint64_t ad = ptx::smem_desc_sw128(sa + kk * 32, 16, 1024);
-          // MN-major tf32 takes the 32-byte-atom swizzle (4-row groups)
-          const uint64_t bd =
-              B_MN ? (FMT == 2 ? ptx::smem_desc_sw128_32b(sb + kk * kInstK * kRowBytes,
-                                                          kChunkBytes, 512)
-                               : ptx::smem_desc_sw128(sb + kk * kInstK * kRowBytes,
-                                                      kChunkBytes, 1024))
-                   : ptx::smem_desc_sw128(sb + kk * 32, 16, 1024);
+          const uint64_t ad = a_mn ? mn_desc(sa, kk) : ptx::smem_desc_sw128(sa + kk * 32, 16, 1024);
+          const uint64_t bd = b_mn ? mn_desc(sb, kk) : ptx::smem_desc_sw128(sb + kk * 32, 16, 1024);
           const uint32_t acc = (kb > 0 || kk > 0) ? 1u : 0u;
           if (CG == 2) {
-            if (FMT == 1) ptx::mma2_bf16(d, ad, bd, kIdesc, acc);
-            else ptx::mma2_tf32(d, ad, bd, kIdesc, acc);
+            if (FMT == 1) ptx::mma2_bf16(d, ad, bd, idesc, acc);
+            else ptx::mma2_tf32(d, ad, bd, idesc, acc);
           } else {
-            if (FMT == 1) ptx::mma_bf16(d, ad, bd, kIdesc, acc);
-            else ptx::mma_tf32(d, ad, bd, kIdesc, acc);
+            if (FMT == 1) ptx::mma_bf16(d, ad, bd, idesc, acc);
+            else ptx::mma_tf32(d, ad, bd, idesc, acc);
           }
         }
         // frees the stage in both CTAs of a pair
@@ -524,7 +562,7 @@ umma_gemm_kernel(const __grid_constant__ UmmaArgs a) {
           for (int j = 0; j < 32; ++j) v[j] *= a.alpha;
           if (a.has_c0) {
             float c0v[32];
-            if (a.tri) {
+            if (a.tri && !a.c0_upper) {
               const int64_t gic = gi < sg.M ? gi : sg.M - 1;
 #pragma unroll
               for (int j = 0; j < 32; ++j) {
@@ -587,7 +625,8 @@ umma_gemm_kernel(const __grid_constant__ UmmaArgs a) {
             ptx::bulk_commit();
           }
           ++nstores;
-          if (a.tri && !diag) {
+          // upper-stored outputs: only tiles on the block diagonal mirror
+          if (a.tri && !diag && !(a.sym_half && tj != ti)) {
             next_stg();
             if (!obf) {
 #pragma unroll
@@ -639,13 +678,15 @@ umma_gemm_kernel(const __grid_constant__ UmmaArgs a) {
         if (a.tri) {
           if (a.has_c0) {
             // 32 independent loads (clamped into the matrix, so they can be
-            // issued together), used only where the element is kept
+            // issued together), used only where the element is kept; an
+            // upper-stored C0 is read at (i, j), otherwise at (j, i)
             const int64_t gic = gi < sg.M ? gi : sg.M - 1;
             float c0v[32];
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
               const int64_t gjc = gj0 + j < sg.N ? gj0 + j : sg.N - 1;
-              c0v[j] = load_c0(sg, b, gjc, gic, a.c0_bf16);
+              c0v[j] = a.c0_upper ? load_c0(sg, b, gic, gjc, a.c0_bf16)
+                                  : load_c0(sg, b, gjc, gic, a.c0_bf16);
             }
 #pragma unroll
             for (int j = 0; j < 32; ++j) v[j] = a.alpha * v[j] + a.beta * c0v[j];
@@ -713,7 +754,7 @@ umma_gemm_kernel(const __grid_constant__ UmmaArgs a) {
           if (mask) store4t(a, to, gr, gc, w, mask);
         }
         __syncwarp();
-        if (a.tri) {
+        if (a.tri && !(a.sym_half && tj != ti)) {
           // mirrored tile: stage transposed [col][row], store row gj
 #pragma unroll
           for (int j = 0; j < 32; ++j) stg[stg_idx(j, lane)] = v[j];
@@ -943,6 +984,12 @@ int launch(const std::vector<GemmDesc>& gs, cudaStream_t stream, int* status) {
   }
   // single workspace output: TMA-store epilogue
   a.tma_out = (g0.direct.empty() && (g0.has_f32 != g0.has_bf16)) ? 1 : 0;
+  a.a_sym = g0.a_sym; a.b_sym = g0.b_sym;
+  a.c0_upper = g0.c0_upper; a.sym_half = g0.sym_half;
+  if ((a.a_sym || a.b_sym) && !(CG == 2 && FMT == 2 && !B_MN))
+    return set_error(OUO_ERR_INVALID_ARG, "upper-stored operands need tf32 K-major pair tiles");
+  if ((a.sym_half || a.c0_upper) && CG != 2)
+    return set_error(OUO_ERR_INVALID_ARG, "upper-stored symmetric outputs need pair tiles");
   int ndirect = 0;
   auto flush = [&]() -> int {
     if (a.nseg == 0) return OUO_OK;
@@ -1006,6 +1053,19 @@ int launch(const std::vector<GemmDesc>& gs, cudaStream_t stream, int* status) {
     else OUO_TRY(make_map(&proto.tmB, g.B, kRowBytes / es, bk, mn_swz));
     proto.M = g.M; proto.N = g.N; proto.K = g.K;
     proto.b4d = b4d ? 1 : 0;
+    if (g.a_sym || g.b_sym) {
+      // the same matrices read transposed, as 32-column MN-major chunks
+      constexpr uint32_t cc = kRowBytes / 4;  // tf32 chunk columns
+      proto.t4d = g.K % cc == 0 ? 1 : 0;
+      const Buf* ops[2] = {&g.A, &g.B};
+      CUtensorMap* maps[2] = {&proto.tmAt, &proto.tmBt};
+      const bool want[2] = {g.a_sym, g.b_sym};
+      for (int q = 0; q < 2; ++q) {
+        if (!want[q]) continue;
+        if (proto.t4d) OUO_TRY(make_map4(maps[q], *ops[q], cc, bk, kTileM / cc, mn_swz));
+        else OUO_TRY(make_map(maps[q], *ops[q], cc, bk, mn_swz));
+      }
+    }
     proto.tiles_n = ceil_div(g.N, BN);
     proto.tiles_per_mat = tiles_per_matrix(g, BN, TR);
     proto.C0 = (g.has_c0 && !g.c0_from_out) ? g.C0.p : nullptr;
@@ -1081,6 +1141,13 @@ int gemm_timing_read(int kind, int* launches, double* total_ms, double* flops) {
   return OUO_OK;
 }
 
+int cta_pair_mode() {
+  const char* env = getenv("OUO_CTA_PAIR");
+  return env && env[0] >= '0' && env[0] <= '2' ? env[0] - '0' : 1;
+}
+
+bool cta_pairs_enabled() { return cta_pair_mode() > 0; }
+
 int gemm_umma_grouped(const std::vector<GemmDesc>& gs, cudaStream_t stream,
                       int* status) {
   if (gs.empty()) return OUO_OK;
@@ -1092,7 +1159,8 @@ int gemm_umma_grouped(const std::vector<GemmDesc>& gs, cudaStream_t stream,
     if (g.tri != g0.tri || g.b_mn != g0.b_mn || g.has_c0 != g0.has_c0 ||
         g.has_f32 != g0.has_f32 || g.has_bf16 != g0.has_bf16 ||
         g.round_tf32 != g0.round_tf32 || g.direct.empty() != g0.direct.empty() ||
-        g.c0_from_out != g0.c0_from_out ||
+        g.c0_from_out != g0.c0_from_out || g.sym_half != g0.sym_half ||
+        g.a_sym != g0.a_sym || g.b_sym != g0.b_sym || g.c0_upper != g0.c0_upper ||
         g.alpha != g0.alpha || g.beta != g0.beta || g.gamma != g0.gamma ||
         (g.has_c0 && g.C0.dtype != g0.C0.dtype) ||
         (!g.direct.empty() && g.direct_dtype != g0.direct_dtype))
@@ -1109,8 +1177,7 @@ int gemm_umma_grouped(const std::vector<GemmDesc>& gs, cudaStream_t stream,
   // CTA pairs (256 x 256 tiles) for wide outputs with more than 128 rows and
   // K-major B.  OUO_CTA_PAIR=0 selects single-CTA 128 x BN tiles throughout;
   // OUO_CTA_PAIR=2 also puts MN-major B (Q X) on pairs.
-  const char* env = getenv("OUO_CTA_PAIR");
-  const int pair_mode = env && env[0] >= '0' && env[0] <= '2' ? env[0] - '0' : 1;
+  const int pair_mode = cta_pair_mode();
   const bool pair = wide && tall && pair_mode > 0 && (!g0.b_mn || pair_mode == 2);
   if (g0.A.dtype == OUO_BF16) {
     if (g0.b_mn) {

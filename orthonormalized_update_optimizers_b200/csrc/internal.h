@@ -86,7 +86,22 @@ struct GemmDesc {
   // With direct outputs: C0 is the output matrix itself (in-place update
   // out = alpha * A op(B) + beta * out).  Non-symmetric outputs only.
   bool c0_from_out = false;
+  // Half-stored symmetric matrices (tf32 / bf16 tensor-core path, CTA-pair
+  // tiles).  A symmetric matrix is "upper-stored" when every 256 x 256 block
+  // on or above the block diagonal holds its values (diagonal blocks in
+  // full) and the blocks below may hold anything.
+  //   sym_half:  the symmetric output is written upper-stored (off-diagonal
+  //              tiles are not mirrored);
+  //   a_sym / b_sym: A / B (K-major, symmetric) are upper-stored: K blocks
+  //              left of the diagonal are read from the transposed block;
+  //   c0_upper:  the symmetric C0 is upper-stored (read at (i, j), j >= i).
+  bool sym_half = false, a_sym = false, b_sym = false, c0_upper = false;
 };
+
+// Whether K-major tensor-core GEMMs with more than 128 output rows and
+// columns run on CTA-pair tiles (OUO_CTA_PAIR, default on); upper-stored
+// symmetric matrices need them.
+bool cta_pairs_enabled();
 
 // Tensor-core GEMM (tcgen05 / TMEM / TMA).  A and B are both bf16
 // (kind::f16) or both fp32 read as tf32 (kind::tf32).

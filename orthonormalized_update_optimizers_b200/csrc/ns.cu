@@ -23,6 +23,8 @@
 #include <algorithm>
 #include <cmath>
 
+#include <cstdlib>
+
 #include "internal.h"
 
 namespace ouo {
@@ -166,8 +168,41 @@ int free_idx(int a, int b) {
 
 // One stage of the iteration over all groups: a single grouped tensor-core
 // launch (bf16 path) or one CUDA-core GEMM per group (fp32 path).
+// Upper-stored symmetric k x k matrices (tensor-core path on CTA-pair
+// tiles): Gram matrices and symmetric products skip the mirrored write of
+// tiles off the block diagonal, and every symmetric fp32 k x k operand (and
+// symmetric C0) is read through its upper blocks.  A product that also
+// writes a bf16 copy (the Q of Q X, read whole as a dense operand) keeps
+// full storage.  Used when the launches run on pair tiles: the bf16 path,
+// pairs enabled, and some k above 128 (so every symmetric launch of the
+// call, which covers all groups, takes pairs).
+// OUO_SYM_HALF=0 keeps full storage.
+bool half_mode(const std::vector<GroupWs>& ws, bool bf) {
+  if (!bf || !cta_pairs_enabled()) return false;
+  const char* env = getenv("OUO_SYM_HALF");
+  if (env && env[0] == '0') return false;
+  for (const GroupWs& w : ws)
+    if (w.A.rows > 128) return true;
+  return false;
+}
+
+void mark_half(std::vector<GemmDesc>& ds, bool half) {
+  if (!half) return;
+  for (GemmDesc& d : ds) {
+    if (!d.tri) continue;
+    d.sym_half = !d.has_bf16;
+    if (d.A.dtype == OUO_F32 && d.A.rows == d.A.cols) d.a_sym = d.b_sym = true;
+    if (d.has_c0) d.c0_upper = true;
+  }
+}
+
 int run_stage(const std::vector<GemmDesc>& ds, bool bf, cudaStream_t s,
-              int* status) {
+              int* status, bool half = false) {
+  if (bf && half) {
+    std::vector<GemmDesc> hd = ds;
+    mark_half(hd, true);
+    return gemm_umma_grouped(hd, s, status);
+  }
   if (bf) return gemm_umma_grouped(ds, s, status);
   for (const GemmDesc& d : ds) OUO_TRY(gemm_simt(d, s));
   return OUO_OK;
@@ -202,6 +237,7 @@ void final_output(GemmDesc& d, const Plan& pl, size_t i, bool bf) {
 // Gram Newton-Schulz, all groups in lockstep (they share the schedule).
 int gram_all(const ouo_ns_params& p, Plan& pl, cudaStream_t s, int* status) {
   const bool bf = p.precision == OUO_PREC_BF16;
+  const bool half = half_mode(pl.ws, bf);
   const Coeffs c = scaled(p);
   const size_t ng = pl.ws.size();
   int xi = 0;  // current X is x0 (0) or x1 (1)
@@ -209,7 +245,7 @@ int gram_all(const ouo_ns_params& p, Plan& pl, cudaStream_t s, int* status) {
   auto Xa = [&](GroupWs& w) -> Buf& { return xi ? w.x0 : w.x1; };
   std::vector<GemmDesc> ds(ng);
   for (size_t i = 0; i < ng; ++i) ds[i] = syrk(Xc(pl.ws[i]), pl.ws[i].A, bf);
-  OUO_TRY(run_stage(ds, bf, s, status));
+  OUO_TRY(run_stage(ds, bf, s, status, half));
   int q = -1;  // buffer holding Q; -1 while Q = I
   for (int t = 1; t <= p.iters; ++t) {
     const bool last = t == p.iters;
@@ -227,7 +263,7 @@ int gram_all(const ouo_ns_params& p, Plan& pl, cudaStream_t s, int* status) {
         ds[i].has_bf16 = true;
       }
     }
-    OUO_TRY(run_stage(ds, bf, s, status));
+    OUO_TRY(run_stage(ds, bf, s, status, half));
     if (q < 0) {
       q = h;  // Q = H I
     } else {
@@ -242,7 +278,7 @@ int gram_all(const ouo_ns_params& p, Plan& pl, cudaStream_t s, int* status) {
           ds[i].has_bf16 = true;
         }
       }
-      OUO_TRY(run_stage(ds, bf, s, status));
+      OUO_TRY(run_stage(ds, bf, s, status, half));
       q = nq;
     }
     if (last) break;
@@ -251,10 +287,10 @@ int gram_all(const ouo_ns_params& p, Plan& pl, cudaStream_t s, int* status) {
         GroupWs& w = pl.ws[i];
         ds[i] = apply_left(bf ? w.qbf : w.kk[q], Xc(w), Xa(w), 1.f, nullptr, 0.f);
       }
-      OUO_TRY(run_stage(ds, bf, s, status));
+      OUO_TRY(run_stage(ds, bf, s, status, half));
       xi ^= 1;
       for (size_t i = 0; i < ng; ++i) ds[i] = syrk(Xc(pl.ws[i]), pl.ws[i].A, bf);
-      OUO_TRY(run_stage(ds, bf, s, status));
+      OUO_TRY(run_stage(ds, bf, s, status, half));
       q = -1;
     } else {
       // A <- H (H A)
@@ -264,14 +300,14 @@ int gram_all(const ouo_ns_params& p, Plan& pl, cudaStream_t s, int* status) {
         ds[i].out_f32 = w.T;
         ds[i].has_f32 = true;
       }
-      OUO_TRY(run_stage(ds, bf, s, status));
+      OUO_TRY(run_stage(ds, bf, s, status, half));
       for (size_t i = 0; i < ng; ++i) {
         GroupWs& w = pl.ws[i];
         ds[i] = symprod(w.kk[h], w.T, 1.f, nullptr, 0.f, 0.f, bf);
         ds[i].out_f32 = w.A;
         ds[i].has_f32 = true;
       }
-      OUO_TRY(run_stage(ds, bf, s, status));
+      OUO_TRY(run_stage(ds, bf, s, status, half));
     }
   }
   if (q < 0) {
@@ -294,6 +330,7 @@ int gram_all(const ouo_ns_params& p, Plan& pl, cudaStream_t s, int* status) {
 // Standard quintic Newton-Schulz, all groups in lockstep.
 int std_all(const ouo_ns_params& p, Plan& pl, cudaStream_t s, int* status) {
   const bool bf = p.precision == OUO_PREC_BF16;
+  const bool half = half_mode(pl.ws, bf);
   const Coeffs c = scaled(p);
   const size_t ng = pl.ws.size();
   int xi = 0;
@@ -302,7 +339,7 @@ int std_all(const ouo_ns_params& p, Plan& pl, cudaStream_t s, int* status) {
   std::vector<GemmDesc> ds(ng);
   for (int t = 1; t <= p.iters; ++t) {
     for (size_t i = 0; i < ng; ++i) ds[i] = syrk(Xc(pl.ws[i]), pl.ws[i].A, bf);
-    OUO_TRY(run_stage(ds, bf, s, status));
+    OUO_TRY(run_stage(ds, bf, s, status, half));
     // B = c' A A + b' A
     for (size_t i = 0; i < ng; ++i) {
       GroupWs& w = pl.ws[i];
@@ -316,7 +353,7 @@ int std_all(const ouo_ns_params& p, Plan& pl, cudaStream_t s, int* status) {
         ds[i].has_f32 = true;
       }
     }
-    OUO_TRY(run_stage(ds, bf, s, status));
+    OUO_TRY(run_stage(ds, bf, s, status, half));
     // X <- a' X + B X   (the last iteration writes the output)
     const bool last = t == p.iters;
     for (size_t i = 0; i < ng; ++i) {
