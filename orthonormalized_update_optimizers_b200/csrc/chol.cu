@@ -24,6 +24,7 @@
 // passes at once).  A non-positive pivot restarts the factorization once
 // with the shift of shifted CholeskyQR, 11 (L r + r (r + 1)) u tr(S); a second
 // failure sets OUO_STATUS_BREAKDOWN and returns L^-1 = I.
+#include <atomic>
 #include <cmath>
 
 #include "internal.h"
@@ -80,13 +81,6 @@ __device__ __forceinline__ void load_blk(float (*t)[kNb + 1], const float* g, in
   for (int e = threadIdx.x; e < kNb * kNb; e += blockDim.x) {
     const int i = e >> 5, j = e & 31;
     t[i][j] = g[(size_t)i * R + j];
-  }
-}
-
-__device__ __forceinline__ void store_blk(float* g, int R, float (*t)[kNb + 1]) {
-  for (int e = threadIdx.x; e < kNb * kNb; e += blockDim.x) {
-    const int i = e >> 5, j = e & 31;
-    g[(size_t)i * R + j] = t[i][j];
   }
 }
 
@@ -403,22 +397,23 @@ int chol_blocked(const float* part, int splits, int r, int64_t L, float* S,
   OUO_CHECK_CUDA(cudaMemsetAsync(ctl, 0, 64, stream));
   // every CTA must be resident at once: at most one per SM times the
   // occupancy, and no more than the widest phase needs
-  static int per_sm[64] = {0};
+  static std::atomic<int> per_sm[64];  // zero-initialized (static storage)
   int dev = 0;
   OUO_CHECK_CUDA(cudaGetDevice(&dev));
   if (dev < 0 || dev >= 64)
     return set_error(OUO_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
-  if (!per_sm[dev]) {
-    int n = 0;
+  int resident = per_sm[dev].load(std::memory_order_relaxed);
+  if (!resident) {
     OUO_CHECK_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(
-        &n, chol_blocked_kernel, kCholThreads, 0));
-    if (n < 1) return set_error(OUO_ERR_UNSUPPORTED, "blocked Cholesky kernel does not fit");
-    per_sm[dev] = n;
+        &resident, chol_blocked_kernel, kCholThreads, 0));
+    if (resident < 1)
+      return set_error(OUO_ERR_UNSUPPORTED, "blocked Cholesky kernel does not fit");
+    per_sm[dev].store(resident, std::memory_order_relaxed);
   }
   const int m = a.nblk - 1;
   int want = m * (m + 1) / 2;
   if (want < 1) want = 1;
-  int grid = num_sms() * (per_sm[dev] < 2 ? per_sm[dev] : 2);
+  int grid = num_sms() * (resident < 2 ? resident : 2);
   if (grid > want) grid = want;
   void* args[] = {&a};
   OUO_CHECK_CUDA(cudaLaunchCooperativeKernel((const void*)chol_blocked_kernel,

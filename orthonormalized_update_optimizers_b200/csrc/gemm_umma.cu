@@ -809,7 +809,7 @@ umma_gemm_kernel(const __grid_constant__ UmmaArgs a) {
 // CUDA events on its stream and its algorithmic flops (symmetric outputs:
 // the upper triangle only) are recorded per kernel kind.  Events come from a
 // pool created when timing is switched on.
-constexpr int kTimingKinds = 8;  // (tri ? 4 : 0) + (tf32 ? 2 : 0) + b_mn
+// kinds: (tri ? 4 : 0) + (tf32 ? 2 : 0) + b_mn
 constexpr int kTimingMax = 4096;
 struct TimingRec {
   cudaEvent_t e0, e1;
@@ -942,13 +942,16 @@ int launch(const std::vector<GemmDesc>& gs, cudaStream_t stream, int* status) {
   // per device: shared-memory opt-in done, and how many CTAs (pairs: CTA
   // pairs) of this kernel can be resident at once -- a persistent grid
   // larger than that would run its last CTAs after the others finish
-  static bool configured[64] = {false};
-  static int resident[64] = {0};
+  static std::mutex setup_mu;
+  static int resident[64] = {0};  // 0: not yet set up on that device
   int dev = 0;
   OUO_CHECK_CUDA(cudaGetDevice(&dev));
   if (dev < 0 || dev >= 64)
     return set_error(OUO_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
-  if (!configured[dev]) {
+  int cap_slots = 0;
+  {
+  std::lock_guard<std::mutex> setup_lock(setup_mu);
+  if (!resident[dev]) {
     OUO_CHECK_CUDA(cudaFuncSetAttribute(
         kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::kSmem));
     int n = num_sms();
@@ -963,7 +966,8 @@ int launch(const std::vector<GemmDesc>& gs, cudaStream_t stream, int* status) {
       n = clusters;
     }
     resident[dev] = n;
-    configured[dev] = true;
+  }
+  cap_slots = resident[dev];
   }
   const GemmDesc& g0 = gs[0];
   UmmaArgs a;
@@ -999,7 +1003,7 @@ int launch(const std::vector<GemmDesc>& gs, cudaStream_t stream, int* status) {
       a.total_tiles += a.seg[s].tiles_per_mat * a.seg[s].nb;
     }
     // one CTA (or CTA pair) per resident slot, at most one per tile
-    const int64_t slots = a.total_tiles < resident[dev] ? a.total_tiles : resident[dev];
+    const int64_t slots = a.total_tiles < cap_slots ? a.total_tiles : cap_slots;
     if (slots >= 1) {
       TimingRec rec;
       bool timed = false;

@@ -88,10 +88,6 @@ GroupWs carve(Arena& ar, const Group& g, const Oriented& o, bool gram,
   return w;
 }
 
-int run_gemm(const GemmDesc& d, bool bf, cudaStream_t s, int* status) {
-  return bf ? gemm_umma(d, s, status) : gemm_simt(d, s);
-}
-
 GemmDesc syrk(const Buf& X, const Buf& out, bool bf) {
   GemmDesc d;
   d.M = d.N = X.rows;
