@@ -208,3 +208,26 @@ def test_single_cta_and_cta_pair_tiles_agree(gram, monkeypatch):
                 assert rel_fro(to64(outs[mode][i]), ref) <= TOL_BF16
         assert rel_fro(to64(outs["1"][i]), to64(outs["0"][i])) <= 1e-2
         assert rel_fro(to64(outs["2"][i]), to64(outs["0"][i])) <= 1e-2
+
+
+@pytest.mark.parametrize("gram", [True, False])
+def test_upper_stored_symmetric_matrices_change_no_bits(gram, monkeypatch):
+    # Upper-stored k x k matrices (the default on pair tiles) read the lower
+    # blocks as the transposed upper blocks -- the very values full storage
+    # mirrors there -- so the result must be bit-identical to full storage
+    # (OUO_SYM_HALF=0).  k = 300 takes the per-chunk transposed loads, k = 512
+    # the 4-D ones.
+    shapes = [(300, 1000), (512, 2048), (1792, 4096)]
+    Xs = [_inputs(s, torch.bfloat16, 90 + i) for i, s in enumerate(shapes)]
+    fn = ouo.gram_ns_orthogonalize if gram else ouo.ns_orthogonalize
+    outs = {}
+    for mode in ("1", "0"):
+        monkeypatch.setenv("OUO_SYM_HALF", mode)
+        Os = [torch.empty_like(x) for x in Xs]
+        fn(Xs, Os, ouo.ns_params())
+        torch.cuda.synchronize()
+        outs[mode] = Os
+    for i, x in enumerate(Xs):
+        assert torch.equal(outs["1"][i], outs["0"][i]), shapes[i]
+    ref = _oracle(to64(Xs[0]), gram)
+    assert rel_fro(to64(outs["1"][0]), ref) <= TOL_BF16
