@@ -353,17 +353,30 @@ struct DionWs {
   Buf ctl;      // barrier counter and flags of the blocked Cholesky
 };
 
-// Ranks from this one up use the blocked multi-CTA Cholesky; the one-CTA
-// kernel keeps smaller ones (measured on 4096 x 4096: equal at r = 64, the
-// blocked kernel 8-23% faster per Dion step from r = 96).
-// OUO_CHOL_BLOCKED_MIN_RANK overrides the threshold (1 to 129).
+// Ranks from blocked_chol_min_rank() up take a blocked Cholesky: the
+// one-CTA kernel with the blocks in shared memory up to
+// smem_chol_max_rank(), the cooperative multi-CTA kernel above it; smaller
+// ranks keep the one-CTA packed-triangle kernel.  Per 4096 x 4096
+// Orth-Dion step the one-CTA blocked kernel is 5-11% faster than the
+// better of the other two from r = 64 to 128, even at r = 192 and 11%
+// slower at r = 256, where the cooperative kernel's wider phases win.
+// OUO_CHOL_BLOCKED_MIN_RANK (1 to 129) and OUO_CHOL_SMEM_MAX_RANK (0 to
+// 256; 0 turns the one-CTA blocked kernel off) override the two bounds.
 int blocked_chol_min_rank() {
   const char* env = getenv("OUO_CHOL_BLOCKED_MIN_RANK");
   if (env) {
     const int v = atoi(env);
     if (v >= 1 && v <= 129) return v;
   }
-  return 65;
+  return 64;
+}
+int smem_chol_max_rank() {
+  const char* env = getenv("OUO_CHOL_SMEM_MAX_RANK");
+  if (env) {
+    const int v = atoi(env);
+    if (v >= 0 && v <= 256) return v;
+  }
+  return 192;
 }
 int64_t padded_rank(int r) { return ceil_div(r, 32) * 32; }
 
@@ -415,11 +428,30 @@ int gram_parts(const Buf& X, const DionWs& w, cudaStream_t s, int* used) {
   return OUO_OK;
 }
 
+__global__ void sum_parts_kernel(const float* part, int splits, int64_t n, float* out) {
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n;
+       e += (int64_t)gridDim.x * blockDim.x) {
+    double s = 0.0;
+    for (int q = 0; q < splits; ++q) s += (double)part[(size_t)q * n + e];
+    out[e] = (float)s;
+  }
+}
+
 // w.Linv = L^-1 where L L^T = sum of `splits` r x r partials at `part`
 // (L_rows: the rows' length, for the shifted retry).
 int cholesky_inverse(const float* part, int splits, int r, int64_t L_rows,
                      const DionWs& w, int* status, cudaStream_t s) {
-  if (r >= blocked_chol_min_rank()) {
+  if (r >= blocked_chol_min_rank() && r <= smem_chol_max_rank() && chol_smem_fits(r)) {
+    if (splits > 1) {  // one wide pass sums the partials; the CTA reads S once
+      const int64_t n = (int64_t)r * r;
+      float* S = reinterpret_cast<float*>(w.S.p);
+      sum_parts_kernel<<<grid_1d(n, 256), 256, 0, s>>>(part, splits, n, S);
+      OUO_CHECK_LAUNCH();
+      part = S;
+      splits = 1;
+    }
+    OUO_TRY(chol_smem(part, splits, r, L_rows, reinterpret_cast<float*>(w.Linv.p), status, s));
+  } else if (r >= blocked_chol_min_rank()) {
     OUO_TRY(chol_blocked(part, splits, r, L_rows, reinterpret_cast<float*>(w.S.p),
                          reinterpret_cast<float*>(w.Linv.p), w.ctl.p, status, s));
   } else {
@@ -702,15 +734,6 @@ namespace {
 
 // out[e] = sum_p part[p][e] in float64, fixed order (the reduction the
 // Cholesky kernels apply to their partials), rounded to fp32.
-__global__ void sum_parts_kernel(const float* part, int splits, int64_t n, float* out) {
-  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n;
-       e += (int64_t)gridDim.x * blockDim.x) {
-    double s = 0.0;
-    for (int q = 0; q < splits; ++q) s += (double)part[(size_t)q * n + e];
-    out[e] = (float)s;
-  }
-}
-
 int64_t pitch4(int64_t n) { return ceil_div(n, 4) * 4; }
 
 // floats of matrix i's block of `red` (256-byte multiple)
