@@ -387,7 +387,7 @@ __global__ void __launch_bounds__(kCholThreads) chol_blocked_kernel(const CholBA
 // S_ij -= L_ip L_jp^T); the inverse is formed one block diagonal at a time,
 // X_ij = -D_i sum_{k=j}^{i-1} L_ik X_kj, from the blocks of X = L^-1
 // already written to the output.  Work items are (block, 8-column group):
-// lane = row, eight accumulators.
+// lane = row, eight accumulators.  S arrives summed (one r x r matrix).
 constexpr int kSmemMaxBlk = 8;
 constexpr int kSmemThreads = 512;
 constexpr int kSmemWarps = kSmemThreads / 32;
@@ -396,8 +396,7 @@ constexpr int kTileF = kNb * kP;  // floats per tile
 constexpr int kStageF = kNb * 9;  // per-warp 32 x 8 staging, pitch 9
 
 struct CholSArgs {
-  const float* part;  // [splits][r][r]
-  int splits;
+  const float* S;     // r x r (ld r), lower triangle read
   int r, R, nblk;
   int64_t L;          // row length of X (for the shift)
   float* Linv;        // R x R output (ld R), lower triangular
@@ -417,6 +416,15 @@ __device__ __forceinline__ int tri_row(int t) {
   while ((bi + 1) * (bi + 2) / 2 <= t) ++bi;
   while (bi * (bi + 1) / 2 > t) --bi;
   return bi;
+}
+
+__device__ __forceinline__ void cp_async4(float* dst_smem, const float* src) {
+  const unsigned d = (unsigned)__cvta_generic_to_shared(dst_smem);
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(d), "l"(src) : "memory");
+}
+
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_all;\n" ::: "memory");
 }
 
 __device__ __forceinline__ void load_row(const float* A, float (&row)[kNb]) {
@@ -468,10 +476,13 @@ __global__ void __launch_bounds__(kSmemThreads, 1) chol_smem_kernel(const CholSA
   float* pan = Dt + kTileF;                // L_ip of the current panel
   float* stg = pan + (size_t)(nb - 1) * kTileF + (size_t)warp * kStageF;
 
-  // blocks of X above the block diagonal are zero
-  for (int e = threadIdx.x; e < R * R; e += blockDim.x) {
-    const int i = e / R, j = e - (e / R) * R;
-    if ((j >> 5) > (i >> 5)) a.Linv[e] = 0.f;
+  // blocks of X above the block diagonal are zero: upper block (bj, bi) for
+  // each strictly lower (bi, bj), 256 float4 per block
+  for (int e = threadIdx.x; e < (nb * (nb - 1) / 2) * 256; e += blockDim.x) {
+    const int t = e >> 8, w = e & 255;
+    const int bi = tri_row(t) + 1, bj = t - bi * (bi - 1) / 2;
+    float* dst = a.Linv + (size_t)(bj * kNb + (w >> 3)) * R + bi * kNb + (w & 7) * 4;
+    *reinterpret_cast<float4*>(dst) = make_float4(0.f, 0.f, 0.f, 0.f);
   }
   bool ok = false;
   for (int attempt = 0; attempt < 2 && !ok; ++attempt) {
@@ -479,9 +490,7 @@ __global__ void __launch_bounds__(kSmemThreads, 1) chol_smem_kernel(const CholSA
     if (attempt == 1) {
       // 11 (L r + r (r + 1)) u tr(S), tr(S) by a fixed-order reduction
       double t = 0.0;
-      for (int i = threadIdx.x; i < r; i += blockDim.x)
-        for (int q = 0; q < a.splits; ++q)
-          t += (double)a.part[(size_t)q * r * r + (size_t)i * r + i];
+      for (int i = threadIdx.x; i < r; i += blockDim.x) t += (double)a.S[(size_t)i * r + i];
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) t += __shfl_xor_sync(0xffffffffu, t, off);
       if (lane == 0) s_red[warp] = t;
@@ -492,26 +501,29 @@ __global__ void __launch_bounds__(kSmemThreads, 1) chol_smem_kernel(const CholSA
       shift = 11.0 * ((double)a.L * r + (double)r * (r + 1)) * u * tr;
       if (!(shift > 0.0)) shift = 1e-30;
     }
-    // lower tiles of S (partials summed in float64, rounded once), padded
-    // with an identity block
-    for (int e = threadIdx.x; e < ntri * kNb * kNb; e += blockDim.x) {
-      const int t = e >> 10, w = e & 1023;
-      const int bi = tri_row(t), bj = t - bi * (bi + 1) / 2;
-      const int ii = w >> 5, jj = w & 31;
-      const int i = bi * kNb + ii, j = bj * kNb + jj;
-      float v = 0.f;
-      if (j <= i) {
-        if (i < r) {
-          double acc = 0.0;
-          for (int q = 0; q < a.splits; ++q)
-            acc += (double)a.part[(size_t)q * r * r + (size_t)i * r + j];
-          if (i == j) acc += shift;
-          v = (float)acc;
-        } else {
-          v = i == j ? 1.f : 0.f;
+    // lower tiles of S, padded with an identity block: asynchronous 4-byte
+    // copies keep many loads in flight without holding registers, which a
+    // single CTA streaming S from memory needs
+    for (int bi = 0, t = 0; bi < nb; ++bi) {
+      for (int bj = 0; bj <= bi; ++bj, ++t) {
+        float* dt = sm + (size_t)t * kTileF;
+        for (int w = threadIdx.x; w < kNb * kNb; w += kSmemThreads) {
+          const int ii = w >> 5, jj = w & 31;
+          const int i = bi * kNb + ii, j = bj * kNb + jj;
+          float* d = dt + ii * kP + jj;
+          if (j <= i && i < r) cp_async4(d, a.S + (size_t)i * r + j);
+          else *d = i == j ? 1.f : 0.f;
         }
       }
-      tile(bi, bj)[ii * kP + jj] = v;
+    }
+    cp_async_wait_all();
+    __syncthreads();
+    if (shift != 0.0) {
+      for (int i = threadIdx.x; i < r; i += kSmemThreads) {
+        float* d = tile(i >> 5, i >> 5) + (i & 31) * kP + (i & 31);
+        *d = (float)((double)*d + shift);
+      }
+      __syncthreads();
     }
     if (threadIdx.x == 0) s_bad = 0;
     __syncthreads();
@@ -626,14 +638,13 @@ size_t chol_blocked_ctl_bytes(int r) { return 64 + (size_t)r * sizeof(double); }
 
 bool chol_smem_fits(int r) { return r >= 1 && ceil_div(r, kNb) <= kSmemMaxBlk; }
 
-int chol_smem(const float* part, int splits, int r, int64_t L, float* Linv, int* status,
+int chol_smem(const float* S, int r, int64_t L, float* Linv, int* status,
               cudaStream_t stream) {
   if (!chol_smem_fits(r))
     return set_error(OUO_ERR_UNSUPPORTED, "one-CTA blocked Cholesky takes 1 <= r <= %d",
                      kSmemMaxBlk * kNb);
   CholSArgs a;
-  a.part = part;
-  a.splits = splits;
+  a.S = S;
   a.r = r;
   a.nblk = (int)ceil_div(r, kNb);
   a.R = a.nblk * kNb;

@@ -357,9 +357,9 @@ struct DionWs {
 // one-CTA kernel with the blocks in shared memory up to
 // smem_chol_max_rank(), the cooperative multi-CTA kernel above it; smaller
 // ranks keep the one-CTA packed-triangle kernel.  Per 4096 x 4096
-// Orth-Dion step the one-CTA blocked kernel is 5-11% faster than the
-// better of the other two from r = 64 to 128, even at r = 192 and 11%
-// slower at r = 256, where the cooperative kernel's wider phases win.
+// Orth-Dion step the one-CTA blocked kernel is 7-11% faster than the
+// better of the other two from r = 64 to 192, 2% at r = 224 and 4% slower
+// at r = 256, where the cooperative kernel's wider phases win.
 // OUO_CHOL_BLOCKED_MIN_RANK (1 to 129) and OUO_CHOL_SMEM_MAX_RANK (0 to
 // 256; 0 turns the one-CTA blocked kernel off) override the two bounds.
 int blocked_chol_min_rank() {
@@ -376,7 +376,7 @@ int smem_chol_max_rank() {
     const int v = atoi(env);
     if (v >= 0 && v <= 256) return v;
   }
-  return 192;
+  return 224;
 }
 int64_t padded_rank(int r) { return ceil_div(r, 32) * 32; }
 
@@ -450,7 +450,7 @@ int cholesky_inverse(const float* part, int splits, int r, int64_t L_rows,
       part = S;
       splits = 1;
     }
-    OUO_TRY(chol_smem(part, splits, r, L_rows, reinterpret_cast<float*>(w.Linv.p), status, s));
+    OUO_TRY(chol_smem(part, r, L_rows, reinterpret_cast<float*>(w.Linv.p), status, s));
   } else if (r >= blocked_chol_min_rank()) {
     OUO_TRY(chol_blocked(part, splits, r, L_rows, reinterpret_cast<float*>(w.S.p),
                          reinterpret_cast<float*>(w.Linv.p), w.ctl.p, status, s));

@@ -140,9 +140,10 @@ size_t chol_blocked_ctl_bytes(int r);
 int chol_blocked(const float* part, int splits, int r, int64_t L, float* S,
                  float* Linv, void* ctl, int* status, cudaStream_t stream);
 // The same factorization and inverse in one CTA with the blocks in shared
-// memory, for 1 <= r <= 256 (chol_smem_fits); no scratch besides Linv.
+// memory, for 1 <= r <= 256 (chol_smem_fits), from one summed r x r matrix
+// S (ld r); no scratch besides Linv.
 bool chol_smem_fits(int r);
-int chol_smem(const float* part, int splits, int r, int64_t L, float* Linv, int* status,
+int chol_smem(const float* S, int r, int64_t L, float* Linv, int* status,
               cudaStream_t stream);
 int convert_buf(const Buf& src, const Buf& dst, cudaStream_t stream);
 

@@ -84,7 +84,7 @@ def test_dion_4096_rank256_20_steps(mode):
 @pytest.mark.parametrize("mode", [odion.COLNORM, odion.QR])
 @pytest.mark.parametrize("shape,r,steps", [((1024, 768), 300, 3), ((1536, 1536), 512, 3)])
 def test_dion_wide_ranks(mode, shape, r, steps):
-    # ranks above 192 take the cooperative multi-CTA Cholesky (r = 300 is
+    # ranks above 224 take the cooperative multi-CTA Cholesky (r = 300 is
     # not a multiple of its 32-wide blocks)
     errs = _run(*shape, r, mode, steps=steps, seed=r)
     for e_m, e_q, e_w in errs:
@@ -109,7 +109,7 @@ def test_cholesky_routes_for_ranks_65_to_256(mode, shape, r, smem_max, monkeypat
 @pytest.mark.parametrize("mode", [odion.COLNORM, odion.QR])
 @pytest.mark.parametrize("shape,r", [((256, 512), 8), ((300, 200), 40)])
 def test_one_cta_blocked_cholesky_at_small_ranks(mode, shape, r, monkeypatch):
-    # OUO_CHOL_BLOCKED_MIN_RANK=1 routes every rank up to 192 to the
+    # OUO_CHOL_BLOCKED_MIN_RANK=1 routes every rank up to 224 to the
     # one-CTA blocked kernel: one block (r = 8) and two ragged blocks (r = 40)
     monkeypatch.setenv("OUO_CHOL_BLOCKED_MIN_RANK", "1")
     errs = _run(*shape, r, mode, steps=3, seed=r + 5)
