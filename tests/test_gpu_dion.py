@@ -50,9 +50,10 @@ def _run(m, n, r, mode, steps, seed, w_dtype=torch.float32, beta=1.0,
         dW_ref = ref["W"] - Wr
         e_w = rel_fro(dW, dW_ref)
         errs.append((e_m, e_q, e_w))
+        # the oracle carries its own state (it never takes a GPU value); with
+        # bf16 weights the comparison is of the update dW, which does not
+        # depend on the weights it is added to
         Mr, Wr, Qr = ref["M"], ref["W"], ref["Q"]
-        if w_dtype == torch.bfloat16:
-            Wr = to64(W)  # bf16 weights: compare the update, carry the stored value
     return errs
 
 
