@@ -231,3 +231,26 @@ def test_upper_stored_symmetric_matrices_change_no_bits(gram, monkeypatch):
         assert torch.equal(outs["1"][i], outs["0"][i]), shapes[i]
     ref = _oracle(to64(Xs[0]), gram)
     assert rel_fro(to64(outs["1"][0]), ref) <= TOL_BF16
+
+
+@pytest.mark.parametrize("gram", [True, False])
+def test_four_d_operand_loads_change_no_bits(gram, monkeypatch):
+    # An MN-major B stage on single-CTA tiles (Q X, B X) is one 4-D TMA load
+    # when the columns split into whole 64-column chunks, else one load per
+    # chunk (OUO_TMA_4D=0 forces the latter).  Both place the same bytes in
+    # shared memory, so the results must be bit-identical.  n = 1000 leaves a
+    # partial chunk and takes the per-chunk loads either way.
+    shapes = [(512, 2048), (256, 4096), (300, 1000)]
+    Xs = [_inputs(s, torch.bfloat16, 110 + i) for i, s in enumerate(shapes)]
+    fn = ouo.gram_ns_orthogonalize if gram else ouo.ns_orthogonalize
+    outs = {}
+    for mode in ("1", "0"):
+        monkeypatch.setenv("OUO_TMA_4D", mode)
+        Os = [torch.empty_like(x) for x in Xs]
+        fn(Xs, Os, ouo.ns_params())
+        torch.cuda.synchronize()
+        outs[mode] = Os
+    for i in range(len(Xs)):
+        assert torch.equal(outs["1"][i], outs["0"][i]), shapes[i]
+    ref = _oracle(to64(Xs[0]), gram)
+    assert rel_fro(to64(outs["1"][0]), ref) <= TOL_BF16
