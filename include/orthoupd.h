@@ -57,7 +57,7 @@ extern "C" {
 /* return codes */
 #define OUO_OK 0
 #define OUO_ERR_INVALID_ARG (-1)  /* bad pointer, shape, ld, alignment, value */
-#define OUO_ERR_UNSUPPORTED (-2)  /* valid request this build does not do    */
+#define OUO_ERR_UNSUPPORTED (-2)  /* valid request the library does not take */
 #define OUO_ERR_WORKSPACE (-3)    /* workspace missing or too small          */
 #define OUO_ERR_CUDA (-4)         /* a CUDA runtime / driver call failed     */
 #define OUO_ERR_NO_DEVICE (-5)    /* no sm_100 device current                */
