@@ -23,7 +23,7 @@ __all__ = [
     "gram_ns_orthogonalize_noalloc",
     "apply_update", "dion_workspace_bytes", "dion_lowrank_step", "dion_effective_rank",
     "DionShardStep", "version",
-    "launch_count", "timing_enable", "timing_read", "batch_empty",
+    "launch_count", "timing_enable", "timing_read", "batch_empty", "check_vector",
 ]
 
 
@@ -35,9 +35,30 @@ def _dtype_code(t: torch.Tensor) -> int:
     raise TypeError(f"unsupported dtype {t.dtype} (float32 or bfloat16)")
 
 
+def check_vector(t: Optional[torch.Tensor], name: str, dtype: torch.dtype,
+                 numel: int, device: Optional[torch.device] = None) -> None:
+    """The library reads and writes `numel` elements of `dtype` at
+    t.data_ptr(): refuse anything else before the pointer reaches it (a wrong
+    dtype or a short buffer would be a silent out-of-bounds access).  None
+    passes (the optional arguments)."""
+    if t is None:
+        return
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.numel() < numel:
+        raise ValueError(f"{name} needs at least {numel} elements, got {t.numel()}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, the matrices on {device}")
+
+
 class MatBatch:
     """A list of 2-D row-major CUDA tensors described once as an ouo_mat
-    array, so repeated calls do not rebuild it."""
+    array, so repeated calls do not rebuild it.  All of them must live on
+    one device."""
 
     def __init__(self, tensors: Iterable[torch.Tensor]):
         self.tensors = list(tensors)
@@ -49,6 +70,8 @@ class MatBatch:
                 raise ValueError("every matrix must be 2-D with unit column stride")
             if not t.is_cuda:
                 raise ValueError("every matrix must be a CUDA tensor")
+            if t.device != self.tensors[0].device:
+                raise ValueError("every matrix of a batch must be on one device")
             self.arr[i] = L.OuoMat(t.data_ptr(), t.shape[0], t.shape[1],
                                    max(t.stride(0), t.shape[1]))
             codes.add(_dtype_code(t))
@@ -158,10 +181,19 @@ def dion_params(rank=None, mu=None, beta=None, lr=None, wd=None,
     return p
 
 
+def _rows(b: MatBatch) -> int:
+    return sum(int(t.shape[0]) for t in b.tensors)
+
+
+def _dev(b: MatBatch) -> Optional[torch.device]:
+    return b.tensors[0].device if b.tensors else None
+
+
 def dion_momentum_update(M, G, mu: float, mode: str = "ema",
                          row_sqnorm: Optional[torch.Tensor] = None,
                          stream=None) -> None:
     Mb, Gb = _batch(M), _batch(G)
+    check_vector(row_sqnorm, "row_sqnorm", torch.float64, _rows(Mb), _dev(Mb))
     code = {"ema": L.OUO_MOMENTUM_EMA, "accum": L.OUO_MOMENTUM_ACCUM}[mode]
     L.check("dion_momentum_update", L.lib().dion_momentum_update(
         Mb.arr, Gb.arr, Mb.n, Gb.dtype, mu, code, _ptr(row_sqnorm),
@@ -177,6 +209,12 @@ def dion3_select_rows(B, row_sqnorm: torch.Tensor, rho: float,
                       ef: bool = True, mu: float = 0.95, eps: float = 1e-7,
                       stream=None) -> None:
     Bb, Xb = _batch(B), _batch(X0)
+    if row_sqnorm is None or idx is None or x0_scale is None:
+        raise ValueError("row_sqnorm, idx and x0_scale are required")
+    nk = sum(dion3_num_selected(int(t.shape[0]), rho) for t in Bb.tensors)
+    check_vector(row_sqnorm, "row_sqnorm", torch.float64, _rows(Bb), _dev(Bb))
+    check_vector(idx, "idx", torch.int32, nk, _dev(Bb))
+    check_vector(x0_scale, "x0_scale", torch.float32, Bb.n, _dev(Bb))
     L.check("dion3_select_rows", L.lib().dion3_select_rows(
         Bb.arr, _ptr(row_sqnorm), Bb.n, rho,
         L.OUO_EF_ROWS if ef else L.OUO_EF_NONE, mu, eps, _ptr(idx), Xb.arr,
@@ -197,6 +235,7 @@ def gram_ns_workspace_bytes(X, params=None) -> int:
 
 def _workspace(nbytes: int, device, given: Optional[torch.Tensor]):
     if given is not None:
+        check_vector(given, "workspace", torch.uint8, nbytes, device)
         return given
     return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
 
@@ -206,6 +245,7 @@ def _run_ns(fname, wsfn, X, O, params, workspace, status, stream):
     p = params or ns_params()
     need = wsfn(Xb, p)
     ws = _workspace(need, Xb.device, workspace)
+    check_vector(status, "status", torch.int32, 1, _dev(Xb))
     fn = getattr(L.lib(), fname)
     L.check(fname, fn(Xb.arr, Xb.dtype, Ob.arr, Ob.dtype, Xb.n, ctypes.byref(p),
                       ctypes.c_void_p(ws.data_ptr()), ws.numel(), _ptr(status),
@@ -231,6 +271,7 @@ def gram_ns_orthogonalize_noalloc(X, O, params=None, status=None,
     calls; calls that overlap on the GPU race) stands in for it."""
     Xb, Ob = _batch(X), _batch(O)
     p = params or ns_params()
+    check_vector(status, "status", torch.int32, 1, _dev(Xb))
     L.check("gram_ns_orthogonalize_noalloc", L.lib().gram_ns_orthogonalize_noalloc(
         Xb.arr, Xb.dtype, Ob.arr, Ob.dtype, Xb.n, ctypes.byref(p), _ptr(status),
         _stream(stream)))
@@ -240,8 +281,11 @@ def apply_update(W, O, lr: float, idx: Optional[torch.Tensor] = None,
                  scale: Optional[Sequence[float]] = None, wd: float = 0.0,
                  stream=None) -> None:
     Wb, Ob = _batch(W), _batch(O)
+    check_vector(idx, "idx", torch.int32, _rows(Ob), _dev(Wb))
     sc = None
     if scale is not None:
+        if len(scale) != Wb.n:
+            raise ValueError("scale needs one value per matrix")
         sc = (ctypes.c_float * Wb.n)(*[float(s) for s in scale])
     L.check("apply_update", L.lib().apply_update(
         Wb.arr, Wb.dtype, Ob.arr, Ob.dtype, _ptr(idx), Wb.n, lr, sc, wd,
@@ -280,12 +324,11 @@ def dion_lowrank_step(M, G, Q_state, W, params, scale=None, workspace=None,
     ws = _workspace(need, Mb.device, workspace)
     sc = None
     if scale is not None:
+        if len(scale) != Mb.n:
+            raise ValueError("scale needs one value per matrix")
         sc = (ctypes.c_float * Mb.n)(*[float(s) for s in scale])
-    if sigma is not None:
-        if sigma.dtype != torch.float32 or not sigma.is_cuda:
-            raise TypeError("sigma must be a float32 CUDA tensor")
-        if sigma.numel() < sum(_ranks(Mb, Qb, params)):
-            raise ValueError("sigma needs sum(ranks) elements")
+    check_vector(sigma, "sigma", torch.float32, sum(_ranks(Mb, Qb, params)), _dev(Mb))
+    check_vector(status, "status", torch.int32, 1, _dev(Mb))
     L.check("dion_lowrank_step", L.lib().dion_lowrank_step_stats(
         Mb.arr, Gb.arr, Gb.dtype, Qb.arr, Wb.arr, Wb.dtype, Mb.n,
         ctypes.byref(params), sc, ctypes.c_void_p(ws.data_ptr()), ws.numel(),
@@ -297,8 +340,10 @@ def dion_effective_rank(sigma: torch.Tensor, ranks: Sequence[int],
     """Per matrix exp(Shannon entropy of sigma_j^2 / sum sigma^2), from the
     sigma that dion_lowrank_step writes; returns a float32 CUDA tensor."""
     n = len(ranks)
+    check_vector(sigma, "sigma", torch.float32, sum(int(r) for r in ranks))
     if erank is None:
         erank = torch.empty(max(n, 1), dtype=torch.float32, device=sigma.device)
+    check_vector(erank, "erank", torch.float32, n, sigma.device)
     rk = (ctypes.c_int * max(n, 1))(*[int(r) for r in ranks])
     L.check("dion_effective_rank", L.lib().dion_effective_rank(
         _ptr(sigma), rk, n, _ptr(erank), _stream(stream)))
@@ -320,6 +365,8 @@ class DionShardStep:
         if len(rows_total) != n:
             raise ValueError("rows_total needs one entry per matrix")
         self.rows = (ctypes.c_int64 * max(n, 1))(*[int(x) for x in rows_total])
+        if scale is not None and len(scale) != n:
+            raise ValueError("scale needs one value per matrix")
         self.scale = None if scale is None else (ctypes.c_float * n)(*[float(x) for x in scale])
         lib = L.lib()
         wsb = lib.dion_shard_workspace_bytes(self.Mb.arr, self.Qb.arr, n, ctypes.byref(params))
@@ -331,6 +378,7 @@ class DionShardStep:
         self.red = torch.empty(max(rf, 64), dtype=torch.float32, device=dev)
 
     def _args(self, status, stream):
+        check_vector(status, "status", torch.int32, 1, self.red.device)
         return (ctypes.byref(self.p), ctypes.c_void_p(self.ws.data_ptr()), self.ws.numel(),
                 _ptr(self.red), _ptr(status), _stream(stream))
 
