@@ -235,7 +235,9 @@ def gram_ns_workspace_bytes(X, params=None) -> int:
 
 def _workspace(nbytes: int, device, given: Optional[torch.Tensor]):
     if given is not None:
-        check_vector(given, "workspace", torch.uint8, nbytes, device)
+        # an empty batch names no device index ("cuda"): check the rest only
+        known = device if getattr(device, "index", None) is not None else None
+        check_vector(given, "workspace", torch.uint8, nbytes, known)
         return given
     return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
 
