@@ -257,9 +257,13 @@ int gram_ns_orthogonalize(const ouo_mat* X, int x_dtype, const ouo_mat* O,
  * library holds the array until the process exits.
  *   - A batch whose gram_ns_workspace_bytes() exceeds the array is refused
  *     with OUO_ERR_WORKSPACE before anything is launched.
- *   - The first call on each device (with that device current) looks up the
- *     array's device address; make that first call before any stream
- *     capture.
+ *   - Every call looks up the array's device address on the current device
+ *     (no allocation).  The first call on a device also loads the library's
+ *     device image there; make that first call before any stream capture.
+ *     The address is never cached, so a device reset (which reloads the
+ *     image, possibly elsewhere) is safe.
+ *   - Arguments are checked as gram_ns_orthogonalize checks them (bad ones
+ *     give OUO_ERR_INVALID_ARG) before the scratch size is computed.
  *   - Every call shares the array; calls whose kernels overlap on the GPU
  *     (e.g. on two unordered streams) race on it.  Each call overwrites what
  *     it reads, so no state carries over between calls.

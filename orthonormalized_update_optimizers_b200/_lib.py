@@ -14,6 +14,11 @@ LIB_PATH = os.path.join(_HERE, "liborthoupd.so")
 
 # ---- constants mirrored from include/orthoupd.h
 OUO_OK = 0
+OUO_ERR_INVALID_ARG = -1
+OUO_ERR_UNSUPPORTED = -2
+OUO_ERR_WORKSPACE = -3
+OUO_ERR_CUDA = -4
+OUO_ERR_NO_DEVICE = -5
 OUO_F32 = 0
 OUO_BF16 = 1
 OUO_MOMENTUM_EMA = 0

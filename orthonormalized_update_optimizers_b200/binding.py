@@ -8,6 +8,7 @@ allocation made here (the library itself never allocates).
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 from typing import Iterable, Optional, Sequence
 
@@ -118,6 +119,37 @@ def _stream(stream) -> ctypes.c_void_p:
     return ctypes.c_void_p(s.cuda_stream)
 
 
+@contextlib.contextmanager
+def _on_device(*batches, stream=None, tensors=()):
+    """Check that every matrix batch, extra tensor and the stream of one call
+    live on one device, and make that device current for the call: the
+    library launches on the current device and looks up per-device state
+    there, so a call whose data sits on another GPU would hand that GPU's
+    pointers to kernels on the wrong one."""
+    dev = None
+    for b in batches:
+        if b is None or not b.tensors:
+            continue
+        if dev is None:
+            dev = b.device
+        elif b.device != dev:
+            raise ValueError(f"a batch is on {b.device}, another on {dev}")
+    for t in tensors:
+        if t is None:
+            continue
+        if dev is None:
+            dev = t.device
+        elif t.device != dev:
+            raise ValueError(f"a buffer is on {t.device}, the matrices on {dev}")
+    if stream is not None and dev is not None and stream.device != dev:
+        raise ValueError(f"the stream is on {stream.device}, the matrices on {dev}")
+    if dev is None:
+        yield None
+        return
+    with torch.cuda.device(dev):
+        yield dev
+
+
 def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
     return None if t is None else t.data_ptr()
 
@@ -195,9 +227,10 @@ def dion_momentum_update(M, G, mu: float, mode: str = "ema",
     Mb, Gb = _batch(M), _batch(G)
     check_vector(row_sqnorm, "row_sqnorm", torch.float64, _rows(Mb), _dev(Mb))
     code = {"ema": L.OUO_MOMENTUM_EMA, "accum": L.OUO_MOMENTUM_ACCUM}[mode]
-    L.check("dion_momentum_update", L.lib().dion_momentum_update(
-        Mb.arr, Gb.arr, Mb.n, Gb.dtype, mu, code, _ptr(row_sqnorm),
-        _stream(stream)))
+    with _on_device(Mb, Gb, stream=stream):
+        L.check("dion_momentum_update", L.lib().dion_momentum_update(
+            Mb.arr, Gb.arr, Mb.n, Gb.dtype, mu, code, _ptr(row_sqnorm),
+            _stream(stream)))
 
 
 def dion3_num_selected(rows: int, rho: float) -> int:
@@ -215,10 +248,11 @@ def dion3_select_rows(B, row_sqnorm: torch.Tensor, rho: float,
     check_vector(row_sqnorm, "row_sqnorm", torch.float64, _rows(Bb), _dev(Bb))
     check_vector(idx, "idx", torch.int32, nk, _dev(Bb))
     check_vector(x0_scale, "x0_scale", torch.float32, Bb.n, _dev(Bb))
-    L.check("dion3_select_rows", L.lib().dion3_select_rows(
-        Bb.arr, _ptr(row_sqnorm), Bb.n, rho,
-        L.OUO_EF_ROWS if ef else L.OUO_EF_NONE, mu, eps, _ptr(idx), Xb.arr,
-        Xb.dtype, _ptr(x0_scale), _stream(stream)))
+    with _on_device(Bb, Xb, stream=stream):
+        L.check("dion3_select_rows", L.lib().dion3_select_rows(
+            Bb.arr, _ptr(row_sqnorm), Bb.n, rho,
+            L.OUO_EF_ROWS if ef else L.OUO_EF_NONE, mu, eps, _ptr(idx), Xb.arr,
+            Xb.dtype, _ptr(x0_scale), _stream(stream)))
 
 
 def ns_workspace_bytes(X, params=None) -> int:
@@ -245,13 +279,14 @@ def _workspace(nbytes: int, device, given: Optional[torch.Tensor]):
 def _run_ns(fname, wsfn, X, O, params, workspace, status, stream):
     Xb, Ob = _batch(X), _batch(O)
     p = params or ns_params()
-    need = wsfn(Xb, p)
-    ws = _workspace(need, Xb.device, workspace)
-    check_vector(status, "status", torch.int32, 1, _dev(Xb))
-    fn = getattr(L.lib(), fname)
-    L.check(fname, fn(Xb.arr, Xb.dtype, Ob.arr, Ob.dtype, Xb.n, ctypes.byref(p),
-                      ctypes.c_void_p(ws.data_ptr()), ws.numel(), _ptr(status),
-                      _stream(stream)))
+    with _on_device(Xb, Ob, stream=stream):
+        need = wsfn(Xb, p)
+        ws = _workspace(need, Xb.device, workspace)
+        check_vector(status, "status", torch.int32, 1, _dev(Xb))
+        fn = getattr(L.lib(), fname)
+        L.check(fname, fn(Xb.arr, Xb.dtype, Ob.arr, Ob.dtype, Xb.n, ctypes.byref(p),
+                          ctypes.c_void_p(ws.data_ptr()), ws.numel(), _ptr(status),
+                          _stream(stream)))
 
 
 def ns_orthogonalize(X, O, params=None, workspace=None, status=None,
@@ -274,9 +309,10 @@ def gram_ns_orthogonalize_noalloc(X, O, params=None, status=None,
     Xb, Ob = _batch(X), _batch(O)
     p = params or ns_params()
     check_vector(status, "status", torch.int32, 1, _dev(Xb))
-    L.check("gram_ns_orthogonalize_noalloc", L.lib().gram_ns_orthogonalize_noalloc(
-        Xb.arr, Xb.dtype, Ob.arr, Ob.dtype, Xb.n, ctypes.byref(p), _ptr(status),
-        _stream(stream)))
+    with _on_device(Xb, Ob, stream=stream):
+        L.check("gram_ns_orthogonalize_noalloc", L.lib().gram_ns_orthogonalize_noalloc(
+            Xb.arr, Xb.dtype, Ob.arr, Ob.dtype, Xb.n, ctypes.byref(p), _ptr(status),
+            _stream(stream)))
 
 
 def apply_update(W, O, lr: float, idx: Optional[torch.Tensor] = None,
@@ -289,9 +325,10 @@ def apply_update(W, O, lr: float, idx: Optional[torch.Tensor] = None,
         if len(scale) != Wb.n:
             raise ValueError("scale needs one value per matrix")
         sc = (ctypes.c_float * Wb.n)(*[float(s) for s in scale])
-    L.check("apply_update", L.lib().apply_update(
-        Wb.arr, Wb.dtype, Ob.arr, Ob.dtype, _ptr(idx), Wb.n, lr, sc, wd,
-        _stream(stream)))
+    with _on_device(Wb, Ob, stream=stream):
+        L.check("apply_update", L.lib().apply_update(
+            Wb.arr, Wb.dtype, Ob.arr, Ob.dtype, _ptr(idx), Wb.n, lr, sc, wd,
+            _stream(stream)))
 
 
 def _ranks(Mb, Qb, params):
@@ -322,8 +359,6 @@ def dion_lowrank_step(M, G, Q_state, W, params, scale=None, workspace=None,
     tensor of sum(ranks) elements) the step also writes the norms of R's
     columns, matrix after matrix."""
     Mb, Gb, Qb, Wb = _batch(M), _batch(G), _batch(Q_state), _batch(W)
-    need = dion_workspace_bytes(Mb, params, Qb)
-    ws = _workspace(need, Mb.device, workspace)
     sc = None
     if scale is not None:
         if len(scale) != Mb.n:
@@ -331,10 +366,13 @@ def dion_lowrank_step(M, G, Q_state, W, params, scale=None, workspace=None,
         sc = (ctypes.c_float * Mb.n)(*[float(s) for s in scale])
     check_vector(sigma, "sigma", torch.float32, sum(_ranks(Mb, Qb, params)), _dev(Mb))
     check_vector(status, "status", torch.int32, 1, _dev(Mb))
-    L.check("dion_lowrank_step", L.lib().dion_lowrank_step_stats(
-        Mb.arr, Gb.arr, Gb.dtype, Qb.arr, Wb.arr, Wb.dtype, Mb.n,
-        ctypes.byref(params), sc, ctypes.c_void_p(ws.data_ptr()), ws.numel(),
-        _ptr(sigma), _ptr(status), _stream(stream)))
+    with _on_device(Mb, Gb, Qb, Wb, stream=stream):
+        need = dion_workspace_bytes(Mb, params, Qb)
+        ws = _workspace(need, Mb.device, workspace)
+        L.check("dion_lowrank_step", L.lib().dion_lowrank_step_stats(
+            Mb.arr, Gb.arr, Gb.dtype, Qb.arr, Wb.arr, Wb.dtype, Mb.n,
+            ctypes.byref(params), sc, ctypes.c_void_p(ws.data_ptr()), ws.numel(),
+            _ptr(sigma), _ptr(status), _stream(stream)))
 
 
 def dion_effective_rank(sigma: torch.Tensor, ranks: Sequence[int],
@@ -347,8 +385,9 @@ def dion_effective_rank(sigma: torch.Tensor, ranks: Sequence[int],
         erank = torch.empty(max(n, 1), dtype=torch.float32, device=sigma.device)
     check_vector(erank, "erank", torch.float32, n, sigma.device)
     rk = (ctypes.c_int * max(n, 1))(*[int(r) for r in ranks])
-    L.check("dion_effective_rank", L.lib().dion_effective_rank(
-        _ptr(sigma), rk, n, _ptr(erank), _stream(stream)))
+    with _on_device(stream=stream, tensors=(sigma, erank)):
+        L.check("dion_effective_rank", L.lib().dion_effective_rank(
+            _ptr(sigma), rk, n, _ptr(erank), _stream(stream)))
     return erank
 
 
@@ -370,6 +409,7 @@ class DionShardStep:
         if scale is not None and len(scale) != n:
             raise ValueError("scale needs one value per matrix")
         self.scale = None if scale is None else (ctypes.c_float * n)(*[float(x) for x in scale])
+        self._check_devices()
         lib = L.lib()
         wsb = lib.dion_shard_workspace_bytes(self.Mb.arr, self.Qb.arr, n, ctypes.byref(params))
         rf = lib.dion_shard_red_floats(self.Mb.arr, self.Qb.arr, n, ctypes.byref(params))
@@ -379,10 +419,18 @@ class DionShardStep:
         self.ws = torch.empty(max(wsb, 256), dtype=torch.uint8, device=dev)
         self.red = torch.empty(max(rf, 64), dtype=torch.float32, device=dev)
 
+    def _check_devices(self):
+        with _on_device(self.Mb, self.Gb, self.Qb, self.Wb):
+            pass
+
     def _args(self, status, stream):
         check_vector(status, "status", torch.int32, 1, self.red.device)
-        return (ctypes.byref(self.p), ctypes.c_void_p(self.ws.data_ptr()), self.ws.numel(),
-                _ptr(self.red), _ptr(status), _stream(stream))
+        if stream is not None and stream.device != self.red.device:
+            raise ValueError(f"the stream is on {stream.device}, the matrices on "
+                             f"{self.red.device}")
+        with torch.cuda.device(self.red.device):
+            return (ctypes.byref(self.p), ctypes.c_void_p(self.ws.data_ptr()),
+                    self.ws.numel(), _ptr(self.red), _ptr(status), _stream(stream))
 
     def project(self, status=None, stream=None) -> None:
         pp, ws, wn, red, st, s = self._args(status, stream)

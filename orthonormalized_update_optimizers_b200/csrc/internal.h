@@ -117,6 +117,11 @@ int gemm_timing_read(int kind, int* launches, double* total_ms, double* flops);
 // CUDA-core fp32 GEMM for the fp32 precision path.
 int gemm_simt(const GemmDesc& g, cudaStream_t stream);
 
+// Argument checks of ns_orthogonalize / gram_ns_orthogonalize (everything
+// but the workspace): OUO_OK or the error code, with the message set.
+int ns_check_call(const ouo_mat* X, int x_dtype, const ouo_mat* O, int o_dtype,
+                  int nmat, const ouo_ns_params* p, int* dev_status);
+
 // ----------------------------------------------------------- other kernels
 struct PrepArgs;  // defined in nsprep.cu
 

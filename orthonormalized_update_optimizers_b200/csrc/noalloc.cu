@@ -12,16 +12,18 @@
 // OUO_NOALLOC_SCRATCH_BYTES bytes; a GPU holds it from the moment this part
 // of the library is loaded on it until the process exits.  Host code cannot
 // use the array's name as a device address (in host code the name is only a
-// stand-in), so the first call on each device, with that device current,
-// looks the address up with cudaGetSymbolAddress and caches it.  That first
-// call on a device should therefore come before any stream capture.
+// stand-in), so every call, with the device current, looks the address up
+// with cudaGetSymbolAddress and checks the result.  The first call on a
+// device also loads the library's device image there (the set-up); make
+// that first call before any stream capture.  The address is not cached:
+// after cudaDeviceReset, or any new primary context, the image is loaded
+// again and the array may sit elsewhere, and a stale address would send the
+// kernels' writes into memory the library does not own.
 //
 // Every call uses the same array, and a call overwrites every part of it it
 // reads, so nothing carries over from one call to the next.  Calls whose
 // kernels overlap on the GPU (for example, issued on two different streams
 // without ordering between them) race on the array.
-#include <mutex>
-
 #include "internal.h"
 
 namespace ouo {
@@ -30,27 +32,14 @@ namespace {
 static __device__ __align__(256) unsigned char
     g_noalloc_scratch[OUO_NOALLOC_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_mu;
-void* g_addr[kMaxDevices] = {nullptr};
-
-// Device address of the scratch array on the current device (looked up once
-// per device).
+// Device address of the scratch array on the current device.
 int scratch_address(void** out) {
-  int dev = 0;
-  OUO_CHECK_CUDA(cudaGetDevice(&dev));
-  if (dev < 0 || dev >= kMaxDevices)
-    return set_error(OUO_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
-  std::lock_guard<std::mutex> lock(g_mu);
-  if (!g_addr[dev]) {
-    void* p = nullptr;
-    cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    if (e != cudaSuccess || !p)
-      return set_error(OUO_ERR_CUDA, "cudaGetSymbolAddress(scratch) failed: %s",
-                       cudaGetErrorString(e));
-    g_addr[dev] = p;
-  }
-  *out = g_addr[dev];
+  void* p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+  if (e != cudaSuccess || !p)
+    return set_error(OUO_ERR_CUDA, "cudaGetSymbolAddress(scratch) failed: %s",
+                     cudaGetErrorString(e));
+  *out = p;
   return OUO_OK;
 }
 
@@ -63,11 +52,10 @@ extern "C" int gram_ns_orthogonalize_noalloc(const ouo_mat* X, int x_dtype,
                                              int* dev_status, void* stream) {
   using namespace ouo;
   clear_error();
-  if (nmat < 0 || nmat > OUO_MAX_BATCH)
-    return set_error(OUO_ERR_INVALID_ARG, "nmat %d out of range", nmat);
-  if (!p) return set_error(OUO_ERR_INVALID_ARG, "NULL ns params");
+  // the same argument checks as gram_ns_orthogonalize, before the size is
+  // computed from those arguments
+  OUO_TRY(ns_check_call(X, x_dtype, O, o_dtype, nmat, p, dev_status));
   if (nmat == 0) return OUO_OK;
-  if (!X) return set_error(OUO_ERR_INVALID_ARG, "X: NULL batch array");
   const size_t need = gram_ns_workspace_bytes(X, nmat, p);
   if (need > (size_t)OUO_NOALLOC_SCRATCH_BYTES)
     return set_error(OUO_ERR_WORKSPACE,

@@ -444,10 +444,10 @@ size_t plan_bytes(const ouo_mat* X, int nmat, const ouo_ns_params* p,
   return ar.used + 256;
 }
 
-int run_ns(const ouo_mat* X, int x_dtype, const ouo_mat* O, int o_dtype,
-           int nmat, const ouo_ns_params* p, void* ws, size_t ws_bytes,
-           int* dev_status, void* stream, bool gram) {
-  clear_error();
+}  // namespace
+
+int ns_check_call(const ouo_mat* X, int x_dtype, const ouo_mat* O, int o_dtype,
+                  int nmat, const ouo_ns_params* p, int* dev_status) {
   if (nmat < 0 || nmat > OUO_MAX_BATCH)
     return set_error(OUO_ERR_INVALID_ARG, "nmat %d out of range", nmat);
   OUO_TRY(validate_params(p));
@@ -457,6 +457,17 @@ int run_ns(const ouo_mat* X, int x_dtype, const ouo_mat* O, int o_dtype,
   OUO_TRY(validate_same_shapes(X, O, nmat, "X", "O"));
   if (dev_status && ((uintptr_t)dev_status % 4))
     return set_error(OUO_ERR_INVALID_ARG, "dev_status misaligned");
+  return OUO_OK;
+}
+
+namespace {
+
+int run_ns(const ouo_mat* X, int x_dtype, const ouo_mat* O, int o_dtype,
+           int nmat, const ouo_ns_params* p, void* ws, size_t ws_bytes,
+           int* dev_status, void* stream, bool gram) {
+  clear_error();
+  OUO_TRY(ns_check_call(X, x_dtype, O, o_dtype, nmat, p, dev_status));
+  if (nmat == 0) return OUO_OK;
   const size_t need = plan_bytes(X, nmat, p, gram, o_dtype);
   if (!ws || ws_bytes < need)
     return set_error(OUO_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given",

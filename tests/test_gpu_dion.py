@@ -46,9 +46,20 @@ def _run(m, n, r, mode, steps, seed, w_dtype=torch.float32, beta=1.0,
         ref = odion.dion_step(Mr, to64(Gs), Qr, Wr, mu, lr, scale, mode, beta=beta)
         e_m = rel_fro(to64(M), ref["M"])
         e_q = rel_fro(to64(Qt).T, ref["Q"])
-        dW = to64(W) - W_before
+        W_after = to64(W)
+        dW = W_after - W_before
         dW_ref = ref["W"] - Wr
-        e_w = rel_fro(dW, dW_ref)
+        if w_dtype == torch.bfloat16:
+            # The kernel adds the update to the bf16 weights in fp32 and
+            # stores the sum rounded to bf16: the stored dW carries one bf16
+            # rounding of the weights (at most 2^-8 relative per element) on
+            # top of the update's own error.  The error is stated as a
+            # fraction of ||dW_ref|| after taking that rounding off.
+            rnd = 2.0 ** -8 * np.linalg.norm(W_after)
+            assert np.linalg.norm(dW_ref) > 4 * rnd  # the check has teeth
+            e_w = max(0.0, np.linalg.norm(dW - dW_ref) - rnd) / np.linalg.norm(dW_ref)
+        else:
+            e_w = rel_fro(dW, dW_ref)
         errs.append((e_m, e_q, e_w))
         # the oracle carries its own state (it never takes a GPU value); with
         # bf16 weights the comparison is of the update dW, which does not
@@ -70,7 +81,7 @@ def test_dion_bf16_weights_and_beta():
     errs = _run(384, 640, 48, odion.QR, steps=2, seed=5, w_dtype=torch.bfloat16,
                 beta=0.5, lr=0.05, scale=2.0)
     for e_m, e_q, e_w in errs:
-        assert e_m <= TOL_BF16 and e_q <= TOL_BF16 and e_w <= 3e-2, errs
+        assert e_m <= TOL_BF16 and e_q <= TOL_BF16 and e_w <= TOL_BF16, errs
 
 
 @pytest.mark.parametrize("mode", [odion.COLNORM, odion.QR])

@@ -4,7 +4,10 @@ gram_ns_orthogonalize_noalloc serves callers that cannot allocate device
 memory (a plugin inside a framework whose pool owns all of it, or a path that
 cannot afford cudaMalloc's implicit synchronization): it runs the same
 kernels as gram_ns_orthogonalize with the library's fixed scratch array in
-place of a caller workspace.  This file is collected last on purpose.
+place of a caller workspace.  Both entry points run the same kernels in the
+same order on the same inputs, and every reduction has a fixed order, so the
+two results must agree bit for bit; the float64 oracle pins both.  This file
+is collected last on purpose.
 """
 import ctypes
 
@@ -14,6 +17,7 @@ import torch
 import orthonormalized_update_optimizers_b200 as ouo
 from orthonormalized_update_optimizers_b200 import _lib as L
 from orthonormalized_update_optimizers_b200 import synth
+from oracle import ns as ons
 
 from ._util import TOL_BF16, rel_fro, to64
 
@@ -47,8 +51,12 @@ def test_noalloc_matches_workspace_entry_on_two_calls():
         assert _noalloc(X, got, p, status) == L.OUO_OK, L.lib().ouo_last_error()
         torch.cuda.synchronize()
         assert status.item() == 0
-        for g, r in zip(got, ref):
-            assert rel_fro(to64(g), to64(r)) <= TOL_BF16, call
+        for i, (g, r) in enumerate(zip(got, ref)):
+            assert torch.equal(g, r), (call, i)
+        # and both against the float64 oracle on the same bf16 inputs
+        o = ons.gram_newton_schulz(to64(X[0]), iters=p.iters,
+                                   restart_after=tuple(p.restart_after[:p.n_restart]))
+        assert rel_fro(to64(got[0]), o) <= TOL_BF16, call
 
 
 def test_noalloc_refuses_batches_beyond_its_array():
@@ -58,5 +66,16 @@ def test_noalloc_refuses_batches_beyond_its_array():
     status = torch.zeros(1, dtype=torch.int32, device=DEV)
     n0 = ouo.launch_count()
     rc = _noalloc(big, big, p, status)
-    assert rc == -3 and b"scratch" in L.lib().ouo_last_error()
+    assert rc == L.OUO_ERR_WORKSPACE and b"scratch" in L.lib().ouo_last_error()
     assert ouo.launch_count() == n0  # nothing was launched
+
+
+def test_noalloc_rejects_bad_parameters_before_sizing():
+    # an unknown precision is an argument error, not a scratch-size refusal
+    p = ouo.ns_params()
+    p.precision = 7
+    X = [torch.zeros(64, 128, dtype=torch.bfloat16, device=DEV)]
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    n0 = ouo.launch_count()
+    assert _noalloc(X, X, p, status) == L.OUO_ERR_INVALID_ARG
+    assert ouo.launch_count() == n0
