@@ -1,7 +1,6 @@
-// Blocked Cholesky factorization and triangular inverse for CholeskyQR on
-// wide ranks: one cooperative multi-CTA launch (chol_blocked), and for
-// r <= 256 a one-CTA kernel that keeps the blocks in shared memory
-// (chol_smem).
+// Blocked Cholesky factorization (and optionally the triangular inverse) for
+// CholeskyQR on ranks above 256: one cooperative multi-CTA launch
+// (chol_blocked).  Ranks up to 256 take the one-CTA kernel of cholqr.cu.
 //
 // Source: "Orth-Dion: Eliminating Geometric Mismatch in Distributed Low-Rank
 // Spectral Optimization", Orth-Dion (the right factor, and in Dion the left
@@ -10,8 +9,8 @@
 // rows L^-1 X are orthonormal, with the implied R = L^T on a positive
 // diagonal (the unique QR).
 //
-// S arrives as `splits` partial Gram matrices, summed here in float64 in a
-// fixed order.  The r x r problem is padded to R = 32 * ceil(r / 32) with an
+// S arrives as `splits` partial Gram matrices in upper storage (entry (i, j)
+// valid for j >= i), summed here in float64 in a fixed order.  The r x r problem is padded to R = 32 * ceil(r / 32) with an
 // identity block and processed in 32 x 32 blocks:
 //   for each block column p:
 //     the diagonal block S_pp = L_pp L_pp^T is factored and inverted
@@ -19,8 +18,11 @@
 //       it (identical bits), and published by CTA 0;
 //     the blocks below it become L_ip = S_ip D_p^T;
 //     the trailing lower blocks are updated S_ij -= L_ip L_jp^T;
-//   then L^-1 by recursive doubling over neighbouring diagonal super-blocks
-//     [[A, 0], [B, C]]^-1 = [[A^-1, 0], [-C^-1 B A^-1, C^-1]].
+//   then (with `inverse`) L^-1 by recursive doubling over neighbouring
+//   diagonal super-blocks [[A, 0], [B, C]]^-1 = [[A^-1, 0], [-C^-1 B A^-1, C^-1]];
+//   without it the strictly lower blocks L_ij stay in S and the inverted
+//   diagonal blocks D_p in the diagonal blocks of Linv (the form the
+//   batched triangular solve of cholqr.cu reads).
 // In the cooperative kernel phases are separated by a grid barrier whose
 // wait is bounded in time (a barrier that runs out sets OUO_STATUS_TIMEOUT
 // and every later barrier passes at once).  In both kernels a non-positive
@@ -49,6 +51,7 @@ struct CholBArgs {
   int* flags;         // [0] pivot failed, [1] barrier timed out
   double* diag;       // unshifted diagonal of S (r values)
   int* status;
+  int inverse;        // form L^-1 (else leave L in S and D_p in Linv)
 };
 
 // Grid-wide barrier over all CTAs of the cooperative launch; the wait is
@@ -100,9 +103,9 @@ __device__ void assemble(const CholBArgs& a, float shift) {
     }
     float v;
     if (i < a.r) {
-      double s = 0.0;
+      double s = 0.0;  // (i, j), j <= i, is stored at (j, i)
       for (int p = 0; p < a.splits; ++p)
-        s += (double)a.part[(size_t)p * a.r * a.r + (size_t)i * a.r + j];
+        s += (double)a.part[(size_t)p * a.r * a.r + (size_t)j * a.r + i];
       if (i == j) {
         a.diag[i] = s;
         s += (double)shift;
@@ -364,8 +367,9 @@ __global__ void __launch_bounds__(kCholThreads) chol_blocked_kernel(const CholBA
          e += (size_t)gridDim.x * blockDim.x) {
       const int i = (int)(e / a.R), j = (int)(e - (e / a.R) * a.R);
       a.Linv[e] = i == j ? 1.f : 0.f;
+      if (!a.inverse && j / kNb < i / kNb) a.S[e] = 0.f;  // L = I
     }
-  } else {
+  } else if (a.inverse) {
     for (int h = 1; h < a.nblk; h *= 2) {
       inv_step1(a, h);
       grid_barrier(a);
@@ -378,297 +382,13 @@ __global__ void __launch_bounds__(kCholThreads) chol_blocked_kernel(const CholBA
     report_status(a.status, OUO_STATUS_TIMEOUT);
 }
 
-// ---------------------------------------------------------------------------
-// One-CTA blocked Cholesky and inverse for r <= 256 (at most 8 x 8 blocks).
-// The lower 32 x 32 blocks of S stay in shared memory for the whole
-// factorization and __syncthreads separates the phases, so no phase waits
-// on a grid barrier.  The block arithmetic is that of the cooperative
-// kernel above (D_p from warp_chol32, L_ip = S_ip D_p^T,
-// S_ij -= L_ip L_jp^T); the inverse is formed one block diagonal at a time,
-// X_ij = -D_i sum_{k=j}^{i-1} L_ik X_kj, from the blocks of X = L^-1
-// already written to the output.  Work items are (block, 8-column group):
-// lane = row, eight accumulators.  S arrives summed (one r x r matrix).
-constexpr int kSmemMaxBlk = 8;
-constexpr int kSmemThreads = 512;
-constexpr int kSmemWarps = kSmemThreads / 32;
-constexpr int kP = 36;            // tile pitch: float4 rows, no bank conflicts
-constexpr int kTileF = kNb * kP;  // floats per tile
-constexpr int kStageF = kNb * 9;  // per-warp 32 x 8 staging, pitch 9
-
-struct CholSArgs {
-  const float* S;     // r x r (ld r), lower triangle read
-  int r, R, nblk;
-  int64_t L;          // row length of X (for the shift)
-  float* Linv;        // R x R output (ld R), lower triangular
-  int* status;
-};
-
-__host__ __device__ constexpr int tri_idx(int bi, int bj) { return bi * (bi + 1) / 2 + bj; }
-
-// lower tiles of S, D_p, the current panel (nblk - 1 tiles), warp staging
-size_t chol_smem_blocked_bytes(int nblk) {
-  const int ntri = nblk * (nblk + 1) / 2;
-  return ((size_t)(ntri + nblk) * kTileF + (size_t)kSmemWarps * kStageF) * sizeof(float);
-}
-
-__device__ __forceinline__ int tri_row(int t) {
-  int bi = (int)((sqrtf(8.f * (float)t + 1.f) - 1.f) * 0.5f);
-  while ((bi + 1) * (bi + 2) / 2 <= t) ++bi;
-  while (bi * (bi + 1) / 2 > t) --bi;
-  return bi;
-}
-
-__device__ __forceinline__ void cp_async4(float* dst_smem, const float* src) {
-  const unsigned d = (unsigned)__cvta_generic_to_shared(dst_smem);
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(d), "l"(src) : "memory");
-}
-
-__device__ __forceinline__ void cp_async_wait_all() {
-  asm volatile("cp.async.wait_all;\n" ::: "memory");
-}
-
-__device__ __forceinline__ void load_row(const float* A, float (&row)[kNb]) {
-  const int lane = threadIdx.x & 31;
-#pragma unroll
-  for (int k = 0; k < kNb; k += 4) {
-    const float4 v = *reinterpret_cast<const float4*>(A + lane * kP + k);
-    row[k] = v.x;
-    row[k + 1] = v.y;
-    row[k + 2] = v.z;
-    row[k + 3] = v.w;
-  }
-}
-
-// acc[c] += sum_k A[lane][k] B[c0 + c][k], c < 8 (tiles of pitch kP)
-__device__ __forceinline__ void rowdot8(const float* A, const float* B, int c0,
-                                        float (&acc)[8]) {
-  float row[kNb];
-  load_row(A, row);
-#pragma unroll
-  for (int c = 0; c < 8; ++c) {
-    const float* b = B + (c0 + c) * kP;
-#pragma unroll
-    for (int k = 0; k < kNb; k += 4) {
-      const float4 v = *reinterpret_cast<const float4*>(b + k);
-      acc[c] = fmaf(row[k], v.x, acc[c]);
-      acc[c] = fmaf(row[k + 1], v.y, acc[c]);
-      acc[c] = fmaf(row[k + 2], v.z, acc[c]);
-      acc[c] = fmaf(row[k + 3], v.w, acc[c]);
-    }
-  }
-}
-
-__device__ __forceinline__ void st8(float* p, const float (&v)[8], float sign) {
-  *reinterpret_cast<float4*>(p) = make_float4(sign * v[0], sign * v[1], sign * v[2], sign * v[3]);
-  *reinterpret_cast<float4*>(p + 4) =
-      make_float4(sign * v[4], sign * v[5], sign * v[6], sign * v[7]);
-}
-
-__global__ void __launch_bounds__(kSmemThreads, 1) chol_smem_kernel(const CholSArgs a) {
-  extern __shared__ __align__(16) float sm[];
-  __shared__ int s_bad;
-  __shared__ double s_red[kSmemWarps];
-  const int nb = a.nblk, R = a.R, r = a.r;
-  const int ntri = nb * (nb + 1) / 2;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  auto tile = [&](int bi, int bj) { return sm + (size_t)tri_idx(bi, bj) * kTileF; };
-  float* Dt = sm + (size_t)ntri * kTileF;  // D_p[i][k] at Dt[i * kP + k]
-  float* pan = Dt + kTileF;                // L_ip of the current panel
-  float* stg = pan + (size_t)(nb - 1) * kTileF + (size_t)warp * kStageF;
-
-  // blocks of X above the block diagonal are zero: upper block (bj, bi) for
-  // each strictly lower (bi, bj), 256 float4 per block
-  for (int e = threadIdx.x; e < (nb * (nb - 1) / 2) * 256; e += blockDim.x) {
-    const int t = e >> 8, w = e & 255;
-    const int bi = tri_row(t) + 1, bj = t - bi * (bi - 1) / 2;
-    float* dst = a.Linv + (size_t)(bj * kNb + (w >> 3)) * R + bi * kNb + (w & 7) * 4;
-    *reinterpret_cast<float4*>(dst) = make_float4(0.f, 0.f, 0.f, 0.f);
-  }
-  bool ok = false;
-  for (int attempt = 0; attempt < 2 && !ok; ++attempt) {
-    double shift = 0.0;
-    if (attempt == 1) {
-      // 11 (L r + r (r + 1)) u tr(S), tr(S) by a fixed-order reduction
-      double t = 0.0;
-      for (int i = threadIdx.x; i < r; i += blockDim.x) t += (double)a.S[(size_t)i * r + i];
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) t += __shfl_xor_sync(0xffffffffu, t, off);
-      if (lane == 0) s_red[warp] = t;
-      __syncthreads();
-      double tr = 0.0;
-      for (int w = 0; w < kSmemWarps; ++w) tr += s_red[w];
-      const double u = 5.9604644775390625e-8;  // 2^-24
-      shift = 11.0 * ((double)a.L * r + (double)r * (r + 1)) * u * tr;
-      if (!(shift > 0.0)) shift = 1e-30;
-    }
-    // lower tiles of S, padded with an identity block: asynchronous 4-byte
-    // copies keep many loads in flight without holding registers, which a
-    // single CTA streaming S from memory needs
-    for (int bi = 0, t = 0; bi < nb; ++bi) {
-      for (int bj = 0; bj <= bi; ++bj, ++t) {
-        float* dt = sm + (size_t)t * kTileF;
-        for (int w = threadIdx.x; w < kNb * kNb; w += kSmemThreads) {
-          const int ii = w >> 5, jj = w & 31;
-          const int i = bi * kNb + ii, j = bj * kNb + jj;
-          float* d = dt + ii * kP + jj;
-          if (j <= i && i < r) cp_async4(d, a.S + (size_t)i * r + j);
-          else *d = i == j ? 1.f : 0.f;
-        }
-      }
-    }
-    cp_async_wait_all();
-    __syncthreads();
-    if (shift != 0.0) {
-      for (int i = threadIdx.x; i < r; i += kSmemThreads) {
-        float* d = tile(i >> 5, i >> 5) + (i & 31) * kP + (i & 31);
-        *d = (float)((double)*d + shift);
-      }
-      __syncthreads();
-    }
-    if (threadIdx.x == 0) s_bad = 0;
-    __syncthreads();
-    bool failed = false;
-    for (int p = 0; p < nb; ++p) {
-      if (warp == 0) {
-        float l[kNb], x[kNb];
-        if (warp_chol32(tile(p, p), kP, l, x)) {
-#pragma unroll
-          for (int i = 0; i < kNb; ++i) {
-            Dt[i * kP + lane] = x[i];
-            a.Linv[(size_t)(p * kNb + i) * R + p * kNb + lane] = x[i];
-          }
-        } else if (lane == 0) {
-          s_bad = 1;
-        }
-      }
-      __syncthreads();
-      if (s_bad) {
-        failed = true;
-        break;
-      }
-      const int m = nb - p - 1;
-      // panel: pan[b] = S_{p+1+b, p} D_p^T
-      for (int it = warp; it < m * 4; it += kSmemWarps) {
-        const int b = it >> 2, c0 = (it & 3) * 8;
-        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        rowdot8(tile(p + 1 + b, p), Dt, c0, acc);
-        st8(pan + (size_t)b * kTileF + lane * kP + c0, acc, 1.f);
-      }
-      __syncthreads();
-      // trailing: S_ij -= L_ip L_jp^T for p < j <= i
-      const int tasks = m * (m + 1) / 2;
-      for (int it = warp; it < tasks * 4; it += kSmemWarps) {
-        const int t = it >> 2, c0 = (it & 3) * 8;
-        const int bi = tri_row(t), bj = t - bi * (bi + 1) / 2;
-        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        rowdot8(pan + (size_t)bi * kTileF, pan + (size_t)bj * kTileF, c0, acc);
-        float* sp = tile(p + 1 + bi, p + 1 + bj) + lane * kP + c0;
-        const float4 s0 = *reinterpret_cast<const float4*>(sp);
-        const float4 s1 = *reinterpret_cast<const float4*>(sp + 4);
-        *reinterpret_cast<float4*>(sp) =
-            make_float4(s0.x - acc[0], s0.y - acc[1], s0.z - acc[2], s0.w - acc[3]);
-        *reinterpret_cast<float4*>(sp + 4) =
-            make_float4(s1.x - acc[4], s1.y - acc[5], s1.z - acc[6], s1.w - acc[7]);
-      }
-      // the panel back into its tiles (read by the inverse)
-      for (int e = threadIdx.x; e < m * kNb * kNb; e += blockDim.x) {
-        const int b = e >> 10, w = e & 1023, ii = w >> 5, jj = w & 31;
-        tile(p + 1 + b, p)[ii * kP + jj] = pan[(size_t)b * kTileF + ii * kP + jj];
-      }
-      __syncthreads();
-    }
-    ok = !failed;
-    __syncthreads();
-  }
-  if (!ok) {
-    if (threadIdx.x == 0) report_status(a.status, OUO_STATUS_BREAKDOWN);
-    for (int e = threadIdx.x; e < R * R; e += blockDim.x) {
-      const int i = e / R, j = e - (e / R) * R;
-      a.Linv[e] = i == j ? 1.f : 0.f;
-    }
-    return;
-  }
-  // X = L^-1 by block diagonals d = 1 .. nb - 1
-  for (int d = 1; d < nb; ++d) {
-    for (int it = warp; it < (nb - d) * 4; it += kSmemWarps) {
-      const int bj = it >> 2, bi = bj + d, c0 = (it & 3) * 8;
-      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      for (int k = bj; k < bi; ++k) {
-        float row[kNb];
-        load_row(tile(bi, k), row);
-        const float* X = a.Linv + (size_t)(k * kNb) * R + bj * kNb + c0;
-#pragma unroll
-        for (int q = 0; q < kNb; ++q) {
-          const float4 x0 = *reinterpret_cast<const float4*>(X + (size_t)q * R);
-          const float4 x1 = *reinterpret_cast<const float4*>(X + (size_t)q * R + 4);
-          acc[0] = fmaf(row[q], x0.x, acc[0]);
-          acc[1] = fmaf(row[q], x0.y, acc[1]);
-          acc[2] = fmaf(row[q], x0.z, acc[2]);
-          acc[3] = fmaf(row[q], x0.w, acc[3]);
-          acc[4] = fmaf(row[q], x1.x, acc[4]);
-          acc[5] = fmaf(row[q], x1.y, acc[5]);
-          acc[6] = fmaf(row[q], x1.z, acc[6]);
-          acc[7] = fmaf(row[q], x1.w, acc[7]);
-        }
-      }
-#pragma unroll
-      for (int c = 0; c < 8; ++c) stg[lane * 9 + c] = acc[c];
-      __syncwarp();
-      const float* Dg = a.Linv + (size_t)(bi * kNb + lane) * R + bi * kNb;
-      float o[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int q = 0; q < kNb; q += 4) {
-        const float4 dv = *reinterpret_cast<const float4*>(Dg + q);
-        const float dq[4] = {dv.x, dv.y, dv.z, dv.w};
-#pragma unroll
-        for (int u = 0; u < 4; ++u)
-#pragma unroll
-          for (int c = 0; c < 8; ++c) o[c] = fmaf(dq[u], stg[(q + u) * 9 + c], o[c]);
-      }
-      st8(a.Linv + (size_t)(bi * kNb + lane) * R + bj * kNb + c0, o, -1.f);
-      __syncwarp();
-    }
-    __syncthreads();
-  }
-}
-
 }  // namespace
 
 size_t chol_blocked_ctl_bytes(int r) { return 64 + (size_t)r * sizeof(double); }
 
-bool chol_smem_fits(int r) { return r >= 1 && ceil_div(r, kNb) <= kSmemMaxBlk; }
-
-int chol_smem(const float* S, int r, int64_t L, float* Linv, int* status,
-              cudaStream_t stream) {
-  if (!chol_smem_fits(r))
-    return set_error(OUO_ERR_UNSUPPORTED, "one-CTA blocked Cholesky takes 1 <= r <= %d",
-                     kSmemMaxBlk * kNb);
-  CholSArgs a;
-  a.S = S;
-  a.r = r;
-  a.nblk = (int)ceil_div(r, kNb);
-  a.R = a.nblk * kNb;
-  a.L = L;
-  a.Linv = Linv;
-  a.status = status;
-  static std::atomic<int> configured[64];  // zero-initialized (static storage)
-  int dev = 0;
-  OUO_CHECK_CUDA(cudaGetDevice(&dev));
-  if (dev < 0 || dev >= 64)
-    return set_error(OUO_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
-  if (!configured[dev].load(std::memory_order_relaxed)) {
-    OUO_CHECK_CUDA(cudaFuncSetAttribute(chol_smem_kernel,
-                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        (int)chol_smem_blocked_bytes(kSmemMaxBlk)));
-    configured[dev].store(1, std::memory_order_relaxed);
-  }
-  chol_smem_kernel<<<1, kSmemThreads, chol_smem_blocked_bytes(a.nblk), stream>>>(a);
-  OUO_CHECK_LAUNCH();
-  return OUO_OK;
-}
-
 int chol_blocked(const float* part, int splits, int r, int64_t L, float* S,
-                 float* Linv, void* ctl, int* status, cudaStream_t stream) {
+                 float* Linv, void* ctl, int* status, cudaStream_t stream,
+                 bool inverse) {
   CholBArgs a;
   a.part = part;
   a.splits = splits;
@@ -682,6 +402,7 @@ int chol_blocked(const float* part, int splits, int r, int64_t L, float* S,
   a.flags = reinterpret_cast<int*>(reinterpret_cast<char*>(ctl) + 16);
   a.diag = reinterpret_cast<double*>(reinterpret_cast<char*>(ctl) + 64);
   a.status = status;
+  a.inverse = inverse ? 1 : 0;
   OUO_CHECK_CUDA(cudaMemsetAsync(ctl, 0, 64, stream));
   // every CTA must be resident at once: at most one per SM times the
   // occupancy, and no more than the widest phase needs

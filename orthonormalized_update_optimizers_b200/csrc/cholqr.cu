@@ -1,0 +1,727 @@
+// Batched CholeskyQR pieces of the Dion / Orth-Dion step: every kernel here
+// takes a table of independent problems (one per matrix of a batch) and
+// runs them in one launch.
+//
+// Source: "Orth-Dion: Eliminating Geometric Mismatch in Distributed Low-Rank
+// Spectral Optimization", Problem Statement (the left factor of the power
+// iteration is orthonormalized) and Orth-Dion (the right factor is too, by
+// QR, instead of Dion's column normalization).  The QR of a block of r rows
+// X (r x L, r <= L) is computed as CholeskyQR: S = X X^T = L L^T, and the
+// rows of L^-1 X are orthonormal with the implied triangular factor L^T on
+// a positive diagonal, i.e. the unique QR factor.
+//
+//   gram     part[s] = X[:, chunk s] X[:, chunk s]^T: 64 x 64 tiles on or
+//            above the diagonal (upper storage), fp32 FMA, the L columns cut
+//            into chunks so that a single matrix fills the GPU.
+//   sum      S = sum_s part[s] in float64, fixed order, rounded to fp32
+//            (upper storage: entries (i, j) with j >= i are valid).
+//   chol     one CTA per matrix (r <= 256): the lower 32 x 32 blocks of S in
+//            shared memory, right-looking blocked Cholesky with one block of
+//            look-ahead; writes the strictly lower blocks L_ij and the
+//            inverses D_i = L_ii^-1 of the diagonal blocks.  A non-positive
+//            pivot restarts once with the shift of shifted CholeskyQR,
+//            11 (L r + r (r + 1)) u tr(S); a second failure reports
+//            OUO_STATUS_BREAKDOWN and writes the identity.
+//   trsm     Y = L^-1 X by block forward substitution, one CTA per 32-column
+//            strip of X: Y_i = D_i (X_i - sum_{k<i} L_ik Y_k).  Optional
+//            second copy and transposed copy of Y.
+//   rows     out = sum_s part[s] (split-K partial products) row by row, with
+//            optional row norms (float64, fixed order) and normalized rows
+//            (Dion's column normalization of R, stored transposed).
+#include <cmath>
+
+#include "internal.h"
+
+namespace ouo {
+namespace {
+
+constexpr int kB = 32;        // Cholesky / solve block
+constexpr int kGT = 64;       // Gram tile
+constexpr int kGK = 32;       // Gram K step
+
+// ------------------------------------------------------------------- gram
+struct GramBatch {
+  CholQrJob job[kChunk];
+  int64_t start[kChunk + 1];  // first work item of every job
+  int njob;
+};
+
+__device__ __forceinline__ int find_job(const int64_t* start, int njob, int64_t item) {
+  int lo = 0, hi = njob - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (start[mid] <= item) lo = mid;
+    else hi = mid - 1;
+  }
+  return lo;
+}
+
+// 256 threads: thread (ty, tx) owns rows ty*4 .. ty*4+3 and columns
+// tx*4 .. tx*4+3 of the 64 x 64 tile (ti, tj), ti <= tj.
+__global__ void __launch_bounds__(256) gram_kernel(const __grid_constant__ GramBatch gb) {
+  __shared__ __align__(16) float As[kGK][kGT + 4];
+  __shared__ __align__(16) float Bs[kGK][kGT + 4];
+  const int j = find_job(gb.start, gb.njob, blockIdx.x);
+  const CholQrJob& jb = gb.job[j];
+  const int tiles = (jb.r + kGT - 1) / kGT;
+  const int pairs = tiles * (tiles + 1) / 2;
+  int64_t t = blockIdx.x - gb.start[j];
+  const int split = (int)(t / pairs);
+  int pr = (int)(t - (int64_t)split * pairs);
+  int ti = 0;
+  while (pr >= tiles - ti) { pr -= tiles - ti; ++ti; }
+  const int tj = ti + pr;
+  const int64_t l0 = (int64_t)split * jb.gchunk;
+  const int64_t l1 = l0 + jb.gchunk < jb.L ? l0 + jb.gchunk : jb.L;
+  const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+  const float* X = jb.X;
+  const int64_t ld = jb.ldx;
+  float acc[4][4];
+#pragma unroll
+  for (int u = 0; u < 4; ++u)
+#pragma unroll
+    for (int v = 0; v < 4; ++v) acc[u][v] = 0.f;
+  // loader: 64 rows x 32 columns per operand = 512 float4, two per thread
+  const int lr = tid >> 3, lc = (tid & 7) * 4;
+  const bool vec = (ld & 3) == 0 && ((uintptr_t)X & 15) == 0;
+  for (int64_t k0 = l0; k0 < l1; k0 += kGK) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int rr = lr + 32 * h;
+      const int ra = ti * kGT + rr, rb = tj * kGT + rr;
+      const int64_t kc = k0 + lc;
+      float va[4] = {0.f, 0.f, 0.f, 0.f}, vb[4] = {0.f, 0.f, 0.f, 0.f};
+      if (vec && kc + 3 < l1) {
+        if (ra < jb.r) {
+          const float4 f = *reinterpret_cast<const float4*>(X + ra * ld + kc);
+          va[0] = f.x; va[1] = f.y; va[2] = f.z; va[3] = f.w;
+        }
+        if (rb < jb.r) {
+          const float4 f = *reinterpret_cast<const float4*>(X + rb * ld + kc);
+          vb[0] = f.x; vb[1] = f.y; vb[2] = f.z; vb[3] = f.w;
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          if (kc + e < l1) {
+            if (ra < jb.r) va[e] = X[ra * ld + kc + e];
+            if (rb < jb.r) vb[e] = X[rb * ld + kc + e];
+          }
+        }
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        As[lc + e][rr] = va[e];
+        Bs[lc + e][rr] = vb[e];
+      }
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int kk = 0; kk < kGK; ++kk) {
+      const float4 a4 = *reinterpret_cast<const float4*>(&As[kk][ty * 4]);
+      const float4 b4 = *reinterpret_cast<const float4*>(&Bs[kk][tx * 4]);
+      const float av[4] = {a4.x, a4.y, a4.z, a4.w};
+      const float bv[4] = {b4.x, b4.y, b4.z, b4.w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int v = 0; v < 4; ++v) acc[u][v] = fmaf(av[u], bv[v], acc[u][v]);
+    }
+    __syncthreads();
+  }
+  float* part = jb.gpart + (size_t)split * jb.r * jb.r;
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int i = ti * kGT + ty * 4 + u;
+    if (i >= jb.r) continue;
+#pragma unroll
+    for (int v = 0; v < 4; ++v) {
+      const int c = tj * kGT + tx * 4 + v;
+      if (c < jb.r) part[(size_t)i * jb.r + c] = acc[u][v];
+    }
+  }
+}
+
+// S[i][j] = sum_s part[s][i][j] (float64, s ascending) for the entries of
+// tiles on or above the diagonal.
+struct SumBatch {
+  const float* part[kChunk];
+  float* S[kChunk];
+  int r[kChunk], splits[kChunk];
+  int64_t start[kChunk + 1];  // prefix sums of r * r
+  int njob;
+};
+
+__global__ void __launch_bounds__(256) sum_kernel(const __grid_constant__ SumBatch sb) {
+  const int64_t total = sb.start[sb.njob];
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total;
+       e += (int64_t)gridDim.x * blockDim.x) {
+    const int j = find_job(sb.start, sb.njob, e);
+    const int64_t w = e - sb.start[j];
+    const int r = sb.r[j];
+    const int i = (int)(w / r), c = (int)(w - (w / r) * r);
+    if (c / kGT < i / kGT) {  // tile below the diagonal: no partials there
+      sb.S[j][w] = 0.f;
+      continue;
+    }
+    double s = 0.0;
+    const float* p = sb.part[j] + w;
+    for (int q = 0; q < sb.splits[j]; ++q) s += (double)p[(size_t)q * r * r];
+    sb.S[j][w] = (float)s;
+  }
+}
+
+// ------------------------------------------------------------------- chol
+constexpr int kCT = 512;             // threads of the Cholesky CTA
+constexpr int kCW = kCT / 32;        // warps
+constexpr int kP = 36;               // tile pitch (16-byte rows, conflict-free row reads)
+constexpr int kTF = kB * kP;         // floats per tile
+constexpr int kMaxNb = 8;            // blocks per side (r <= 256)
+
+struct CholBatch {
+  const float* S[kChunk];   // r x r, upper storage, ld r
+  float* Lb[kChunk];        // R x R, ld R
+  int r[kChunk];
+  int64_t L[kChunk];        // length of the rows (for the shift)
+  int njob;
+  int* status;
+};
+
+size_t chol_smem_bytes(int nb) {
+  const int ntri = nb * (nb + 1) / 2;
+  // lower tiles, D of the current block, the panel (nb - 1 tiles)
+  return (size_t)(ntri + 1 + (nb > 1 ? nb - 1 : 0)) * kTF * sizeof(float);
+}
+
+__device__ __forceinline__ int tri_index(int bi, int bj) { return bi * (bi + 1) / 2 + bj; }
+
+__device__ __forceinline__ int tri_row_of(int t) {
+  int bi = (int)((sqrtf(8.f * (float)t + 1.f) - 1.f) * 0.5f);
+  while ((bi + 1) * (bi + 2) / 2 <= t) ++bi;
+  while (bi * (bi + 1) / 2 > t) --bi;
+  return bi;
+}
+
+// One warp: factor the 32 x 32 block T (pitch kP, lower triangle used),
+// T = L L^T, leaving L in T, and write D = L^-1 (lower triangular, zeros
+// above) to Dt (pitch kP) and to global memory at g (row pitch ldg).
+// Returns false on a non-positive or non-finite pivot (the same in every
+// lane).
+__device__ __noinline__ bool chol_inv32(float* T, float* Dt, float* g, int64_t ldg) {
+  const unsigned full = 0xffffffffu;
+  const int lane = threadIdx.x & 31;
+  bool ok = true;
+  float my_inv = 0.f;  // 1 / L[lane][lane]
+  {
+    // row `lane` of the block in registers, right-looking: the pivot and
+    // the column below it are broadcast by shuffles
+    float l[kB];
+#pragma unroll
+    for (int k = 0; k < kB; k += 4) {
+      const float4 v = *reinterpret_cast<const float4*>(T + lane * kP + k);
+      l[k] = v.x; l[k + 1] = v.y; l[k + 2] = v.z; l[k + 3] = v.w;
+    }
+#pragma unroll
+    for (int k = 0; k < kB; ++k) {
+      const float piv = __shfl_sync(full, l[k], k);
+      // a bad pivot is the same in every lane; the sweep runs on (its
+      // values are discarded) so that the loop stays fully unrolled
+      if (!(piv > 0.f) || !(piv < INFINITY)) ok = false;
+      const float rs = rsqrtf(piv);
+      if (lane == k) { l[k] = piv * rs; my_inv = rs; }
+      else if (lane > k) l[k] *= rs;
+      const float lk = l[k];
+#pragma unroll
+      for (int j = k + 1; j < kB; ++j) {
+        const float ljk = __shfl_sync(full, lk, j);
+        if (lane >= j) l[j] = fmaf(-lk, ljk, l[j]);
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < kB; k += 4)
+      *reinterpret_cast<float4*>(T + lane * kP + k) = make_float4(l[k], l[k + 1], l[k + 2], l[k + 3]);
+  }
+  __syncwarp();
+  // column `lane` of L^-1 by a column sweep: x[k] = acc[k] / L[k][k], then
+  // every later row r loses L[r][k] x[k] (L read back from T, broadcast)
+  float acc[kB];
+#pragma unroll
+  for (int r = 0; r < kB; ++r) acc[r] = r == lane ? 1.f : 0.f;
+#pragma unroll
+  for (int k = 0; k < kB; ++k) {
+    const float xk = acc[k] * __shfl_sync(full, my_inv, k);
+    acc[k] = xk;
+#pragma unroll
+    for (int r = k + 1; r < kB; ++r) acc[r] = fmaf(-T[r * kP + k], xk, acc[r]);
+  }
+  // acc[r] = D[r][lane]; lanes write column `lane`
+#pragma unroll
+  for (int r = 0; r < kB; ++r) {
+    Dt[r * kP + lane] = acc[r];
+    g[(int64_t)r * ldg + lane] = acc[r];
+  }
+  return ok;
+}
+
+// acc[c] += sum_k A[lane][k] B[c0 + c][k], c < 8 (tiles of pitch kP)
+__device__ __forceinline__ void rowdot8(const float* A, const float* B, int c0, float (&acc)[8]) {
+  const int lane = threadIdx.x & 31;
+  float row[kB];
+#pragma unroll
+  for (int k = 0; k < kB; k += 4) {
+    const float4 v = *reinterpret_cast<const float4*>(A + lane * kP + k);
+    row[k] = v.x; row[k + 1] = v.y; row[k + 2] = v.z; row[k + 3] = v.w;
+  }
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    const float* bp = B + (c0 + c) * kP;
+#pragma unroll
+    for (int k = 0; k < kB; k += 4) {
+      const float4 v = *reinterpret_cast<const float4*>(bp + k);
+      acc[c] = fmaf(row[k], v.x, acc[c]);
+      acc[c] = fmaf(row[k + 1], v.y, acc[c]);
+      acc[c] = fmaf(row[k + 2], v.z, acc[c]);
+      acc[c] = fmaf(row[k + 3], v.w, acc[c]);
+    }
+  }
+}
+
+// tile(bi, bj) -= A B^T over columns c0 .. c0 + 7 (row = lane)
+__device__ __forceinline__ void sub_rowdot8(float* Tt, const float* A, const float* B, int c0) {
+  const int lane = threadIdx.x & 31;
+  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  rowdot8(A, B, c0, acc);
+  float* sp = Tt + lane * kP + c0;
+  const float4 s0 = *reinterpret_cast<const float4*>(sp);
+  const float4 s1 = *reinterpret_cast<const float4*>(sp + 4);
+  *reinterpret_cast<float4*>(sp) =
+      make_float4(s0.x - acc[0], s0.y - acc[1], s0.z - acc[2], s0.w - acc[3]);
+  *reinterpret_cast<float4*>(sp + 4) =
+      make_float4(s1.x - acc[4], s1.y - acc[5], s1.z - acc[6], s1.w - acc[7]);
+}
+
+__global__ void __launch_bounds__(kCT, 1) chol_kernel(const __grid_constant__ CholBatch cb) {
+  extern __shared__ __align__(16) float sm[];
+  __shared__ int s_bad;
+  __shared__ double s_red[kCW];
+  const int job = blockIdx.x;
+  const float* S = cb.S[job];
+  float* Lb = cb.Lb[job];
+  const int r = cb.r[job];
+  const int nb = (r + kB - 1) / kB, R = nb * kB;
+  const int ntri = nb * (nb + 1) / 2;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  auto tile = [&](int bi, int bj) { return sm + (size_t)tri_index(bi, bj) * kTF; };
+  float* Dt = sm + (size_t)ntri * kTF;
+  float* pan = Dt + kTF;
+  auto gblk = [&](int bi, int bj) { return Lb + (size_t)bi * kB * R + (size_t)bj * kB; };
+
+  bool ok = false;
+  for (int attempt = 0; attempt < 2 && !ok; ++attempt) {
+    double shift = 0.0;
+    if (attempt == 1) {
+      double t = 0.0;
+      for (int i = threadIdx.x; i < r; i += kCT) t += (double)S[(size_t)i * r + i];
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) t += __shfl_xor_sync(0xffffffffu, t, off);
+      if (lane == 0) s_red[warp] = t;
+      __syncthreads();
+      double tr = 0.0;
+      for (int w = 0; w < kCW; ++w) tr += s_red[w];
+      const double u = 5.9604644775390625e-8;  // 2^-24
+      shift = 11.0 * ((double)cb.L[job] * r + (double)r * (r + 1)) * u * tr;
+      if (!(shift > 0.0)) shift = 1e-30;
+      __syncthreads();
+    }
+    // lower tiles from the upper storage: tile (bi, bj)[ii][jj] = S[j][i]
+    // with i = bi*32 + ii, j = bj*32 + jj, identity padding past r.
+    // Asynchronous 4-byte copies keep the whole matrix in flight at once
+    // (one CTA streaming it with one load per thread at a time would wait
+    // on memory latency for every element).
+    for (int e = threadIdx.x; e < ntri * kB * kB; e += kCT) {
+      const int tt = e >> 10, w = e & 1023, jj = w >> 5, ii = w & 31;
+      const int bi = tri_row_of(tt), bj = tt - bi * (bi + 1) / 2;
+      const int i = bi * kB + ii, j = bj * kB + jj;
+      float* d = sm + (size_t)tt * kTF + ii * kP + jj;
+      if (i < r && j < r && j <= i) {
+        const unsigned da = (unsigned)__cvta_generic_to_shared(d);
+        asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(da),
+                     "l"(S + (size_t)j * r + i) : "memory");
+      } else {
+        *d = i == j ? 1.f : 0.f;
+      }
+    }
+    asm volatile("cp.async.wait_all;\n" ::: "memory");
+    __syncthreads();
+    if (shift != 0.0) {
+      for (int i = threadIdx.x; i < r; i += kCT) {
+        float* d = tile(i / kB, i / kB) + (i % kB) * kP + (i % kB);
+        *d = (float)((double)*d + shift);
+      }
+    }
+    if (threadIdx.x == 0) s_bad = 0;
+    __syncthreads();
+    if (warp == 0 && !chol_inv32(tile(0, 0), Dt, gblk(0, 0), R) && lane == 0) s_bad = 1;
+    __syncthreads();
+    bool failed = s_bad != 0;
+    for (int p = 0; p < nb && !failed; ++p) {
+      const int m = nb - 1 - p;
+      if (m == 0) break;
+      // panel: pan[b] = S(p+1+b, p) D_p^T
+      for (int it = warp; it < 4 * m; it += kCW) {
+        const int bb = it >> 2, c0 = (it & 3) * 8;
+        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        rowdot8(tile(p + 1 + bb, p), Dt, c0, acc);
+        float* dst = pan + (size_t)bb * kTF + lane * kP + c0;
+        *reinterpret_cast<float4*>(dst) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+        *reinterpret_cast<float4*>(dst + 4) = make_float4(acc[4], acc[5], acc[6], acc[7]);
+      }
+      __syncthreads();
+      // the panel blocks L_{p+1+b, p} to global memory
+      for (int e = threadIdx.x; e < m * kB * kB; e += kCT) {
+        const int bb = e >> 10, w = e & 1023, ii = w >> 5, jj = w & 31;
+        gblk(p + 1 + bb, p)[(size_t)ii * R + jj] = pan[(size_t)bb * kTF + ii * kP + jj];
+      }
+      // look-ahead: the next diagonal block first (warps 0-3), then warp 0
+      // factors it while the other warps finish the trailing update
+      if (warp < 4) {
+        sub_rowdot8(tile(p + 1, p + 1), pan, pan, warp * 8);
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        if (warp == 0 && !chol_inv32(tile(p + 1, p + 1), Dt, gblk(p + 1, p + 1), R) && lane == 0)
+          s_bad = 1;
+      }
+      if (warp > 0) {
+        // trailing: S(p+1+bi, p+1+bj) -= pan[bi] pan[bj]^T, bj <= bi, except (0, 0)
+        const int tasks = m * (m + 1) / 2 - 1;
+        for (int it = warp - 1; it < 4 * tasks; it += kCW - 1) {
+          const int t = (it >> 2) + 1, c0 = (it & 3) * 8;
+          const int bi = tri_row_of(t), bj = t - bi * (bi + 1) / 2;
+          sub_rowdot8(tile(p + 1 + bi, p + 1 + bj), pan + (size_t)bi * kTF,
+                      pan + (size_t)bj * kTF, c0);
+        }
+      }
+      __syncthreads();
+      failed = s_bad != 0;
+    }
+    ok = !failed;
+    __syncthreads();
+  }
+  if (!ok) {
+    // breakdown survived the shift: L^-1 = I (the solve copies X)
+    if (threadIdx.x == 0) report_status(cb.status, OUO_STATUS_BREAKDOWN);
+    for (int e = threadIdx.x; e < R * R; e += kCT) {
+      const int i = e / R, j = e - (e / R) * R;
+      if (j / kB <= i / kB) Lb[e] = i == j ? 1.f : 0.f;
+    }
+  }
+}
+
+// ------------------------------------------------------------------- trsm
+constexpr int kSP = 36;  // strip pitch (32 columns + pad, 16-byte rows)
+
+struct TrsmBatch {
+  CholQrJob job[kChunk];
+  int64_t start[kChunk + 1];  // first strip of every job
+  int njob;
+};
+
+__global__ void __launch_bounds__(256) trsm_kernel(const __grid_constant__ TrsmBatch tb) {
+  extern __shared__ __align__(16) float xs[];  // R x kSP
+  const int j = find_job(tb.start, tb.njob, blockIdx.x);
+  const CholQrJob& jb = tb.job[j];
+  const int64_t c0g = (blockIdx.x - tb.start[j]) * kB;  // first column of the strip
+  const int r = jb.r, nb = (r + kB - 1) / kB, R = nb * kB;
+  const int tid = threadIdx.x;
+  const int64_t ncol = jb.L - c0g < kB ? jb.L - c0g : kB;
+  // strip in: xs[i][c] = X[i][c0g + c], zero past r or L
+  {
+    const bool vec = (jb.ldx & 3) == 0 && ((uintptr_t)jb.X & 15) == 0 && ncol == kB;
+    for (int e = tid; e < R * 8; e += 256) {
+      const int i = e >> 3, c = (e & 7) * 4;
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (i < r) {
+        const float* src = jb.X + (int64_t)i * jb.ldx + c0g + c;
+        if (vec) {
+          v = *reinterpret_cast<const float4*>(src);
+        } else {
+          float t[4] = {0.f, 0.f, 0.f, 0.f};
+          for (int q = 0; q < 4; ++q)
+            if (c + q < ncol) t[q] = src[q];
+          v = make_float4(t[0], t[1], t[2], t[3]);
+        }
+      }
+      *reinterpret_cast<float4*>(xs + i * kSP + c) = v;
+    }
+  }
+  __syncthreads();
+  const int row = tid >> 3, cc = (tid & 7) * 4;
+  const float* Lb = jb.Lb;
+  for (int i = 0; i < nb; ++i) {
+    // Y_i = D_i X_i
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    {
+      const float* Drow = (jb.Dd ? jb.Dd : Lb) + (size_t)(i * kB + row) * R + i * kB;
+#pragma unroll
+      for (int k = 0; k < kB; k += 4) {
+        const float4 d = __ldg(reinterpret_cast<const float4*>(Drow + k));
+        const float dv[4] = {d.x, d.y, d.z, d.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float4 x = *reinterpret_cast<const float4*>(xs + (i * kB + k + q) * kSP + cc);
+          acc.x = fmaf(dv[q], x.x, acc.x);
+          acc.y = fmaf(dv[q], x.y, acc.y);
+          acc.z = fmaf(dv[q], x.z, acc.z);
+          acc.w = fmaf(dv[q], x.w, acc.w);
+        }
+      }
+    }
+    __syncthreads();
+    *reinterpret_cast<float4*>(xs + (i * kB + row) * kSP + cc) = acc;
+    __syncthreads();
+    // X_b -= L_bi Y_i for the blocks below
+    for (int bb = i + 1; bb < nb; ++bb) {
+      const float* Lrow = Lb + (size_t)(bb * kB + row) * R + i * kB;
+      float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int k = 0; k < kB; k += 4) {
+        const float4 l = __ldg(reinterpret_cast<const float4*>(Lrow + k));
+        const float lv[4] = {l.x, l.y, l.z, l.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float4 y = *reinterpret_cast<const float4*>(xs + (i * kB + k + q) * kSP + cc);
+          s.x = fmaf(lv[q], y.x, s.x);
+          s.y = fmaf(lv[q], y.y, s.y);
+          s.z = fmaf(lv[q], y.z, s.z);
+          s.w = fmaf(lv[q], y.w, s.w);
+        }
+      }
+      float* xp = xs + (bb * kB + row) * kSP + cc;
+      float4 x = *reinterpret_cast<float4*>(xp);
+      x.x -= s.x; x.y -= s.y; x.z -= s.z; x.w -= s.w;
+      *reinterpret_cast<float4*>(xp) = x;
+    }
+    __syncthreads();
+  }
+  // out: Y (and its copy) row-major, Y^T (L x r)
+  for (int e = tid; e < r * 8; e += 256) {
+    const int i = e >> 3, c = (e & 7) * 4;
+    const float4 v = *reinterpret_cast<const float4*>(xs + i * kSP + c);
+    const float vv[4] = {v.x, v.y, v.z, v.w};
+    float* outs[2] = {jb.Y, jb.Y2};
+    const int64_t lds[2] = {jb.ldy, jb.ldy2};
+#pragma unroll
+    for (int o = 0; o < 2; ++o) {
+      if (!outs[o]) continue;
+      float* dst = outs[o] + (int64_t)i * lds[o] + c0g + c;
+      if (ncol == kB && (lds[o] & 3) == 0 && ((uintptr_t)outs[o] & 15) == 0) {
+        *reinterpret_cast<float4*>(dst) = v;
+      } else {
+        for (int q = 0; q < 4; ++q)
+          if (c + q < ncol) dst[q] = vv[q];
+      }
+    }
+  }
+  if (jb.Yt) {
+    for (int c = 0; c < ncol; ++c)
+      for (int i = tid; i < r; i += 256) jb.Yt[(c0g + c) * jb.ldyt + i] = xs[i * kSP + c];
+  }
+}
+
+// ------------------------------------------------------------------- rows
+struct RowsBatch {
+  RowsJob job[kChunk];
+  int64_t start[kChunk + 1];  // first row of every job
+  int njob;
+  float eps;
+};
+
+__global__ void __launch_bounds__(256) rows_kernel(const __grid_constant__ RowsBatch rb) {
+  __shared__ double red[8];
+  const int j = find_job(rb.start, rb.njob, blockIdx.x);
+  const RowsJob& jb = rb.job[j];
+  const int64_t c = blockIdx.x - rb.start[j];
+  const int64_t n = jb.n;
+  const float* src = jb.part + c * jb.ldp;
+  const bool vec = (jb.ldp & 3) == 0 && (jb.sp & 3) == 0 && ((uintptr_t)jb.part & 15) == 0 &&
+                   (!jb.out || ((jb.ldo & 3) == 0 && ((uintptr_t)jb.out & 15) == 0));
+  const bool want_norm = jb.sigma || jb.qn;
+  double ss = 0.0;
+  float* orow = jb.out ? jb.out + c * jb.ldo : nullptr;
+  if (vec) {
+    for (int64_t e = 4 * (int64_t)threadIdx.x; e < (n & ~3LL); e += 4 * blockDim.x) {
+      float4 v = *reinterpret_cast<const float4*>(src + e);
+      for (int q = 1; q < jb.ks; ++q) {
+        const float4 w = *reinterpret_cast<const float4*>(src + q * jb.sp + e);
+        v.x += w.x; v.y += w.y; v.z += w.z; v.w += w.w;
+      }
+      if (orow) *reinterpret_cast<float4*>(orow + e) = v;
+      if (want_norm)
+        ss += (double)v.x * v.x + (double)v.y * v.y + (double)v.z * v.z + (double)v.w * v.w;
+    }
+  }
+  for (int64_t e = (vec ? (n & ~3LL) : 0) + threadIdx.x; e < n; e += blockDim.x) {
+    float v = src[e];
+    for (int q = 1; q < jb.ks; ++q) v += src[q * jb.sp + e];
+    if (orow) orow[e] = v;
+    if (want_norm) ss += (double)v * v;
+  }
+  if (!want_norm) return;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+  __syncthreads();
+  double tot = 0.0;
+  for (int w = 0; w < 8; ++w) tot += red[w];
+  const double nrm = sqrt(tot);
+  if (jb.sigma && threadIdx.x == 0) jb.sigma[c] = (float)nrm;
+  if (!jb.qn) return;
+  const float inv = (float)(1.0 / (nrm + (double)rb.eps));
+  // the summed row is read back from where this thread wrote it (orow), or
+  // summed again from the partials
+  for (int64_t e = threadIdx.x; e < n; e += blockDim.x) {
+    float v;
+    if (orow) {
+      v = orow[e];
+    } else {
+      v = src[e];
+      for (int q = 1; q < jb.ks; ++q) v += src[q * jb.sp + e];
+    }
+    const float qv = v * inv;
+    jb.qn[c * jb.ldq + e] = qv;
+    if (jb.q2) jb.q2[c * jb.ldq2 + e] = qv;
+  }
+}
+
+unsigned grid_cap(int64_t n, int per_block) {
+  int64_t b = ceil_div(n, per_block);
+  const int64_t cap = (int64_t)num_sms() * 8;
+  if (b > cap) b = cap;
+  return (unsigned)(b < 1 ? 1 : b);
+}
+
+int set_smem_attr(const void* fn, size_t bytes) {
+  static int done[64][4] = {{0}};
+  int dev = 0;
+  OUO_CHECK_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return set_error(OUO_ERR_UNSUPPORTED, "device ordinal %d", dev);
+  const int slot = fn == (const void*)chol_kernel ? 0 : 1;
+  if (!done[dev][slot]) {
+    OUO_CHECK_CUDA(cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        slot == 0 ? (int)chol_smem_bytes(kMaxNb)
+                                                  : (int)(1024 * kSP * sizeof(float))));
+    done[dev][slot] = 1;
+  }
+  (void)bytes;
+  return OUO_OK;
+}
+
+}  // namespace
+
+int cholqr_gram_splits(int r, int64_t L) {
+  const int tiles = (int)ceil_div(r, kGT);
+  const int pairs = tiles * (tiles + 1) / 2;
+  int64_t want = ceil_div((int64_t)num_sms() * 2, pairs);
+  const int64_t maxs = ceil_div(L, 256);  // at least 256 columns per split
+  if (want > maxs) want = maxs;
+  if (want < 1) want = 1;
+  if (want > 64) want = 64;
+  return (int)want;
+}
+
+int cholqr_gram(const std::vector<CholQrJob>& jobs, cudaStream_t s) {
+  for (size_t c0 = 0; c0 < jobs.size(); c0 += kChunk) {
+    const int cn = (int)(jobs.size() - c0 < (size_t)kChunk ? jobs.size() - c0 : kChunk);
+    GramBatch gb;
+    SumBatch sb;
+    gb.njob = sb.njob = cn;
+    gb.start[0] = sb.start[0] = 0;
+    int64_t total_sum = 0;
+    for (int i = 0; i < cn; ++i) {
+      CholQrJob jb = jobs[c0 + i];
+      const int tiles = (int)ceil_div(jb.r, kGT);
+      const int64_t splits = ceil_div(jb.L, jb.gchunk);
+      gb.job[i] = jb;
+      gb.start[i + 1] = gb.start[i] + splits * (tiles * (tiles + 1) / 2);
+      sb.part[i] = jb.gpart;
+      sb.S[i] = jb.S;
+      sb.r[i] = jb.r;
+      sb.splits[i] = (int)splits;
+      sb.start[i + 1] = sb.start[i] + (int64_t)jb.r * jb.r;
+      total_sum += (int64_t)jb.r * jb.r;
+    }
+    gram_kernel<<<(unsigned)gb.start[cn], 256, 0, s>>>(gb);
+    OUO_CHECK_LAUNCH();
+    sum_kernel<<<grid_cap(total_sum, 256), 256, 0, s>>>(sb);
+    OUO_CHECK_LAUNCH();
+  }
+  return OUO_OK;
+}
+
+bool cholqr_small_rank(int r) { return r >= 1 && r <= kMaxNb * kB; }
+
+int cholqr_factor(const std::vector<CholQrJob>& jobs, int* status, cudaStream_t s) {
+  OUO_TRY(set_smem_attr((const void*)chol_kernel, 0));
+  for (size_t c0 = 0; c0 < jobs.size(); c0 += kChunk) {
+    const int cn = (int)(jobs.size() - c0 < (size_t)kChunk ? jobs.size() - c0 : kChunk);
+    CholBatch cb;
+    cb.njob = cn;
+    cb.status = status;
+    int nbmax = 1;
+    for (int i = 0; i < cn; ++i) {
+      const CholQrJob& jb = jobs[c0 + i];
+      if (!cholqr_small_rank(jb.r))
+        return set_error(OUO_ERR_UNSUPPORTED, "one-CTA Cholesky takes r <= %d", kMaxNb * kB);
+      cb.S[i] = jb.S;
+      cb.Lb[i] = jb.Lb;
+      cb.r[i] = jb.r;
+      cb.L[i] = jb.L;
+      const int nb = (int)ceil_div(jb.r, kB);
+      if (nb > nbmax) nbmax = nb;
+    }
+    chol_kernel<<<cn, kCT, chol_smem_bytes(nbmax), s>>>(cb);
+    OUO_CHECK_LAUNCH();
+  }
+  return OUO_OK;
+}
+
+int cholqr_apply(const std::vector<CholQrJob>& jobs, cudaStream_t s) {
+  OUO_TRY(set_smem_attr((const void*)trsm_kernel, 0));
+  for (size_t c0 = 0; c0 < jobs.size(); c0 += kChunk) {
+    const int cn = (int)(jobs.size() - c0 < (size_t)kChunk ? jobs.size() - c0 : kChunk);
+    TrsmBatch tb;
+    tb.njob = cn;
+    tb.start[0] = 0;
+    int Rmax = kB;
+    for (int i = 0; i < cn; ++i) {
+      const CholQrJob& jb = jobs[c0 + i];
+      const int R = (int)(ceil_div(jb.r, kB) * kB);
+      if (R > 1024) return set_error(OUO_ERR_UNSUPPORTED, "triangular solve takes r <= 1024");
+      if (R > Rmax) Rmax = R;
+      tb.job[i] = jb;
+      tb.start[i + 1] = tb.start[i] + ceil_div(jb.L, kB);
+    }
+    trsm_kernel<<<(unsigned)tb.start[cn], 256, (size_t)Rmax * kSP * sizeof(float), s>>>(tb);
+    OUO_CHECK_LAUNCH();
+  }
+  return OUO_OK;
+}
+
+int rows_reduce(const std::vector<RowsJob>& jobs, float eps, cudaStream_t s) {
+  for (size_t c0 = 0; c0 < jobs.size(); c0 += kChunk) {
+    const int cn = (int)(jobs.size() - c0 < (size_t)kChunk ? jobs.size() - c0 : kChunk);
+    RowsBatch rb;
+    rb.njob = cn;
+    rb.eps = eps;
+    rb.start[0] = 0;
+    for (int i = 0; i < cn; ++i) {
+      rb.job[i] = jobs[c0 + i];
+      rb.start[i + 1] = rb.start[i] + jobs[c0 + i].rows;
+    }
+    if (rb.start[cn] == 0) continue;
+    rows_kernel<<<(unsigned)rb.start[cn], 256, 0, s>>>(rb);
+    OUO_CHECK_LAUNCH();
+  }
+  return OUO_OK;
+}
+
+}  // namespace ouo

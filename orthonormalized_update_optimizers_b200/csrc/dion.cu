@@ -1,4 +1,4 @@
-// Dion / Orth-Dion low-rank step.
+// Dion / Orth-Dion low-rank step, batched across the matrices of a call.
 //
 // Source: "Orth-Dion: Eliminating Geometric Mismatch in Distributed Low-Rank
 // Spectral Optimization" -- Problem Statement (rank-r factors from a single
@@ -8,253 +8,34 @@
 // Contributions (error-feedback coefficient beta); "Dion: The Distributed
 // Orthonormal Update Revolution Is Here", Technical details.
 //
-// Per matrix (B is the momentum buffer after B = M + G, m x n fp32):
-//   Pt = Qt B^T                      (r x m; Qt = Q_prev^T is the state)
+// Per matrix (B is the momentum buffer after B = M + G, m x n fp32; the
+// state Qt is the right factor transposed, r x n):
+//   Pt = Qt B^T                      (r x m)
 //   Pt <- rows orthonormalized       (CholeskyQR2: P = orth(B Q_prev))
 //   Rt = Pt B                        (r x n; R = B^T P)
 //   Qt_new = rows of Rt normalized   (Dion)  or  rows orthonormalized (Orth-Dion)
 //   M <- beta B - (beta - mu) P Rt   (residual buffer / error feedback)
 //   W <- (1 - lr wd) W - lr s P Qt_new
 //   state <- Qt_new
-// Working in the transposed layouts keeps every large product on the
-// tcgen05 GEMM (tf32 operands, fp32 accumulation) with K-major A.  The
-// orthonormalization works on r x L row blocks X: S = X X^T in fp32 (split
-// over L, partial sums added in float64 in a fixed order), S = L L^T by a
-// one-CTA Cholesky (r <= 64) or the blocked cooperative Cholesky of chol.cu
-// (wider ranks), L inverted, X <- L^-1 X (rows orthonormal; the
-// implied R = L^T has a positive diagonal, the unique QR).  Two passes
-// (CholeskyQR2).  A failed pivot retries with the shift of shifted
-// CholeskyQR (11 (L r + r (r + 1)) u ||X||_F^2); a second failure sets
-// OUO_STATUS_BREAKDOWN.
+// Every stage is one batched launch over all matrices (or a few, for very
+// large batches): the momentum pass; the two projections on the tensor
+// cores (tf32 operands, fp32 accumulation), grouped by shape and split
+// along K when a matrix alone has too few output tiles to fill the GPU; the
+// CholeskyQR passes (Gram matrices, one Cholesky CTA per matrix, block
+// triangular solves; cholqr.cu); the row reductions / column
+// normalization; and the two in-place rank-r updates.  Per-matrix choices
+// (split counts, Gram chunks, tile shapes) depend only on that matrix's
+// shape and rank, so a batch computes what one call per matrix computes,
+// bit for bit.
 #include <cmath>
 #include <cstdlib>
+#include <map>
+#include <tuple>
 
 #include "internal.h"
 
 namespace ouo {
 namespace {
-
-// --------------------------------------------------------------- Gram S
-constexpr int kGT = 32;  // Gram tile
-
-struct GramArgs {
-  const float* X;
-  int64_t ld;
-  int r;
-  int64_t L, chunk;
-  float* part;  // [splits][r][r]
-  int tiles;    // ceil(r / 32)
-};
-
-// grid.x: upper tile pairs (ti <= tj), grid.y: split of the L range.
-__global__ void __launch_bounds__(256) gram_partial_kernel(const GramArgs a) {
-  __shared__ float xi[kGT][kGT + 1];
-  __shared__ float xj[kGT][kGT + 1];
-  int t = blockIdx.x, ti = 0;
-  while (t >= a.tiles - ti) { t -= a.tiles - ti; ++ti; }
-  const int tj = ti + t;
-  const int64_t l0 = (int64_t)blockIdx.y * a.chunk;
-  const int64_t l1 = l0 + a.chunk < a.L ? l0 + a.chunk : a.L;
-  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
-  for (int64_t k0 = l0; k0 < l1; k0 += kGT) {
-    for (int e = threadIdx.x; e < kGT * kGT; e += 256) {
-      const int rr = e >> 5, kk = e & 31;
-      const int64_t k = k0 + kk;
-      const int ri = ti * kGT + rr, rj = tj * kGT + rr;
-      xi[kk][rr] = (ri < a.r && k < l1) ? a.X[ri * a.ld + k] : 0.f;
-      xj[kk][rr] = (rj < a.r && k < l1) ? a.X[rj * a.ld + k] : 0.f;
-    }
-    __syncthreads();
-#pragma unroll 8
-    for (int kk = 0; kk < kGT; ++kk) {
-      const float bj = xj[kk][tx];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) acc[u] = __fmaf_rn(xi[kk][ty + 8 * u], bj, acc[u]);
-    }
-    __syncthreads();
-  }
-  float* part = a.part + (size_t)blockIdx.y * a.r * a.r;
-  const int j = tj * kGT + tx;
-#pragma unroll
-  for (int u = 0; u < 4; ++u) {
-    const int i = ti * kGT + ty + 8 * u;
-    if (i < a.r && j < a.r) {
-      part[(size_t)i * a.r + j] = acc[u];
-      part[(size_t)j * a.r + i] = acc[u];
-    }
-  }
-}
-
-// ---------------------------------------------------- Cholesky + inverse
-// One CTA, ranks up to 128 (by default up to 64; larger ones use the
-// blocked kernel in chol.cu).
-// S is summed from the partials in float64 (fixed order) and kept as a
-// packed lower triangle (fp32) in shared memory.
-// Cholesky S = L L^T in place, then L^-1 in place, then written as a full
-// lower-triangular r x r row-major fp32 matrix.
-__device__ __forceinline__ int tri_at(int i, int j) {  // j <= i
-  return i * (i + 1) / 2 + j;
-}
-
-struct CholArgs {
-  const float* part;
-  int splits;
-  int r;
-  int64_t L;        // length of the rows of X (for the shift)
-  float* Linv;      // r x r out, row pitch ldl
-  int64_t ldl;
-  int* status;
-};
-
-__device__ void chol_load(const CholArgs& a, float* tri, float shift) {
-  const int n = a.r * (a.r + 1) / 2;
-  for (int e = threadIdx.x; e < n; e += blockDim.x) {
-    // invert e -> (i, j), j <= i
-    int i = (int)((sqrtf(8.f * (float)e + 1.f) - 1.f) * 0.5f);
-    while (tri_at(i + 1, 0) <= e) ++i;
-    while (tri_at(i, 0) > e) --i;
-    const int j = e - tri_at(i, 0);
-    double s = 0.0;
-    for (int p = 0; p < a.splits; ++p)
-      s += (double)a.part[(size_t)p * a.r * a.r + (size_t)i * a.r + j];
-    if (i == j) s += (double)shift;
-    tri[e] = (float)s;
-  }
-  __syncthreads();
-}
-
-// Right-looking Cholesky in place; returns false if a pivot is not positive.
-__device__ bool chol_factor(const CholArgs& a, float* tri, int* s_fail) {
-  const int r = a.r;
-  if (threadIdx.x == 0) *s_fail = 0;
-  __syncthreads();
-  for (int k = 0; k < r; ++k) {
-    const float piv = tri[tri_at(k, k)];
-    if (!(piv > 0.f) || !isfinite(piv)) {
-      if (threadIdx.x == 0) *s_fail = 1;
-      __syncthreads();
-      return false;
-    }
-    const float d = sqrtf(piv);
-    const float inv = 1.0f / d;
-    __syncthreads();
-    if (threadIdx.x == 0) tri[tri_at(k, k)] = d;
-    for (int i = k + 1 + threadIdx.x; i < r; i += blockDim.x) tri[tri_at(i, k)] *= inv;
-    __syncthreads();
-    // trailing update S[i][j] -= L[i][k] L[j][k], k < j <= i
-    const int m = r - k - 1;
-    const int cnt = m * (m + 1) / 2;
-    for (int e = threadIdx.x; e < cnt; e += blockDim.x) {
-      int ii = (int)((sqrtf(8.f * (float)e + 1.f) - 1.f) * 0.5f);
-      while ((ii + 1) * (ii + 2) / 2 <= e) ++ii;
-      while (ii * (ii + 1) / 2 > e) --ii;
-      const int jj = e - ii * (ii + 1) / 2;
-      const int i = k + 1 + ii, j = k + 1 + jj;
-      tri[tri_at(i, j)] -= tri[tri_at(i, k)] * tri[tri_at(j, k)];
-    }
-    __syncthreads();
-  }
-  return true;
-}
-
-// In-place inverse of the packed lower-triangular L (column j from the
-// last to the first: L^-1[j+1:, j] = -L^-1[j+1:, j+1:] L[j+1:, j] / L[j][j]).
-__device__ void tri_invert(const CholArgs& a, float* tri, float* tmp) {
-  const int r = a.r;
-  for (int j = r - 1; j >= 0; --j) {
-    const float djj = 1.0f / tri[tri_at(j, j)];
-    // tmp = L[j+1:, j] (original column)
-    for (int i = j + 1 + threadIdx.x; i < r; i += blockDim.x) tmp[i] = tri[tri_at(i, j)];
-    __syncthreads();
-    for (int i = j + 1 + threadIdx.x; i < r; i += blockDim.x) {
-      float s = 0.f;
-      for (int k = j + 1; k <= i; ++k) s = __fmaf_rn(tri[tri_at(i, k)], tmp[k], s);
-      tri[tri_at(i, j)] = -s * djj;
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) tri[tri_at(j, j)] = djj;
-    __syncthreads();
-  }
-}
-
-__global__ void __launch_bounds__(1024) chol_inv_kernel(const CholArgs a) {
-  extern __shared__ float sm[];
-  __shared__ int s_fail;
-  const int r = a.r;
-  float* tri = sm;
-  float* tmp = sm + r * (r + 1) / 2;
-  chol_load(a, tri, 0.f);
-  if (!chol_factor(a, tri, &s_fail)) {
-    // shifted CholeskyQR: 11 (L r + r (r + 1)) u ||X||_F^2, ||X||_F^2 = tr S
-    __shared__ float s_trace;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      double tr = 0.0;
-      for (int i = 0; i < r; ++i)
-        for (int p = 0; p < a.splits; ++p)
-          tr += (double)a.part[(size_t)p * r * r + (size_t)i * r + i];
-      const double u = 5.9604644775390625e-8;  // 2^-24
-      s_trace = (float)(11.0 * ((double)a.L * r + (double)r * (r + 1)) * u * tr);
-    }
-    __syncthreads();
-    chol_load(a, tri, s_trace > 0.f ? s_trace : 1e-30f);
-    if (!chol_factor(a, tri, &s_fail)) {
-      if (threadIdx.x == 0) report_status(a.status, OUO_STATUS_BREAKDOWN);
-      // keep going with unit pivots where the factorization failed
-      __syncthreads();
-      for (int e = threadIdx.x; e < r * (r + 1) / 2; e += blockDim.x) tri[e] = 0.f;
-      __syncthreads();
-      for (int i = threadIdx.x; i < r; i += blockDim.x) tri[tri_at(i, i)] = 1.f;
-      __syncthreads();
-    }
-  }
-  tri_invert(a, tri, tmp);
-  for (int e = threadIdx.x; e < r * r; e += blockDim.x) {
-    const int i = e / r, j = e - (e / r) * r;
-    a.Linv[(int64_t)i * a.ldl + j] = j <= i ? tri[tri_at(i, j)] : 0.f;
-  }
-}
-
-// ------------------------------------------------------ row normalization
-// Q[c][:] = R[c][:] / (||R[c][:]||_2 + eps); one block per row, float64
-// sum of squares in a fixed order.
-__global__ void __launch_bounds__(256)
-rownorm_kernel(const float* R, int64_t ldr, float* Q, int64_t ldq, int64_t n,
-               float eps) {
-  __shared__ double part[8];
-  const int64_t c = blockIdx.x;
-  const float* row = R + c * ldr;
-  double acc = 0.0;
-  for (int64_t j = threadIdx.x; j < n; j += blockDim.x) acc += (double)row[j] * row[j];
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-  if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = acc;
-  __syncthreads();
-  double tot = 0.0;
-  for (int w = 0; w < 8; ++w) tot += part[w];
-  const float inv = (float)(1.0 / (sqrt(tot) + (double)eps));
-  for (int64_t j = threadIdx.x; j < n; j += blockDim.x) Q[c * ldq + j] = row[j] * inv;
-}
-
-// sigma[c] = ||R[c][:]||_2 (float64 sum of squares in a fixed order).
-__global__ void __launch_bounds__(256)
-rownorm_only_kernel(const float* R, int64_t ldr, int64_t n, float* sigma) {
-  __shared__ double part[8];
-  const int64_t c = blockIdx.x;
-  const float* row = R + c * ldr;
-  double acc = 0.0;
-  for (int64_t j = threadIdx.x; j < n; j += blockDim.x) acc += (double)row[j] * row[j];
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-  if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = acc;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    double tot = 0.0;
-    for (int w = 0; w < 8; ++w) tot += part[w];
-    sigma[c] = (float)sqrt(tot);
-  }
-}
 
 // One block per matrix: exp(-sum p ln p), p_j = sigma_j^2 / sum sigma^2.
 struct ERankArgs {
@@ -294,105 +75,122 @@ __global__ void __launch_bounds__(256) erank_kernel(const ERankArgs a) {
   if (threadIdx.x == 0) a.erank[i] = tot > 0.0 ? (float)exp(red[0]) : 0.f;
 }
 
-// --------------------------------------------------------------- helpers
-__global__ void transpose_kernel(const float* src, int64_t lds, float* dst,
-                                 int64_t ldd, int64_t rows, int64_t cols) {
-  __shared__ float t[32][33];
-  const int64_t r0 = (int64_t)blockIdx.y * 32, c0 = (int64_t)blockIdx.x * 32;
-  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;  // 32 x 8
-  for (int y = ty; y < 32; y += 8) {
-    const int64_t r = r0 + y, c = c0 + tx;
-    t[y][tx] = (r < rows && c < cols) ? src[r * lds + c] : 0.f;
-  }
-  __syncthreads();
-  for (int y = ty; y < 32; y += 8) {
-    const int64_t r = c0 + y, c = r0 + tx;  // dst is cols x rows
-    if (r < cols && c < rows) dst[r * ldd + c] = t[tx][y];
-  }
+int64_t pitch4(int64_t n) { return ceil_div(n, 4) * 4; }
+int pad32(int r) { return (int)(ceil_div(r, 32) * 32); }
+
+// Split-K of a projection with an M x N fp32 output and depth K: only a
+// matrix whose own output tiles cannot fill the GPU is split, into ranges
+// of at least 1024 along K.  Depends on the shape alone.
+int proj_ksplit(int64_t M, int64_t N, int64_t K) {
+  const int64_t ctas = ceil_div(M, 128) * ceil_div(N, 256);
+  if (ctas >= 64) return 1;
+  int64_t ks = ceil_div(128, ctas);
+  int64_t kmax = K / 1024;
+  if (kmax < 1) kmax = 1;
+  if (ks > kmax) ks = kmax;
+  if (ks > 8) ks = 8;
+  return gemm_ksplit_used(K, (int)ks, OUO_F32);
 }
 
-__global__ void copy2d_kernel(const float* src, int64_t lds, float* dst,
-                              int64_t ldd, int64_t rows, int64_t cols) {
-  const int64_t total = rows * cols;
-  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total;
-       e += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t r = e / cols, c = e - (e / cols) * cols;
-    dst[r * ldd + c] = src[r * lds + c];
-  }
+int64_t gram_chunk(int r, int64_t L) {
+  const int sp = cholqr_gram_splits(r, L);
+  return ceil_div(ceil_div(L, sp), 32) * 32;
 }
+int64_t gram_nsplit(int r, int64_t L) { return ceil_div(L, gram_chunk(r, L)); }
 
-unsigned grid_1d(int64_t n, int per_block) {
-  int64_t b = ceil_div(n, per_block);
-  int64_t cap = (int64_t)num_sms() * 8;
-  if (b > cap) b = cap;
-  return (unsigned)(b < 1 ? 1 : b);
-}
-
-// Packed triangle (plus r floats) the one-CTA kernel keeps in shared
-// memory: at most 33 KB for the ranks it serves (r <= 128).
-size_t chol_smem_bytes(int r) { return ((size_t)r * (r + 1) / 2 + r) * sizeof(float); }
-
-int gram_splits(int r, int64_t L) {
-  const int tiles = (int)ceil_div(r, kGT);
-  const int pairs = tiles * (tiles + 1) / 2;
-  int64_t want = ceil_div((int64_t)num_sms() * 4, pairs);
-  int64_t maxs = ceil_div(L, 256);  // at least 256 columns per split
-  if (want > maxs) want = maxs;
-  if (want < 1) want = 1;
-  if (want > 64) want = 64;
-  return (int)want;
-}
-
-struct DionWs {
-  Buf Pa, Pb;   // r x m
-  Buf P;        // m x r
-  Buf Ra, Rb;   // r x n
-  Buf part;     // [64][r][r]
-  Buf Linv;     // R x R (R = r rounded up to 32)
-  Buf S;        // R x R (blocked Cholesky)
-  Buf ctl;      // barrier counter and flags of the blocked Cholesky
+// Matrices of one (rows, cols, rank) in a call, with their workspace.
+struct DGroup {
+  int64_t m = 0, n = 0;
+  int r = 0;
+  std::vector<int> members;  // indices into the caller's batch
+  int ks1 = 1, ks2 = 1;      // K splits of Pt = Qt B^T and Rt = Pt B
+  Buf Pt, P, Rt, Qn;         // r x m, m x r, r x n, r x n per member
+  Buf kp1, kp2;              // split-K partials (the same memory)
+  Buf S, Lb, Ld;             // r x r summed Gram; R x R factors
+  float* gpart = nullptr;    // Gram partials, gstride floats per member
+  int64_t gstride = 0;
+  char* ctl = nullptr;       // cooperative Cholesky control (r > 256)
+  size_t ctl_stride = 0;
 };
 
-// Ranks from blocked_chol_min_rank() up take a blocked Cholesky: the
-// one-CTA kernel with the blocks in shared memory up to
-// smem_chol_max_rank(), the cooperative multi-CTA kernel above it; smaller
-// ranks keep the one-CTA packed-triangle kernel.  Per 4096 x 4096
-// Orth-Dion step the one-CTA blocked kernel is 7-11% faster than the
-// better of the other two from r = 64 to 192, 2% at r = 224 and 4% slower
-// at r = 256, where the cooperative kernel's wider phases win.
-// OUO_CHOL_BLOCKED_MIN_RANK (1 to 129) and OUO_CHOL_SMEM_MAX_RANK (0 to
-// 256; 0 turns the one-CTA blocked kernel off) override the two bounds.
-int blocked_chol_min_rank() {
-  const char* env = getenv("OUO_CHOL_BLOCKED_MIN_RANK");
-  if (env) {
-    const int v = atoi(env);
-    if (v >= 1 && v <= 129) return v;
-  }
-  return 64;
+Buf view(const Buf& b, int64_t first, int64_t nb) {
+  Buf v = b;
+  v.p = b.p ? b.p + (size_t)first * b.stride * elem_size(b.dtype) : nullptr;
+  v.nb = nb;
+  return v;
 }
-int smem_chol_max_rank() {
-  const char* env = getenv("OUO_CHOL_SMEM_MAX_RANK");
-  if (env) {
-    const int v = atoi(env);
-    if (v >= 0 && v <= 256) return v;
-  }
-  return 224;
-}
-int64_t padded_rank(int r) { return ceil_div(r, 32) * 32; }
 
-DionWs carve_dion(Arena& ar, int64_t m, int64_t n, int r) {
-  DionWs w;
-  w.Pa = ar.take(OUO_F32, 1, r, m);
-  w.Pb = ar.take(OUO_F32, 1, r, m);
-  w.P = ar.take(OUO_F32, 1, m, r);
-  w.Ra = ar.take(OUO_F32, 1, r, n);
-  w.Rb = ar.take(OUO_F32, 1, r, n);
-  w.part = ar.take(OUO_F32, 64, r, r);
-  const int64_t R = padded_rank(r);
-  w.Linv = ar.take(OUO_F32, 1, R, R);
-  w.S = ar.take(OUO_F32, 1, R, R);
-  w.ctl = ar.take(OUO_F32, 1, 1, (int64_t)ceil_div(chol_blocked_ctl_bytes(r), 4));
-  return w;
+Buf take_bytes(Arena& ar, size_t bytes) {
+  Buf b = ar.take(OUO_F32, 1, 1, (int64_t)ceil_div((int64_t)bytes, 4));
+  return b;
+}
+
+std::vector<DGroup> plan(const ouo_mat* M, int nmat, const int* ranks, Arena& ar) {
+  std::vector<DGroup> gs;
+  std::map<std::tuple<int64_t, int64_t, int>, int> where;
+  for (int i = 0; i < nmat; ++i) {
+    auto key = std::make_tuple(M[i].rows, M[i].cols, ranks[i]);
+    auto it = where.find(key);
+    if (it == where.end()) {
+      where[key] = (int)gs.size();
+      DGroup g;
+      g.m = M[i].rows;
+      g.n = M[i].cols;
+      g.r = ranks[i];
+      gs.push_back(g);
+      gs.back().members.push_back(i);
+    } else {
+      gs[it->second].members.push_back(i);
+    }
+  }
+  for (DGroup& g : gs) {
+    const int64_t nb = (int64_t)g.members.size();
+    const int64_t m = g.m, n = g.n;
+    const int r = g.r, R = pad32(r);
+    g.ks1 = proj_ksplit(r, m, n);
+    g.ks2 = proj_ksplit(r, n, m);
+    g.Pt = ar.take(OUO_F32, nb, r, m);
+    g.P = ar.take(OUO_F32, nb, m, r);
+    g.Rt = ar.take(OUO_F32, nb, r, n);
+    g.Qn = ar.take(OUO_F32, nb, r, n);
+    {
+      // the two partial sets are used one after the other: one region
+      const int64_t f1 = g.ks1 > 1 ? g.ks1 * (int64_t)r * pitch4(m) : 0;
+      const int64_t f2 = g.ks2 > 1 ? g.ks2 * (int64_t)r * pitch4(n) : 0;
+      Buf region = take_bytes(ar, (size_t)nb * (size_t)(f1 > f2 ? f1 : f2) * 4 + 256);
+      g.kp1 = Buf();
+      g.kp1.p = region.p;
+      g.kp1.dtype = OUO_F32;
+      g.kp1.rows = r;
+      g.kp1.cols = m;
+      g.kp1.ld = pitch4(m);
+      g.kp1.stride = r * pitch4(m);
+      g.kp1.nb = nb * g.ks1;
+      g.kp2 = g.kp1;
+      g.kp2.cols = n;
+      g.kp2.ld = pitch4(n);
+      g.kp2.stride = r * pitch4(n);
+      g.kp2.nb = nb * g.ks2;
+    }
+    const int64_t gs_m = gram_nsplit(r, m), gs_n = gram_nsplit(r, n);
+    g.gstride = (gs_m > gs_n ? gs_m : gs_n) * (int64_t)r * r;
+    g.gstride = ceil_div(g.gstride, 64) * 64;
+    g.gpart = reinterpret_cast<float*>(take_bytes(ar, (size_t)nb * g.gstride * 4).p);
+    g.S = ar.take(OUO_F32, nb, r, r);
+    g.Lb = ar.take(OUO_F32, nb, R, R);
+    if (!cholqr_small_rank(r)) {
+      g.Ld = ar.take(OUO_F32, nb, R, R);
+      g.ctl_stride = align_up(chol_blocked_ctl_bytes(r), 256);
+      g.ctl = take_bytes(ar, (size_t)nb * g.ctl_stride).p;
+    }
+  }
+  return gs;
+}
+
+size_t plan_bytes(const ouo_mat* M, int nmat, const int* ranks) {
+  Arena ar{nullptr, 0, 0, true};
+  plan(M, nmat, ranks, ar);
+  return ar.used + 256;
 }
 
 Buf caller_buf(const ouo_mat& m, int dtype) {
@@ -407,99 +205,349 @@ Buf caller_buf(const ouo_mat& m, int dtype) {
   return b;
 }
 
-// Partial Gram matrices of the rows of X (r x L) into w.part: returns the
-// number of partials written (their float64 sum is X X^T).
-int gram_parts(const Buf& X, const DionWs& w, cudaStream_t s, int* used) {
-  const int r = (int)X.rows;
-  const int64_t L = X.cols;
-  GramArgs ga;
-  ga.X = reinterpret_cast<const float*>(X.p);
-  ga.ld = X.ld;
-  ga.r = r;
-  ga.L = L;
-  const int splits = gram_splits(r, L);
-  ga.chunk = ceil_div(ceil_div(L, splits), kGT) * kGT;
-  *used = (int)ceil_div(L, ga.chunk);
-  ga.part = reinterpret_cast<float*>(w.part.p);
-  ga.tiles = (int)ceil_div(r, kGT);
-  dim3 grid((unsigned)(ga.tiles * (ga.tiles + 1) / 2), (unsigned)*used);
-  gram_partial_kernel<<<grid, 256, 0, s>>>(ga);
-  OUO_CHECK_LAUNCH();
-  return OUO_OK;
+// The members' caller matrices as one evenly strided batch, when they are
+// laid out that way (same ld, equal byte steps, 16-byte multiple, no
+// overlap); false otherwise.
+bool caller_uniform(const ouo_mat* mats, const std::vector<int>& mem, int dtype, Buf* out) {
+  const ouo_mat& f = mats[mem[0]];
+  const int64_t es = (int64_t)elem_size(dtype);
+  if (mem.size() == 1) {
+    *out = caller_buf(f, dtype);
+    return true;
+  }
+  const int64_t step = reinterpret_cast<const char*>(mats[mem[1]].ptr) -
+                       reinterpret_cast<const char*>(f.ptr);
+  if (step <= 0 || step % 16 || step % es || step < f.rows * f.ld * es) return false;
+  for (size_t k = 0; k < mem.size(); ++k) {
+    const ouo_mat& x = mats[mem[k]];
+    if (x.ld != f.ld || reinterpret_cast<const char*>(x.ptr) !=
+                            reinterpret_cast<const char*>(f.ptr) + (int64_t)k * step)
+      return false;
+  }
+  *out = caller_buf(f, dtype);
+  out->stride = step / es;
+  out->nb = (int64_t)mem.size();
+  return true;
 }
 
-__global__ void sum_parts_kernel(const float* part, int splits, int64_t n, float* out) {
-  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n;
-       e += (int64_t)gridDim.x * blockDim.x) {
-    double s = 0.0;
-    for (int q = 0; q < splits; ++q) s += (double)part[(size_t)q * n + e];
-    out[e] = (float)s;
+// Descriptors of one GEMM stage for a group whose A and / or B operands are
+// caller matrices: one descriptor over the whole group when the caller
+// operands are evenly strided, else one per member.
+void add_descs(std::vector<GemmDesc>& out, const GemmDesc& proto, const DGroup& g,
+               const ouo_mat* Acall, const ouo_mat* Bcall, const Buf& Aws, const Buf& Bws,
+               const Buf& Ows) {
+  const int64_t nb = (int64_t)g.members.size();
+  Buf A = Aws, B = Bws;
+  bool uniform = true;
+  if (Acall) uniform = uniform && caller_uniform(Acall, g.members, OUO_F32, &A);
+  if (Bcall) uniform = uniform && caller_uniform(Bcall, g.members, OUO_F32, &B);
+  if (uniform) {
+    GemmDesc d = proto;
+    d.nb = nb;
+    d.A = A;
+    d.B = B;
+    d.out_f32 = Ows;
+    out.push_back(d);
+    return;
+  }
+  const int64_t per = Ows.nb / nb;  // outputs per member (K splits)
+  for (int64_t k = 0; k < nb; ++k) {
+    GemmDesc d = proto;
+    d.nb = 1;
+    d.A = Acall ? caller_buf(Acall[g.members[k]], OUO_F32) : view(Aws, k, 1);
+    d.B = Bcall ? caller_buf(Bcall[g.members[k]], OUO_F32) : view(Bws, k, 1);
+    d.out_f32 = view(Ows, k * per, per);
+    out.push_back(d);
   }
 }
 
-// w.Linv = L^-1 where L L^T = sum of `splits` r x r partials at `part`
-// (L_rows: the rows' length, for the shifted retry).
-int cholesky_inverse(const float* part, int splits, int r, int64_t L_rows,
-                     const DionWs& w, int* status, cudaStream_t s) {
-  if (r >= blocked_chol_min_rank() && r <= smem_chol_max_rank() && chol_smem_fits(r)) {
-    if (splits > 1) {  // one wide pass sums the partials; the CTA reads S once
-      const int64_t n = (int64_t)r * r;
-      float* S = reinterpret_cast<float*>(w.S.p);
-      sum_parts_kernel<<<grid_1d(n, 256), 256, 0, s>>>(part, splits, n, S);
-      OUO_CHECK_LAUNCH();
-      part = S;
-      splits = 1;
+// Which CholeskyQR jobs of a pass take the one-CTA Cholesky.
+int orth_factor(std::vector<CholQrJob>& jobs, const std::vector<const DGroup*>& owner,
+                const std::vector<int64_t>& mem, int* status, cudaStream_t s) {
+  std::vector<CholQrJob> small;
+  for (size_t k = 0; k < jobs.size(); ++k) {
+    if (cholqr_small_rank(jobs[k].r)) {
+      small.push_back(jobs[k]);
+      continue;
     }
-    OUO_TRY(chol_smem(part, r, L_rows, reinterpret_cast<float*>(w.Linv.p), status, s));
-  } else if (r >= blocked_chol_min_rank()) {
-    OUO_TRY(chol_blocked(part, splits, r, L_rows, reinterpret_cast<float*>(w.S.p),
-                         reinterpret_cast<float*>(w.Linv.p), w.ctl.p, status, s));
-  } else {
-    CholArgs ca;
-    ca.part = part;
-    ca.splits = splits;
-    ca.r = r;
-    ca.L = L_rows;
-    ca.Linv = reinterpret_cast<float*>(w.Linv.p);
-    ca.ldl = w.Linv.ld;
-    ca.status = status;
-    chol_inv_kernel<<<1, 1024, chol_smem_bytes(r), s>>>(ca);
-    OUO_CHECK_LAUNCH();
+    const DGroup& g = *owner[k];
+    const int64_t i = mem[k];
+    OUO_TRY(chol_blocked(jobs[k].S, 1, jobs[k].r, jobs[k].L, jobs[k].Lb,
+                         const_cast<float*>(jobs[k].Dd), g.ctl + (size_t)i * g.ctl_stride,
+                         status, s, false));
+  }
+  return cholqr_factor(small, status, s);
+}
+
+// One CholeskyQR pass over every job: Gram, Cholesky, triangular solve.
+// With `gram_done`, S already holds the (summed) Gram matrices.
+int orth_pass(std::vector<CholQrJob>& jobs, const std::vector<const DGroup*>& owner,
+              const std::vector<int64_t>& mem, int* status, cudaStream_t s, bool gram_done) {
+  if (jobs.empty()) return OUO_OK;
+  if (!gram_done) OUO_TRY(cholqr_gram(jobs, s));
+  OUO_TRY(orth_factor(jobs, owner, mem, status, s));
+  return cholqr_apply(jobs, s);
+}
+
+// A CholeskyQR job on member i of group g (rows X, length L), factor
+// buffers from the group.
+CholQrJob orth_job(const DGroup& g, int64_t i, const float* X, int64_t ldx, int64_t L) {
+  CholQrJob j;
+  j.X = X;
+  j.ldx = ldx;
+  j.r = g.r;
+  j.L = L;
+  j.gchunk = gram_chunk(g.r, L);
+  j.gpart = g.gpart + i * g.gstride;
+  j.S = reinterpret_cast<float*>(view(g.S, i, 1).p);
+  j.Lb = reinterpret_cast<float*>(view(g.Lb, i, 1).p);
+  j.Dd = g.Ld.p ? reinterpret_cast<const float*>(view(g.Ld, i, 1).p) : nullptr;
+  return j;
+}
+
+float* fp(const Buf& b, int64_t i) { return reinterpret_cast<float*>(view(b, i, 1).p); }
+
+// Stage: Pt = Qt B^T for every matrix (split-K partials summed into Pt).
+int stage_project(const std::vector<DGroup>& gs, const ouo_mat* M, const ouo_mat* Q,
+                  int* status, cudaStream_t s) {
+  std::vector<GemmDesc> ds;
+  std::vector<RowsJob> red;
+  for (const DGroup& g : gs) {
+    GemmDesc d;
+    d.M = g.r; d.N = g.m; d.K = g.n;
+    d.has_f32 = true;
+    d.ksplit = g.ks1;
+    d.per_desc_tiles = true;
+    add_descs(ds, d, g, Q, M, Buf(), Buf(), g.ks1 > 1 ? g.kp1 : g.Pt);
+    if (g.ks1 > 1) {
+      for (int64_t i = 0; i < (int64_t)g.members.size(); ++i) {
+        RowsJob rj;
+        rj.part = fp(g.kp1, i * g.ks1);
+        rj.ldp = g.kp1.ld;
+        rj.sp = g.kp1.stride;
+        rj.ks = g.ks1;
+        rj.rows = g.r;
+        rj.n = g.m;
+        rj.out = fp(g.Pt, i);
+        rj.ldo = g.Pt.ld;
+        red.push_back(rj);
+      }
+    }
+  }
+  OUO_TRY(gemm_umma_grouped(ds, s, status));
+  return rows_reduce(red, 0.f, s);
+}
+
+// Stage: passes pass_from .. pass_to - 1 of CholeskyQR2 on every Pt, in
+// place; the second solve also writes P = Pt^T.
+int stage_orth_p(const std::vector<DGroup>& gs, int* status, cudaStream_t s, int pass_from,
+                 int pass_to) {
+  for (int pass = pass_from; pass < pass_to; ++pass) {
+    std::vector<CholQrJob> jobs;
+    std::vector<const DGroup*> own;
+    std::vector<int64_t> mem;
+    for (const DGroup& g : gs) {
+      for (int64_t i = 0; i < (int64_t)g.members.size(); ++i) {
+        CholQrJob j = orth_job(g, i, fp(g.Pt, i), g.Pt.ld, g.m);
+        j.Y = fp(g.Pt, i);
+        j.ldy = g.Pt.ld;
+        if (pass == 1) {
+          j.Yt = fp(g.P, i);
+          j.ldyt = g.P.ld;
+        }
+        jobs.push_back(j);
+        own.push_back(&g);
+        mem.push_back(i);
+      }
+    }
+    OUO_TRY(orth_pass(jobs, own, mem, status, s, false));
   }
   return OUO_OK;
 }
 
-// dst = Linv src (r x L, fp32 SIMT)
-int apply_linv(const DionWs& w, int r, const Buf& src, const Buf& dst, cudaStream_t s) {
-  GemmDesc d;
-  d.M = r;
-  d.N = src.cols;
-  d.K = r;
-  d.nb = 1;
-  d.A = w.Linv;
-  d.B = src;
-  d.b_mn = 1;
-  d.out_f32 = dst;
-  d.has_f32 = true;
-  return gemm_simt(d, s);
+// Stage: Rt = Pt B into `dst(g, i)` (Rt of the workspace, or the
+// caller-summed buffer of the row-sharded step), split-K partials summed.
+template <class Dst>
+int stage_rproject(const std::vector<DGroup>& gs, const ouo_mat* M, Dst dst, int* status,
+                   cudaStream_t s) {
+  std::vector<GemmDesc> ds;
+  std::vector<RowsJob> red;
+  for (const DGroup& g : gs) {
+    GemmDesc d;
+    d.M = g.r; d.N = g.n; d.K = g.m;
+    d.b_mn = 1;
+    d.has_f32 = true;
+    d.ksplit = g.ks2;
+    d.per_desc_tiles = true;
+    if (g.ks2 > 1) {
+      add_descs(ds, d, g, nullptr, M, g.Pt, Buf(), g.kp2);
+      for (int64_t i = 0; i < (int64_t)g.members.size(); ++i) {
+        RowsJob rj;
+        rj.part = fp(g.kp2, i * g.ks2);
+        rj.ldp = g.kp2.ld;
+        rj.sp = g.kp2.stride;
+        rj.ks = g.ks2;
+        rj.rows = g.r;
+        rj.n = g.n;
+        int64_t ld = 0;
+        rj.out = dst(g, i, &ld);
+        rj.ldo = ld;
+        red.push_back(rj);
+      }
+    } else {
+      // outputs straight into dst: per member when dst is not one batch
+      std::vector<GemmDesc> one;
+      add_descs(one, d, g, nullptr, M, g.Pt, Buf(), g.Rt);
+      int64_t ld0 = 0;
+      float* base = dst(g, 0, &ld0);
+      if (base == fp(g.Rt, 0)) {
+        for (auto& x : one) ds.push_back(x);
+      } else {
+        for (int64_t i = 0; i < (int64_t)g.members.size(); ++i) {
+          GemmDesc di = d;
+          di.nb = 1;
+          di.A = view(g.Pt, i, 1);
+          di.B = caller_buf(M[g.members[i]], OUO_F32);
+          int64_t ld = 0;
+          Buf o;
+          o.p = reinterpret_cast<char*>(dst(g, i, &ld));
+          o.dtype = OUO_F32;
+          o.rows = g.r;
+          o.cols = g.n;
+          o.ld = ld;
+          o.stride = g.r * ld;
+          o.nb = 1;
+          di.out_f32 = o;
+          ds.push_back(di);
+        }
+      }
+    }
+  }
+  OUO_TRY(gemm_umma_grouped(ds, s, status));
+  return rows_reduce(red, 0.f, s);
 }
 
-// Rows of X (r x L, workspace) made orthonormal into Y: two CholeskyQR
-// passes (X -> tmp -> Y); X is clobbered.
-int orth_rows(Buf X, Buf tmp, Buf Y, const DionWs& w, cudaStream_t s,
-              int* status) {
-  const int r = (int)X.rows;
-  Buf src = X;
+// Stage: from Rt (rt(g, i), row pitch ldr): sigma (optional), and Q_new^T
+// into Qn and the caller's state -- column normalization (Dion) or
+// CholeskyQR2 (Orth-Dion).
+template <class Rtp>
+int stage_qnew(const std::vector<DGroup>& gs, Rtp rt, const ouo_mat* Q_state,
+               const ouo_dion_params* p, float* sigma, const std::vector<int64_t>& sig_off,
+               int* status, cudaStream_t s) {
+  std::vector<RowsJob> rows;
+  for (const DGroup& g : gs) {
+    for (int64_t i = 0; i < (int64_t)g.members.size(); ++i) {
+      const int bi = g.members[i];
+      const bool colnorm = p->norm_mode == OUO_DION_COLNORM;
+      if (!colnorm && !sigma) continue;
+      int64_t ld = 0;
+      RowsJob rj;
+      rj.part = rt(g, i, &ld);
+      rj.ldp = ld;
+      rj.sp = 0;
+      rj.ks = 1;
+      rj.rows = g.r;
+      rj.n = g.n;
+      rj.sigma = sigma ? sigma + sig_off[bi] : nullptr;
+      if (colnorm) {
+        rj.qn = fp(g.Qn, i);
+        rj.ldq = g.Qn.ld;
+        rj.q2 = reinterpret_cast<float*>(Q_state[bi].ptr);
+        rj.ldq2 = Q_state[bi].ld;
+      }
+      rows.push_back(rj);
+    }
+  }
+  OUO_TRY(rows_reduce(rows, p->eps, s));
+  if (p->norm_mode == OUO_DION_COLNORM) return OUO_OK;
   for (int pass = 0; pass < 2; ++pass) {
-    Buf dst = pass == 0 ? tmp : Y;
-    int used = 0;
-    OUO_TRY(gram_parts(src, w, s, &used));
-    OUO_TRY(cholesky_inverse(reinterpret_cast<const float*>(w.part.p), used, r, src.cols,
-                             w, status, s));
-    OUO_TRY(apply_linv(w, r, src, dst, s));
-    src = dst;
+    std::vector<CholQrJob> jobs;
+    std::vector<const DGroup*> own;
+    std::vector<int64_t> mem;
+    for (const DGroup& g : gs) {
+      for (int64_t i = 0; i < (int64_t)g.members.size(); ++i) {
+        int64_t ld = 0;
+        float* x = pass == 0 ? rt(g, i, &ld) : fp(g.Qn, i);
+        if (pass == 1) ld = g.Qn.ld;
+        CholQrJob j = orth_job(g, i, x, ld, g.n);
+        j.Y = fp(g.Qn, i);
+        j.ldy = g.Qn.ld;
+        if (pass == 1) {
+          const int bi = g.members[i];
+          j.Y2 = reinterpret_cast<float*>(Q_state[bi].ptr);
+          j.ldy2 = Q_state[bi].ld;
+        }
+        jobs.push_back(j);
+        own.push_back(&g);
+        mem.push_back(i);
+      }
+    }
+    OUO_TRY(orth_pass(jobs, own, mem, status, s, false));
   }
   return OUO_OK;
+}
+
+// Stage: M <- beta B - (beta - mu) P Rt and W <- (1 - lr wd) W - lr s P Qn,
+// in place in the caller's matrices.
+template <class Rtp>
+int stage_update(const std::vector<DGroup>& gs, Rtp rt, const ouo_mat* M, const ouo_mat* W,
+                 int w_dtype, const ouo_dion_params* p, const float* scale, int* status,
+                 cudaStream_t s) {
+  std::vector<GemmDesc> dm, dw;
+  for (const DGroup& g : gs) {
+    const int64_t nb = (int64_t)g.members.size();
+    GemmDesc d;
+    d.M = g.m; d.N = g.n; d.K = g.r; d.nb = nb;
+    d.A = g.P;
+    d.b_mn = 1;
+    d.has_c0 = true;
+    d.c0_from_out = true;
+    d.per_desc_tiles = true;
+    // M update: B = Rt (the workspace batch, or the caller-summed rows)
+    int64_t ld0 = 0;
+    float* r0 = rt(g, 0, &ld0);
+    const bool rt_ws = r0 == fp(g.Rt, 0);
+    for (int64_t i = 0; i < (rt_ws ? 1 : nb); ++i) {
+      GemmDesc x = d;
+      x.alpha = -(p->beta - p->mu);
+      x.beta = p->beta;
+      x.direct_dtype = OUO_F32;
+      if (rt_ws) {
+        x.B = g.Rt;
+        for (int64_t k = 0; k < nb; ++k)
+          x.direct.push_back(MatRef{M[g.members[k]].ptr, M[g.members[k]].ld});
+      } else {
+        int64_t ld = 0;
+        Buf b;
+        b.p = reinterpret_cast<char*>(rt(g, i, &ld));
+        b.dtype = OUO_F32;
+        b.rows = g.r;
+        b.cols = g.n;
+        b.ld = ld;
+        b.stride = g.r * ld;
+        b.nb = 1;
+        x.B = b;
+        x.nb = 1;
+        x.A = view(g.P, i, 1);
+        x.direct.push_back(MatRef{M[g.members[i]].ptr, M[g.members[i]].ld});
+      }
+      dm.push_back(x);
+    }
+    // W update: B = Qn, per-matrix alpha = -lr * scale
+    GemmDesc y = d;
+    y.B = g.Qn;
+    y.beta = 1.0f - p->lr * p->wd;
+    y.alpha = -p->lr;
+    y.direct_dtype = w_dtype;
+    for (int64_t k = 0; k < nb; ++k) {
+      const int bi = g.members[k];
+      y.direct.push_back(MatRef{W[bi].ptr, W[bi].ld});
+      y.direct_alpha.push_back(-p->lr * (scale ? scale[bi] : 1.0f));
+    }
+    dw.push_back(y);
+  }
+  OUO_TRY(gemm_umma_grouped(dm, s, status));
+  return gemm_umma_grouped(dw, s, status);
 }
 
 int validate_dion(const ouo_dion_params* p) {
@@ -510,12 +558,6 @@ int validate_dion(const ouo_dion_params* p) {
   return OUO_OK;
 }
 
-size_t dion_plan_bytes(const ouo_mat* M, int nmat, const int* ranks) {
-  Arena ar{nullptr, 0, 0, true};
-  for (int i = 0; i < nmat; ++i) carve_dion(ar, M[i].rows, M[i].cols, ranks[i]);
-  return ar.used + 256;
-}
-
 }  // namespace
 }  // namespace ouo
 
@@ -523,7 +565,7 @@ extern "C" size_t dion_workspace_bytes(const ouo_mat* M, int nmat,
                                        const ouo_dion_params* p) {
   if (!M || !p || nmat <= 0 || nmat > OUO_MAX_BATCH || p->rank < 1) return 0;
   std::vector<int> ranks((size_t)nmat, p->rank);
-  return ouo::dion_plan_bytes(M, nmat, ranks.data());
+  return ouo::plan_bytes(M, nmat, ranks.data());
 }
 
 extern "C" size_t dion_workspace_bytes_ranks(const ouo_mat* M, const int* ranks,
@@ -531,7 +573,7 @@ extern "C" size_t dion_workspace_bytes_ranks(const ouo_mat* M, const int* ranks,
   if (!M || !ranks || !p || nmat <= 0 || nmat > OUO_MAX_BATCH) return 0;
   for (int i = 0; i < nmat; ++i)
     if (ranks[i] < 1) return 0;
-  return ouo::dion_plan_bytes(M, nmat, ranks);
+  return ouo::plan_bytes(M, nmat, ranks);
 }
 
 extern "C" int dion_lowrank_step(const ouo_mat* M, const ouo_mat* G,
@@ -565,12 +607,18 @@ extern "C" int dion_lowrank_step_stats(const ouo_mat* M, const ouo_mat* G,
   if (p->rank < 0) return set_error(OUO_ERR_INVALID_ARG, "rank %d < 0", p->rank);
   // per-matrix ranks: p->rank, or Q_state[i].rows when p->rank == 0
   std::vector<int> ranks((size_t)nmat);
+  std::vector<int64_t> sig_off((size_t)nmat);
+  int64_t so = 0;
   for (int i = 0; i < nmat; ++i) {
     const int r = p->rank ? p->rank : (int)Q_state[i].rows;
     ranks[i] = r;
+    sig_off[i] = so;
+    so += r;
     if (r < 1 || r > M[i].rows || r > M[i].cols)
       return set_error(OUO_ERR_INVALID_ARG, "rank %d outside [1, min(rows, cols)] for M[%d]",
                        r, i);
+    if (r > 1024)
+      return set_error(OUO_ERR_UNSUPPORTED, "rank %d above 1024 (M[%d])", r, i);
     if (Q_state[i].rows != r || Q_state[i].cols != M[i].cols)
       return set_error(OUO_ERR_INVALID_ARG,
                        "Q_state[%d] must be r x cols (%d x %lld, the transposed factor)",
@@ -584,7 +632,7 @@ extern "C" int dion_lowrank_step_stats(const ouo_mat* M, const ouo_mat* G,
     return set_error(OUO_ERR_INVALID_ARG, "dev_status misaligned");
   if (sigma && ((uintptr_t)sigma % 4))
     return set_error(OUO_ERR_INVALID_ARG, "sigma misaligned");
-  const size_t need = dion_plan_bytes(M, nmat, ranks.data());
+  const size_t need = plan_bytes(M, nmat, ranks.data());
   if (!ws || ws_bytes < need)
     return set_error(OUO_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given",
                      need, ws_bytes);
@@ -596,101 +644,16 @@ extern "C" int dion_lowrank_step_stats(const ouo_mat* M, const ouo_mat* G,
   OUO_TRY(dion_momentum_update(M, G, nmat, g_dtype, p->mu, OUO_MOMENTUM_ACCUM,
                                nullptr, stream));
   Arena ar{reinterpret_cast<char*>(ws), ws_bytes, 0, false};
-  const float mu = p->mu, beta = p->beta;
-  int64_t sig_off = 0;
-  for (int i = 0; i < nmat; ++i) {
-    const int64_t m = M[i].rows, n = M[i].cols;
-    const int r = ranks[i];
-    DionWs w = carve_dion(ar, m, n, r);
-    const Buf Bm = caller_buf(M[i], OUO_F32);
-    const Buf Qt = caller_buf(Q_state[i], OUO_F32);
-    // Pt = Qt B^T  (r x m)
-    {
-      GemmDesc d;
-      d.M = r; d.N = m; d.K = n; d.nb = 1;
-      d.A = Qt;
-      d.B = Bm;
-      d.out_f32 = w.Pa;
-      d.has_f32 = true;
-      OUO_TRY(gemm_umma(d, s, dev_status));
-    }
-    // rows of Pt orthonormal (P = orth(B Q_prev)) -> Pa
-    OUO_TRY(orth_rows(w.Pa, w.Pb, w.Pa, w, s, dev_status));
-    // Rt = Pt B  (r x n)
-    {
-      GemmDesc d;
-      d.M = r; d.N = n; d.K = m; d.nb = 1;
-      d.A = w.Pa;
-      d.B = Bm;
-      d.b_mn = 1;
-      d.out_f32 = w.Ra;
-      d.has_f32 = true;
-      OUO_TRY(gemm_umma(d, s, dev_status));
-    }
-    // the power iteration's singular-value estimates: ||rows of Rt||
-    if (sigma) {
-      rownorm_only_kernel<<<r, 256, 0, s>>>(reinterpret_cast<const float*>(w.Ra.p), w.Ra.ld,
-                                            n, sigma + sig_off);
-      OUO_CHECK_LAUNCH();
-    }
-    sig_off += r;
-    // P = Pt^T (m x r), the K-major left operand of the updates
-    {
-      dim3 grid((unsigned)ceil_div(m, 32), (unsigned)ceil_div(r, 32));
-      transpose_kernel<<<grid, 256, 0, s>>>(reinterpret_cast<const float*>(w.Pa.p),
-                                            w.Pa.ld, reinterpret_cast<float*>(w.P.p),
-                                            w.P.ld, r, m);
-      OUO_CHECK_LAUNCH();
-    }
-    // M <- beta B - (beta - mu) P Rt   (in place over B)
-    {
-      GemmDesc d;
-      d.M = m; d.N = n; d.K = r; d.nb = 1;
-      d.A = w.P;
-      d.B = w.Ra;
-      d.b_mn = 1;
-      d.alpha = -(beta - mu);
-      d.beta = beta;
-      d.has_c0 = true;
-      d.direct = {MatRef{M[i].ptr, M[i].ld}};
-      d.direct_dtype = OUO_F32;
-      d.c0_from_out = true;
-      OUO_TRY(gemm_umma(d, s, dev_status));
-    }
-    // Qt_new: rows of Rt normalized (Dion) or orthonormalized (Orth-Dion) -> Rb
-    Buf Qn = w.Rb;
-    if (p->norm_mode == OUO_DION_COLNORM) {
-      rownorm_kernel<<<r, 256, 0, s>>>(reinterpret_cast<const float*>(w.Ra.p), w.Ra.ld,
-                                       reinterpret_cast<float*>(w.Rb.p), w.Rb.ld, n,
-                                       p->eps);
-      OUO_CHECK_LAUNCH();
-    } else {
-      OUO_TRY(orth_rows(w.Ra, w.Rb, w.Ra, w, s, dev_status));
-      Qn = w.Ra;
-    }
-    // W <- (1 - lr wd) W - lr s P Qt_new
-    {
-      const float sc = scale ? scale[i] : 1.0f;
-      GemmDesc d;
-      d.M = m; d.N = n; d.K = r; d.nb = 1;
-      d.A = w.P;
-      d.B = Qn;
-      d.b_mn = 1;
-      d.alpha = -p->lr * sc;
-      d.beta = 1.0f - p->lr * p->wd;
-      d.has_c0 = true;
-      d.direct = {MatRef{W[i].ptr, W[i].ld}};
-      d.direct_dtype = w_dtype;
-      d.c0_from_out = true;
-      OUO_TRY(gemm_umma(d, s, dev_status));
-    }
-    // state <- Qt_new
-    copy2d_kernel<<<grid_1d((int64_t)r * n, 256), 256, 0, s>>>(
-        reinterpret_cast<const float*>(Qn.p), Qn.ld,
-        reinterpret_cast<float*>(Q_state[i].ptr), Q_state[i].ld, r, n);
-    OUO_CHECK_LAUNCH();
-  }
-  return OUO_OK;
+  const std::vector<DGroup> gs = plan(M, nmat, ranks.data(), ar);
+  auto rt_ws = [](const DGroup& g, int64_t i, int64_t* ld) {
+    *ld = g.Rt.ld;
+    return fp(g.Rt, i);
+  };
+  OUO_TRY(stage_project(gs, M, Q_state, dev_status, s));
+  OUO_TRY(stage_orth_p(gs, dev_status, s, 0, 2));
+  OUO_TRY(stage_rproject(gs, M, rt_ws, dev_status, s));
+  OUO_TRY(stage_qnew(gs, rt_ws, Q_state, p, sigma, sig_off, dev_status, s));
+  return stage_update(gs, rt_ws, M, W, w_dtype, p, scale, dev_status, s);
 }
 
 extern "C" int dion_effective_rank(const float* sigma, const int* ranks, int nmat,
@@ -728,13 +691,10 @@ extern "C" int dion_effective_rank(const float* sigma, const int* ranks, int nma
 // r x r Gram matrices of P^T and the r x n product P^T B are the only
 // quantities summed across ranks (by the caller, between the calls below);
 // everything else is local to a rank's rows, and the right factor is
-// formed redundantly on every rank.
+// formed redundantly on every rank.  The four calls run the same batched
+// stages as dion_lowrank_step, so one rank reproduces it bit for bit.
 namespace ouo {
 namespace {
-
-// out[e] = sum_p part[p][e] in float64, fixed order (the reduction the
-// Cholesky kernels apply to their partials), rounded to fp32.
-int64_t pitch4(int64_t n) { return ceil_div(n, 4) * 4; }
 
 // floats of matrix i's block of `red` (256-byte multiple)
 int64_t red_block(int r, int64_t n) {
@@ -756,6 +716,8 @@ int shard_ranks(const ouo_mat* M, const ouo_mat* Q_state, int nmat,
     ranks[i] = r;
     if (r < 1 || r > M[i].cols)
       return set_error(OUO_ERR_INVALID_ARG, "rank %d outside [1, cols] for M[%d]", r, i);
+    if (r > 1024)
+      return set_error(OUO_ERR_UNSUPPORTED, "rank %d above 1024 (M[%d])", r, i);
     if (Q_state[i].rows != r || Q_state[i].cols != M[i].cols)
       return set_error(OUO_ERR_INVALID_ARG, "Q_state[%d] must be r x cols", i);
     if (!vec16(M[i], OUO_F32) || !vec16(Q_state[i], OUO_F32))
@@ -773,7 +735,7 @@ int shard_common(const ouo_mat* M, const ouo_mat* Q_state, int nmat,
     return set_error(OUO_ERR_INVALID_ARG, "dev_status misaligned");
   if (!red || ((uintptr_t)red % 256))
     return set_error(OUO_ERR_INVALID_ARG, "red must be a 256-byte aligned device buffer");
-  const size_t need = dion_plan_bytes(M, nmat, ranks.data());
+  const size_t need = plan_bytes(M, nmat, ranks.data());
   if (!ws || ws_bytes < need)
     return set_error(OUO_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given",
                      need, ws_bytes);
@@ -782,12 +744,88 @@ int shard_common(const ouo_mat* M, const ouo_mat* Q_state, int nmat,
   return require_sm100();
 }
 
-int sum_parts(const DionWs& w, int used, int r, float* out, cudaStream_t s) {
-  const int64_t n = (int64_t)r * r;
-  sum_parts_kernel<<<grid_1d(n, 256), 256, 0, s>>>(reinterpret_cast<const float*>(w.part.p),
-                                                   used, n, out);
-  OUO_CHECK_LAUNCH();
-  return OUO_OK;
+// Offsets (floats) of every batch matrix's block of `red`.
+std::vector<int64_t> red_offsets(const ouo_mat* M, const std::vector<int>& ranks) {
+  std::vector<int64_t> off(ranks.size());
+  int64_t o = 0;
+  for (size_t i = 0; i < ranks.size(); ++i) {
+    off[i] = o;
+    o += red_block(ranks[i], M[i].cols);
+  }
+  return off;
+}
+
+// The Gram matrices of every Pt, summed into S = the matrix's block of red.
+int gram_into_red(const std::vector<DGroup>& gs, float* red, const std::vector<int64_t>& off,
+                  int64_t (*rows_of)(const DGroup&), cudaStream_t s) {
+  std::vector<CholQrJob> jobs;
+  for (const DGroup& g : gs) {
+    for (int64_t i = 0; i < (int64_t)g.members.size(); ++i) {
+      CholQrJob j = orth_job(g, i, fp(g.Pt, i), g.Pt.ld, rows_of(g));
+      j.S = red + off[g.members[i]];
+      jobs.push_back(j);
+    }
+  }
+  return cholqr_gram(jobs, s);
+}
+
+int64_t local_rows(const DGroup& g) { return g.m; }
+
+// orth1 (second = false) and orth2 (second = true): Cholesky of the summed
+// Gram matrices in red, the solve on the local rows of Pt, then red = the
+// next pass's Gram matrices (orth1) or P^T B (orth2).
+int shard_orth(const ouo_mat* M, const ouo_mat* Q_state, int nmat,
+               const ouo_dion_params* p, const int64_t* rows_total, void* ws,
+               size_t ws_bytes, float* red, int* dev_status, void* stream, bool second) {
+  clear_error();
+  if (nmat < 0 || nmat > OUO_MAX_BATCH)
+    return set_error(OUO_ERR_INVALID_ARG, "nmat %d out of range", nmat);
+  if (nmat == 0) return OUO_OK;
+  if (!rows_total) return set_error(OUO_ERR_INVALID_ARG, "NULL rows_total");
+  std::vector<int> ranks;
+  OUO_TRY(shard_common(M, Q_state, nmat, p, ws, ws_bytes, red, dev_status, ranks));
+  for (int i = 0; i < nmat; ++i)
+    if (rows_total[i] < ranks[i] || rows_total[i] < M[i].rows)
+      return set_error(OUO_ERR_INVALID_ARG, "rows_total[%d] smaller than rank or local rows", i);
+  cudaStream_t s = (cudaStream_t)stream;
+  Arena ar{reinterpret_cast<char*>(ws), ws_bytes, 0, false};
+  const std::vector<DGroup> gs = plan(M, nmat, ranks.data(), ar);
+  const std::vector<int64_t> off = red_offsets(M, ranks);
+  std::vector<CholQrJob> jobs;
+  std::vector<const DGroup*> own;
+  std::vector<int64_t> mem;
+  for (const DGroup& g : gs) {
+    for (int64_t i = 0; i < (int64_t)g.members.size(); ++i) {
+      const int bi = g.members[i];
+      // the shift of a retry takes the global row count
+      CholQrJob j = orth_job(g, i, fp(g.Pt, i), g.Pt.ld, rows_total[bi]);
+      j.S = red + off[bi];
+      j.Y = fp(g.Pt, i);
+      j.ldy = g.Pt.ld;
+      if (second) {
+        j.Yt = fp(g.P, i);
+        j.ldyt = g.P.ld;
+      }
+      // the solve runs over the local rows
+      jobs.push_back(j);
+      own.push_back(&g);
+      mem.push_back(i);
+    }
+  }
+  OUO_TRY(orth_factor(jobs, own, mem, dev_status, s));
+  for (CholQrJob& j : jobs) j.L = 0;
+  {
+    size_t k = 0;
+    for (const DGroup& g : gs)
+      for (int64_t i = 0; i < (int64_t)g.members.size(); ++i) jobs[k++].L = g.m;
+  }
+  OUO_TRY(cholqr_apply(jobs, s));
+  if (!second) return gram_into_red(gs, red, off, local_rows, s);
+  auto dst = [&](const DGroup& g, int64_t i, int64_t* ld) {
+    *ld = pitch4(g.n);
+    return red + off[g.members[i]];
+  };
+  return stage_rproject(gs, M, dst, dev_status, s);
 }
 
 }  // namespace
@@ -801,7 +839,7 @@ extern "C" size_t dion_shard_workspace_bytes(const ouo_mat* M, const ouo_mat* Q_
     ranks[i] = p->rank ? p->rank : (int)Q_state[i].rows;
     if (ranks[i] < 1) return 0;
   }
-  return ouo::dion_plan_bytes(M, nmat, ranks.data());
+  return ouo::plan_bytes(M, nmat, ranks.data());
 }
 
 extern "C" size_t dion_shard_red_floats(const ouo_mat* M, const ouo_mat* Q_state, int nmat,
@@ -833,80 +871,10 @@ extern "C" int dion_shard_project(const ouo_mat* M, const ouo_mat* G, int g_dtyp
   OUO_TRY(dion_momentum_update(M, G, nmat, g_dtype, p->mu, OUO_MOMENTUM_ACCUM, nullptr,
                                stream));
   Arena ar{reinterpret_cast<char*>(ws), ws_bytes, 0, false};
-  int64_t off = 0;
-  for (int i = 0; i < nmat; ++i) {
-    const int r = ranks[i];
-    const int64_t m = M[i].rows, n = M[i].cols;
-    DionWs w = carve_dion(ar, m, n, r);
-    GemmDesc d;  // P^T = Q^T B^T (r x m local)
-    d.M = r; d.N = m; d.K = n; d.nb = 1;
-    d.A = caller_buf(Q_state[i], OUO_F32);
-    d.B = caller_buf(M[i], OUO_F32);
-    d.out_f32 = w.Pa;
-    d.has_f32 = true;
-    OUO_TRY(gemm_umma(d, s, dev_status));
-    int used = 0;
-    OUO_TRY(gram_parts(w.Pa, w, s, &used));
-    OUO_TRY(sum_parts(w, used, r, red + off, s));
-    off += red_block(r, n);
-  }
-  return OUO_OK;
+  const std::vector<DGroup> gs = plan(M, nmat, ranks.data(), ar);
+  OUO_TRY(stage_project(gs, M, Q_state, dev_status, s));
+  return gram_into_red(gs, red, red_offsets(M, ranks), local_rows, s);
 }
-
-namespace ouo {
-namespace {
-// orth1 (second = false) and orth2 (second = true)
-int shard_orth(const ouo_mat* M, const ouo_mat* Q_state, int nmat,
-               const ouo_dion_params* p, const int64_t* rows_total, void* ws,
-               size_t ws_bytes, float* red, int* dev_status, void* stream, bool second) {
-  clear_error();
-  if (nmat < 0 || nmat > OUO_MAX_BATCH)
-    return set_error(OUO_ERR_INVALID_ARG, "nmat %d out of range", nmat);
-  if (nmat == 0) return OUO_OK;
-  if (!rows_total) return set_error(OUO_ERR_INVALID_ARG, "NULL rows_total");
-  std::vector<int> ranks;
-  OUO_TRY(shard_common(M, Q_state, nmat, p, ws, ws_bytes, red, dev_status, ranks));
-  for (int i = 0; i < nmat; ++i)
-    if (rows_total[i] < ranks[i] || rows_total[i] < M[i].rows)
-      return set_error(OUO_ERR_INVALID_ARG, "rows_total[%d] smaller than rank or local rows", i);
-  cudaStream_t s = (cudaStream_t)stream;
-  Arena ar{reinterpret_cast<char*>(ws), ws_bytes, 0, false};
-  int64_t off = 0;
-  for (int i = 0; i < nmat; ++i) {
-    const int r = ranks[i];
-    const int64_t m = M[i].rows, n = M[i].cols;
-    DionWs w = carve_dion(ar, m, n, r);
-    OUO_TRY(cholesky_inverse(red + off, 1, r, rows_total[i], w, dev_status, s));
-    if (!second) {
-      OUO_TRY(apply_linv(w, r, w.Pa, w.Pb, s));
-      int used = 0;
-      OUO_TRY(gram_parts(w.Pb, w, s, &used));
-      OUO_TRY(sum_parts(w, used, r, red + off, s));
-    } else {
-      OUO_TRY(apply_linv(w, r, w.Pb, w.Pa, s));
-      Buf rt;  // P^T B (r x n) into the exchange buffer
-      rt.p = reinterpret_cast<char*>(red + off);
-      rt.dtype = OUO_F32;
-      rt.rows = r;
-      rt.cols = n;
-      rt.ld = pitch4(n);
-      rt.stride = rt.rows * rt.ld;
-      rt.nb = 1;
-      GemmDesc d;
-      d.M = r; d.N = n; d.K = m; d.nb = 1;
-      d.A = w.Pa;
-      d.B = caller_buf(M[i], OUO_F32);
-      d.b_mn = 1;
-      d.out_f32 = rt;
-      d.has_f32 = true;
-      OUO_TRY(gemm_umma(d, s, dev_status));
-    }
-    off += red_block(r, n);
-  }
-  return OUO_OK;
-}
-}  // namespace
-}  // namespace ouo
 
 extern "C" int dion_shard_orth1(const ouo_mat* M, const ouo_mat* Q_state, int nmat,
                                 const ouo_dion_params* p, const int64_t* rows_total,
@@ -943,67 +911,14 @@ extern "C" int dion_shard_update(const ouo_mat* M, const ouo_mat* Q_state,
       return set_error(OUO_ERR_INVALID_ARG, "W rows must be on 16-byte boundaries (%d)", i);
   cudaStream_t s = (cudaStream_t)stream;
   Arena ar{reinterpret_cast<char*>(ws), ws_bytes, 0, false};
-  const float mu = p->mu, beta = p->beta;
-  int64_t off = 0;
-  for (int i = 0; i < nmat; ++i) {
-    const int r = ranks[i];
-    const int64_t m = M[i].rows, n = M[i].cols;
-    DionWs w = carve_dion(ar, m, n, r);
-    // R^T (summed over ranks) into the workspace
-    copy2d_kernel<<<grid_1d((int64_t)r * n, 256), 256, 0, s>>>(
-        red + off, pitch4(n), reinterpret_cast<float*>(w.Ra.p), w.Ra.ld, r, n);
-    OUO_CHECK_LAUNCH();
-    {
-      dim3 grid((unsigned)ceil_div(m, 32), (unsigned)ceil_div(r, 32));
-      transpose_kernel<<<grid, 256, 0, s>>>(reinterpret_cast<const float*>(w.Pa.p),
-                                            w.Pa.ld, reinterpret_cast<float*>(w.P.p),
-                                            w.P.ld, r, m);
-      OUO_CHECK_LAUNCH();
-    }
-    {  // M <- beta B - (beta - mu) P R^T (local rows)
-      GemmDesc d;
-      d.M = m; d.N = n; d.K = r; d.nb = 1;
-      d.A = w.P;
-      d.B = w.Ra;
-      d.b_mn = 1;
-      d.alpha = -(beta - mu);
-      d.beta = beta;
-      d.has_c0 = true;
-      d.direct = {MatRef{M[i].ptr, M[i].ld}};
-      d.direct_dtype = OUO_F32;
-      d.c0_from_out = true;
-      OUO_TRY(gemm_umma(d, s, dev_status));
-    }
-    Buf Qn = w.Rb;
-    if (p->norm_mode == OUO_DION_COLNORM) {
-      rownorm_kernel<<<r, 256, 0, s>>>(reinterpret_cast<const float*>(w.Ra.p), w.Ra.ld,
-                                       reinterpret_cast<float*>(w.Rb.p), w.Rb.ld, n,
-                                       p->eps);
-      OUO_CHECK_LAUNCH();
-    } else {
-      OUO_TRY(orth_rows(w.Ra, w.Rb, w.Ra, w, s, dev_status));
-      Qn = w.Ra;
-    }
-    {  // W <- (1 - lr wd) W - lr s P Q_new^T (local rows)
-      const float sc = scale ? scale[i] : 1.0f;
-      GemmDesc d;
-      d.M = m; d.N = n; d.K = r; d.nb = 1;
-      d.A = w.P;
-      d.B = Qn;
-      d.b_mn = 1;
-      d.alpha = -p->lr * sc;
-      d.beta = 1.0f - p->lr * p->wd;
-      d.has_c0 = true;
-      d.direct = {MatRef{W[i].ptr, W[i].ld}};
-      d.direct_dtype = w_dtype;
-      d.c0_from_out = true;
-      OUO_TRY(gemm_umma(d, s, dev_status));
-    }
-    copy2d_kernel<<<grid_1d((int64_t)r * n, 256), 256, 0, s>>>(
-        reinterpret_cast<const float*>(Qn.p), Qn.ld,
-        reinterpret_cast<float*>(Q_state[i].ptr), Q_state[i].ld, r, n);
-    OUO_CHECK_LAUNCH();
-    off += red_block(r, n);
-  }
-  return OUO_OK;
+  const std::vector<DGroup> gs = plan(M, nmat, ranks.data(), ar);
+  const std::vector<int64_t> off = red_offsets(M, ranks);
+  // R^T (summed over the ranks) is read where the caller left it
+  auto rt_red = [&](const DGroup& g, int64_t i, int64_t* ld) {
+    *ld = pitch4(g.n);
+    return red + off[g.members[i]];
+  };
+  std::vector<int64_t> no_sig((size_t)nmat, 0);
+  OUO_TRY(stage_qnew(gs, rt_red, Q_state, p, nullptr, no_sig, dev_status, s));
+  return stage_update(gs, rt_red, M, W, w_dtype, p, scale, dev_status, s);
 }

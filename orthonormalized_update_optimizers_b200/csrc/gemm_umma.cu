@@ -86,6 +86,12 @@ struct Segment {
   CUtensorMap tmAt;
   CUtensorMap tmBt;
   int t4d;
+  // split-K: the K blocks of every output tile are divided into `ksplit`
+  // ranges of `kbc` blocks; range s of matrix b is written to output matrix
+  // b * ksplit + s (workspace outputs only), to be summed by the caller
+  int ksplit;
+  int64_t kbc;
+  int64_t tiles_2d;  // output tiles of one matrix (tiles_per_mat / ksplit)
 };
 
 constexpr int kMaxSeg = 6;
@@ -103,6 +109,9 @@ struct UmmaArgs {
   int* status;
   void* dptr[kChunk];
   int64_t dld[kChunk];
+  // per-matrix alpha of direct outputs (has_dalpha), else `alpha` for all
+  float dalpha[kChunk];
+  int has_dalpha;
 };
 
 template <int BN, int CG>
@@ -133,14 +142,18 @@ __host__ __device__ __forceinline__ int64_t tri_jmin(int64_t i, int BN, int TR) 
 // tile column).
 __device__ __forceinline__ int decode_tile(const UmmaArgs& a, int BN, int TR,
                                            int64_t tile, int64_t* b,
-                                           int64_t* ti, int64_t* tj) {
+                                           int64_t* ti, int64_t* tj,
+                                           int64_t* ks) {
   int g = 0;
   while (g + 1 < a.nseg && tile >= a.seg[g + 1].tile_start) ++g;
   const Segment& sg = a.seg[g];
   int64_t t = tile - sg.tile_start;
   *b = t / sg.tiles_per_mat;
   t -= *b * sg.tiles_per_mat;
+  *ks = 0;
   if (!a.tri) {
+    *ks = t / sg.tiles_2d;
+    t -= *ks * sg.tiles_2d;
     *ti = t / sg.tiles_n;
     *tj = t - *ti * sg.tiles_n;
     return g;
@@ -346,14 +359,16 @@ umma_gemm_kernel(const __grid_constant__ UmmaArgs a) {
     int64_t issued = 0;
     for (int64_t tile = tile0; ok && tile < a.total_tiles;
          tile += tile_step) {
-      int64_t b, ti, tj;
-      const int g = decode_tile(a, BN, TR, tile, &b, &ti, &tj);
+      int64_t b, ti, tj, ks;
+      const int g = decode_tile(a, BN, TR, tile, &b, &ti, &tj, &ks);
       const Segment& sg = a.seg[g];
       const int64_t nk = (sg.K + kBK - 1) / kBK;
+      const int64_t kb0 = ks * sg.kbc;
+      const int64_t kb1 = kb0 + sg.kbc < nk ? kb0 + sg.kbc : nk;
       const int32_t z = (int32_t)(sg.b0 + b);
       const int32_t arow = (int32_t)(ti * TR + rank * kTileM);
       const int32_t bcol = (int32_t)(tj * BN + rank * C::kBRows);
-      for (int64_t kb = 0; kb < nk; ++kb) {
+      for (int64_t kb = kb0; kb < kb1; ++kb) {
         if (!ptx::mbar_wait(&empty[stage], phase ^ 1, abort_flag)) {
           ok = false;
           break;
@@ -434,9 +449,11 @@ umma_gemm_kernel(const __grid_constant__ UmmaArgs a) {
     int64_t local = 0;
     for (int64_t tile = tile0; ok && tile < a.total_tiles;
          tile += tile_step, ++local) {
-      int64_t b, ti, tj;
-      const int g = decode_tile(a, BN, TR, tile, &b, &ti, &tj);
+      int64_t b, ti, tj, ks;
+      const int g = decode_tile(a, BN, TR, tile, &b, &ti, &tj, &ks);
       const int64_t nk = (a.seg[g].K + kBK - 1) / kBK;
+      const int64_t kb0 = ks * a.seg[g].kbc;
+      const int64_t kb1 = kb0 + a.seg[g].kbc < nk ? kb0 + a.seg[g].kbc : nk;
       const uint32_t buf = (uint32_t)(local & 1);
       const uint32_t tphase = (uint32_t)((local >> 1) & 1);
       if (!ptx::mbar_wait(&tempty[buf], tphase ^ 1, abort_flag)) {
@@ -445,7 +462,7 @@ umma_gemm_kernel(const __grid_constant__ UmmaArgs a) {
       }
       ptx::tc_fence_after();
       const uint32_t d = tmem_base + buf * BN;
-      for (int64_t kb = 0; kb < nk; ++kb) {
+      for (int64_t kb = kb0; kb < kb1; ++kb) {
         if (!ptx::mbar_wait(&full[stage], phase, abort_flag)) {
           ok = false;
           break;
@@ -469,7 +486,7 @@ umma_gemm_kernel(const __grid_constant__ UmmaArgs a) {
         for (uint32_t kk = 0; kk < kBK / kInstK; ++kk) {
           const uint64_t ad = a_mn ? mn_desc(sa, kk) : ptx::smem_desc_sw128(sa + kk * 32, 16, 1024);
           const uint64_t bd = b_mn ? mn_desc(sb, kk) : ptx::smem_desc_sw128(sb + kk * 32, 16, 1024);
-          const uint32_t acc = (kb > 0 || kk > 0) ? 1u : 0u;
+          const uint32_t acc = (kb > kb0 || kk > 0) ? 1u : 0u;
           if (CG == 2) {
             if (FMT == 1) ptx::mma2_bf16(d, ad, bd, idesc, acc);
             else ptx::mma2_tf32(d, ad, bd, idesc, acc);
@@ -505,11 +522,52 @@ umma_gemm_kernel(const __grid_constant__ UmmaArgs a) {
     uint32_t nstores = 0;  // bulk stores issued by this warp
     for (int64_t tile = tile0; tile < a.total_tiles;
          tile += tile_step, ++local) {
-      int64_t b, ti, tj;
-      const int g = decode_tile(a, BN, TR, tile, &b, &ti, &tj);
+      int64_t b, ti, tj, ks;
+      const int g = decode_tile(a, BN, TR, tile, &b, &ti, &tj, &ks);
       const Segment& sg = a.seg[g];
       const uint32_t buf = (uint32_t)(local & 1);
       const uint32_t tphase = (uint32_t)((local >> 1) & 1);
+      // Non-symmetric outputs with a C0 (a workspace matrix, or the output
+      // itself for in-place updates) are written through the direct path
+      // below; their C0 is prefetched one 32 x 32 chunk ahead into
+      // registers, the first chunk before the accumulator is waited for,
+      // so that every epilogue warp keeps a chunk of loads in flight.
+      constexpr int kCh = BN / 64;  // 32-column chunks per warp (half a tile)
+      const bool pf = !a.tma_out && !a.tri && a.has_c0;
+      const int64_t pf_row = ti * TR + rank * kTileM + q * 32;
+      const int pf_sr = lane >> 3, pf_sc = 4 * (lane & 7);
+      const uint32_t pf_half = (uint32_t)((warp - 2) >> 2);
+      const TileOut pf_to = tile_out(a, sg, b);
+      // C0 element (pf_row + pf_sr, column 0 of this warp's half), its
+      // element size and the byte step between it-rows (4 matrix rows)
+      const int pf_es = a.c0_out ? (a.has_f32 ? 4 : 2) : (a.c0_bf16 ? 2 : 4);
+      const int64_t pf_ld = a.c0_out ? (a.has_f32 ? pf_to.ldf : pf_to.ldh) : sg.ldc0;
+      const char* pf_base = nullptr;
+      if (pf) {
+        const int64_t e0 = (pf_row + pf_sr) * pf_ld + tj * BN + pf_half * (BN / 2) + pf_sc;
+        pf_base = a.c0_out
+            ? (a.has_f32 ? reinterpret_cast<const char*>(pf_to.f) : reinterpret_cast<const char*>(pf_to.h)) + e0 * pf_es
+            : reinterpret_cast<const char*>(sg.C0) + ((sg.b0 + b) * sg.sc0 + e0) * pf_es;
+      }
+      // C0 of (chunk c, it-row it): rows pf_row + 4 it + pf_sr, 16 bytes,
+      // for chunks inside the matrix (edge chunks load where they are used)
+      auto pf_full = [&](int c) {
+        return pf_row + 32 <= sg.M && tj * BN + pf_half * (BN / 2) + c * 32 + 32 <= sg.N;
+      };
+      auto pf_load = [&](int c, int it) {
+        const char* p0 = pf_base + (int64_t)c * 32 * pf_es + (int64_t)it * 4 * pf_ld * pf_es;
+        if (pf_es == 4) return __ldg(reinterpret_cast<const float4*>(p0));
+        const uint2 u = __ldg(reinterpret_cast<const uint2*>(p0));
+        return make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xffff0000u),
+                           __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xffff0000u));
+      };
+      // one chunk of C0 in flight: slot `it` is refilled with the next
+      // chunk's value as soon as the current chunk has taken it
+      float4 pfe[8];
+      if (pf && pf_full(0)) {
+#pragma unroll
+        for (int it = 0; it < 8; ++it) pfe[it] = pf_load(0, it);
+      }
       // one lane polls the barrier; the warp follows through __syncwarp
       int ok = 1;
       if (lane == 0) ok = ptx::mbar_wait(&tfull[buf], tphase, abort_flag) ? 1 : 0;
@@ -549,7 +607,7 @@ umma_gemm_kernel(const __grid_constant__ UmmaArgs a) {
           __syncwarp();
         };
         const uint32_t half = (uint32_t)((warp - 2) >> 2);
-        const int32_t z = (int32_t)(sg.b0 + b);
+        const int32_t z = (int32_t)((sg.b0 + b) * sg.ksplit + ks);
         const bool obf = a.has_bf16 != 0;
 #pragma unroll 1
         for (uint32_t c0 = half * (BN / 2); c0 < (half + 1) * (BN / 2); c0 += 32) {
@@ -652,6 +710,79 @@ umma_gemm_kernel(const __grid_constant__ UmmaArgs a) {
         }
         continue;
       }
+      if (!a.tri) {
+        // Non-symmetric direct (or dual) outputs.  This warp owns tile rows
+        // q*32 .. q*32+31 (TMEM lanes) and one half of the columns, in
+        // 32 x 32 chunks: finished with row = lane, staged in shared
+        // memory, and stored 16 bytes per lane, 8 lanes per 128-byte row,
+        // 4 rows per instruction, with the prefetched C0 added on the way.
+        const float alpha = (a.has_dalpha && sg.direct) ? a.dalpha[sg.dbase + b] : a.alpha;
+        float* stg = epi_smem + (warp - 2) * (C::kStg * 32 * 32);
+#pragma unroll 1
+        for (int c = 0; c < kCh; ++c) {
+          const int64_t gj0 = tj * BN + pf_half * (BN / 2) + c * 32;
+          const bool next_full = pf && c + 1 < kCh && pf_full(c + 1);
+          if (pf_row >= sg.M || gj0 >= sg.N) continue;  // outside the output
+          const bool full_chunk = pf_row + 32 <= sg.M && gj0 + 32 <= sg.N;
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {  // two 16-column TMEM loads
+            float v[16];
+            ptx::tmem_ld16(tmem_base + ((q * 32u) << 16) + buf * BN +
+                               (uint32_t)(pf_half * (BN / 2) + c * 32 + hh * 16), v);
+#pragma unroll
+            for (int j = 0; j < 16; j += 4)
+              *reinterpret_cast<float4*>(stg + stg_idx(lane, hh * 16 + j)) =
+                  make_float4(alpha * v[j], alpha * v[j + 1], alpha * v[j + 2], alpha * v[j + 3]);
+          }
+          __syncwarp();
+#pragma unroll
+          for (int it = 0; it < 8; ++it) {
+            const int rr = it * 4 + pf_sr;
+            const int64_t gr = pf_row + rr, gc = gj0 + pf_sc;
+            float4 w = *reinterpret_cast<const float4*>(stg + stg_idx(rr, pf_sc));
+            uint32_t mask = 0xFu;
+            if (!full_chunk) {
+              mask = 0;
+#pragma unroll
+              for (int t = 0; t < 4; ++t)
+                if (gr < sg.M && gc + t < sg.N) mask |= 1u << t;
+            }
+            if (pf) {
+              float4 e = pfe[it];
+              if (next_full) pfe[it] = pf_load(c + 1, it);
+              if (!full_chunk) {
+                float x[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int t = 0; t < 4; ++t)
+                  if (mask & (1u << t))
+                    x[t] = a.c0_out ? load_out1(a, pf_to, gr, gc + t)
+                                    : load_c0(sg, b, gr, gc + t, a.c0_bf16);
+                e = make_float4(x[0], x[1], x[2], x[3]);
+              }
+              w.x += a.beta * e.x;
+              w.y += a.beta * e.y;
+              w.z += a.beta * e.z;
+              w.w += a.beta * e.w;
+            }
+            if (a.gamma != 0.f && gr >= gc && gr < gc + 4) {
+              if (gr == gc) w.x += a.gamma;
+              if (gr == gc + 1) w.y += a.gamma;
+              if (gr == gc + 2) w.z += a.gamma;
+              if (gr == gc + 3) w.w += a.gamma;
+            }
+            if (mask) store4t(a, pf_to, gr, gc, w, mask);
+          }
+          __syncwarp();
+        }
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          if (CG == 2) ptx::mbar_arrive_cluster(tempty_lead + buf * 8u);
+          else ptx::mbar_arrive(&tempty[buf]);
+        }
+        continue;
+      }
+      // Symmetric direct (or dual) outputs.
       // This warp owns tile rows q*32 .. q*32+31 (TMEM lanes) and one half
       // of the columns; each chunk is 32 rows x 32 columns.  Values are
       // finished with row = lane (where the symmetric C0 read (j, i) is
@@ -979,6 +1110,7 @@ int launch(const std::vector<GemmDesc>& gs, cudaStream_t stream, int* status) {
   a.has_f32 = g0.has_f32; a.round_tf32 = g0.round_tf32;
   a.has_bf16 = g0.has_bf16;
   a.status = status;
+  a.has_dalpha = !g0.direct_alpha.empty() ? 1 : 0;
   if (!g0.direct.empty()) {
     a.has_f32 = g0.direct_dtype == OUO_F32;
     a.has_bf16 = g0.direct_dtype == OUO_BF16;
@@ -1071,7 +1203,15 @@ int launch(const std::vector<GemmDesc>& gs, cudaStream_t stream, int* status) {
       }
     }
     proto.tiles_n = ceil_div(g.N, BN);
-    proto.tiles_per_mat = tiles_per_matrix(g, BN, TR);
+    proto.tiles_2d = tiles_per_matrix(g, BN, TR);
+    {
+      const int64_t nk = ceil_div(g.K, (int64_t)bk);
+      int64_t ksp = g.ksplit < 1 ? 1 : g.ksplit;
+      if (ksp > nk) ksp = nk;
+      proto.kbc = ceil_div(nk, ksp);
+      proto.ksplit = (int)ceil_div(nk, proto.kbc);  // every range non-empty
+    }
+    proto.tiles_per_mat = proto.tiles_2d * proto.ksplit;
     proto.C0 = (g.has_c0 && !g.c0_from_out) ? g.C0.p : nullptr;
     proto.ldc0 = g.C0.ld; proto.sc0 = g.C0.stride;
     proto.Of = g.has_f32 ? reinterpret_cast<float*>(g.out_f32.p) : nullptr;
@@ -1098,6 +1238,7 @@ int launch(const std::vector<GemmDesc>& gs, cudaStream_t stream, int* status) {
         for (int64_t i = 0; i < nb; ++i) {
           a.dptr[ndirect + i] = g.direct[b0 + i].p;
           a.dld[ndirect + i] = g.direct[b0 + i].ld;
+          a.dalpha[ndirect + i] = a.has_dalpha ? g.direct_alpha[b0 + i] : g.alpha;
         }
         ndirect += (int)nb;
       }
@@ -1145,6 +1286,15 @@ int gemm_timing_read(int kind, int* launches, double* total_ms, double* flops) {
   return OUO_OK;
 }
 
+int gemm_ksplit_used(int64_t K, int ksplit, int dtype) {
+  const int64_t bk = kRowBytes / (dtype == OUO_BF16 ? 2 : 4);
+  const int64_t nk = ceil_div(K, bk);
+  int64_t ksp = ksplit < 1 ? 1 : ksplit;
+  if (ksp > nk) ksp = nk;
+  const int64_t kbc = ceil_div(nk, ksp);
+  return (int)ceil_div(nk, kbc);
+}
+
 int cta_pair_mode() {
   const char* env = getenv("OUO_CTA_PAIR");
   return env && env[0] >= '0' && env[0] <= '2' ? env[0] - '0' : 1;
@@ -1152,37 +1302,10 @@ int cta_pair_mode() {
 
 bool cta_pairs_enabled() { return cta_pair_mode() > 0; }
 
-int gemm_umma_grouped(const std::vector<GemmDesc>& gs, cudaStream_t stream,
-                      int* status) {
-  if (gs.empty()) return OUO_OK;
+// One launch kind: operand type, B majorness, CTA pairs, tile width.
+int launch_kind(const std::vector<GemmDesc>& gs, bool pair, bool wide, cudaStream_t stream,
+                int* status) {
   const GemmDesc& g0 = gs[0];
-  bool wide = false, tall = false;
-  for (const GemmDesc& g : gs) {
-    if (g.A.dtype != g.B.dtype || g.A.dtype != g0.A.dtype)
-      return set_error(OUO_ERR_UNSUPPORTED, "tensor-core GEMM needs equal operand types");
-    if (g.tri != g0.tri || g.b_mn != g0.b_mn || g.has_c0 != g0.has_c0 ||
-        g.has_f32 != g0.has_f32 || g.has_bf16 != g0.has_bf16 ||
-        g.round_tf32 != g0.round_tf32 || g.direct.empty() != g0.direct.empty() ||
-        g.c0_from_out != g0.c0_from_out || g.sym_half != g0.sym_half ||
-        g.a_sym != g0.a_sym || g.b_sym != g0.b_sym || g.c0_upper != g0.c0_upper ||
-        g.alpha != g0.alpha || g.beta != g0.beta || g.gamma != g0.gamma ||
-        (g.has_c0 && g.C0.dtype != g0.C0.dtype) ||
-        (!g.direct.empty() && g.direct_dtype != g0.direct_dtype))
-      return set_error(OUO_ERR_INVALID_ARG, "grouped GEMM descriptors differ");
-    if (g.tri && (g.M != g.N || g.b_mn))
-      return set_error(OUO_ERR_INVALID_ARG, "symmetric GEMM needs M == N, K-major B");
-    if (!g.direct.empty() && (int64_t)g.direct.size() != g.nb)
-      return set_error(OUO_ERR_INVALID_ARG, "direct output table size mismatch");
-    if (g.c0_from_out && (g.direct.empty() || g.tri))
-      return set_error(OUO_ERR_INVALID_ARG, "in-place C0 needs direct, non-symmetric outputs");
-    wide = wide || g.N > 128;
-    tall = tall || g.M > 128;
-  }
-  // CTA pairs (256 x 256 tiles) for wide outputs with more than 128 rows and
-  // K-major B.  OUO_CTA_PAIR=0 selects single-CTA 128 x BN tiles throughout;
-  // OUO_CTA_PAIR=2 also puts MN-major B (Q X) on pairs.
-  const int pair_mode = cta_pair_mode();
-  const bool pair = wide && tall && pair_mode > 0 && (!g0.b_mn || pair_mode == 2);
   if (g0.A.dtype == OUO_BF16) {
     if (g0.b_mn) {
       if (pair) return launch<256, 1, 1, 2>(gs, stream, status);
@@ -1197,6 +1320,60 @@ int gemm_umma_grouped(const std::vector<GemmDesc>& gs, cudaStream_t stream,
   }
   if (pair) return launch<256, 2, 0, 2>(gs, stream, status);
   return wide ? launch<256, 2, 0, 1>(gs, stream, status) : launch<128, 2, 0, 1>(gs, stream, status);
+}
+
+int gemm_umma_grouped(const std::vector<GemmDesc>& gs, cudaStream_t stream,
+                      int* status) {
+  if (gs.empty()) return OUO_OK;
+  const GemmDesc& g0 = gs[0];
+  bool wide = false, tall = false, per_desc = false;
+  for (const GemmDesc& g : gs) {
+    if (g.A.dtype != g.B.dtype || g.A.dtype != g0.A.dtype)
+      return set_error(OUO_ERR_UNSUPPORTED, "tensor-core GEMM needs equal operand types");
+    if (g.tri != g0.tri || g.b_mn != g0.b_mn || g.has_c0 != g0.has_c0 ||
+        g.has_f32 != g0.has_f32 || g.has_bf16 != g0.has_bf16 ||
+        g.round_tf32 != g0.round_tf32 || g.direct.empty() != g0.direct.empty() ||
+        g.c0_from_out != g0.c0_from_out || g.sym_half != g0.sym_half ||
+        g.a_sym != g0.a_sym || g.b_sym != g0.b_sym || g.c0_upper != g0.c0_upper ||
+        (g.alpha != g0.alpha && g0.direct_alpha.empty()) || g.beta != g0.beta ||
+        g.gamma != g0.gamma || g.direct_alpha.empty() != g0.direct_alpha.empty() ||
+        (g.has_c0 && g.C0.dtype != g0.C0.dtype) ||
+        (!g.direct.empty() && g.direct_dtype != g0.direct_dtype))
+      return set_error(OUO_ERR_INVALID_ARG, "grouped GEMM descriptors differ");
+    if (g.tri && (g.M != g.N || g.b_mn))
+      return set_error(OUO_ERR_INVALID_ARG, "symmetric GEMM needs M == N, K-major B");
+    if (!g.direct.empty() && (int64_t)g.direct.size() != g.nb)
+      return set_error(OUO_ERR_INVALID_ARG, "direct output table size mismatch");
+    if (g.c0_from_out && (g.direct.empty() || g.tri))
+      return set_error(OUO_ERR_INVALID_ARG, "in-place C0 needs direct, non-symmetric outputs");
+    if (!g.direct_alpha.empty() && (int64_t)g.direct_alpha.size() != g.nb)
+      return set_error(OUO_ERR_INVALID_ARG, "direct alpha table size mismatch");
+    if (g.ksplit > 1 && (g.tri || !g.direct.empty() || g.has_c0 || g.has_f32 == g.has_bf16))
+      return set_error(OUO_ERR_INVALID_ARG,
+                       "split-K needs one workspace output, no C0, non-symmetric");
+    wide = wide || g.N > 128;
+    tall = tall || g.M > 128;
+    per_desc = per_desc || g.per_desc_tiles;
+  }
+  // CTA pairs (256 x 256 tiles) for wide outputs with more than 128 rows and
+  // K-major B.  OUO_CTA_PAIR=0 selects single-CTA 128 x BN tiles throughout;
+  // OUO_CTA_PAIR=2 also puts MN-major B (Q X) on pairs.
+  const int pair_mode = cta_pair_mode();
+  auto pair_of = [&](bool w, bool t) {
+    return w && t && pair_mode > 0 && (!g0.b_mn || pair_mode == 2);
+  };
+  if (!per_desc) return launch_kind(gs, pair_of(wide, tall), wide, stream, status);
+  // every descriptor keeps its own tile shape: one launch per shape in use
+  for (int kind = 0; kind < 3; ++kind) {
+    std::vector<GemmDesc> part;
+    for (const GemmDesc& g : gs) {
+      const bool w = g.N > 128, pr = pair_of(w, g.M > 128);
+      const int k = pr ? 2 : (w ? 1 : 0);
+      if (k == kind) part.push_back(g);
+    }
+    if (!part.empty()) OUO_TRY(launch_kind(part, kind == 2, kind >= 1, stream, status));
+  }
+  return OUO_OK;
 }
 
 int gemm_umma(const GemmDesc& g, cudaStream_t stream, int* status) {

@@ -96,7 +96,24 @@ struct GemmDesc {
   //              left of the diagonal are read from the transposed block;
   //   c0_upper:  the symmetric C0 is upper-stored (read at (i, j), j >= i).
   bool sym_half = false, a_sym = false, b_sym = false, c0_upper = false;
+  // Per-matrix alpha of direct outputs (one value per batch matrix); empty:
+  // `alpha` for every matrix.
+  std::vector<float> direct_alpha;
+  // Split-K (tensor-core path, one workspace output, no C0, non-symmetric):
+  // the K range is cut into up to `ksplit` equal ranges of whole K blocks;
+  // range s of matrix b is written to output matrix b * ksplit' + s, where
+  // ksplit' = gemm_ksplit_used(K, ksplit, dtype) <= ksplit (no empty range).
+  // The output buffer holds nb * ksplit' matrices; the caller sums them.
+  int ksplit = 1;
+  // Tile shape (CTA pair or not, 128 or 256 columns) chosen for this
+  // descriptor alone instead of for the whole grouped launch, so that a
+  // matrix is computed the same way whatever it is batched with.
+  bool per_desc_tiles = false;
 };
+
+// Number of K ranges a split-K GEMM of depth K over `dtype` operands
+// actually uses for a requested `ksplit` (every range non-empty).
+int gemm_ksplit_used(int64_t K, int ksplit, int dtype);
 
 // Whether K-major tensor-core GEMMs with more than 128 output rows and
 // columns run on CTA-pair tiles (OUO_CTA_PAIR, default on); upper-stored
@@ -137,19 +154,71 @@ int ns_writeout(const Buf& y, const ouo_mat* O, int o_dtype, const Group& grp,
 // Fill nb identity matrices (fp32 and / or bf16 copies).
 int fill_identity(const Buf& q, cudaStream_t stream);
 
-// Blocked Cholesky + triangular inverse (chol.cu): S = sum of `splits`
-// partial r x r Gram matrices; writes L^-1 into Linv (R x R, ld R, R = r
-// rounded up to 32).  S is R x R scratch (ld R); ctl is
+// --------------------------------------------------- batched CholeskyQR
+// One r x L block of rows to orthonormalize (cholqr.cu): Gram matrix S =
+// X X^T, Cholesky S = L L^T, Y = L^-1 X (rows orthonormal, the QR factor
+// with a positive diagonal).  Every pointer is device memory.
+struct CholQrJob {
+  const float* X = nullptr;  // r x L, row pitch ldx (16-byte rows preferred)
+  int64_t ldx = 0;
+  int r = 0;
+  int64_t L = 0;
+  int64_t gchunk = 0;        // Gram: columns per split (multiple of 32)
+  float* gpart = nullptr;    // Gram partials [ceil(L / gchunk)][r][r]
+  float* S = nullptr;        // summed Gram, r x r, upper storage (j >= i valid)
+  float* Lb = nullptr;       // R x R (R = r rounded up to 32), ld R: the
+                             // strictly lower 32 x 32 blocks of L
+  const float* Dd = nullptr; // R x R, ld R: D_i = L_ii^-1 on the diagonal
+                             // blocks (nullptr: they are in Lb)
+  float* Y = nullptr;        // L^-1 X, r x L (may be X itself)
+  int64_t ldy = 0;
+  float* Y2 = nullptr;       // optional copy of Y
+  int64_t ldy2 = 0;
+  float* Yt = nullptr;       // optional transpose of Y, L x r
+  int64_t ldyt = 0;
+};
+// Gram splits for an r x L block (columns per split = ceil(L / splits),
+// rounded up to 32).
+int cholqr_gram_splits(int r, int64_t L);
+// Gram partials and their float64 sum S, for every job (2 launches).
+int cholqr_gram(const std::vector<CholQrJob>& jobs, cudaStream_t s);
+// Whether the one-CTA Cholesky takes rank r (1 <= r <= 256).
+bool cholqr_small_rank(int r);
+// S -> Lb (strictly lower blocks of L and D_i on the diagonal blocks), one
+// CTA per job, r <= 256; breakdown after the shifted retry sets
+// OUO_STATUS_BREAKDOWN and writes the identity.
+int cholqr_factor(const std::vector<CholQrJob>& jobs, int* status, cudaStream_t s);
+// Y = L^-1 X (and Y2, Yt) for every job, r <= 1024.
+int cholqr_apply(const std::vector<CholQrJob>& jobs, cudaStream_t s);
+
+// Rows of the sum of `ks` partial matrices (sp floats apart, row pitch
+// ldp), with optional row norms (float64, fixed order) and normalized rows
+// v / (||v|| + eps).
+struct RowsJob {
+  const float* part = nullptr;
+  int64_t ldp = 0, sp = 0;
+  int ks = 1;
+  int64_t rows = 0, n = 0;
+  float* out = nullptr;      // optional summed rows
+  int64_t ldo = 0;
+  float* sigma = nullptr;    // optional row norms
+  float* qn = nullptr;       // optional normalized rows
+  int64_t ldq = 0;
+  float* q2 = nullptr;       // optional copy of qn
+  int64_t ldq2 = 0;
+};
+int rows_reduce(const std::vector<RowsJob>& jobs, float eps, cudaStream_t s);
+
+// Cooperative blocked Cholesky for ranks above 256 (chol.cu): S = sum of
+// `splits` partial r x r Gram matrices in upper storage.  With `inverse`,
+// writes L^-1 into Linv (R x R, ld R, R = r rounded up to 32); without it,
+// leaves the strictly lower blocks of L in S (R x R, ld R) and the inverted
+// diagonal blocks in the diagonal blocks of Linv.  ctl is
 // chol_blocked_ctl_bytes(r) bytes of 8-byte aligned scratch.
 size_t chol_blocked_ctl_bytes(int r);
 int chol_blocked(const float* part, int splits, int r, int64_t L, float* S,
-                 float* Linv, void* ctl, int* status, cudaStream_t stream);
-// The same factorization and inverse in one CTA with the blocks in shared
-// memory, for 1 <= r <= 256 (chol_smem_fits), from one summed r x r matrix
-// S (ld r); no scratch besides Linv.
-bool chol_smem_fits(int r);
-int chol_smem(const float* S, int r, int64_t L, float* Linv, int* status,
-              cudaStream_t stream);
+                 float* Linv, void* ctl, int* status, cudaStream_t stream,
+                 bool inverse);
 int convert_buf(const Buf& src, const Buf& dst, cudaStream_t stream);
 
 }  // namespace ouo

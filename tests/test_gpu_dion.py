@@ -104,38 +104,24 @@ def test_dion_wide_ranks(mode, shape, r, steps):
 
 
 @pytest.mark.parametrize("mode", [odion.COLNORM, odion.QR])
-@pytest.mark.parametrize("shape,r", [((640, 512), 65), ((512, 300), 100),
-                                     ((768, 1024), 200), ((1024, 1024), 256)])
-@pytest.mark.parametrize("smem_max", ["256", "0"])
-def test_cholesky_routes_for_ranks_65_to_256(mode, shape, r, smem_max, monkeypatch):
-    # Both blocked Cholesky kernels at every block count they may serve:
-    # OUO_CHOL_SMEM_MAX_RANK=256 sends ranks up to 256 to the one-CTA kernel
-    # (blocks in shared memory), 0 sends them all to the cooperative one.
-    # Both must follow the oracle; r = 65, 100 and 200 leave ragged blocks.
-    monkeypatch.setenv("OUO_CHOL_SMEM_MAX_RANK", smem_max)
+@pytest.mark.parametrize("shape,r", [((256, 512), 8), ((300, 200), 40), ((640, 512), 65),
+                                     ((512, 300), 100), ((768, 1024), 200),
+                                     ((1024, 1024), 256)])
+def test_one_cta_cholesky_ranks_up_to_256(mode, shape, r):
+    # ranks up to 256 take the one-CTA blocked Cholesky: one block (r = 8),
+    # ragged last blocks (40, 65, 100, 200) and all eight blocks (256)
     errs = _run(*shape, r, mode, steps=3, seed=3 * r + 1)
     for e_m, e_q, e_w in errs:
         assert e_m <= TOL_BF16 and e_q <= TOL_BF16 and e_w <= TOL_BF16, errs
 
 
-@pytest.mark.parametrize("mode", [odion.COLNORM, odion.QR])
-@pytest.mark.parametrize("shape,r", [((256, 512), 8), ((300, 200), 40)])
-def test_one_cta_blocked_cholesky_at_small_ranks(mode, shape, r, monkeypatch):
-    # OUO_CHOL_BLOCKED_MIN_RANK=1 routes every rank up to 224 to the
-    # one-CTA blocked kernel: one block (r = 8) and two ragged blocks (r = 40)
-    monkeypatch.setenv("OUO_CHOL_BLOCKED_MIN_RANK", "1")
-    errs = _run(*shape, r, mode, steps=3, seed=r + 5)
-    for e_m, e_q, e_w in errs:
-        assert e_m <= TOL_BF16 and e_q <= TOL_BF16 and e_w <= TOL_BF16, errs
-
-
-@pytest.mark.parametrize("smem_max", ["256", "0"])
-def test_zero_gradient_takes_the_shifted_retry(smem_max, monkeypatch):
+@pytest.mark.parametrize("r", [96, 300])
+def test_zero_gradient_takes_the_shifted_retry(r):
     # B = 0 makes every Gram matrix zero: the first factorization meets a
     # zero pivot, the shifted retry (tr S = 0, so the smallest positive
-    # shift) succeeds, and the step leaves M at zero and W unchanged.
-    monkeypatch.setenv("OUO_CHOL_SMEM_MAX_RANK", smem_max)
-    m, n, r = 512, 384, 96
+    # shift) succeeds, and the step leaves M at zero and W unchanged.  r = 96
+    # runs the one-CTA Cholesky, r = 300 the cooperative one.
+    m, n = 512, 384
     M = torch.zeros(m, n, device=DEV)
     G = torch.zeros(m, n, dtype=torch.bfloat16, device=DEV)
     W = synth.gaussian((m, n), 5, 0.02, torch.float32, DEV)
