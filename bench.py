@@ -53,6 +53,10 @@ def _args():
     ap.add_argument("--layers", type=int, default=32)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-dion", action="store_true",
+                    help="skip the Dion / Orth-Dion measurements of the JSON line")
+    ap.add_argument("--no-sweep", action="store_true",
+                    help="skip the standard-vs-Gram crossover points of the JSON line")
     ap.add_argument("--cpu-sample-layers", type=int, default=1)
     ap.add_argument("--micro", choices=["gram", "dion"], default=None,
                     help="one kernel-level case for profiling: Gram NS on --nb blocks "
@@ -315,14 +319,20 @@ def run_ours(args):
     parts = shard.plan_partition(mn, world, RHO)
     own = parts[rank]
     lay = shard.ExchangeLayout(mn, parts, RHO)
-    Gs, Ms = [], []
-    for i in own:
+    # every operand laid out one block per shape (the layout the grouped
+    # launches read without copies)
+    own_mn = [mn[i] for i in own]
+    Gs = ouo.batch_empty(own_mn, torch.bfloat16, dev)
+    Ms = ouo.batch_empty(own_mn, torch.float32, dev)
+    for k, i in enumerate(own):
         m, n = mn[i]
-        Gs.append(synth.lowrank_plus_noise(m, n, 32, 0.01, synth.seed_for(3, i),
-                                           torch.bfloat16, dev))
-        Ms.append(torch.zeros(m, n, dtype=torch.float32, device=dev))
-    Ws = [synth.gaussian((m, n), synth.seed_for(3, 1000 + i), 0.02, torch.bfloat16, dev)
-          for i, (m, n) in enumerate(mn)]
+        Gs[k].copy_(synth.lowrank_plus_noise(m, n, 32, 0.01, synth.seed_for(3, i),
+                                             torch.bfloat16, dev))
+        Ms[k].zero_()
+    Ws = ouo.batch_empty(mn, torch.bfloat16, dev)
+    for i, (m, n) in enumerate(mn):
+        Ws[i].copy_(synth.gaussian((m, n), synth.seed_for(3, 1000 + i), 0.02,
+                                   torch.bfloat16, dev))
     ks = [lay.k[i] for i in own]
     assert ks == [ouo.dion3_num_selected(mn[i][0], RHO) for i in own]
     keys = torch.empty(max(1, sum(mn[i][0] for i in own)), dtype=torch.float64, device=dev)
@@ -415,41 +425,31 @@ def run_ours(args):
     barrier()
     launches = ouo.launch_count() - n0
     ms = max_over_ranks(e0.elapsed_time(e1) / args.steps)
-    # --- the Gram-NS stage alone (dominant tensor-core kernels)
-    g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    g0.record()
-    for _ in range(args.steps):
-        if own:
-            ouo.gram_ns_orthogonalize(Xb, Ob, params, workspace=ws, status=status)
-    g1.record()
-    barrier()
-    gram_ms = max_over_ranks(g0.elapsed_time(g1) / args.steps)
-    # --- the momentum kernel alone (HBM-bound)
-    m0, m1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    m0.record()
-    for _ in range(args.steps):
+    # --- the step's parts, timed inside full steps: events recorded between
+    # the calls of each step, so the parts add up to the step
+    part_names = ("momentum", "selection", "gram_ns", "update")
+    pev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    for k in range(args.steps):
+        ev = pev[k]
+        ev[0].record()
         if own:
             ouo.dion_momentum_update(Mb, Gb, MU, "accum", keys)
-    m1.record()
-    barrier()
-    mom_ms = max_over_ranks(m0.elapsed_time(m1) / args.steps)
-    # --- row selection + gather, and the weight update (HBM-bound), alone
-    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    s0.record()
-    for _ in range(args.steps):
+        ev[1].record()
         if own:
             ouo.dion3_select_rows(Mb, keys, RHO, idx, Xb, scale, ef=True, mu=MU)
-    s1.record()
+        ev[2].record()
+        if own:
+            ouo.gram_ns_orthogonalize(Xb, Ob, params, workspace=ws, status=status)
+        ev[3].record()
+        exchange_and_update()
+        ev[4].record()
     barrier()
-    sel_ms = max_over_ranks(s0.elapsed_time(s1) / args.steps)
-    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a0.record()
-    for _ in range(args.steps):
-        for Wb_r, Ob_r, idx_r, sc_r in segs:
-            ouo.apply_update(Wb_r, Ob_r, LR, idx=idx_r, scale=sc_r)
-    a1.record()
-    barrier()
-    app_ms = max_over_ranks(a0.elapsed_time(a1) / args.steps)
+    part_ms = {}
+    for j, nm in enumerate(part_names):
+        part_ms[nm] = max_over_ranks(
+            sum(pev[k][j].elapsed_time(pev[k][j + 1]) for k in range(args.steps)) / args.steps)
+    mom_ms, sel_ms = part_ms["momentum"], part_ms["selection"]
+    gram_ms, app_ms = part_ms["gram_ns"], part_ms["update"]
     # --- per-launch timing of every tensor-core GEMM launch of full steps
     # (CUDA events recorded by the library around each launch, on its stream)
     ouo.timing_enable(True)
@@ -490,22 +490,28 @@ def run_ours(args):
     mom_gbs = mom_bytes / (mom_ms * 1e-3) / 1e9 if mom_ms > 0 else 0.0
     mom_launches = -(-len(own) // 128)
     # The dominant kernel of the step by device time: a GEMM kind or the
-    # momentum kernel.  Kernels timed inside full steps use the sustained
-    # dense-bf16 peak (tf32 at the nominal tf32/bf16 ratio).
+    # momentum kernel.  The step lasts tens of milliseconds, far shorter than
+    # the seconds-long loop the sustained peak was taken in, so the burst
+    # dense-bf16 peak is the denominator (tf32 at the nominal tf32/bf16
+    # ratio); the sustained one is reported beside it.
     p_bf_s = peaks["bf16_tflops_sustained"]
     traffic = _traffic()
     dom_name, dom = max(kinds.items(), key=lambda kv: kv[1]["ms_per_step"]) if kinds else (None, None)
     if dom is not None and dom["ms_per_step"] > mom_ms:
         is_tf32 = "tf32" in dom_name
-        peak = p_bf_s * (TF32_RATIO if is_tf32 else 1.0)
+        ratio = TF32_RATIO if is_tf32 else 1.0
+        peak = p_bf * ratio
+        peak_s = p_bf_s * ratio
         roofline = {"bound": "tensor", "kernel": f"umma_gemm_kernel ({dom_name})",
                     "achieved": dom["tflops"], "peak": round(peak, 1), "unit": "TFLOP/s",
                     "frac": round(dom["tflops"] / peak, 4),
                     "traffic": traffic.get("umma_gemm_kernel tf32 symmetric")
                     if "tf32 symmetric" in dom_name else None,
-                    "peak_note": f"{'tf32 = ' if is_tf32 else ''}measured sustained bf16 "
-                                 f"{p_bf_s}{' x 0.489 nominal tf32/bf16' if is_tf32 else ''} "
-                                 f"({peaks['source']})",
+                    "peak_note": f"{'tf32 = ' if is_tf32 else ''}burst bf16 {p_bf}"
+                                 f"{' x 0.489 nominal tf32/bf16' if is_tf32 else ''} "
+                                 f"({peaks['source']}); tf32 is not measured on its own",
+                    "peak_sustained": round(peak_s, 1),
+                    "frac_of_sustained": round(dom["tflops"] / peak_s, 4),
                     "units": "algorithmic flops per launch (symmetric outputs: upper "
                              "triangle) / CUDA-event launch time"}
     else:
@@ -536,6 +542,9 @@ def run_ours(args):
                          "ms_per_step": round(mom_ms, 4),
                          "launches_per_step": mom_launches},
         "matrices_per_s": round(len(mn) / (ms * 1e-3), 1),
+        "parts": {nm: {"ms_per_step": round(v, 4)} for nm, v in part_ms.items()},
+        "parts_note": "device time of each call, events between the calls inside the same "
+                      "full steps (they add up to the step)",
         "kernels": kinds,
         "elementwise": _elementwise(sel_ms, app_ms, own, all_kn, lay, peaks),
         "gpu_launches": int(launches),
@@ -548,6 +557,13 @@ def run_ours(args):
         result["e2e"] = e2e_measure(args, chunks, step_chunk, exchange_and_update, idx, scale,
                                     barrier, max_over_ranks)
 
+    if world == 1 and not args.no_dion:
+        del ws
+        torch.cuda.empty_cache()
+        result["dion"] = dion_measure(args, Ms, Gs, Ws, mn, dev, peaks)
+    if world == 1 and not args.no_sweep:
+        torch.cuda.empty_cache()
+        result["sweep"] = sweep_points(args, dev, peaks)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(args)
     if rank == 0:
@@ -555,6 +571,144 @@ def run_ours(args):
     if dist is not None:
         dist.barrier()
         dist.destroy_process_group()
+
+
+DION_BYTES_PER_ELEM = 30  # B = M + G (10), two reads of B (8), M update (8), bf16 W (4)
+
+
+def _timed(fn, steps, warmup):
+    import torch
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / steps
+
+
+def _dion_line(ms, elems, rank, peaks):
+    """ms, and the step's fraction of its HBM and tf32 bounds."""
+    gbs = DION_BYTES_PER_ELEM * elems / (ms * 1e-3) / 1e9
+    tfl = 8.0 * elems * rank / (ms * 1e-3) / 1e12
+    p_tf = peaks["bf16_tflops"] * TF32_RATIO
+    return {"ms": round(ms, 4), "hbm_gbs": round(gbs, 1),
+            "frac_hbm": round(gbs / peaks["hbm_gbs"], 4),
+            "tflops_tf32": round(tfl, 1), "frac_tf32": round(tfl / p_tf, 4),
+            "hbm_bound_ms": round(DION_BYTES_PER_ELEM * elems / (peaks["hbm_gbs"] * 1e9) * 1e3, 4)}
+
+
+def dion_measure(args, Ms, Gs, Ws, mn, dev, peaks):
+    """Dion / Orth-Dion steps at rank 256: one 4096 x 4096 matrix (bf16
+    low-rank(64) + noise gradient), and the whole 8B-shaped parameter set in
+    one grouped call (the step's buffers, one block per shape; right factors
+    one block per weight shape).  Device time per step after warm-up;
+    fractions against the algorithmic HBM bytes (30 per element) and the
+    tf32 flops (8 m n r)."""
+    import torch
+    import orthonormalized_update_optimizers_b200 as ouo
+    from orthonormalized_update_optimizers_b200 import synth
+    K, W = max(3, min(args.steps, 5)), max(3, args.warmup)
+    r = 256
+    out = {"rank": r, "bytes_per_element": DION_BYTES_PER_ELEM,
+           "flops": "8 m n r (tf32)", "peak_note": f"HBM {peaks['hbm_gbs']} GB/s, tf32 = "
+           f"bf16 {peaks['bf16_tflops']} x 0.489 ({peaks['source']})"}
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    m = n = 4096
+    G = synth.lowrank_plus_noise(m, n, 64, 0.02, synth.seed_for(2, 0), torch.bfloat16, dev)
+    q0 = torch.linalg.qr(synth.dion_q0(n, r, 1).to(dev))[0].T.contiguous()
+    single = {}
+    for mode, label in (("colnorm", "dion"), ("qr", "orth_dion")):
+        M = torch.zeros(m, n, dtype=torch.float32, device=dev)
+        Wt = synth.gaussian((m, n), 5, 0.02, torch.bfloat16, dev)
+        Qt = q0.clone()
+        p = ouo.dion_params(rank=r, norm_mode=mode)
+        wsd = torch.empty(ouo.dion_workspace_bytes([M], p), dtype=torch.uint8, device=dev)
+        ms = _timed(lambda: ouo.dion_lowrank_step([M], [G], [Qt], [Wt], p, workspace=wsd,
+                                                  status=status), K, W)
+        single[label] = _dion_line(ms, m * n, r, peaks)
+        del M, Wt, Qt, wsd
+    out["matrix_4096x4096"] = single
+    # the 8B-shaped set in one call; right factors in one block per shape
+    qshapes = {}
+    for i, (mm, nn) in enumerate(mn):
+        qshapes.setdefault((mm, nn), []).append(i)
+    Qs = [None] * len(mn)
+    for (mm, nn), members in qshapes.items():
+        blk = torch.empty((len(members), r, nn), dtype=torch.float32, device=dev)
+        for k, i in enumerate(members):
+            blk[k].copy_(q0[:, :nn] if nn == n else
+                         torch.linalg.qr(synth.dion_q0(nn, r, 1).to(dev))[0].T)
+            Qs[i] = blk[k]
+    Mb, Gb, Wb, Qb = ouo.MatBatch(Ms), ouo.MatBatch(Gs), ouo.MatBatch(Ws), ouo.MatBatch(Qs)
+    elems = sum(a * b for a, b in mn)
+    scales = [math.sqrt(max(1.0, a / b)) for a, b in mn]
+    grouped = {}
+    for mode, label in (("colnorm", "dion"), ("qr", "orth_dion")):
+        p = ouo.dion_params(rank=r, norm_mode=mode)
+        need = ouo.dion_workspace_bytes(Mb, p)
+        free = torch.cuda.mem_get_info()[0]
+        if need > free - (2 << 30):
+            grouped[label] = {"skipped": f"workspace {need} B, {free} B free"}
+            continue
+        wsd = torch.empty(need, dtype=torch.uint8, device=dev)
+        ms = _timed(lambda: ouo.dion_lowrank_step(Mb, Gb, Qb, Wb, p, scale=scales,
+                                                  workspace=wsd, status=status),
+                    max(2, K - 2), 2)
+        grouped[label] = dict(_dion_line(ms, elems, r, peaks), workspace_bytes=need)
+        del wsd
+        torch.cuda.empty_cache()
+    out["llama8b_set_grouped"] = dict(grouped, matrices=len(mn), params=elems)
+    out["device_status"] = int(status.item())
+    return out
+
+
+def sweep_points(args, dev, peaks):
+    """Standard vs Gram Newton-Schulz at the crossover shapes of the sweep
+    (m = 1024, n / m = 1, 4, 16; bf16 low-rank(64) + noise, normalization
+    on, 5 iterations, one batch of about 2^29 elements per shape).  The
+    full sweep is ``--sweep``."""
+    import torch
+    import orthonormalized_update_optimizers_b200 as ouo
+    from orthonormalized_update_optimizers_b200 import synth
+    K, W = max(3, min(args.steps, 5)), max(3, args.warmup)
+    p_bf = peaks["bf16_tflops"]
+    p_tf = p_bf * TF32_RATIO
+    rows = []
+    for m, n in ((1024, 1024), (1024, 4096), (1024, 16384)):
+        nb = max(1, min(64, (1 << 29) // (m * n)))
+        X = ouo.batch_empty([(m, n)] * nb, torch.bfloat16, dev)
+        for i in range(nb):
+            X[i].copy_(synth.lowrank_plus_noise(m, n, 64, 0.02, synth.seed_for(4, 100 * i + n // m),
+                                                torch.bfloat16, dev))
+        O = [torch.empty_like(x) for x in X]
+        Xb, Ob = ouo.MatBatch(X), ouo.MatBatch(O)
+        row = {"m": m, "n": n, "batch": nb}
+        kk = min(m, n)
+        std_tf = ITERS * kk * kk * (kk + 1)
+        std_bf = std_ns_flops(m, n) - std_tf
+        gbf, gtf = gram_ns_flops(m, n)
+        for name, fn_name, bf, tf in (("standard", "ns_orthogonalize", std_bf, std_tf),
+                                      ("gram", "gram_ns_orthogonalize", gbf, gtf)):
+            params = ouo.ns_params()
+            wsb = getattr(ouo, fn_name.replace("orthogonalize", "workspace_bytes"))(Xb, params)
+            wsn = torch.empty(wsb, dtype=torch.uint8, device=dev)
+            fn = getattr(ouo, fn_name)
+            ms = _timed(lambda: fn(Xb, Ob, params, workspace=wsn), K, W)
+            tfl = nb * (bf + tf) / (ms * 1e-3) / 1e12
+            pk = (bf + tf) / (bf / p_bf + tf / p_tf)
+            row[name] = {"ms": round(ms, 4), "tflops": round(tfl, 1),
+                         "frac_of_peak": round(tfl / pk, 4)}
+            del wsn
+        row["gram_speedup"] = round(row["standard"]["ms"] / row["gram"]["ms"], 3)
+        rows.append(row)
+        del X, O, Xb, Ob
+        torch.cuda.empty_cache()
+    return {"points": rows, "peak_note": f"bf16 {p_bf} ({peaks['source']}, burst), tf32 = "
+            "bf16 x 0.489, weighted by each point's bf16 / tf32 flops"}
 
 
 def _elementwise(sel_ms, app_ms, own, all_kn, lay, peaks):

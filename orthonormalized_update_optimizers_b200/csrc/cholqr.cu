@@ -57,10 +57,15 @@ __device__ __forceinline__ int find_job(const int64_t* start, int njob, int64_t 
 }
 
 // 256 threads: thread (ty, tx) owns rows ty*4 .. ty*4+3 and columns
-// tx*4 .. tx*4+3 of the 64 x 64 tile (ti, tj), ti <= tj.
+// tx*4 .. tx*4+3 of the 64 x 64 tile (ti, tj), ti <= tj.  The K range of the
+// split is walked in steps of 32 columns with a register-staged double
+// buffer: the next step's operands are loaded from global memory while the
+// current step's are multiplied out of shared memory.  Loads: thread t
+// reads row t % 64, columns 4 (t / 64) .. +3 and 16 + 4 (t / 64) .. +3, and
+// stores them transposed (As[k][row]) without bank conflicts.
 __global__ void __launch_bounds__(256) gram_kernel(const __grid_constant__ GramBatch gb) {
-  __shared__ __align__(16) float As[kGK][kGT + 4];
-  __shared__ __align__(16) float Bs[kGK][kGT + 4];
+  __shared__ __align__(16) float As[2][kGK][kGT + 4];
+  __shared__ __align__(16) float Bs[2][kGK][kGT + 4];
   const int j = find_job(gb.start, gb.njob, blockIdx.x);
   const CholQrJob& jb = gb.job[j];
   const int tiles = (jb.r + kGT - 1) / kGT;
@@ -81,15 +86,14 @@ __global__ void __launch_bounds__(256) gram_kernel(const __grid_constant__ GramB
   for (int u = 0; u < 4; ++u)
 #pragma unroll
     for (int v = 0; v < 4; ++v) acc[u][v] = 0.f;
-  // loader: 64 rows x 32 columns per operand = 512 float4, two per thread
-  const int lr = tid >> 3, lc = (tid & 7) * 4;
+  const int lr = tid & 63, lc = (tid >> 6) * 4;
+  const int ra = ti * kGT + lr, rb = tj * kGT + lr;
   const bool vec = (ld & 3) == 0 && ((uintptr_t)X & 15) == 0;
-  for (int64_t k0 = l0; k0 < l1; k0 += kGK) {
+  float4 na[2], nb2[2];  // the next step's operands
+  auto fetch = [&](int64_t k0) {
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-      const int rr = lr + 32 * h;
-      const int ra = ti * kGT + rr, rb = tj * kGT + rr;
-      const int64_t kc = k0 + lc;
+      const int64_t kc = k0 + lc + 16 * h;
       float va[4] = {0.f, 0.f, 0.f, 0.f}, vb[4] = {0.f, 0.f, 0.f, 0.f};
       if (vec && kc + 3 < l1) {
         if (ra < jb.r) {
@@ -109,17 +113,33 @@ __global__ void __launch_bounds__(256) gram_kernel(const __grid_constant__ GramB
           }
         }
       }
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        As[lc + e][rr] = va[e];
-        Bs[lc + e][rr] = vb[e];
-      }
+      na[h] = make_float4(va[0], va[1], va[2], va[3]);
+      nb2[h] = make_float4(vb[0], vb[1], vb[2], vb[3]);
     }
-    __syncthreads();
+  };
+  auto stash = [&](int buf) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int c = lc + 16 * h;
+      As[buf][c][lr] = na[h].x; As[buf][c + 1][lr] = na[h].y;
+      As[buf][c + 2][lr] = na[h].z; As[buf][c + 3][lr] = na[h].w;
+      Bs[buf][c][lr] = nb2[h].x; Bs[buf][c + 1][lr] = nb2[h].y;
+      Bs[buf][c + 2][lr] = nb2[h].z; Bs[buf][c + 3][lr] = nb2[h].w;
+    }
+  };
+  if (l0 < l1) {
+    fetch(l0);
+    stash(0);
+  }
+  __syncthreads();
+  int buf = 0;
+  for (int64_t k0 = l0; k0 < l1; k0 += kGK) {
+    const bool more = k0 + kGK < l1;
+    if (more) fetch(k0 + kGK);
 #pragma unroll 8
     for (int kk = 0; kk < kGK; ++kk) {
-      const float4 a4 = *reinterpret_cast<const float4*>(&As[kk][ty * 4]);
-      const float4 b4 = *reinterpret_cast<const float4*>(&Bs[kk][tx * 4]);
+      const float4 a4 = *reinterpret_cast<const float4*>(&As[buf][kk][ty * 4]);
+      const float4 b4 = *reinterpret_cast<const float4*>(&Bs[buf][kk][tx * 4]);
       const float av[4] = {a4.x, a4.y, a4.z, a4.w};
       const float bv[4] = {b4.x, b4.y, b4.z, b4.w};
 #pragma unroll
@@ -127,17 +147,23 @@ __global__ void __launch_bounds__(256) gram_kernel(const __grid_constant__ GramB
 #pragma unroll
         for (int v = 0; v < 4; ++v) acc[u][v] = fmaf(av[u], bv[v], acc[u][v]);
     }
+    if (more) stash(buf ^ 1);
     __syncthreads();
+    buf ^= 1;
   }
   float* part = jb.gpart + (size_t)split * jb.r * jb.r;
 #pragma unroll
   for (int u = 0; u < 4; ++u) {
     const int i = ti * kGT + ty * 4 + u;
     if (i >= jb.r) continue;
+    const int c = tj * kGT + tx * 4;
+    if (c + 3 < jb.r && (jb.r & 3) == 0) {
+      *reinterpret_cast<float4*>(part + (size_t)i * jb.r + c) =
+          make_float4(acc[u][0], acc[u][1], acc[u][2], acc[u][3]);
+    } else {
 #pragma unroll
-    for (int v = 0; v < 4; ++v) {
-      const int c = tj * kGT + tx * 4 + v;
-      if (c < jb.r) part[(size_t)i * jb.r + c] = acc[u][v];
+      for (int v = 0; v < 4; ++v)
+        if (c + v < jb.r) part[(size_t)i * jb.r + c + v] = acc[u][v];
     }
   }
 }
@@ -172,7 +198,7 @@ __global__ void __launch_bounds__(256) sum_kernel(const __grid_constant__ SumBat
 }
 
 // ------------------------------------------------------------------- chol
-constexpr int kCT = 512;             // threads of the Cholesky CTA
+constexpr int kCT = 384;             // threads of the Cholesky CTA
 constexpr int kCW = kCT / 32;        // warps
 constexpr int kP = 36;               // tile pitch (16-byte rows, conflict-free row reads)
 constexpr int kTF = kB * kP;         // floats per tile
@@ -203,47 +229,42 @@ __device__ __forceinline__ int tri_row_of(int t) {
 }
 
 // One warp: factor the 32 x 32 block T (pitch kP, lower triangle used),
-// T = L L^T, leaving L in T, and write D = L^-1 (lower triangular, zeros
-// above) to Dt (pitch kP) and to global memory at g (row pitch ldg).
-// Returns false on a non-positive or non-finite pivot (the same in every
-// lane).
-__device__ __noinline__ bool chol_inv32(float* T, float* Dt, float* g, int64_t ldg) {
+// T = L L^T, and write D = L^-1 (lower triangular, zeros above) to Dt
+// (pitch kP) and to global memory at g (row pitch ldg).  Returns false on a
+// non-positive or non-finite pivot (the same in every lane).
+//   factor:  row `lane` of the block in registers, right-looking; the
+//            pivot and the column below it are broadcast by shuffles.
+//   inverse: column `lane` of L^-1 by a column sweep, x[k] = acc[k] /
+//            L[k][k], then every later row r loses L[r][k] x[k]; L[r][k] is
+//            a shuffle from lane r (independent of x, so the shuffles of a
+//            step overlap).
+__device__ __noinline__ bool chol_inv32(const float* T, float* Dt, float* g, int64_t ldg) {
   const unsigned full = 0xffffffffu;
   const int lane = threadIdx.x & 31;
   bool ok = true;
   float my_inv = 0.f;  // 1 / L[lane][lane]
-  {
-    // row `lane` of the block in registers, right-looking: the pivot and
-    // the column below it are broadcast by shuffles
-    float l[kB];
+  float l[kB];
 #pragma unroll
-    for (int k = 0; k < kB; k += 4) {
-      const float4 v = *reinterpret_cast<const float4*>(T + lane * kP + k);
-      l[k] = v.x; l[k + 1] = v.y; l[k + 2] = v.z; l[k + 3] = v.w;
-    }
-#pragma unroll
-    for (int k = 0; k < kB; ++k) {
-      const float piv = __shfl_sync(full, l[k], k);
-      // a bad pivot is the same in every lane; the sweep runs on (its
-      // values are discarded) so that the loop stays fully unrolled
-      if (!(piv > 0.f) || !(piv < INFINITY)) ok = false;
-      const float rs = rsqrtf(piv);
-      if (lane == k) { l[k] = piv * rs; my_inv = rs; }
-      else if (lane > k) l[k] *= rs;
-      const float lk = l[k];
-#pragma unroll
-      for (int j = k + 1; j < kB; ++j) {
-        const float ljk = __shfl_sync(full, lk, j);
-        if (lane >= j) l[j] = fmaf(-lk, ljk, l[j]);
-      }
-    }
-#pragma unroll
-    for (int k = 0; k < kB; k += 4)
-      *reinterpret_cast<float4*>(T + lane * kP + k) = make_float4(l[k], l[k + 1], l[k + 2], l[k + 3]);
+  for (int k = 0; k < kB; k += 4) {
+    const float4 v = *reinterpret_cast<const float4*>(T + lane * kP + k);
+    l[k] = v.x; l[k + 1] = v.y; l[k + 2] = v.z; l[k + 3] = v.w;
   }
-  __syncwarp();
-  // column `lane` of L^-1 by a column sweep: x[k] = acc[k] / L[k][k], then
-  // every later row r loses L[r][k] x[k] (L read back from T, broadcast)
+#pragma unroll
+  for (int k = 0; k < kB; ++k) {
+    const float piv = __shfl_sync(full, l[k], k);
+    // a bad pivot is the same in every lane; the sweep runs on (its values
+    // are discarded) so that the loop stays fully unrolled
+    if (!(piv > 0.f) || !(piv < INFINITY)) ok = false;
+    const float rs = rsqrtf(piv);
+    if (lane == k) { l[k] = piv * rs; my_inv = rs; }
+    else if (lane > k) l[k] *= rs;
+    const float lk = l[k];
+#pragma unroll
+    for (int j = k + 1; j < kB; ++j) {
+      const float ljk = __shfl_sync(full, lk, j);
+      if (lane >= j) l[j] = fmaf(-lk, ljk, l[j]);
+    }
+  }
   float acc[kB];
 #pragma unroll
   for (int r = 0; r < kB; ++r) acc[r] = r == lane ? 1.f : 0.f;
@@ -252,7 +273,8 @@ __device__ __noinline__ bool chol_inv32(float* T, float* Dt, float* g, int64_t l
     const float xk = acc[k] * __shfl_sync(full, my_inv, k);
     acc[k] = xk;
 #pragma unroll
-    for (int r = k + 1; r < kB; ++r) acc[r] = fmaf(-T[r * kP + k], xk, acc[r]);
+    for (int r = k + 1; r < kB; ++r)
+      acc[r] = fmaf(-__shfl_sync(full, l[k], r), xk, acc[r]);
   }
   // acc[r] = D[r][lane]; lanes write column `lane`
 #pragma unroll
@@ -263,41 +285,95 @@ __device__ __noinline__ bool chol_inv32(float* T, float* Dt, float* g, int64_t l
   return ok;
 }
 
-// acc[c] += sum_k A[lane][k] B[c0 + c][k], c < 8 (tiles of pitch kP)
-__device__ __forceinline__ void rowdot8(const float* A, const float* B, int c0, float (&acc)[8]) {
-  const int lane = threadIdx.x & 31;
-  float row[kB];
+// One warp: the 32 x 32 block product A B^T of two 32 x 32 tiles (pitch
+// kP) on the tensor cores, with fp32 accuracy from three tf32 products per
+// term (x = hi + lo, hi the tf32 rounding of x: A B^T ~ lo_A hi_B + hi_A lo_B
+// + hi_A hi_B, the tiny lo_A lo_B dropped).  c[mi][ni] is the m16n8 tile
+// (mi, ni) in the mma.sync accumulator layout: rows 16 mi + g (+8), columns
+// 8 ni + 2 t (+1), g = lane / 4, t = lane % 4.
+__device__ __forceinline__ void split_tf32(float x, uint32_t& hi, uint32_t& lo) {
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(hi) : "f"(x));
+  lo = __float_as_uint(x - __uint_as_float(hi));
+}
+
+__device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4],
+                                         const uint32_t (&b)[2]) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 "
+      "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+__device__ __forceinline__ void block_abt(const float* A, const float* B, float (&c)[2][4][4]) {
+  const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
 #pragma unroll
-  for (int k = 0; k < kB; k += 4) {
-    const float4 v = *reinterpret_cast<const float4*>(A + lane * kP + k);
-    row[k] = v.x; row[k + 1] = v.y; row[k + 2] = v.z; row[k + 3] = v.w;
-  }
+  for (int mi = 0; mi < 2; ++mi)
 #pragma unroll
-  for (int c = 0; c < 8; ++c) {
-    const float* bp = B + (c0 + c) * kP;
+    for (int ni = 0; ni < 4; ++ni)
 #pragma unroll
-    for (int k = 0; k < kB; k += 4) {
-      const float4 v = *reinterpret_cast<const float4*>(bp + k);
-      acc[c] = fmaf(row[k], v.x, acc[c]);
-      acc[c] = fmaf(row[k + 1], v.y, acc[c]);
-      acc[c] = fmaf(row[k + 2], v.z, acc[c]);
-      acc[c] = fmaf(row[k + 3], v.w, acc[c]);
+      for (int e = 0; e < 4; ++e) c[mi][ni][e] = 0.f;
+#pragma unroll
+  for (int ks = 0; ks < 4; ++ks) {
+    const int k0 = 8 * ks + t;
+    uint32_t ah[2][4], al[2][4], bh[4][2], bl[4][2];
+#pragma unroll
+    for (int mi = 0; mi < 2; ++mi) {
+      const float* a0 = A + (16 * mi + g) * kP + k0;
+      split_tf32(a0[0], ah[mi][0], al[mi][0]);
+      split_tf32(a0[8 * kP], ah[mi][1], al[mi][1]);
+      split_tf32(a0[4], ah[mi][2], al[mi][2]);
+      split_tf32(a0[8 * kP + 4], ah[mi][3], al[mi][3]);
     }
+#pragma unroll
+    for (int ni = 0; ni < 4; ++ni) {
+      const float* b0 = B + (8 * ni + g) * kP + k0;
+      split_tf32(b0[0], bh[ni][0], bl[ni][0]);
+      split_tf32(b0[4], bh[ni][1], bl[ni][1]);
+    }
+#pragma unroll
+    for (int mi = 0; mi < 2; ++mi)
+#pragma unroll
+      for (int ni = 0; ni < 4; ++ni) {
+        mma_tf32(c[mi][ni], al[mi], bh[ni]);
+        mma_tf32(c[mi][ni], ah[mi], bl[ni]);
+        mma_tf32(c[mi][ni], ah[mi], bh[ni]);
+      }
   }
 }
 
-// tile(bi, bj) -= A B^T over columns c0 .. c0 + 7 (row = lane)
-__device__ __forceinline__ void sub_rowdot8(float* Tt, const float* A, const float* B, int c0) {
-  const int lane = threadIdx.x & 31;
-  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-  rowdot8(A, B, c0, acc);
-  float* sp = Tt + lane * kP + c0;
-  const float4 s0 = *reinterpret_cast<const float4*>(sp);
-  const float4 s1 = *reinterpret_cast<const float4*>(sp + 4);
-  *reinterpret_cast<float4*>(sp) =
-      make_float4(s0.x - acc[0], s0.y - acc[1], s0.z - acc[2], s0.w - acc[3]);
-  *reinterpret_cast<float4*>(sp + 4) =
-      make_float4(s1.x - acc[4], s1.y - acc[5], s1.z - acc[6], s1.w - acc[7]);
+// T -= A B^T (32 x 32 tiles, pitch kP), one warp.
+__device__ __forceinline__ void block_sub_abt(float* T, const float* A, const float* B) {
+  const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+  float c[2][4][4];
+  block_abt(A, B, c);
+#pragma unroll
+  for (int mi = 0; mi < 2; ++mi)
+#pragma unroll
+    for (int ni = 0; ni < 4; ++ni)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        float2* p = reinterpret_cast<float2*>(T + (16 * mi + g + 8 * h) * kP + 8 * ni + 2 * t);
+        float2 v = *p;
+        v.x -= c[mi][ni][2 * h];
+        v.y -= c[mi][ni][2 * h + 1];
+        *p = v;
+      }
+}
+
+// T = A B^T (32 x 32 tiles, pitch kP), one warp.
+__device__ __forceinline__ void block_set_abt(float* T, const float* A, const float* B) {
+  const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+  float c[2][4][4];
+  block_abt(A, B, c);
+#pragma unroll
+  for (int mi = 0; mi < 2; ++mi)
+#pragma unroll
+    for (int ni = 0; ni < 4; ++ni)
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+        *reinterpret_cast<float2*>(T + (16 * mi + g + 8 * h) * kP + 8 * ni + 2 * t) =
+            make_float2(c[mi][ni][2 * h], c[mi][ni][2 * h + 1]);
 }
 
 __global__ void __launch_bounds__(kCT, 1) chol_kernel(const __grid_constant__ CholBatch cb) {
@@ -367,37 +443,29 @@ __global__ void __launch_bounds__(kCT, 1) chol_kernel(const __grid_constant__ Ch
     for (int p = 0; p < nb && !failed; ++p) {
       const int m = nb - 1 - p;
       if (m == 0) break;
-      // panel: pan[b] = S(p+1+b, p) D_p^T
-      for (int it = warp; it < 4 * m; it += kCW) {
-        const int bb = it >> 2, c0 = (it & 3) * 8;
-        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        rowdot8(tile(p + 1 + bb, p), Dt, c0, acc);
-        float* dst = pan + (size_t)bb * kTF + lane * kP + c0;
-        *reinterpret_cast<float4*>(dst) = make_float4(acc[0], acc[1], acc[2], acc[3]);
-        *reinterpret_cast<float4*>(dst + 4) = make_float4(acc[4], acc[5], acc[6], acc[7]);
-      }
+      // panel: pan[b] = S(p+1+b, p) D_p^T, one warp per block
+      for (int bb = warp; bb < m; bb += kCW)
+        block_set_abt(pan + (size_t)bb * kTF, tile(p + 1 + bb, p), Dt);
       __syncthreads();
       // the panel blocks L_{p+1+b, p} to global memory
       for (int e = threadIdx.x; e < m * kB * kB; e += kCT) {
         const int bb = e >> 10, w = e & 1023, ii = w >> 5, jj = w & 31;
         gblk(p + 1 + bb, p)[(size_t)ii * R + jj] = pan[(size_t)bb * kTF + ii * kP + jj];
       }
-      // look-ahead: the next diagonal block first (warps 0-3), then warp 0
-      // factors it while the other warps finish the trailing update
-      if (warp < 4) {
-        sub_rowdot8(tile(p + 1, p + 1), pan, pan, warp * 8);
-        asm volatile("bar.sync 1, 128;" ::: "memory");
-        if (warp == 0 && !chol_inv32(tile(p + 1, p + 1), Dt, gblk(p + 1, p + 1), R) && lane == 0)
-          s_bad = 1;
-      }
-      if (warp > 0) {
+      // look-ahead: warp 0 updates the next diagonal block and factors it
+      // while the other warps finish the trailing update
+      if (warp == 0) {
+        block_sub_abt(tile(p + 1, p + 1), pan, pan);
+        __syncwarp();
+        if (!chol_inv32(tile(p + 1, p + 1), Dt, gblk(p + 1, p + 1), R) && lane == 0) s_bad = 1;
+      } else {
         // trailing: S(p+1+bi, p+1+bj) -= pan[bi] pan[bj]^T, bj <= bi, except (0, 0)
         const int tasks = m * (m + 1) / 2 - 1;
-        for (int it = warp - 1; it < 4 * tasks; it += kCW - 1) {
-          const int t = (it >> 2) + 1, c0 = (it & 3) * 8;
-          const int bi = tri_row_of(t), bj = t - bi * (bi + 1) / 2;
-          sub_rowdot8(tile(p + 1 + bi, p + 1 + bj), pan + (size_t)bi * kTF,
-                      pan + (size_t)bj * kTF, c0);
+        for (int it = warp - 1; it < tasks; it += kCW - 1) {
+          const int tt = it + 1;
+          const int bi = tri_row_of(tt), bj = tt - bi * (bi + 1) / 2;
+          block_sub_abt(tile(p + 1 + bi, p + 1 + bj), pan + (size_t)bi * kTF,
+                        pan + (size_t)bj * kTF);
         }
       }
       __syncthreads();
@@ -417,7 +485,7 @@ __global__ void __launch_bounds__(kCT, 1) chol_kernel(const __grid_constant__ Ch
 }
 
 // ------------------------------------------------------------------- trsm
-constexpr int kSP = 36;  // strip pitch (32 columns + pad, 16-byte rows)
+constexpr int kSP = 36;  // row pitch of the strip and block buffers (floats)
 
 struct TrsmBatch {
   CholQrJob job[kChunk];
@@ -425,14 +493,61 @@ struct TrsmBatch {
   int njob;
 };
 
+__device__ __forceinline__ void cp_async16(float* dst, const float* src) {
+  const unsigned d = (unsigned)__cvta_generic_to_shared(dst);
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(d), "l"(src) : "memory");
+}
+
+// Y = L^-1 X on one 32-column strip, block row by block row:
+//   Y_i = D_i X_i;  X_j -= L_ji Y_i for the blocks j > i below.
+// The products run in rounds: a round is D_i X_i, or up to four updates
+// L_ji Y_i, one per group of 64 threads (a thread owns rows ro, ro+8,
+// ro+16, ro+24 and four columns of a 32 x 32 block).  The blocks of L a
+// round needs are copied into shared memory (cp.async) one round ahead.
 __global__ void __launch_bounds__(256) trsm_kernel(const __grid_constant__ TrsmBatch tb) {
-  extern __shared__ __align__(16) float xs[];  // R x kSP
-  const int j = find_job(tb.start, tb.njob, blockIdx.x);
-  const CholQrJob& jb = tb.job[j];
-  const int64_t c0g = (blockIdx.x - tb.start[j]) * kB;  // first column of the strip
+  extern __shared__ __align__(16) float sm[];
+  const int job = find_job(tb.start, tb.njob, blockIdx.x);
+  const CholQrJob& jb = tb.job[job];
+  const int64_t c0g = (blockIdx.x - tb.start[job]) * kB;  // first column of the strip
   const int r = jb.r, nb = (r + kB - 1) / kB, R = nb * kB;
-  const int tid = threadIdx.x;
+  float* xs = sm;                                   // R x kSP
+  float* blk = sm + (size_t)R * kSP;                // [2][4][32][kSP]
+  const int tid = threadIdx.x, grp = tid >> 6, t64 = tid & 63;
+  const int ro = t64 >> 3, cc = 4 * (t64 & 7);
   const int64_t ncol = jb.L - c0g < kB ? jb.L - c0g : kB;
+  const float* Lb = jb.Lb;
+  const float* Dd = jb.Dd ? jb.Dd : jb.Lb;
+  // rounds: for every block row i, one D round, then ceil((nb-1-i)/4)
+  // update rounds
+  auto round_of = [&](int t, int* i, int* j0) {
+    for (int b = 0; b < nb; ++b) {
+      const int nu = (nb - 1 - b + 3) / 4;
+      if (t == 0) { *i = b; *j0 = -1; return; }
+      if (t <= nu) { *i = b; *j0 = b + 1 + 4 * (t - 1); return; }
+      t -= 1 + nu;
+    }
+    *i = -1;
+    *j0 = -1;
+  };
+  int nrounds = 0;
+  for (int b = 0; b < nb; ++b) nrounds += 1 + (nb - 1 - b + 3) / 4;
+  auto prefetch = [&](int t) {
+    if (t >= nrounds) return;
+    int i, j0;
+    round_of(t, &i, &j0);
+    float* dst = blk + (size_t)(t & 1) * 4 * kB * kSP;
+    // thread: row tid >> 3, 16-byte column group tid & 7 of each block
+    const int br = tid >> 3, bc = 4 * (tid & 7);
+    if (j0 < 0) {
+      cp_async16(dst + br * kSP + bc, Dd + (size_t)(i * kB + br) * R + i * kB + bc);
+    } else {
+      for (int g = 0; g < 4 && j0 + g < nb; ++g)
+        cp_async16(dst + (size_t)g * kB * kSP + br * kSP + bc,
+                   Lb + (size_t)((j0 + g) * kB + br) * R + i * kB + bc);
+    }
+  };
+  prefetch(0);
+  asm volatile("cp.async.commit_group;\n" ::: "memory");
   // strip in: xs[i][c] = X[i][c0g + c], zero past r or L
   {
     const bool vec = (jb.ldx & 3) == 0 && ((uintptr_t)jb.X & 15) == 0 && ncol == kB;
@@ -444,64 +559,73 @@ __global__ void __launch_bounds__(256) trsm_kernel(const __grid_constant__ TrsmB
         if (vec) {
           v = *reinterpret_cast<const float4*>(src);
         } else {
-          float t[4] = {0.f, 0.f, 0.f, 0.f};
+          float t4[4] = {0.f, 0.f, 0.f, 0.f};
           for (int q = 0; q < 4; ++q)
-            if (c + q < ncol) t[q] = src[q];
-          v = make_float4(t[0], t[1], t[2], t[3]);
+            if (c + q < ncol) t4[q] = src[q];
+          v = make_float4(t4[0], t4[1], t4[2], t4[3]);
         }
       }
       *reinterpret_cast<float4*>(xs + i * kSP + c) = v;
     }
   }
-  __syncthreads();
-  const int row = tid >> 3, cc = (tid & 7) * 4;
-  const float* Lb = jb.Lb;
-  for (int i = 0; i < nb; ++i) {
-    // Y_i = D_i X_i
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    {
-      const float* Drow = (jb.Dd ? jb.Dd : Lb) + (size_t)(i * kB + row) * R + i * kB;
+  for (int t = 0; t < nrounds; ++t) {
+    prefetch(t + 1);
+    asm volatile("cp.async.commit_group;\n" ::: "memory");
+    asm volatile("cp.async.wait_group 1;\n" ::: "memory");
+    __syncthreads();
+    int i, j0;
+    round_of(t, &i, &j0);
+    const float* bb = blk + (size_t)(t & 1) * 4 * kB * kSP + (size_t)grp * kB * kSP;
+    const bool active = j0 < 0 ? grp == 0 : j0 + grp < nb;
+    float acc[4][4];
 #pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+      for (int v = 0; v < 4; ++v) acc[u][v] = 0.f;
+    if (active) {
+      const float* yi = xs + (size_t)(i * kB) * kSP + cc;
+#pragma unroll 2
       for (int k = 0; k < kB; k += 4) {
-        const float4 d = __ldg(reinterpret_cast<const float4*>(Drow + k));
-        const float dv[4] = {d.x, d.y, d.z, d.w};
+        float a[4][4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float4 w = *reinterpret_cast<const float4*>(bb + (ro + 8 * u) * kSP + k);
+          a[u][0] = w.x; a[u][1] = w.y; a[u][2] = w.z; a[u][3] = w.w;
+        }
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          const float4 x = *reinterpret_cast<const float4*>(xs + (i * kB + k + q) * kSP + cc);
-          acc.x = fmaf(dv[q], x.x, acc.x);
-          acc.y = fmaf(dv[q], x.y, acc.y);
-          acc.z = fmaf(dv[q], x.z, acc.z);
-          acc.w = fmaf(dv[q], x.w, acc.w);
+          const float4 y = *reinterpret_cast<const float4*>(yi + (k + q) * kSP);
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            acc[u][0] = fmaf(a[u][q], y.x, acc[u][0]);
+            acc[u][1] = fmaf(a[u][q], y.y, acc[u][1]);
+            acc[u][2] = fmaf(a[u][q], y.z, acc[u][2]);
+            acc[u][3] = fmaf(a[u][q], y.w, acc[u][3]);
+          }
         }
       }
     }
-    __syncthreads();
-    *reinterpret_cast<float4*>(xs + (i * kB + row) * kSP + cc) = acc;
-    __syncthreads();
-    // X_b -= L_bi Y_i for the blocks below
-    for (int bb = i + 1; bb < nb; ++bb) {
-      const float* Lrow = Lb + (size_t)(bb * kB + row) * R + i * kB;
-      float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (j0 < 0) {
+      __syncthreads();  // every read of X_i is done before Y_i replaces it
+      if (active) {
 #pragma unroll
-      for (int k = 0; k < kB; k += 4) {
-        const float4 l = __ldg(reinterpret_cast<const float4*>(Lrow + k));
-        const float lv[4] = {l.x, l.y, l.z, l.w};
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float4 y = *reinterpret_cast<const float4*>(xs + (i * kB + k + q) * kSP + cc);
-          s.x = fmaf(lv[q], y.x, s.x);
-          s.y = fmaf(lv[q], y.y, s.y);
-          s.z = fmaf(lv[q], y.z, s.z);
-          s.w = fmaf(lv[q], y.w, s.w);
-        }
+        for (int u = 0; u < 4; ++u)
+          *reinterpret_cast<float4*>(xs + (size_t)(i * kB + ro + 8 * u) * kSP + cc) =
+              make_float4(acc[u][0], acc[u][1], acc[u][2], acc[u][3]);
       }
-      float* xp = xs + (bb * kB + row) * kSP + cc;
-      float4 x = *reinterpret_cast<float4*>(xp);
-      x.x -= s.x; x.y -= s.y; x.z -= s.z; x.w -= s.w;
-      *reinterpret_cast<float4*>(xp) = x;
+    } else if (active) {
+      const int jb2 = j0 + grp;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        float* xp = xs + (size_t)(jb2 * kB + ro + 8 * u) * kSP + cc;
+        float4 x = *reinterpret_cast<float4*>(xp);
+        x.x -= acc[u][0]; x.y -= acc[u][1]; x.z -= acc[u][2]; x.w -= acc[u][3];
+        *reinterpret_cast<float4*>(xp) = x;
+      }
     }
     __syncthreads();
   }
+  asm volatile("cp.async.wait_group 0;\n" ::: "memory");
   // out: Y (and its copy) row-major, Y^T (L x r)
   for (int e = tid; e < r * 8; e += 256) {
     const int i = e >> 3, c = (e & 7) * 4;
@@ -521,11 +645,17 @@ __global__ void __launch_bounds__(256) trsm_kernel(const __grid_constant__ TrsmB
       }
     }
   }
-  if (jb.Yt) {
+  if (jb.Yt || jb.Ytb) {
     for (int c = 0; c < ncol; ++c)
-      for (int i = tid; i < r; i += 256) jb.Yt[(c0g + c) * jb.ldyt + i] = xs[i * kSP + c];
+      for (int i = tid; i < r; i += 256) {
+        const float v = xs[i * kSP + c];
+        if (jb.Yt) jb.Yt[(c0g + c) * jb.ldyt + i] = v;
+        if (jb.Ytb) jb.Ytb[(c0g + c) * jb.ldytb + i] = f32_to_bf16(v);
+      }
   }
 }
+
+size_t trsm_smem_bytes(int R) { return ((size_t)R * kSP + 2 * 4 * kB * kSP) * sizeof(float); }
 
 // ------------------------------------------------------------------- rows
 struct RowsBatch {
@@ -543,7 +673,9 @@ __global__ void __launch_bounds__(256) rows_kernel(const __grid_constant__ RowsB
   const int64_t n = jb.n;
   const float* src = jb.part + c * jb.ldp;
   const bool vec = (jb.ldp & 3) == 0 && (jb.sp & 3) == 0 && ((uintptr_t)jb.part & 15) == 0 &&
-                   (!jb.out || ((jb.ldo & 3) == 0 && ((uintptr_t)jb.out & 15) == 0));
+                   (!jb.out || ((jb.ldo & 3) == 0 && ((uintptr_t)jb.out & 15) == 0)) &&
+                   (!jb.outb || ((jb.ldob & 3) == 0 && ((uintptr_t)jb.outb & 7) == 0));
+  uint16_t* brow = jb.outb ? jb.outb + c * jb.ldob : nullptr;
   const bool want_norm = jb.sigma || jb.qn;
   double ss = 0.0;
   float* orow = jb.out ? jb.out + c * jb.ldo : nullptr;
@@ -555,6 +687,12 @@ __global__ void __launch_bounds__(256) rows_kernel(const __grid_constant__ RowsB
         v.x += w.x; v.y += w.y; v.z += w.z; v.w += w.w;
       }
       if (orow) *reinterpret_cast<float4*>(orow + e) = v;
+      if (brow) {
+        uint2 u;
+        u.x = pack_bf16x2(v.x, v.y);
+        u.y = pack_bf16x2(v.z, v.w);
+        *reinterpret_cast<uint2*>(brow + e) = u;
+      }
       if (want_norm)
         ss += (double)v.x * v.x + (double)v.y * v.y + (double)v.z * v.z + (double)v.w * v.w;
     }
@@ -563,6 +701,7 @@ __global__ void __launch_bounds__(256) rows_kernel(const __grid_constant__ RowsB
     float v = src[e];
     for (int q = 1; q < jb.ks; ++q) v += src[q * jb.sp + e];
     if (orow) orow[e] = v;
+    if (brow) brow[e] = f32_to_bf16(v);
     if (want_norm) ss += (double)v * v;
   }
   if (!want_norm) return;
@@ -608,7 +747,7 @@ int set_smem_attr(const void* fn, size_t bytes) {
   if (!done[dev][slot]) {
     OUO_CHECK_CUDA(cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         slot == 0 ? (int)chol_smem_bytes(kMaxNb)
-                                                  : (int)(1024 * kSP * sizeof(float))));
+                                                  : (int)trsm_smem_bytes(1024)));
     done[dev][slot] = 1;
   }
   (void)bytes;
@@ -700,7 +839,7 @@ int cholqr_apply(const std::vector<CholQrJob>& jobs, cudaStream_t s) {
       tb.job[i] = jb;
       tb.start[i + 1] = tb.start[i] + ceil_div(jb.L, kB);
     }
-    trsm_kernel<<<(unsigned)tb.start[cn], 256, (size_t)Rmax * kSP * sizeof(float), s>>>(tb);
+    trsm_kernel<<<(unsigned)tb.start[cn], 256, trsm_smem_bytes(Rmax), s>>>(tb);
     OUO_CHECK_LAUNCH();
   }
   return OUO_OK;

@@ -105,6 +105,7 @@ struct DGroup {
   std::vector<int> members;  // indices into the caller's batch
   int ks1 = 1, ks2 = 1;      // K splits of Pt = Qt B^T and Rt = Pt B
   Buf Pt, P, Rt, Qn;         // r x m, m x r, r x n, r x n per member
+  Buf Pb, Rtb;               // bf16 copies of P and Rt (the M update's operands)
   Buf kp1, kp2;              // split-K partials (the same memory)
   Buf S, Lb, Ld;             // r x r summed Gram; R x R factors
   float* gpart = nullptr;    // Gram partials, gstride floats per member
@@ -153,6 +154,8 @@ std::vector<DGroup> plan(const ouo_mat* M, int nmat, const int* ranks, Arena& ar
     g.P = ar.take(OUO_F32, nb, m, r);
     g.Rt = ar.take(OUO_F32, nb, r, n);
     g.Qn = ar.take(OUO_F32, nb, r, n);
+    g.Pb = ar.take(OUO_BF16, nb, m, r);
+    g.Rtb = ar.take(OUO_BF16, nb, r, n);
     {
       // the two partial sets are used one after the other: one region
       const int64_t f1 = g.ks1 > 1 ? g.ks1 * (int64_t)r * pitch4(m) : 0;
@@ -354,6 +357,8 @@ int stage_orth_p(const std::vector<DGroup>& gs, int* status, cudaStream_t s, int
         if (pass == 1) {
           j.Yt = fp(g.P, i);
           j.ldyt = g.P.ld;
+          j.Ytb = reinterpret_cast<uint16_t*>(view(g.Pb, i, 1).p);
+          j.ldytb = g.Pb.ld;
         }
         jobs.push_back(j);
         own.push_back(&g);
@@ -439,7 +444,6 @@ int stage_qnew(const std::vector<DGroup>& gs, Rtp rt, const ouo_mat* Q_state,
     for (int64_t i = 0; i < (int64_t)g.members.size(); ++i) {
       const int bi = g.members[i];
       const bool colnorm = p->norm_mode == OUO_DION_COLNORM;
-      if (!colnorm && !sigma) continue;
       int64_t ld = 0;
       RowsJob rj;
       rj.part = rt(g, i, &ld);
@@ -448,6 +452,8 @@ int stage_qnew(const std::vector<DGroup>& gs, Rtp rt, const ouo_mat* Q_state,
       rj.ks = 1;
       rj.rows = g.r;
       rj.n = g.n;
+      rj.outb = reinterpret_cast<uint16_t*>(view(g.Rtb, i, 1).p);  // the M update's operand
+      rj.ldob = g.Rtb.ld;
       rj.sigma = sigma ? sigma + sig_off[bi] : nullptr;
       if (colnorm) {
         rj.qn = fp(g.Qn, i);
@@ -488,63 +494,79 @@ int stage_qnew(const std::vector<DGroup>& gs, Rtp rt, const ouo_mat* Q_state,
 }
 
 // Stage: M <- beta B - (beta - mu) P Rt and W <- (1 - lr wd) W - lr s P Qn,
-// in place in the caller's matrices.
-template <class Rtp>
-int stage_update(const std::vector<DGroup>& gs, Rtp rt, const ouo_mat* M, const ouo_mat* W,
+// in place in the caller's matrices.  Both are rank-r updates whose C0 is
+// the output itself: the GEMM's TMA epilogue loads each C0 box, adds the
+// product and stores it back (bulk copies only).  With K = r the operand
+// tiles weigh as much as the output they update, so both run on CTA-pair
+// tiles (half the operand bytes per output), and the M update takes bf16
+// operands (P and Rt rounded once: its product is scaled by beta - mu and
+// lands in the momentum buffer, so the rounding is far inside the
+// tolerance).  The weight update keeps tf32 operands, so that Orth-Dion's
+// update stays a partial isometry to fp32-level accuracy.  Outputs are
+// described to the TMA as one evenly strided batch per group when the
+// caller's matrices are laid out that way, else one matrix per segment.
+int stage_update(const std::vector<DGroup>& gs, const ouo_mat* M, const ouo_mat* W,
                  int w_dtype, const ouo_dion_params* p, const float* scale, int* status,
                  cudaStream_t s) {
   std::vector<GemmDesc> dm, dw;
   for (const DGroup& g : gs) {
     const int64_t nb = (int64_t)g.members.size();
     GemmDesc d;
-    d.M = g.m; d.N = g.n; d.K = g.r; d.nb = nb;
-    d.A = g.P;
+    d.M = g.m; d.N = g.n; d.K = g.r;
     d.b_mn = 1;
     d.has_c0 = true;
     d.c0_from_out = true;
     d.per_desc_tiles = true;
-    // M update: B = Rt (the workspace batch, or the caller-summed rows)
-    int64_t ld0 = 0;
-    float* r0 = rt(g, 0, &ld0);
-    const bool rt_ws = r0 == fp(g.Rt, 0);
-    for (int64_t i = 0; i < (rt_ws ? 1 : nb); ++i) {
-      GemmDesc x = d;
-      x.alpha = -(p->beta - p->mu);
-      x.beta = p->beta;
-      x.direct_dtype = OUO_F32;
-      if (rt_ws) {
-        x.B = g.Rt;
-        for (int64_t k = 0; k < nb; ++k)
-          x.direct.push_back(MatRef{M[g.members[k]].ptr, M[g.members[k]].ld});
-      } else {
-        int64_t ld = 0;
-        Buf b;
-        b.p = reinterpret_cast<char*>(rt(g, i, &ld));
-        b.dtype = OUO_F32;
-        b.rows = g.r;
-        b.cols = g.n;
-        b.ld = ld;
-        b.stride = g.r * ld;
-        b.nb = 1;
-        x.B = b;
-        x.nb = 1;
-        x.A = view(g.P, i, 1);
-        x.direct.push_back(MatRef{M[g.members[i]].ptr, M[g.members[i]].ld});
-      }
+    d.pair_mn = true;
+    // M update (fp32 output)
+    GemmDesc x = d;
+    x.alpha = -(p->beta - p->mu);
+    x.beta = p->beta;
+    x.has_f32 = true;
+    Buf mo;
+    if (caller_uniform(M, g.members, OUO_F32, &mo)) {
+      x.nb = nb;
+      x.A = g.Pb;
+      x.B = g.Rtb;
+      x.out_f32 = mo;
       dm.push_back(x);
+    } else {
+      for (int64_t k = 0; k < nb; ++k) {
+        GemmDesc xi = x;
+        xi.nb = 1;
+        xi.A = view(g.Pb, k, 1);
+        xi.B = view(g.Rtb, k, 1);
+        xi.out_f32 = caller_buf(M[g.members[k]], OUO_F32);
+        dm.push_back(xi);
+      }
     }
-    // W update: B = Qn, per-matrix alpha = -lr * scale
+    // W update (caller dtype), per-matrix alpha = -lr * scale
     GemmDesc y = d;
-    y.B = g.Qn;
     y.beta = 1.0f - p->lr * p->wd;
     y.alpha = -p->lr;
-    y.direct_dtype = w_dtype;
-    for (int64_t k = 0; k < nb; ++k) {
-      const int bi = g.members[k];
-      y.direct.push_back(MatRef{W[bi].ptr, W[bi].ld});
-      y.direct_alpha.push_back(-p->lr * (scale ? scale[bi] : 1.0f));
+    y.has_f32 = w_dtype == OUO_F32;
+    y.has_bf16 = w_dtype == OUO_BF16;
+    Buf wo;
+    auto alpha_of = [&](int64_t k) { return -p->lr * (scale ? scale[g.members[k]] : 1.0f); };
+    if (caller_uniform(W, g.members, w_dtype, &wo)) {
+      y.nb = nb;
+      y.A = g.P;
+      y.B = g.Qn;
+      (w_dtype == OUO_F32 ? y.out_f32 : y.out_bf16) = wo;
+      for (int64_t k = 0; k < nb; ++k) y.direct_alpha.push_back(alpha_of(k));
+      dw.push_back(y);
+    } else {
+      for (int64_t k = 0; k < nb; ++k) {
+        GemmDesc yi = y;
+        yi.nb = 1;
+        yi.A = view(g.P, k, 1);
+        yi.B = view(g.Qn, k, 1);
+        (w_dtype == OUO_F32 ? yi.out_f32 : yi.out_bf16) =
+            caller_buf(W[g.members[k]], w_dtype);
+        yi.direct_alpha.push_back(alpha_of(k));
+        dw.push_back(yi);
+      }
     }
-    dw.push_back(y);
   }
   OUO_TRY(gemm_umma_grouped(dm, s, status));
   return gemm_umma_grouped(dw, s, status);
@@ -653,7 +675,7 @@ extern "C" int dion_lowrank_step_stats(const ouo_mat* M, const ouo_mat* G,
   OUO_TRY(stage_orth_p(gs, dev_status, s, 0, 2));
   OUO_TRY(stage_rproject(gs, M, rt_ws, dev_status, s));
   OUO_TRY(stage_qnew(gs, rt_ws, Q_state, p, sigma, sig_off, dev_status, s));
-  return stage_update(gs, rt_ws, M, W, w_dtype, p, scale, dev_status, s);
+  return stage_update(gs, M, W, w_dtype, p, scale, dev_status, s);
 }
 
 extern "C" int dion_effective_rank(const float* sigma, const int* ranks, int nmat,
@@ -805,6 +827,8 @@ int shard_orth(const ouo_mat* M, const ouo_mat* Q_state, int nmat,
       if (second) {
         j.Yt = fp(g.P, i);
         j.ldyt = g.P.ld;
+        j.Ytb = reinterpret_cast<uint16_t*>(view(g.Pb, i, 1).p);
+        j.ldytb = g.Pb.ld;
       }
       // the solve runs over the local rows
       jobs.push_back(j);
@@ -920,5 +944,5 @@ extern "C" int dion_shard_update(const ouo_mat* M, const ouo_mat* Q_state,
   };
   std::vector<int64_t> no_sig((size_t)nmat, 0);
   OUO_TRY(stage_qnew(gs, rt_red, Q_state, p, nullptr, no_sig, dev_status, s));
-  return stage_update(gs, rt_red, M, W, w_dtype, p, scale, dev_status, s);
+  return stage_update(gs, M, W, w_dtype, p, scale, dev_status, s);
 }

@@ -129,7 +129,7 @@ struct Cfg {
   // per epilogue warp: a 32 x 32 fp32 staging buffer
   static constexpr uint32_t kEpiBytes = kEpiWarps * kStg * 32 * 32 * 4;
   static constexpr size_t kSmem =
-      1024 + (size_t)kStages * kStageBytes + 256 + kEpiBytes;
+      1024 + (size_t)kStages * kStageBytes + 512 + kEpiBytes;
 };
 
 // First column tile of row tile i (tiles of TR rows) that reaches the
@@ -309,6 +309,10 @@ umma_gemm_kernel(const __grid_constant__ UmmaArgs a) {
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
   // per stage: bit 0 = A tile MN-major (transposed block), bit 1 = B tile
   volatile uint32_t* stage_fmt = reinterpret_cast<volatile uint32_t*>(tmem_holder + 2);
+  // in-place TMA epilogue: one barrier per staging buffer of every epilogue
+  // warp, completed by the TMA load of a C0 box into that buffer
+  uint64_t* c0bar = reinterpret_cast<uint64_t*>(
+      (reinterpret_cast<uintptr_t>(stage_fmt + C::kStages) + 7) & ~(uintptr_t)7);
   // per-warp 4 KB staging buffers, 1024-byte aligned (the TMA swizzle
   // patterns are computed from absolute shared-memory address bits)
   float* epi_smem = reinterpret_cast<float*>(smem + C::kStages * C::kStageBytes);
@@ -329,6 +333,7 @@ umma_gemm_kernel(const __grid_constant__ UmmaArgs a) {
       ptx::mbar_init(&tempty[s], kEpiWarps * CG);  // one arrival per epilogue warp
     }
     ptx::mbar_init(drain, 1);
+    for (int i = 0; i < kEpiWarps * C::kStg; ++i) ptx::mbar_init(&c0bar[i], 1);
     *abort_flag = 0;
     ptx::fence_barrier_init();
     for (int g = 0; g < a.nseg; ++g) {
@@ -520,6 +525,7 @@ umma_gemm_kernel(const __grid_constant__ UmmaArgs a) {
     // accumulator-free barrier of the pair's even CTA (cluster address)
     const uint32_t tempty_lead = CG == 2 ? ptx::mapa(ptx::smem_u32(tempty), 0) : 0u;
     uint32_t nstores = 0;  // bulk stores issued by this warp
+    uint32_t nc0[2] = {0u, 0u};  // C0 box loads waited for, per staging buffer
     for (int64_t tile = tile0; tile < a.total_tiles;
          tile += tile_step, ++local) {
       int64_t b, ti, tj, ks;
@@ -561,6 +567,32 @@ umma_gemm_kernel(const __grid_constant__ UmmaArgs a) {
         return make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xffff0000u),
                            __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xffff0000u));
       };
+      // The C0 rows this warp will read for the next tile (and, on the
+      // first tile, for this one) are prefetched into L2 before the
+      // accumulator is waited for: lane l prefetches row l of the warp's
+      // 32 x BN/2 region, so that a whole tile of C0 loads is in flight per
+      // SM and the register loads below mostly hit L2.
+      if (pf) {
+        auto l2_region = [&](int64_t tl) {
+          int64_t b2, ti2, tj2, ks2;
+          const int g2 = decode_tile(a, BN, TR, tl, &b2, &ti2, &tj2, &ks2);
+          const Segment& s2 = a.seg[g2];
+          const int64_t row = ti2 * TR + rank * kTileM + q * 32 + lane;
+          const int64_t col = tj2 * BN + pf_half * (BN / 2);
+          if (row >= s2.M || col >= s2.N) return;
+          const TileOut o2 = tile_out(a, s2, b2);
+          const int64_t ld2 = a.c0_out ? (a.has_f32 ? o2.ldf : o2.ldh) : s2.ldc0;
+          const char* base = a.c0_out
+              ? (a.has_f32 ? reinterpret_cast<const char*>(o2.f) : reinterpret_cast<const char*>(o2.h))
+              : reinterpret_cast<const char*>(s2.C0) + (s2.b0 + b2) * s2.sc0 * pf_es;
+          const char* p0 = base + (row * ld2 + col) * pf_es;
+          const int64_t ncols = s2.N - col < BN / 2 ? s2.N - col : BN / 2;
+          for (int64_t off = 0; off < ncols * pf_es; off += 128)
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(p0 + off));
+        };
+        if (local == 0) l2_region(tile);
+        if (tile + tile_step < a.total_tiles) l2_region(tile + tile_step);
+      }
       // one chunk of C0 in flight: slot `it` is refilled with the next
       // chunk's value as soon as the current chunk has taken it
       float4 pfe[8];
@@ -580,6 +612,110 @@ umma_gemm_kernel(const __grid_constant__ UmmaArgs a) {
         break;
       }
       ptx::tc_fence_after();
+      if (a.tma_out && a.c0_out) {
+        // In-place update through the TMA (non-symmetric outputs): the C0
+        // box of a 32 x 32 chunk is loaded by the TMA into a staging buffer
+        // (the layout of the store box), the finished chunk alpha acc +
+        // beta C0 replaces it there, and a bulk tensor store writes it back.
+        // With two staging buffers (CTA pairs) the next chunk's C0 is
+        // loaded while this one is finished.  Loads and stores are async
+        // bulk copies: no per-thread global access in the epilogue.
+        const int64_t row_base = ti * TR + rank * kTileM + q * 32;
+        const uint32_t half = (uint32_t)((warp - 2) >> 2);
+        float* const stg_base = epi_smem + (warp - 2) * (C::kStg * 32 * 32);
+        uint64_t* const bars = c0bar + (warp - 2) * C::kStg;
+        const int32_t z = (int32_t)(sg.b0 + b);
+        const bool obf = a.has_bf16 != 0;
+        const uint32_t box_bytes = obf ? 2048u : 4096u;
+        const float alpha = a.has_dalpha ? a.dalpha[sg.dbase + b] : a.alpha;
+        // chunks of this warp inside the output
+        int nch = 0;
+        for (int c = 0; c < kCh; ++c)
+          if (row_base < sg.M && tj * BN + half * (BN / 2) + c * 32 < sg.N) nch = c + 1;
+        auto c0_load = [&](int c) {
+          const uint32_t sb = nstores & (C::kStg - 1);  // buffer of this chunk's store
+          float* dst = stg_base + sb * (32 * 32);
+          if (lane == 0) {
+            // the buffer's previous store has finished reading it
+            if (C::kStg == 2) ptx::bulk_wait_read1();
+            else ptx::bulk_wait_read0();
+            ptx::mbar_arrive_expect_tx(&bars[sb], box_bytes);
+            ptx::tma_load_3d(dst, &sg.tmC, &bars[sb],
+                             (int32_t)(tj * BN + half * (BN / 2) + c * 32), (int32_t)row_base, z);
+          }
+        };
+        bool ok_c0 = true;
+        if (nch > 0) c0_load(0);
+#pragma unroll 1
+        for (int c = 0; c < nch; ++c) {
+          const uint32_t sb = nstores & (C::kStg - 1);
+          const uint32_t ph = (nc0[sb] & 1u);
+          float* stg = stg_base + sb * (32 * 32);
+          uint16_t* stg16 = reinterpret_cast<uint16_t*>(stg);
+          const int64_t gj0 = tj * BN + half * (BN / 2) + c * 32;
+          float v[32];
+          ptx::tmem_ld32(tmem_base + ((q * 32u) << 16) + buf * BN + half * (BN / 2) + c * 32, v);
+          // C0 of this chunk has landed
+          int okw = 1;
+          if (lane == 0) okw = ptx::mbar_wait(&bars[sb], ph, abort_flag) ? 1 : 0;
+          okw = __shfl_sync(0xffffffffu, okw, 0);
+          ++nc0[sb];
+          if (!okw) {
+            if (lane == 0) {
+              *abort_flag = 1;
+              report_status(a.status, OUO_STATUS_TIMEOUT);
+            }
+            ok_c0 = false;
+            break;
+          }
+          if (!obf) {
+#pragma unroll
+            for (int j = 0; j < 32; j += 4) {
+              float4* pp = reinterpret_cast<float4*>(stg + stg_idx(lane, j));
+              const float4 e = *pp;
+              *pp = make_float4(alpha * v[j] + a.beta * e.x, alpha * v[j + 1] + a.beta * e.y,
+                                alpha * v[j + 2] + a.beta * e.z, alpha * v[j + 3] + a.beta * e.w);
+            }
+          } else {
+#pragma unroll
+            for (int qq = 0; qq < 4; ++qq) {
+              uint4* pp = reinterpret_cast<uint4*>(stg16 + stg16_idx(lane, 8 * qq));
+              const uint4 e = *pp;
+              const uint32_t ew[4] = {e.x, e.y, e.z, e.w};
+              uint32_t ow[4];
+#pragma unroll
+              for (int h = 0; h < 4; ++h) {
+                const float lo = __uint_as_float(ew[h] << 16), hi = __uint_as_float(ew[h] & 0xffff0000u);
+                ow[h] = pack_bf16x2(alpha * v[8 * qq + 2 * h] + a.beta * lo,
+                                    alpha * v[8 * qq + 2 * h + 1] + a.beta * hi);
+              }
+              *pp = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+            }
+          }
+          ptx::fence_async_shared();
+          __syncwarp();
+          if (lane == 0) {
+            ptx::tma_store_3d(&sg.tmC, stg, (int32_t)gj0, (int32_t)row_base, z);
+            ptx::bulk_commit();
+          }
+          ++nstores;
+          if (c + 1 < nch) c0_load(c + 1);
+        }
+        if (!ok_c0) {
+          // loads still in flight land before the CTA's shared memory goes
+          if (lane == 0)
+            for (int i = 0; i < C::kStg; ++i)
+              ptx::mbar_wait_timed(&bars[i], nc0[i] & 1u, 100000000ull);
+          break;
+        }
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          if (CG == 2) ptx::mbar_arrive_cluster(tempty_lead + buf * 8u);
+          else ptx::mbar_arrive(&tempty[buf]);
+        }
+        continue;
+      }
       if (a.tma_out) {
         // Finished values (row = lane) are staged in the TMA's swizzled box
         // layout (fp32: 128-byte rows, 16-byte chunks XOR row % 8; bf16:
@@ -774,11 +910,15 @@ umma_gemm_kernel(const __grid_constant__ UmmaArgs a) {
           }
           __syncwarp();
         }
+        // The accumulator is free once this warp's TMEM reads have
+        // completed (tcgen05.wait::ld): the arrival is relaxed, so that it
+        // does not wait for the warp's global stores to be performed (a
+        // release arrival would, once per tile).
         ptx::tc_fence_before();
         __syncwarp();
         if (lane == 0) {
-          if (CG == 2) ptx::mbar_arrive_cluster(tempty_lead + buf * 8u);
-          else ptx::mbar_arrive(&tempty[buf]);
+          if (CG == 2) ptx::mbar_arrive_cluster_relaxed(tempty_lead + buf * 8u);
+          else ptx::mbar_arrive_relaxed(&tempty[buf]);
         }
         continue;
       }
@@ -910,9 +1050,9 @@ umma_gemm_kernel(const __grid_constant__ UmmaArgs a) {
       }
       ptx::tc_fence_before();
       __syncwarp();
-      if (lane == 0) {
-        if (CG == 2) ptx::mbar_arrive_cluster(tempty_lead + buf * 8u);
-        else ptx::mbar_arrive(&tempty[buf]);
+      if (lane == 0) {  // relaxed, as in the non-symmetric direct path
+        if (CG == 2) ptx::mbar_arrive_cluster_relaxed(tempty_lead + buf * 8u);
+        else ptx::mbar_arrive_relaxed(&tempty[buf]);
       }
     }
     // bulk stores complete before the CTA (and its shared memory) goes away
@@ -1120,6 +1260,11 @@ int launch(const std::vector<GemmDesc>& gs, cudaStream_t stream, int* status) {
   }
   // single workspace output: TMA-store epilogue
   a.tma_out = (g0.direct.empty() && (g0.has_f32 != g0.has_bf16)) ? 1 : 0;
+  // in-place update through the TMA: C0 is the output matrix itself
+  if (a.tma_out && g0.c0_from_out) {
+    a.c0_out = 1;
+    a.has_c0 = 1;
+  }
   a.a_sym = g0.a_sym; a.b_sym = g0.b_sym;
   a.c0_upper = g0.c0_upper; a.sym_half = g0.sym_half;
   if ((a.a_sym || a.b_sym) && !(CG == 2 && FMT == 2 && !B_MN))
@@ -1226,18 +1371,19 @@ int launch(const std::vector<GemmDesc>& gs, cudaStream_t stream, int* status) {
     }
     int64_t b0 = 0;
     while (b0 < g.nb) {
-      if (a.nseg == kMaxSeg || (proto.direct && ndirect == kChunk)) OUO_TRY(flush());
+      const bool tabled = proto.direct || a.has_dalpha;  // per-matrix table slots
+      if (a.nseg == kMaxSeg || (tabled && ndirect == kChunk)) OUO_TRY(flush());
       int64_t nb = g.nb - b0;
-      if (proto.direct && nb > kChunk - ndirect) nb = kChunk - ndirect;
+      if (tabled && nb > kChunk - ndirect) nb = kChunk - ndirect;
       Segment& sg = a.seg[a.nseg++];
       sg = proto;
       sg.b0 = b0;
       sg.nb = nb;
-      if (proto.direct) {
+      if (tabled) {
         sg.dbase = ndirect;
         for (int64_t i = 0; i < nb; ++i) {
-          a.dptr[ndirect + i] = g.direct[b0 + i].p;
-          a.dld[ndirect + i] = g.direct[b0 + i].ld;
+          a.dptr[ndirect + i] = proto.direct ? g.direct[b0 + i].p : nullptr;
+          a.dld[ndirect + i] = proto.direct ? g.direct[b0 + i].ld : 0;
           a.dalpha[ndirect + i] = a.has_dalpha ? g.direct_alpha[b0 + i] : g.alpha;
         }
         ndirect += (int)nb;
@@ -1344,8 +1490,9 @@ int gemm_umma_grouped(const std::vector<GemmDesc>& gs, cudaStream_t stream,
       return set_error(OUO_ERR_INVALID_ARG, "symmetric GEMM needs M == N, K-major B");
     if (!g.direct.empty() && (int64_t)g.direct.size() != g.nb)
       return set_error(OUO_ERR_INVALID_ARG, "direct output table size mismatch");
-    if (g.c0_from_out && (g.direct.empty() || g.tri))
-      return set_error(OUO_ERR_INVALID_ARG, "in-place C0 needs direct, non-symmetric outputs");
+    if (g.c0_from_out && (g.tri || (g.direct.empty() && g.has_f32 == g.has_bf16)))
+      return set_error(OUO_ERR_INVALID_ARG,
+                       "in-place C0 needs non-symmetric direct outputs or one output matrix");
     if (!g.direct_alpha.empty() && (int64_t)g.direct_alpha.size() != g.nb)
       return set_error(OUO_ERR_INVALID_ARG, "direct alpha table size mismatch");
     if (g.ksplit > 1 && (g.tri || !g.direct.empty() || g.has_c0 || g.has_f32 == g.has_bf16))
@@ -1359,15 +1506,15 @@ int gemm_umma_grouped(const std::vector<GemmDesc>& gs, cudaStream_t stream,
   // K-major B.  OUO_CTA_PAIR=0 selects single-CTA 128 x BN tiles throughout;
   // OUO_CTA_PAIR=2 also puts MN-major B (Q X) on pairs.
   const int pair_mode = cta_pair_mode();
-  auto pair_of = [&](bool w, bool t) {
-    return w && t && pair_mode > 0 && (!g0.b_mn || pair_mode == 2);
+  auto pair_of = [&](bool w, bool t, bool mn_ok) {
+    return w && t && pair_mode > 0 && (!g0.b_mn || pair_mode == 2 || mn_ok);
   };
-  if (!per_desc) return launch_kind(gs, pair_of(wide, tall), wide, stream, status);
+  if (!per_desc) return launch_kind(gs, pair_of(wide, tall, false), wide, stream, status);
   // every descriptor keeps its own tile shape: one launch per shape in use
   for (int kind = 0; kind < 3; ++kind) {
     std::vector<GemmDesc> part;
     for (const GemmDesc& g : gs) {
-      const bool w = g.N > 128, pr = pair_of(w, g.M > 128);
+      const bool w = g.N > 128, pr = pair_of(w, g.M > 128, g.pair_mn);
       const int k = pr ? 2 : (w ? 1 : 0);
       if (k == kind) part.push_back(g);
     }

@@ -109,6 +109,10 @@ struct GemmDesc {
   // descriptor alone instead of for the whole grouped launch, so that a
   // matrix is computed the same way whatever it is batched with.
   bool per_desc_tiles = false;
+  // With per_desc_tiles: CTA-pair tiles also for an MN-major B (by default
+  // only K-major B takes them).  Pairs halve the operand bytes per output
+  // element, which is what a short-K GEMM with an in-place C0 runs out of.
+  bool pair_mn = false;
 };
 
 // Number of K ranges a split-K GEMM of depth K over `dtype` operands
@@ -176,6 +180,8 @@ struct CholQrJob {
   int64_t ldy2 = 0;
   float* Yt = nullptr;       // optional transpose of Y, L x r
   int64_t ldyt = 0;
+  uint16_t* Ytb = nullptr;   // optional bf16 copy of the transpose, L x r
+  int64_t ldytb = 0;
 };
 // Gram splits for an r x L block (columns per split = ceil(L / splits),
 // rounded up to 32).
@@ -201,6 +207,8 @@ struct RowsJob {
   int64_t rows = 0, n = 0;
   float* out = nullptr;      // optional summed rows
   int64_t ldo = 0;
+  uint16_t* outb = nullptr;  // optional bf16 copy of the summed rows
+  int64_t ldob = 0;
   float* sigma = nullptr;    // optional row norms
   float* qn = nullptr;       // optional normalized rows
   int64_t ldq = 0;
