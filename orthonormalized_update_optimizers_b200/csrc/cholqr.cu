@@ -13,8 +13,8 @@
 //   gram     part[s] = X[:, chunk s] X[:, chunk s]^T: 64 x 64 tiles on or
 //            above the diagonal (upper storage), fp32 FMA, the L columns cut
 //            into chunks so that a single matrix fills the GPU.
-//   sum      S = sum_s part[s] in float64, fixed order, rounded to fp32
-//            (upper storage: entries (i, j) with j >= i are valid).
+//   sum      S = sum_s part[s] in float64, fixed order, rounded to fp32,
+//            written in full (symmetric).
 //   chol     one CTA per matrix (r <= 256): the lower 32 x 32 blocks of S in
 //            shared memory, right-looking blocked Cholesky with one block of
 //            look-ahead; writes the strictly lower blocks L_ij and the
@@ -168,8 +168,8 @@ __global__ void __launch_bounds__(256) gram_kernel(const __grid_constant__ GramB
   }
 }
 
-// S[i][j] = sum_s part[s][i][j] (float64, s ascending) for the entries of
-// tiles on or above the diagonal.
+// S[i][j] = sum_s part[s][i][j] (float64, s ascending), the partials read at
+// (j, i) for tiles below the diagonal: S in full symmetric storage.
 struct SumBatch {
   const float* part[kChunk];
   float* S[kChunk];
@@ -186,12 +186,11 @@ __global__ void __launch_bounds__(256) sum_kernel(const __grid_constant__ SumBat
     const int64_t w = e - sb.start[j];
     const int r = sb.r[j];
     const int i = (int)(w / r), c = (int)(w - (w / r) * r);
-    if (c / kGT < i / kGT) {  // tile below the diagonal: no partials there
-      sb.S[j][w] = 0.f;
-      continue;
-    }
+    // entries of tiles below the diagonal are the mirror of (c, i), which
+    // the Gram kernel computed: S is written in full (symmetric)
+    const int64_t src = (c / kGT < i / kGT) ? (int64_t)c * r + i : w;
     double s = 0.0;
-    const float* p = sb.part[j] + w;
+    const float* p = sb.part[j] + src;
     for (int q = 0; q < sb.splits[j]; ++q) s += (double)p[(size_t)q * r * r];
     sb.S[j][w] = (float)s;
   }
@@ -215,8 +214,9 @@ struct CholBatch {
 
 size_t chol_smem_bytes(int nb) {
   const int ntri = nb * (nb + 1) / 2;
-  // lower tiles, D of the current block, the panel (nb - 1 tiles)
-  return (size_t)(ntri + 1 + (nb > 1 ? nb - 1 : 0)) * kTF * sizeof(float);
+  // lower tiles, D of the current block, the panel (nb - 1 tiles), the
+  // factoring warp's column scratch
+  return (size_t)(ntri + 2 + (nb > 1 ? nb - 1 : 0)) * kTF * sizeof(float);
 }
 
 __device__ __forceinline__ int tri_index(int bi, int bj) { return bi * (bi + 1) / 2 + bj; }
@@ -230,19 +230,22 @@ __device__ __forceinline__ int tri_row_of(int t) {
 
 // One warp: factor the 32 x 32 block T (pitch kP, lower triangle used),
 // T = L L^T, and write D = L^-1 (lower triangular, zeros above) to Dt
-// (pitch kP) and to global memory at g (row pitch ldg).  Returns false on a
-// non-positive or non-finite pivot (the same in every lane).
-//   factor:  row `lane` of the block in registers, right-looking; the
-//            pivot and the column below it are broadcast by shuffles.
+// (pitch kP) and to global memory at g (row pitch ldg).  `col` is 32 x kP
+// floats of shared scratch of this warp.  Returns false on a non-positive
+// or non-finite pivot (the same in every lane).
+//   factor:  row `lane` of the block in registers, right-looking.  Every
+//            lane takes the pivot by one shuffle and forms 1/sqrt itself;
+//            the scaled column k is broadcast through shared memory (one
+//            store per lane, 16-byte reads), not by one shuffle per entry,
+//            which would serialize 31 shuffles per pivot.
 //   inverse: column `lane` of L^-1 by a column sweep, x[k] = acc[k] /
-//            L[k][k], then every later row r loses L[r][k] x[k]; L[r][k] is
-//            a shuffle from lane r (independent of x, so the shuffles of a
-//            step overlap).
-__device__ __noinline__ bool chol_inv32(const float* T, float* Dt, float* g, int64_t ldg) {
+//            L[k][k], then every later row r loses L[r][k] x[k]; column k of
+//            L is read from its transposed copy in `col`.
+__device__ __noinline__ bool chol_inv32(const float* T, float* Dt, float* g, int64_t ldg,
+                                        float* col) {
   const unsigned full = 0xffffffffu;
   const int lane = threadIdx.x & 31;
   bool ok = true;
-  float my_inv = 0.f;  // 1 / L[lane][lane]
   float l[kB];
 #pragma unroll
   for (int k = 0; k < kB; k += 4) {
@@ -256,26 +259,44 @@ __device__ __noinline__ bool chol_inv32(const float* T, float* Dt, float* g, int
     // are discarded) so that the loop stays fully unrolled
     if (!(piv > 0.f) || !(piv < INFINITY)) ok = false;
     const float rs = rsqrtf(piv);
-    if (lane == k) { l[k] = piv * rs; my_inv = rs; }
-    else if (lane > k) l[k] *= rs;
-    const float lk = l[k];
+    l[k] = lane == k ? piv * rs : l[k] * rs;  // L[lane][k] (lanes above k: unused)
+    // column k (rows > k) to every lane: col row k holds L[.][k], and its
+    // padding column 32 holds 1 / L[k][k]
+    col[k * kP + lane] = l[k];
+    if (lane == 0) col[k * kP + kB] = rs;
+    __syncwarp();
+    if (k + 1 < kB) {
+      const float lk = l[k];
 #pragma unroll
-    for (int j = k + 1; j < kB; ++j) {
-      const float ljk = __shfl_sync(full, lk, j);
-      if (lane >= j) l[j] = fmaf(-lk, ljk, l[j]);
+      for (int j4 = ((k + 1) >> 2) << 2; j4 < kB; j4 += 4) {
+        const float4 c4 = *reinterpret_cast<const float4*>(col + k * kP + j4);
+        const float cj[4] = {c4.x, c4.y, c4.z, c4.w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int j = j4 + u;
+          if (j > k && lane >= j) l[j] = fmaf(-lk, cj[u], l[j]);
+        }
+      }
     }
   }
+  // col row k now holds column k of L (rows k..31 valid)
   float acc[kB];
 #pragma unroll
   for (int r = 0; r < kB; ++r) acc[r] = r == lane ? 1.f : 0.f;
 #pragma unroll
   for (int k = 0; k < kB; ++k) {
-    const float xk = acc[k] * __shfl_sync(full, my_inv, k);
+    const float xk = acc[k] * col[k * kP + kB];
     acc[k] = xk;
 #pragma unroll
-    for (int r = k + 1; r < kB; ++r)
-      acc[r] = fmaf(-__shfl_sync(full, l[k], r), xk, acc[r]);
+    for (int r4 = ((k + 1) >> 2) << 2; r4 < kB; r4 += 4) {
+      const float4 c4 = *reinterpret_cast<const float4*>(col + k * kP + r4);
+      const float cr[4] = {c4.x, c4.y, c4.z, c4.w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (r4 + u > k) acc[r4 + u] = fmaf(-cr[u], xk, acc[r4 + u]);
+    }
   }
+  __syncwarp();
   // acc[r] = D[r][lane]; lanes write column `lane`
 #pragma unroll
   for (int r = 0; r < kB; ++r) {
@@ -285,95 +306,41 @@ __device__ __noinline__ bool chol_inv32(const float* T, float* Dt, float* g, int
   return ok;
 }
 
-// One warp: the 32 x 32 block product A B^T of two 32 x 32 tiles (pitch
-// kP) on the tensor cores, with fp32 accuracy from three tf32 products per
-// term (x = hi + lo, hi the tf32 rounding of x: A B^T ~ lo_A hi_B + hi_A lo_B
-// + hi_A hi_B, the tiny lo_A lo_B dropped).  c[mi][ni] is the m16n8 tile
-// (mi, ni) in the mma.sync accumulator layout: rows 16 mi + g (+8), columns
-// 8 ni + 2 t (+1), g = lane / 4, t = lane % 4.
-__device__ __forceinline__ void split_tf32(float x, uint32_t& hi, uint32_t& lo) {
-  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(hi) : "f"(x));
-  lo = __float_as_uint(x - __uint_as_float(hi));
-}
-
-__device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4],
-                                         const uint32_t (&b)[2]) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 "
-      "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
-}
-
-__device__ __forceinline__ void block_abt(const float* A, const float* B, float (&c)[2][4][4]) {
-  const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+// acc[c] += sum_k A[lane][k] B[c0 + c][k], c < 8 (tiles of pitch kP)
+__device__ __forceinline__ void rowdot8(const float* A, const float* B, int c0, float (&acc)[8]) {
+  const int lane = threadIdx.x & 31;
+  float row[kB];
 #pragma unroll
-  for (int mi = 0; mi < 2; ++mi)
+  for (int k = 0; k < kB; k += 4) {
+    const float4 v = *reinterpret_cast<const float4*>(A + lane * kP + k);
+    row[k] = v.x; row[k + 1] = v.y; row[k + 2] = v.z; row[k + 3] = v.w;
+  }
 #pragma unroll
-    for (int ni = 0; ni < 4; ++ni)
+  for (int c = 0; c < 8; ++c) {
+    const float* bp = B + (c0 + c) * kP;
 #pragma unroll
-      for (int e = 0; e < 4; ++e) c[mi][ni][e] = 0.f;
-#pragma unroll
-  for (int ks = 0; ks < 4; ++ks) {
-    const int k0 = 8 * ks + t;
-    uint32_t ah[2][4], al[2][4], bh[4][2], bl[4][2];
-#pragma unroll
-    for (int mi = 0; mi < 2; ++mi) {
-      const float* a0 = A + (16 * mi + g) * kP + k0;
-      split_tf32(a0[0], ah[mi][0], al[mi][0]);
-      split_tf32(a0[8 * kP], ah[mi][1], al[mi][1]);
-      split_tf32(a0[4], ah[mi][2], al[mi][2]);
-      split_tf32(a0[8 * kP + 4], ah[mi][3], al[mi][3]);
+    for (int k = 0; k < kB; k += 4) {
+      const float4 v = *reinterpret_cast<const float4*>(bp + k);
+      acc[c] = fmaf(row[k], v.x, acc[c]);
+      acc[c] = fmaf(row[k + 1], v.y, acc[c]);
+      acc[c] = fmaf(row[k + 2], v.z, acc[c]);
+      acc[c] = fmaf(row[k + 3], v.w, acc[c]);
     }
-#pragma unroll
-    for (int ni = 0; ni < 4; ++ni) {
-      const float* b0 = B + (8 * ni + g) * kP + k0;
-      split_tf32(b0[0], bh[ni][0], bl[ni][0]);
-      split_tf32(b0[4], bh[ni][1], bl[ni][1]);
-    }
-#pragma unroll
-    for (int mi = 0; mi < 2; ++mi)
-#pragma unroll
-      for (int ni = 0; ni < 4; ++ni) {
-        mma_tf32(c[mi][ni], al[mi], bh[ni]);
-        mma_tf32(c[mi][ni], ah[mi], bl[ni]);
-        mma_tf32(c[mi][ni], ah[mi], bh[ni]);
-      }
   }
 }
 
-// T -= A B^T (32 x 32 tiles, pitch kP), one warp.
-__device__ __forceinline__ void block_sub_abt(float* T, const float* A, const float* B) {
-  const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-  float c[2][4][4];
-  block_abt(A, B, c);
-#pragma unroll
-  for (int mi = 0; mi < 2; ++mi)
-#pragma unroll
-    for (int ni = 0; ni < 4; ++ni)
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        float2* p = reinterpret_cast<float2*>(T + (16 * mi + g + 8 * h) * kP + 8 * ni + 2 * t);
-        float2 v = *p;
-        v.x -= c[mi][ni][2 * h];
-        v.y -= c[mi][ni][2 * h + 1];
-        *p = v;
-      }
-}
-
-// T = A B^T (32 x 32 tiles, pitch kP), one warp.
-__device__ __forceinline__ void block_set_abt(float* T, const float* A, const float* B) {
-  const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-  float c[2][4][4];
-  block_abt(A, B, c);
-#pragma unroll
-  for (int mi = 0; mi < 2; ++mi)
-#pragma unroll
-    for (int ni = 0; ni < 4; ++ni)
-#pragma unroll
-      for (int h = 0; h < 2; ++h)
-        *reinterpret_cast<float2*>(T + (16 * mi + g + 8 * h) * kP + 8 * ni + 2 * t) =
-            make_float2(c[mi][ni][2 * h], c[mi][ni][2 * h + 1]);
+// tile -= A B^T over columns c0 .. c0 + 7 (row = lane)
+__device__ __forceinline__ void sub_rowdot8(float* Tt, const float* A, const float* B, int c0) {
+  const int lane = threadIdx.x & 31;
+  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  rowdot8(A, B, c0, acc);
+  float* sp = Tt + lane * kP + c0;
+  const float4 s0 = *reinterpret_cast<const float4*>(sp);
+  const float4 s1 = *reinterpret_cast<const float4*>(sp + 4);
+  *reinterpret_cast<float4*>(sp) =
+      make_float4(s0.x - acc[0], s0.y - acc[1], s0.z - acc[2], s0.w - acc[3]);
+  *reinterpret_cast<float4*>(sp + 4) =
+      make_float4(s1.x - acc[4], s1.y - acc[5], s1.z - acc[6], s1.w - acc[7]);
 }
 
 __global__ void __launch_bounds__(kCT, 1) chol_kernel(const __grid_constant__ CholBatch cb) {
@@ -389,7 +356,8 @@ __global__ void __launch_bounds__(kCT, 1) chol_kernel(const __grid_constant__ Ch
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   auto tile = [&](int bi, int bj) { return sm + (size_t)tri_index(bi, bj) * kTF; };
   float* Dt = sm + (size_t)ntri * kTF;
-  float* pan = Dt + kTF;
+  float* col = Dt + kTF;   // column scratch of the factoring warp
+  float* pan = col + kTF;
   auto gblk = [&](int bi, int bj) { return Lb + (size_t)bi * kB * R + (size_t)bj * kB; };
 
   bool ok = false;
@@ -409,22 +377,26 @@ __global__ void __launch_bounds__(kCT, 1) chol_kernel(const __grid_constant__ Ch
       if (!(shift > 0.0)) shift = 1e-30;
       __syncthreads();
     }
-    // lower tiles from the upper storage: tile (bi, bj)[ii][jj] = S[j][i]
-    // with i = bi*32 + ii, j = bj*32 + jj, identity padding past r.
-    // Asynchronous 4-byte copies keep the whole matrix in flight at once
-    // (one CTA streaming it with one load per thread at a time would wait
-    // on memory latency for every element).
-    for (int e = threadIdx.x; e < ntri * kB * kB; e += kCT) {
-      const int tt = e >> 10, w = e & 1023, jj = w >> 5, ii = w & 31;
-      const int bi = tri_row_of(tt), bj = tt - bi * (bi + 1) / 2;
-      const int i = bi * kB + ii, j = bj * kB + jj;
-      float* d = sm + (size_t)tt * kTF + ii * kP + jj;
-      if (i < r && j < r && j <= i) {
-        const unsigned da = (unsigned)__cvta_generic_to_shared(d);
-        asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(da),
-                     "l"(S + (size_t)j * r + i) : "memory");
-      } else {
-        *d = i == j ? 1.f : 0.f;
+    // lower tiles of S (full symmetric storage, ld r): row ii of tile
+    // (bi, bj) is 32 consecutive floats of row bi*32 + ii, copied as eight
+    // 16-byte asynchronous copies when the rows allow it; identity padding
+    // past r
+    {
+      const bool vec = (r & 3) == 0 && ((uintptr_t)S & 15) == 0;
+      for (int e = threadIdx.x; e < ntri * kB * 8; e += kCT) {
+        const int tt = e >> 8, w = e & 255, ii = w >> 3, c4 = (w & 7) * 4;
+        const int bi = tri_row_of(tt), bj = tt - bi * (bi + 1) / 2;
+        const int i = bi * kB + ii, j = bj * kB + c4;
+        float* d = sm + (size_t)tt * kTF + ii * kP + c4;
+        if (vec && i < r && j + 3 < r) {
+          const unsigned da = (unsigned)__cvta_generic_to_shared(d);
+          asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(da),
+                       "l"(S + (size_t)i * r + j) : "memory");
+        } else {
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            d[u] = (i < r && j + u < r) ? S[(size_t)i * r + j + u] : (i == j + u ? 1.f : 0.f);
+        }
       }
     }
     asm volatile("cp.async.wait_all;\n" ::: "memory");
@@ -437,35 +409,45 @@ __global__ void __launch_bounds__(kCT, 1) chol_kernel(const __grid_constant__ Ch
     }
     if (threadIdx.x == 0) s_bad = 0;
     __syncthreads();
-    if (warp == 0 && !chol_inv32(tile(0, 0), Dt, gblk(0, 0), R) && lane == 0) s_bad = 1;
+    if (warp == 0 && !chol_inv32(tile(0, 0), Dt, gblk(0, 0), R, col) && lane == 0) s_bad = 1;
     __syncthreads();
     bool failed = s_bad != 0;
     for (int p = 0; p < nb && !failed; ++p) {
       const int m = nb - 1 - p;
       if (m == 0) break;
-      // panel: pan[b] = S(p+1+b, p) D_p^T, one warp per block
-      for (int bb = warp; bb < m; bb += kCW)
-        block_set_abt(pan + (size_t)bb * kTF, tile(p + 1 + bb, p), Dt);
-      __syncthreads();
-      // the panel blocks L_{p+1+b, p} to global memory
-      for (int e = threadIdx.x; e < m * kB * kB; e += kCT) {
-        const int bb = e >> 10, w = e & 1023, ii = w >> 5, jj = w & 31;
-        gblk(p + 1 + bb, p)[(size_t)ii * R + jj] = pan[(size_t)bb * kTF + ii * kP + jj];
+      // panel: pan[b] = S(p+1+b, p) D_p^T, items (block, 8 columns)
+      for (int it = warp; it < 4 * m; it += kCW) {
+        const int bb = it >> 2, c0 = (it & 3) * 8;
+        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        rowdot8(tile(p + 1 + bb, p), Dt, c0, acc);
+        float* dst = pan + (size_t)bb * kTF + lane * kP + c0;
+        *reinterpret_cast<float4*>(dst) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+        *reinterpret_cast<float4*>(dst + 4) = make_float4(acc[4], acc[5], acc[6], acc[7]);
       }
-      // look-ahead: warp 0 updates the next diagonal block and factors it
-      // while the other warps finish the trailing update
-      if (warp == 0) {
-        block_sub_abt(tile(p + 1, p + 1), pan, pan);
-        __syncwarp();
-        if (!chol_inv32(tile(p + 1, p + 1), Dt, gblk(p + 1, p + 1), R) && lane == 0) s_bad = 1;
-      } else {
+      __syncthreads();
+      // the panel blocks L_{p+1+b, p} to global memory (16-byte stores)
+      for (int e = threadIdx.x; e < m * kB * 8; e += kCT) {
+        const int bb = e >> 8, w = e & 255, ii = w >> 3, c4 = (w & 7) * 4;
+        *reinterpret_cast<float4*>(gblk(p + 1 + bb, p) + (size_t)ii * R + c4) =
+            *reinterpret_cast<const float4*>(pan + (size_t)bb * kTF + ii * kP + c4);
+      }
+      // look-ahead: warps 0-3 update the next diagonal block, then warp 0
+      // factors it while the other warps finish the trailing update
+      if (warp < 4) {
+        sub_rowdot8(tile(p + 1, p + 1), pan, pan, warp * 8);
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        if (warp == 0 && !chol_inv32(tile(p + 1, p + 1), Dt, gblk(p + 1, p + 1), R, col) &&
+            lane == 0)
+          s_bad = 1;
+      }
+      if (warp > 0) {
         // trailing: S(p+1+bi, p+1+bj) -= pan[bi] pan[bj]^T, bj <= bi, except (0, 0)
         const int tasks = m * (m + 1) / 2 - 1;
-        for (int it = warp - 1; it < tasks; it += kCW - 1) {
-          const int tt = it + 1;
+        for (int it = warp - 1; it < 4 * tasks; it += kCW - 1) {
+          const int tt = (it >> 2) + 1, c0 = (it & 3) * 8;
           const int bi = tri_row_of(tt), bj = tt - bi * (bi + 1) / 2;
-          block_sub_abt(tile(p + 1 + bi, p + 1 + bj), pan + (size_t)bi * kTF,
-                        pan + (size_t)bj * kTF);
+          sub_rowdot8(tile(p + 1 + bi, p + 1 + bj), pan + (size_t)bi * kTF,
+                      pan + (size_t)bj * kTF, c0);
         }
       }
       __syncthreads();
