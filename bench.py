@@ -58,10 +58,11 @@ def _args():
     ap.add_argument("--no-sweep", action="store_true",
                     help="skip the standard-vs-Gram crossover points of the JSON line")
     ap.add_argument("--cpu-sample-layers", type=int, default=1)
-    ap.add_argument("--micro", choices=["gram", "dion"], default=None,
+    ap.add_argument("--micro", choices=["gram", "dion", "dion_set"], default=None,
                     help="one kernel-level case for profiling: Gram NS on --nb blocks "
-                         "of --m x --n bf16, or one Dion / Orth-Dion matrix --m x --n "
-                         "at --rank (--mode colnorm|qr)")
+                         "of --m x --n bf16, one Dion / Orth-Dion matrix --m x --n "
+                         "at --rank (--mode colnorm|qr), or the 8B-shaped set of "
+                         "--layers layers in one grouped Dion / Orth-Dion call")
     ap.add_argument("--nb", type=int, default=32)
     ap.add_argument("--m", type=int, default=1792)
     ap.add_argument("--n", type=int, default=4096)
@@ -909,6 +910,32 @@ def run_micro(args):
         fn = lambda: ouo.gram_ns_orthogonalize(Xb, Ob, p, workspace=ws)  # noqa: E731
         flops = args.nb * sum(gram_ns_flops(m, n))
         case = f"Gram NS, {args.nb} x bf16 {m}x{n}"
+    elif args.micro == "dion_set":
+        r = args.rank
+        shapes = [(a, b) for _, a, b in synth.llama8b_shapes(args.layers)]
+        Ms = ouo.batch_empty(shapes, torch.float32, dev)
+        Gs = ouo.batch_empty(shapes, torch.bfloat16, dev)
+        Ws = ouo.batch_empty(shapes, torch.bfloat16, dev)
+        Qs = ouo.batch_empty([(r, b) for _, b in shapes], torch.float32, dev)
+        q0 = {}
+        for i, (a, b) in enumerate(shapes):
+            Gs[i].copy_(synth.lowrank_plus_noise(a, b, 64, 0.02, synth.seed_for(4, 100 + i),
+                                                 torch.bfloat16, dev))
+            Ms[i].zero_()
+            Ws[i].copy_(synth.gaussian((a, b), synth.seed_for(4, 600 + i), 0.02,
+                                       torch.bfloat16, dev))
+            if b not in q0:
+                q0[b] = torch.linalg.qr(synth.dion_q0(b, r, 1).to(dev))[0].T.contiguous()
+            Qs[i].copy_(q0[b])
+        Mb, Gb, Wb, Qb = ouo.MatBatch(Ms), ouo.MatBatch(Gs), ouo.MatBatch(Ws), ouo.MatBatch(Qs)
+        p = ouo.dion_params(rank=r, norm_mode=args.mode)
+        scales = [math.sqrt(max(1.0, a / b)) for a, b in shapes]
+        ws = torch.empty(ouo.dion_workspace_bytes(Mb, p), dtype=torch.uint8, device=dev)
+        fn = lambda: ouo.dion_lowrank_step(Mb, Gb, Qb, Wb, p, scale=scales,  # noqa: E731
+                                           workspace=ws)
+        flops = 8 * r * sum(a * b for a, b in shapes)
+        case = (f"{'Orth-Dion' if args.mode == 'qr' else 'Dion'} step, 8B-shaped set, "
+                f"{args.layers} layer(s), {len(shapes)} matrices, r={r}")
     else:
         r = args.rank
         G = synth.lowrank_plus_noise(m, n, 64, 0.02, synth.seed_for(4, 7), torch.bfloat16, dev)

@@ -10,11 +10,12 @@
 // rows of L^-1 X are orthonormal with the implied triangular factor L^T on
 // a positive diagonal, i.e. the unique QR factor.
 //
-//   gram     part[s] = X[:, chunk s] X[:, chunk s]^T: 64 x 64 tiles on or
-//            above the diagonal (upper storage), fp32 FMA, the L columns cut
-//            into chunks so that a single matrix fills the GPU.
-//   sum      S = sum_s part[s] in float64, fixed order, rounded to fp32,
-//            written in full (symmetric).
+//   gram     on the tensor cores, split-tf32: lo = 2 (X - tf32(X)), then
+//            part[s] = tf32(X) [tf32(X) | tf32(lo)]^T over K range s of
+//            two passes (one tcgen05 GEMM, split-K so that a single matrix
+//            fills the GPU), and S = sym(sum_s part[s]) in float64, fixed
+//            order, rounded to fp32 and written in full: X X^T up to the
+//            residual-residual term (2^-20 relative) and fp32 accumulation.
 //   chol     one CTA per matrix (r <= 256): the lower 32 x 32 blocks of S in
 //            shared memory, right-looking blocked Cholesky with one block of
 //            look-ahead; writes the strictly lower blocks L_ij and the
@@ -36,16 +37,8 @@ namespace ouo {
 namespace {
 
 constexpr int kB = 32;        // Cholesky / solve block
-constexpr int kGT = 64;       // Gram tile
-constexpr int kGK = 32;       // Gram K step
 
 // ------------------------------------------------------------------- gram
-struct GramBatch {
-  CholQrJob job[kChunk];
-  int64_t start[kChunk + 1];  // first work item of every job
-  int njob;
-};
-
 __device__ __forceinline__ int find_job(const int64_t* start, int njob, int64_t item) {
   int lo = 0, hi = njob - 1;
   while (lo < hi) {
@@ -56,143 +49,102 @@ __device__ __forceinline__ int find_job(const int64_t* start, int njob, int64_t 
   return lo;
 }
 
-// 256 threads: thread (ty, tx) owns rows ty*4 .. ty*4+3 and columns
-// tx*4 .. tx*4+3 of the 64 x 64 tile (ti, tj), ti <= tj.  The K range of the
-// split is walked in steps of 32 columns with a register-staged double
-// buffer: the next step's operands are loaded from global memory while the
-// current step's are multiplied out of shared memory.  Loads: thread t
-// reads row t % 64, columns 4 (t / 64) .. +3 and 16 + 4 (t / 64) .. +3, and
-// stores them transposed (As[k][row]) without bank conflicts.
-__global__ void __launch_bounds__(256) gram_kernel(const __grid_constant__ GramBatch gb) {
-  __shared__ __align__(16) float As[2][kGK][kGT + 4];
-  __shared__ __align__(16) float Bs[2][kGK][kGT + 4];
-  const int j = find_job(gb.start, gb.njob, blockIdx.x);
-  const CholQrJob& jb = gb.job[j];
-  const int tiles = (jb.r + kGT - 1) / kGT;
-  const int pairs = tiles * (tiles + 1) / 2;
-  int64_t t = blockIdx.x - gb.start[j];
-  const int split = (int)(t / pairs);
-  int pr = (int)(t - (int64_t)split * pairs);
-  int ti = 0;
-  while (pr >= tiles - ti) { pr -= tiles - ti; ++ti; }
-  const int tj = ti + pr;
-  const int64_t l0 = (int64_t)split * jb.gchunk;
-  const int64_t l1 = l0 + jb.gchunk < jb.L ? l0 + jb.gchunk : jb.L;
-  const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
-  const float* X = jb.X;
-  const int64_t ld = jb.ldx;
-  float acc[4][4];
-#pragma unroll
-  for (int u = 0; u < 4; ++u)
-#pragma unroll
-    for (int v = 0; v < 4; ++v) acc[u][v] = 0.f;
-  const int lr = tid & 63, lc = (tid >> 6) * 4;
-  const int ra = ti * kGT + lr, rb = tj * kGT + lr;
-  const bool vec = (ld & 3) == 0 && ((uintptr_t)X & 15) == 0;
-  float4 na[2], nb2[2];  // the next step's operands
-  auto fetch = [&](int64_t k0) {
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int64_t kc = k0 + lc + 16 * h;
-      float va[4] = {0.f, 0.f, 0.f, 0.f}, vb[4] = {0.f, 0.f, 0.f, 0.f};
-      if (vec && kc + 3 < l1) {
-        if (ra < jb.r) {
-          const float4 f = *reinterpret_cast<const float4*>(X + ra * ld + kc);
-          va[0] = f.x; va[1] = f.y; va[2] = f.z; va[3] = f.w;
-        }
-        if (rb < jb.r) {
-          const float4 f = *reinterpret_cast<const float4*>(X + rb * ld + kc);
-          vb[0] = f.x; vb[1] = f.y; vb[2] = f.z; vb[3] = f.w;
-        }
-      } else {
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          if (kc + e < l1) {
-            if (ra < jb.r) va[e] = X[ra * ld + kc + e];
-            if (rb < jb.r) vb[e] = X[rb * ld + kc + e];
-          }
-        }
-      }
-      na[h] = make_float4(va[0], va[1], va[2], va[3]);
-      nb2[h] = make_float4(vb[0], vb[1], vb[2], vb[3]);
-    }
-  };
-  auto stash = [&](int buf) {
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int c = lc + 16 * h;
-      As[buf][c][lr] = na[h].x; As[buf][c + 1][lr] = na[h].y;
-      As[buf][c + 2][lr] = na[h].z; As[buf][c + 3][lr] = na[h].w;
-      Bs[buf][c][lr] = nb2[h].x; Bs[buf][c + 1][lr] = nb2[h].y;
-      Bs[buf][c + 2][lr] = nb2[h].z; Bs[buf][c + 3][lr] = nb2[h].w;
-    }
-  };
-  if (l0 < l1) {
-    fetch(l0);
-    stash(0);
-  }
-  __syncthreads();
-  int buf = 0;
-  for (int64_t k0 = l0; k0 < l1; k0 += kGK) {
-    const bool more = k0 + kGK < l1;
-    if (more) fetch(k0 + kGK);
-#pragma unroll 8
-    for (int kk = 0; kk < kGK; ++kk) {
-      const float4 a4 = *reinterpret_cast<const float4*>(&As[buf][kk][ty * 4]);
-      const float4 b4 = *reinterpret_cast<const float4*>(&Bs[buf][kk][tx * 4]);
-      const float av[4] = {a4.x, a4.y, a4.z, a4.w};
-      const float bv[4] = {b4.x, b4.y, b4.z, b4.w};
-#pragma unroll
-      for (int u = 0; u < 4; ++u)
-#pragma unroll
-        for (int v = 0; v < 4; ++v) acc[u][v] = fmaf(av[u], bv[v], acc[u][v]);
-    }
-    if (more) stash(buf ^ 1);
-    __syncthreads();
-    buf ^= 1;
-  }
-  float* part = jb.gpart + (size_t)split * jb.r * jb.r;
-#pragma unroll
-  for (int u = 0; u < 4; ++u) {
-    const int i = ti * kGT + ty * 4 + u;
-    if (i >= jb.r) continue;
-    const int c = tj * kGT + tx * 4;
-    if (c + 3 < jb.r && (jb.r & 3) == 0) {
-      *reinterpret_cast<float4*>(part + (size_t)i * jb.r + c) =
-          make_float4(acc[u][0], acc[u][1], acc[u][2], acc[u][3]);
-    } else {
-#pragma unroll
-      for (int v = 0; v < 4; ++v)
-        if (c + v < jb.r) part[(size_t)i * jb.r + c + v] = acc[u][v];
-    }
-  }
+// Residual operand of the split-tf32 Gram: lo = 2 (x - tf32(x)), where
+// tf32(x) keeps the sign, exponent and top 10 mantissa bits of x (the
+// tensor core's reading of an fp32 operand).  x - tf32(x) is exact in fp32,
+// and so is the factor 2.  One CTA per row of every job.
+struct LoBatch {
+  const float* X[kChunk];
+  float* lo[kChunk];
+  int64_t ld[kChunk], L[kChunk];
+  int64_t start[kChunk + 1];  // prefix sums of the jobs' rows
+  int njob;
+};
+
+__device__ __forceinline__ float resid2(float x) {
+  const float h = __uint_as_float(__float_as_uint(x) & 0xffffe000u);
+  return 2.f * (x - h);
 }
 
-// S[i][j] = sum_s part[s][i][j] (float64, s ascending), the partials read at
-// (j, i) for tiles below the diagonal: S in full symmetric storage.
+__global__ void __launch_bounds__(256) lo_kernel(const __grid_constant__ LoBatch lb) {
+  const int j = find_job(lb.start, lb.njob, blockIdx.x);
+  const int64_t row = blockIdx.x - lb.start[j];
+  const float* x = lb.X[j] + row * lb.ld[j];
+  float* o = lb.lo[j] + row * lb.ld[j];
+  const int64_t L = lb.L[j], L4 = L >> 2;
+  // rows start on 16-byte boundaries (ld a multiple of 4, aligned bases)
+  const float4* x4 = reinterpret_cast<const float4*>(x);
+  float4* o4 = reinterpret_cast<float4*>(o);
+  for (int64_t c = threadIdx.x; c < L4; c += blockDim.x) {
+    const float4 v = x4[c];
+    o4[c] = make_float4(resid2(v.x), resid2(v.y), resid2(v.z), resid2(v.w));
+  }
+  for (int64_t c = 4 * L4 + threadIdx.x; c < L; c += blockDim.x) o[c] = resid2(x[c]);
+}
+
+// S = (U + U^T) / 2 with U = sum_s part[s] (float64, s ascending), the
+// partials r x r with row pitch pitch4(r), one after another.  With
+// U = X^ X^T + 2 X^ lo'^T (X^ = tf32(X), lo' = X - X^), the symmetric part is
+// X^ X^T + X^ lo'^T + lo' X^T = X X^T - lo' lo'^T.  S is written in full.
+// One CTA per pair of 32 x 32 tiles (bi, bj), bi <= bj: thread (ty, tx)
+// sums U at rows bi*32 + ty + 8k, column bj*32 + tx, and at the mirrored
+// position, both reads along rows; the mirrored sums meet their partners
+// through shared memory.
 struct SumBatch {
   const float* part[kChunk];
   float* S[kChunk];
   int r[kChunk], splits[kChunk];
-  int64_t start[kChunk + 1];  // prefix sums of r * r
+  int64_t start[kChunk + 1];  // prefix sums of the jobs' tile pairs
   int njob;
 };
 
 __global__ void __launch_bounds__(256) sum_kernel(const __grid_constant__ SumBatch sb) {
-  const int64_t total = sb.start[sb.njob];
-  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total;
-       e += (int64_t)gridDim.x * blockDim.x) {
-    const int j = find_job(sb.start, sb.njob, e);
-    const int64_t w = e - sb.start[j];
-    const int r = sb.r[j];
-    const int i = (int)(w / r), c = (int)(w - (w / r) * r);
-    // entries of tiles below the diagonal are the mirror of (c, i), which
-    // the Gram kernel computed: S is written in full (symmetric)
-    const int64_t src = (c / kGT < i / kGT) ? (int64_t)c * r + i : w;
-    double s = 0.0;
-    const float* p = sb.part[j] + src;
-    for (int q = 0; q < sb.splits[j]; ++q) s += (double)p[(size_t)q * r * r];
-    sb.S[j][w] = (float)s;
+  __shared__ double mir[32][33];
+  const int j = find_job(sb.start, sb.njob, blockIdx.x);
+  const int r = sb.r[j];
+  const int nt = (r + 31) / 32;
+  int pr = (int)(blockIdx.x - sb.start[j]);
+  int bi = 0;
+  while (pr >= nt - bi) { pr -= nt - bi; ++bi; }
+  const int bj = bi + pr;
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+  const int64_t ldp = (r + 3) & ~3;
+  const size_t sp = (size_t)r * ldp;
+  const float* p = sb.part[j];
+  double u[4] = {0.0, 0.0, 0.0, 0.0}, v[4] = {0.0, 0.0, 0.0, 0.0};
+  const int cu = bj * 32 + tx, cv = bi * 32 + tx;
+  for (int q = 0; q < sb.splits[j]; ++q) {
+    const float* pq = p + q * sp;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int ru = bi * 32 + ty + 8 * k, rv = bj * 32 + ty + 8 * k;
+      if (ru < r && cu < r) u[k] += (double)pq[(size_t)ru * ldp + cu];
+      if (rv < r && cv < r) v[k] += (double)pq[(size_t)rv * ldp + cv];
+    }
+  }
+  // v[k] = sum U[bj*32 + ty + 8k][bi*32 + tx]: element (tx, ty + 8k) of
+  // the tile (bi, bj) of U^T
+#pragma unroll
+  for (int k = 0; k < 4; ++k) mir[ty + 8 * k][tx] = v[k];
+  __syncthreads();
+  float* S = sb.S[j];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int i = bi * 32 + ty + 8 * k, c = bj * 32 + tx;
+    const double w = 0.5 * (u[k] + mir[tx][ty + 8 * k]);
+    if (i < r && c < r) S[(size_t)i * r + c] = (float)w;
+    u[k] = w;
+  }
+  if (bi == bj) return;
+  // the mirrored tile (bj, bi) of S, rows along tx
+  __syncthreads();
+#pragma unroll
+  for (int k = 0; k < 4; ++k) mir[ty + 8 * k][tx] = u[k];
+  __syncthreads();
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int i = bj * 32 + ty + 8 * k, c = bi * 32 + tx;
+    if (i < r && c < r) S[(size_t)i * r + c] = (float)mir[tx][ty + 8 * k];
   }
 }
 
@@ -738,41 +690,116 @@ int set_smem_attr(const void* fn, size_t bytes) {
 
 }  // namespace
 
-int cholqr_gram_splits(int r, int64_t L) {
-  const int tiles = (int)ceil_div(r, kGT);
-  const int pairs = tiles * (tiles + 1) / 2;
-  int64_t want = ceil_div((int64_t)num_sms() * 2, pairs);
-  const int64_t maxs = ceil_div(L, 256);  // at least 256 columns per split
-  if (want > maxs) want = maxs;
+int cholqr_gram_ksplit(int r, int64_t L) {
+  (void)r;
+  // K ranges of at least 32 tf32 K blocks (the two passes counted), at
+  // most 64: a lone matrix spreads over enough CTAs to keep the Gram short,
+  // and a large batch writes few partials.  Depends on L alone.
+  const int64_t nkv = 2 * ceil_div(L, (int64_t)32);
+  int64_t want = nkv / 32;
   if (want < 1) want = 1;
   if (want > 64) want = 64;
-  return (int)want;
+  return gemm_ksplit_used(L, (int)want, OUO_F32, 2);
 }
 
-int cholqr_gram(const std::vector<CholQrJob>& jobs, cudaStream_t s) {
+int64_t cholqr_gram_part_floats(int r, int64_t L) {
+  return (int64_t)cholqr_gram_ksplit(r, L) * r * ((r + 3) & ~3);
+}
+
+int cholqr_gram(const std::vector<CholQrJob>& jobs, int* status, cudaStream_t s) {
+  if (jobs.empty()) return OUO_OK;
+  // residuals
   for (size_t c0 = 0; c0 < jobs.size(); c0 += kChunk) {
     const int cn = (int)(jobs.size() - c0 < (size_t)kChunk ? jobs.size() - c0 : kChunk);
-    GramBatch gb;
-    SumBatch sb;
-    gb.njob = sb.njob = cn;
-    gb.start[0] = sb.start[0] = 0;
-    int64_t total_sum = 0;
+    LoBatch lb;
+    lb.njob = cn;
+    lb.start[0] = 0;
     for (int i = 0; i < cn; ++i) {
-      CholQrJob jb = jobs[c0 + i];
-      const int tiles = (int)ceil_div(jb.r, kGT);
-      const int64_t splits = ceil_div(jb.L, jb.gchunk);
-      gb.job[i] = jb;
-      gb.start[i + 1] = gb.start[i] + splits * (tiles * (tiles + 1) / 2);
+      const CholQrJob& jb = jobs[c0 + i];
+      if ((jb.ldx & 3) || ((uintptr_t)jb.X & 15) || ((uintptr_t)jb.Xlo & 15))
+        return set_error(OUO_ERR_INVALID_ARG, "Gram operands need 16-byte rows");
+      lb.X[i] = jb.X;
+      lb.lo[i] = jb.Xlo;
+      lb.ld[i] = jb.ldx;
+      lb.L[i] = jb.L;
+      lb.start[i + 1] = lb.start[i] + jb.r;
+    }
+    lo_kernel<<<(unsigned)lb.start[cn], 256, 0, s>>>(lb);
+    OUO_CHECK_LAUNCH();
+  }
+  // partial Gram matrices: one two-pass GEMM descriptor per run of jobs
+  // that sit evenly strided in memory (the members of a group)
+  std::vector<GemmDesc> ds;
+  size_t k = 0;
+  while (k < jobs.size()) {
+    const CholQrJob& j0 = jobs[k];
+    const int ks = cholqr_gram_ksplit(j0.r, j0.L);
+    const int64_t ldp = (j0.r + 3) & ~3;
+    const int64_t pf = (int64_t)ks * j0.r * ldp;
+    size_t e = k + 1;
+    int64_t xs = 0, ls = 0;
+    if (e < jobs.size()) {
+      xs = jobs[e].X - j0.X;
+      ls = jobs[e].Xlo - j0.Xlo;
+    }
+    while (e < jobs.size()) {
+      const CholQrJob& je = jobs[e];
+      const int64_t d = (int64_t)(e - k);
+      if (je.r != j0.r || je.L != j0.L || je.ldx != j0.ldx || xs < j0.r * j0.ldx ||
+          xs != ls || je.X != j0.X + d * xs || je.Xlo != j0.Xlo + d * ls ||
+          je.gpart != j0.gpart + d * pf)
+        break;
+      ++e;
+    }
+    const int64_t cnt = (int64_t)(e - k);
+    if (cnt == 1) xs = j0.r * j0.ldx;
+    GemmDesc d;
+    d.M = j0.r; d.N = j0.r; d.K = j0.L; d.nb = cnt;
+    Buf x;
+    x.p = reinterpret_cast<char*>(const_cast<float*>(j0.X));
+    x.dtype = OUO_F32;
+    x.rows = j0.r;
+    x.cols = j0.L;
+    x.ld = j0.ldx;
+    x.stride = xs;
+    x.nb = cnt;
+    d.A = x;
+    d.B = x;
+    d.B2 = x;
+    d.B2.p = reinterpret_cast<char*>(j0.Xlo);
+    d.npass = 2;
+    d.b_lo = 2;  // pass 1 reads B from the residuals
+    d.has_f32 = true;
+    Buf o;
+    o.p = reinterpret_cast<char*>(j0.gpart);
+    o.dtype = OUO_F32;
+    o.rows = j0.r;
+    o.cols = j0.r;
+    o.ld = ldp;
+    o.stride = j0.r * ldp;
+    o.nb = cnt * ks;
+    d.out_f32 = o;
+    d.ksplit = ks;
+    d.per_desc_tiles = true;
+    ds.push_back(d);
+    k = e;
+  }
+  OUO_TRY(gemm_umma_grouped(ds, s, status));
+  for (size_t c0 = 0; c0 < jobs.size(); c0 += kChunk) {
+    const int cn = (int)(jobs.size() - c0 < (size_t)kChunk ? jobs.size() - c0 : kChunk);
+    SumBatch sb;
+    sb.njob = cn;
+    sb.start[0] = 0;
+    for (int i = 0; i < cn; ++i) {
+      const CholQrJob& jb = jobs[c0 + i];
       sb.part[i] = jb.gpart;
       sb.S[i] = jb.S;
       sb.r[i] = jb.r;
-      sb.splits[i] = (int)splits;
-      sb.start[i + 1] = sb.start[i] + (int64_t)jb.r * jb.r;
-      total_sum += (int64_t)jb.r * jb.r;
+      sb.splits[i] = cholqr_gram_ksplit(jb.r, jb.L);
+      const int64_t nt = ceil_div(jb.r, 32);
+      sb.start[i + 1] = sb.start[i] + nt * (nt + 1) / 2;
     }
-    gram_kernel<<<(unsigned)gb.start[cn], 256, 0, s>>>(gb);
-    OUO_CHECK_LAUNCH();
-    sum_kernel<<<grid_cap(total_sum, 256), 256, 0, s>>>(sb);
+    sum_kernel<<<(unsigned)sb.start[cn], 256, 0, s>>>(sb);
     OUO_CHECK_LAUNCH();
   }
   return OUO_OK;

@@ -92,12 +92,6 @@ int proj_ksplit(int64_t M, int64_t N, int64_t K) {
   return gemm_ksplit_used(K, (int)ks, OUO_F32);
 }
 
-int64_t gram_chunk(int r, int64_t L) {
-  const int sp = cholqr_gram_splits(r, L);
-  return ceil_div(ceil_div(L, sp), 32) * 32;
-}
-int64_t gram_nsplit(int r, int64_t L) { return ceil_div(L, gram_chunk(r, L)); }
-
 // Matrices of one (rows, cols, rank) in a call, with their workspace.
 struct DGroup {
   int64_t m = 0, n = 0;
@@ -107,6 +101,7 @@ struct DGroup {
   Buf Pt, P, Rt, Qn;         // r x m, m x r, r x n, r x n per member
   Buf Pb, Rtb;               // bf16 copies of P and Rt (the M update's operands)
   Buf kp1, kp2;              // split-K partials (the same memory)
+  float* lo = nullptr;       // Gram residual operands (the same memory again)
   Buf S, Lb, Ld;             // r x r summed Gram; R x R factors
   float* gpart = nullptr;    // Gram partials, gstride floats per member
   int64_t gstride = 0;
@@ -157,10 +152,16 @@ std::vector<DGroup> plan(const ouo_mat* M, int nmat, const int* ranks, Arena& ar
     g.Pb = ar.take(OUO_BF16, nb, m, r);
     g.Rtb = ar.take(OUO_BF16, nb, r, n);
     {
-      // the two partial sets are used one after the other: one region
+      // the two partial sets and the Gram residuals are used one after the
+      // other: one region (residuals of member i at i times the stride of
+      // the Gram's input, at most the largest of the inputs' strides)
       const int64_t f1 = g.ks1 > 1 ? g.ks1 * (int64_t)r * pitch4(m) : 0;
       const int64_t f2 = g.ks2 > 1 ? g.ks2 * (int64_t)r * pitch4(n) : 0;
-      Buf region = take_bytes(ar, (size_t)nb * (size_t)(f1 > f2 ? f1 : f2) * 4 + 256);
+      int64_t f = f1 > f2 ? f1 : f2;
+      const int64_t xs[4] = {g.Pt.stride, g.Rt.stride, g.Qn.stride, (int64_t)r * pitch4(n)};
+      for (int64_t x : xs) f = x > f ? x : f;
+      Buf region = take_bytes(ar, (size_t)nb * (size_t)f * 4 + 256);
+      g.lo = reinterpret_cast<float*>(region.p);
       g.kp1 = Buf();
       g.kp1.p = region.p;
       g.kp1.dtype = OUO_F32;
@@ -175,9 +176,8 @@ std::vector<DGroup> plan(const ouo_mat* M, int nmat, const int* ranks, Arena& ar
       g.kp2.stride = r * pitch4(n);
       g.kp2.nb = nb * g.ks2;
     }
-    const int64_t gs_m = gram_nsplit(r, m), gs_n = gram_nsplit(r, n);
-    g.gstride = (gs_m > gs_n ? gs_m : gs_n) * (int64_t)r * r;
-    g.gstride = ceil_div(g.gstride, 64) * 64;
+    const int64_t gp_m = cholqr_gram_part_floats(r, m), gp_n = cholqr_gram_part_floats(r, n);
+    g.gstride = gp_m > gp_n ? gp_m : gp_n;
     g.gpart = reinterpret_cast<float*>(take_bytes(ar, (size_t)nb * g.gstride * 4).p);
     g.S = ar.take(OUO_F32, nb, r, r);
     g.Lb = ar.take(OUO_F32, nb, R, R);
@@ -287,21 +287,24 @@ int orth_factor(std::vector<CholQrJob>& jobs, const std::vector<const DGroup*>& 
 int orth_pass(std::vector<CholQrJob>& jobs, const std::vector<const DGroup*>& owner,
               const std::vector<int64_t>& mem, int* status, cudaStream_t s, bool gram_done) {
   if (jobs.empty()) return OUO_OK;
-  if (!gram_done) OUO_TRY(cholqr_gram(jobs, s));
+  if (!gram_done) OUO_TRY(cholqr_gram(jobs, status, s));
   OUO_TRY(orth_factor(jobs, owner, mem, status, s));
   return cholqr_apply(jobs, s);
 }
 
-// A CholeskyQR job on member i of group g (rows X, length L), factor
-// buffers from the group.
-CholQrJob orth_job(const DGroup& g, int64_t i, const float* X, int64_t ldx, int64_t L) {
+// A CholeskyQR job on member i of group g (rows X, length L; the members'
+// inputs `xstride` floats apart), factor buffers from the group.  Gram
+// partials and residuals are laid out evenly over the members, so that
+// the group's Gram is one GEMM descriptor.
+CholQrJob orth_job(const DGroup& g, int64_t i, const float* X, int64_t ldx, int64_t L,
+                   int64_t xstride) {
   CholQrJob j;
   j.X = X;
   j.ldx = ldx;
   j.r = g.r;
   j.L = L;
-  j.gchunk = gram_chunk(g.r, L);
-  j.gpart = g.gpart + i * g.gstride;
+  j.Xlo = g.lo + i * xstride;
+  j.gpart = g.gpart + i * cholqr_gram_part_floats(g.r, L);
   j.S = reinterpret_cast<float*>(view(g.S, i, 1).p);
   j.Lb = reinterpret_cast<float*>(view(g.Lb, i, 1).p);
   j.Dd = g.Ld.p ? reinterpret_cast<const float*>(view(g.Ld, i, 1).p) : nullptr;
@@ -351,7 +354,7 @@ int stage_orth_p(const std::vector<DGroup>& gs, int* status, cudaStream_t s, int
     std::vector<int64_t> mem;
     for (const DGroup& g : gs) {
       for (int64_t i = 0; i < (int64_t)g.members.size(); ++i) {
-        CholQrJob j = orth_job(g, i, fp(g.Pt, i), g.Pt.ld, g.m);
+        CholQrJob j = orth_job(g, i, fp(g.Pt, i), g.Pt.ld, g.m, g.Pt.stride);
         j.Y = fp(g.Pt, i);
         j.ldy = g.Pt.ld;
         if (pass == 1) {
@@ -472,10 +475,24 @@ int stage_qnew(const std::vector<DGroup>& gs, Rtp rt, const ouo_mat* Q_state,
     std::vector<int64_t> mem;
     for (const DGroup& g : gs) {
       for (int64_t i = 0; i < (int64_t)g.members.size(); ++i) {
-        int64_t ld = 0;
-        float* x = pass == 0 ? rt(g, i, &ld) : fp(g.Qn, i);
-        if (pass == 1) ld = g.Qn.ld;
-        CholQrJob j = orth_job(g, i, x, ld, g.n);
+        int64_t ld = 0, xst = 0;
+        float* x = nullptr;
+        if (pass == 0) {
+          x = rt(g, i, &ld);
+          // residuals spaced like the inputs when those are evenly spaced
+          // (the workspace's Rt), so that the group is one Gram descriptor
+          xst = (int64_t)g.r * ld;
+          if (g.members.size() > 1) {
+            int64_t l1 = 0;
+            const int64_t d = rt(g, 1, &l1) - rt(g, 0, &l1);
+            if (d >= xst && d <= g.Rt.stride) xst = d;
+          }
+        } else {
+          x = fp(g.Qn, i);
+          ld = g.Qn.ld;
+          xst = g.Qn.stride;
+        }
+        CholQrJob j = orth_job(g, i, x, ld, g.n, xst);
         j.Y = fp(g.Qn, i);
         j.ldy = g.Qn.ld;
         if (pass == 1) {
@@ -779,16 +796,16 @@ std::vector<int64_t> red_offsets(const ouo_mat* M, const std::vector<int>& ranks
 
 // The Gram matrices of every Pt, summed into S = the matrix's block of red.
 int gram_into_red(const std::vector<DGroup>& gs, float* red, const std::vector<int64_t>& off,
-                  int64_t (*rows_of)(const DGroup&), cudaStream_t s) {
+                  int64_t (*rows_of)(const DGroup&), int* status, cudaStream_t s) {
   std::vector<CholQrJob> jobs;
   for (const DGroup& g : gs) {
     for (int64_t i = 0; i < (int64_t)g.members.size(); ++i) {
-      CholQrJob j = orth_job(g, i, fp(g.Pt, i), g.Pt.ld, rows_of(g));
+      CholQrJob j = orth_job(g, i, fp(g.Pt, i), g.Pt.ld, rows_of(g), g.Pt.stride);
       j.S = red + off[g.members[i]];
       jobs.push_back(j);
     }
   }
-  return cholqr_gram(jobs, s);
+  return cholqr_gram(jobs, status, s);
 }
 
 int64_t local_rows(const DGroup& g) { return g.m; }
@@ -820,7 +837,7 @@ int shard_orth(const ouo_mat* M, const ouo_mat* Q_state, int nmat,
     for (int64_t i = 0; i < (int64_t)g.members.size(); ++i) {
       const int bi = g.members[i];
       // the shift of a retry takes the global row count
-      CholQrJob j = orth_job(g, i, fp(g.Pt, i), g.Pt.ld, rows_total[bi]);
+      CholQrJob j = orth_job(g, i, fp(g.Pt, i), g.Pt.ld, rows_total[bi], g.Pt.stride);
       j.S = red + off[bi];
       j.Y = fp(g.Pt, i);
       j.ldy = g.Pt.ld;
@@ -844,7 +861,7 @@ int shard_orth(const ouo_mat* M, const ouo_mat* Q_state, int nmat,
       for (int64_t i = 0; i < (int64_t)g.members.size(); ++i) jobs[k++].L = g.m;
   }
   OUO_TRY(cholqr_apply(jobs, s));
-  if (!second) return gram_into_red(gs, red, off, local_rows, s);
+  if (!second) return gram_into_red(gs, red, off, local_rows, dev_status, s);
   auto dst = [&](const DGroup& g, int64_t i, int64_t* ld) {
     *ld = pitch4(g.n);
     return red + off[g.members[i]];
@@ -897,7 +914,7 @@ extern "C" int dion_shard_project(const ouo_mat* M, const ouo_mat* G, int g_dtyp
   Arena ar{reinterpret_cast<char*>(ws), ws_bytes, 0, false};
   const std::vector<DGroup> gs = plan(M, nmat, ranks.data(), ar);
   OUO_TRY(stage_project(gs, M, Q_state, dev_status, s));
-  return gram_into_red(gs, red, red_offsets(M, ranks), local_rows, s);
+  return gram_into_red(gs, red, red_offsets(M, ranks), local_rows, dev_status, s);
 }
 
 extern "C" int dion_shard_orth1(const ouo_mat* M, const ouo_mat* Q_state, int nmat,

@@ -92,6 +92,10 @@ struct Segment {
   int ksplit;
   int64_t kbc;
   int64_t tiles_2d;  // output tiles of one matrix (tiles_per_mat / ksplit)
+  // split-tf32 passes: the K blocks are walked `npass` times; pass q reads
+  // A from UmmaArgs::lo_map[segment][0] when bit q of a_lo is set (B from
+  // lo_map[segment][1] for b_lo)
+  int npass, a_lo, b_lo;
 };
 
 constexpr int kMaxSeg = 6;
@@ -112,19 +116,26 @@ struct UmmaArgs {
   // per-matrix alpha of direct outputs (has_dalpha), else `alpha` for all
   float dalpha[kChunk];
   int has_dalpha;
+  // residual operands of the split-tf32 passes, per segment (A, B); kept
+  // out of Segment so that the fields every tile reads stay compact
+  CUtensorMap lo_map[kMaxSeg][2];
 };
+static_assert(sizeof(UmmaArgs) <= 32764, "kernel parameters above the 32 KB limit");
 
-template <int BN, int CG>
+// UPD: in-place rank-r updates (K = r, short main loops): fewer operand
+// stages, four staging buffers per epilogue warp, so that three C0 boxes
+// per warp are in flight.
+template <int BN, int CG, int UPD = 0>
 struct Cfg {
   static constexpr uint32_t kTileRows = kTileM * CG;  // rows of one scheduled tile
   static constexpr uint32_t kBRows = (uint32_t)BN / CG;  // B rows (N) staged per CTA
   static constexpr uint32_t kABytes = kTileM * kRowBytes;      // 16 KB
   static constexpr uint32_t kBBytes = kBRows * kRowBytes;      // 16/32 KB
   static constexpr uint32_t kStageBytes = kABytes + kBBytes;
-  static constexpr int kStages = CG == 2 ? 5 : (BN == 256 ? 4 : 6);
+  static constexpr int kStages = UPD ? 3 : (CG == 2 ? 5 : (BN == 256 ? 4 : 6));
   // epilogue staging buffers per warp: two where shared memory allows, so a
   // bulk store can still be reading one while the next chunk fills the other
-  static constexpr int kStg = CG == 2 ? 2 : 1;
+  static constexpr int kStg = UPD ? 4 : (CG == 2 ? 2 : 1);
   static constexpr uint32_t kTmemCols = 2 * BN;
   // per epilogue warp: a 32 x 32 fp32 staging buffer
   static constexpr uint32_t kEpiBytes = kEpiWarps * kStg * 32 * 32 * 4;
@@ -284,10 +295,10 @@ __device__ __forceinline__ void load_c0x4(const Segment& sg, int64_t b,
   }
 }
 
-template <int BN, int FMT /*1 bf16, 2 tf32*/, int B_MN, int CG /*CTAs per tile*/>
+template <int BN, int FMT /*1 bf16, 2 tf32*/, int B_MN, int CG /*CTAs per tile*/, int UPD>
 __global__ void __launch_bounds__(kThreads, 1)
 umma_gemm_kernel(const __grid_constant__ UmmaArgs a) {
-  using C = Cfg<BN, CG>;
+  using C = Cfg<BN, CG, UPD>;
   constexpr int TR = (int)C::kTileRows;
   constexpr uint32_t kEs = FMT == 1 ? 2 : 4;           // element bytes
   constexpr uint32_t kBK = kRowBytes / kEs;            // K elements per stage
@@ -367,17 +378,28 @@ umma_gemm_kernel(const __grid_constant__ UmmaArgs a) {
       int64_t b, ti, tj, ks;
       const int g = decode_tile(a, BN, TR, tile, &b, &ti, &tj, &ks);
       const Segment& sg = a.seg[g];
-      const int64_t nk = (sg.K + kBK - 1) / kBK;
+      const int64_t nkr = (sg.K + kBK - 1) / kBK;  // K blocks of one pass
+      const int64_t nk = nkr * sg.npass;
       const int64_t kb0 = ks * sg.kbc;
       const int64_t kb1 = kb0 + sg.kbc < nk ? kb0 + sg.kbc : nk;
       const int32_t z = (int32_t)(sg.b0 + b);
       const int32_t arow = (int32_t)(ti * TR + rank * kTileM);
       const int32_t bcol = (int32_t)(tj * BN + rank * C::kBRows);
-      for (int64_t kb = kb0; kb < kb1; ++kb) {
+      // pass and K block within the pass, advanced by counting (no division
+      // per stage); the operands of the pass
+      int64_t pass = kb0 >= nkr ? kb0 / nkr : 0;
+      int64_t kb = kb0 - pass * nkr;
+      for (int64_t kbv = kb0; kbv < kb1; ++kbv, ++kb) {
+        if (kb == nkr) {
+          kb = 0;
+          ++pass;
+        }
         if (!ptx::mbar_wait(&empty[stage], phase ^ 1, abort_flag)) {
           ok = false;
           break;
         }
+        const CUtensorMap* mA = ((sg.a_lo >> pass) & 1) ? &a.lo_map[g][0] : &sg.tmA;
+        const CUtensorMap* mB = ((sg.b_lo >> pass) & 1) ? &a.lo_map[g][1] : &sg.tmB;
         // Upper-stored symmetric operands: a K stage left of the tile's block
         // diagonal (256-wide blocks, pair tiles) comes from the transposed
         // block.  Both CTAs of a pair take the same decision.
@@ -408,20 +430,20 @@ umma_gemm_kernel(const __grid_constant__ UmmaArgs a) {
           }
         };
         if (at) load_t(sa, &sg.tmAt, arow);
-        else load(sa, &sg.tmA, (int32_t)(kb * kBK), arow);
+        else load(sa, mA, (int32_t)(kb * kBK), arow);
         if (bt) {
           load_t(sb, &sg.tmBt, bcol);
         } else if (!B_MN) {
-          load(sb, &sg.tmB, (int32_t)(kb * kBK), bcol);
+          load(sb, mB, (int32_t)(kb * kBK), bcol);
         } else if (CG == 1 && sg.b4d) {
           // (chunk column, K row, chunk, matrix): the chunks land back to
           // back, the layout the per-chunk loads produce
-          ptx::tma_load_4d(sb, &sg.tmB, &full[stage], 0, (int32_t)(kb * kBK),
+          ptx::tma_load_4d(sb, mB, &full[stage], 0, (int32_t)(kb * kBK),
                            (int32_t)(bcol / kChunkCols), z);
         } else {
 #pragma unroll
           for (uint32_t c = 0; c < C::kBRows / kChunkCols; ++c)
-            load(sb + c * kChunkBytes, &sg.tmB, (int32_t)(bcol + c * kChunkCols),
+            load(sb + c * kChunkBytes, mB, (int32_t)(bcol + c * kChunkCols),
                  (int32_t)(kb * kBK));
         }
         ++issued;
@@ -456,7 +478,7 @@ umma_gemm_kernel(const __grid_constant__ UmmaArgs a) {
          tile += tile_step, ++local) {
       int64_t b, ti, tj, ks;
       const int g = decode_tile(a, BN, TR, tile, &b, &ti, &tj, &ks);
-      const int64_t nk = (a.seg[g].K + kBK - 1) / kBK;
+      const int64_t nk = (a.seg[g].K + kBK - 1) / kBK * a.seg[g].npass;
       const int64_t kb0 = ks * a.seg[g].kbc;
       const int64_t kb1 = kb0 + a.seg[g].kbc < nk ? kb0 + a.seg[g].kbc : nk;
       const uint32_t buf = (uint32_t)(local & 1);
@@ -525,7 +547,8 @@ umma_gemm_kernel(const __grid_constant__ UmmaArgs a) {
     // accumulator-free barrier of the pair's even CTA (cluster address)
     const uint32_t tempty_lead = CG == 2 ? ptx::mapa(ptx::smem_u32(tempty), 0) : 0u;
     uint32_t nstores = 0;  // bulk stores issued by this warp
-    uint32_t nc0[2] = {0u, 0u};  // C0 box loads waited for, per staging buffer
+    uint32_t c0ph = 0u;    // bit s: parity of the C0 box loads waited for in buffer s
+    uint32_t c0pend = 0u;  // bit s: a C0 box load into buffer s not yet waited for
     for (int64_t tile = tile0; tile < a.total_tiles;
          tile += tile_step, ++local) {
       int64_t b, ti, tj, ks;
@@ -533,72 +556,46 @@ umma_gemm_kernel(const __grid_constant__ UmmaArgs a) {
       const Segment& sg = a.seg[g];
       const uint32_t buf = (uint32_t)(local & 1);
       const uint32_t tphase = (uint32_t)((local >> 1) & 1);
-      // Non-symmetric outputs with a C0 (a workspace matrix, or the output
-      // itself for in-place updates) are written through the direct path
-      // below; their C0 is prefetched one 32 x 32 chunk ahead into
-      // registers, the first chunk before the accumulator is waited for,
-      // so that every epilogue warp keeps a chunk of loads in flight.
       constexpr int kCh = BN / 64;  // 32-column chunks per warp (half a tile)
-      const bool pf = !a.tma_out && !a.tri && a.has_c0;
-      const int64_t pf_row = ti * TR + rank * kTileM + q * 32;
-      const int pf_sr = lane >> 3, pf_sc = 4 * (lane & 7);
-      const uint32_t pf_half = (uint32_t)((warp - 2) >> 2);
-      const TileOut pf_to = tile_out(a, sg, b);
-      // C0 element (pf_row + pf_sr, column 0 of this warp's half), its
-      // element size and the byte step between it-rows (4 matrix rows)
-      const int pf_es = a.c0_out ? (a.has_f32 ? 4 : 2) : (a.c0_bf16 ? 2 : 4);
-      const int64_t pf_ld = a.c0_out ? (a.has_f32 ? pf_to.ldf : pf_to.ldh) : sg.ldc0;
-      const char* pf_base = nullptr;
-      if (pf) {
-        const int64_t e0 = (pf_row + pf_sr) * pf_ld + tj * BN + pf_half * (BN / 2) + pf_sc;
-        pf_base = a.c0_out
-            ? (a.has_f32 ? reinterpret_cast<const char*>(pf_to.f) : reinterpret_cast<const char*>(pf_to.h)) + e0 * pf_es
-            : reinterpret_cast<const char*>(sg.C0) + ((sg.b0 + b) * sg.sc0 + e0) * pf_es;
+      // In-place update through the TMA (non-symmetric outputs): the C0 box
+      // of a 32 x 32 chunk is loaded by the TMA into a staging buffer (the
+      // layout of the store box), the finished chunk alpha acc + beta C0
+      // replaces it there, and a bulk tensor store writes it back.  Up to
+      // kStg - 1 chunks ahead are in flight (one with a single buffer); the
+      // first ones are requested before the accumulator is waited for, so
+      // that they load while the tile's MMAs run.  Loads and stores are
+      // async bulk copies: no per-thread global access in the epilogue.
+      const bool inplace = a.tma_out && a.c0_out;
+      constexpr int kAhead = C::kStg > 1 ? C::kStg - 1 : 1;
+      const int64_t ip_row = ti * TR + rank * kTileM + q * 32;
+      const uint32_t ip_half = (uint32_t)((warp - 2) >> 2);
+      float* const ip_stg = epi_smem + (warp - 2) * (C::kStg * 32 * 32);
+      uint64_t* const ip_bars = c0bar + (warp - 2) * C::kStg;
+      const int32_t ip_z = (int32_t)(sg.b0 + b);
+      const uint32_t ip_box = a.has_bf16 ? 2048u : 4096u;
+      const uint32_t ip_base = nstores;  // chunk c stages in buffer (ip_base + c) % kStg
+      int nch = 0;  // chunks of this warp inside the output
+      if (inplace) {
+        for (int c = 0; c < kCh; ++c)
+          if (ip_row < sg.M && tj * BN + ip_half * (BN / 2) + c * 32 < sg.N) nch = c + 1;
       }
-      // C0 of (chunk c, it-row it): rows pf_row + 4 it + pf_sr, 16 bytes,
-      // for chunks inside the matrix (edge chunks load where they are used)
-      auto pf_full = [&](int c) {
-        return pf_row + 32 <= sg.M && tj * BN + pf_half * (BN / 2) + c * 32 + 32 <= sg.N;
+      auto c0_issue = [&](int c) {  // lane 0
+        const uint32_t sb = (ip_base + (uint32_t)c) & (C::kStg - 1);
+        ptx::mbar_arrive_expect_tx(&ip_bars[sb], ip_box);
+        ptx::tma_load_3d(ip_stg + sb * (32 * 32), &sg.tmC, &ip_bars[sb],
+                         (int32_t)(tj * BN + ip_half * (BN / 2) + c * 32), (int32_t)ip_row, ip_z);
+        c0pend |= 1u << sb;
       };
-      auto pf_load = [&](int c, int it) {
-        const char* p0 = pf_base + (int64_t)c * 32 * pf_es + (int64_t)it * 4 * pf_ld * pf_es;
-        if (pf_es == 4) return __ldg(reinterpret_cast<const float4*>(p0));
-        const uint2 u = __ldg(reinterpret_cast<const uint2*>(p0));
-        return make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xffff0000u),
-                           __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xffff0000u));
+      // loads in flight land before the CTA's shared memory goes away
+      auto c0_drain = [&]() {
+        if (lane == 0)
+          for (int i = 0; i < C::kStg; ++i)
+            if ((c0pend >> i) & 1u)
+              ptx::mbar_wait_timed(&ip_bars[i], (c0ph >> i) & 1u, 100000000ull);
       };
-      // The C0 rows this warp will read for the next tile (and, on the
-      // first tile, for this one) are prefetched into L2 before the
-      // accumulator is waited for: lane l prefetches row l of the warp's
-      // 32 x BN/2 region, so that a whole tile of C0 loads is in flight per
-      // SM and the register loads below mostly hit L2.
-      if (pf) {
-        auto l2_region = [&](int64_t tl) {
-          int64_t b2, ti2, tj2, ks2;
-          const int g2 = decode_tile(a, BN, TR, tl, &b2, &ti2, &tj2, &ks2);
-          const Segment& s2 = a.seg[g2];
-          const int64_t row = ti2 * TR + rank * kTileM + q * 32 + lane;
-          const int64_t col = tj2 * BN + pf_half * (BN / 2);
-          if (row >= s2.M || col >= s2.N) return;
-          const TileOut o2 = tile_out(a, s2, b2);
-          const int64_t ld2 = a.c0_out ? (a.has_f32 ? o2.ldf : o2.ldh) : s2.ldc0;
-          const char* base = a.c0_out
-              ? (a.has_f32 ? reinterpret_cast<const char*>(o2.f) : reinterpret_cast<const char*>(o2.h))
-              : reinterpret_cast<const char*>(s2.C0) + (s2.b0 + b2) * s2.sc0 * pf_es;
-          const char* p0 = base + (row * ld2 + col) * pf_es;
-          const int64_t ncols = s2.N - col < BN / 2 ? s2.N - col : BN / 2;
-          for (int64_t off = 0; off < ncols * pf_es; off += 128)
-            asm volatile("prefetch.global.L2 [%0];" ::"l"(p0 + off));
-        };
-        if (local == 0) l2_region(tile);
-        if (tile + tile_step < a.total_tiles) l2_region(tile + tile_step);
-      }
-      // one chunk of C0 in flight: slot `it` is refilled with the next
-      // chunk's value as soon as the current chunk has taken it
-      float4 pfe[8];
-      if (pf && pf_full(0)) {
-#pragma unroll
-        for (int it = 0; it < 8; ++it) pfe[it] = pf_load(0, it);
+      if (inplace && nch > 0 && lane == 0) {
+        ptx::bulk_wait_read0();  // earlier stores have read their buffers
+        for (int c = 0; c < nch && c < kAhead; ++c) c0_issue(c);
       }
       // one lane polls the barrier; the warp follows through __syncwarp
       int ok = 1;
@@ -609,57 +606,27 @@ umma_gemm_kernel(const __grid_constant__ UmmaArgs a) {
           *abort_flag = 1;
           report_status(a.status, OUO_STATUS_TIMEOUT);
         }
+        c0_drain();
         break;
       }
       ptx::tc_fence_after();
-      if (a.tma_out && a.c0_out) {
-        // In-place update through the TMA (non-symmetric outputs): the C0
-        // box of a 32 x 32 chunk is loaded by the TMA into a staging buffer
-        // (the layout of the store box), the finished chunk alpha acc +
-        // beta C0 replaces it there, and a bulk tensor store writes it back.
-        // With two staging buffers (CTA pairs) the next chunk's C0 is
-        // loaded while this one is finished.  Loads and stores are async
-        // bulk copies: no per-thread global access in the epilogue.
-        const int64_t row_base = ti * TR + rank * kTileM + q * 32;
-        const uint32_t half = (uint32_t)((warp - 2) >> 2);
-        float* const stg_base = epi_smem + (warp - 2) * (C::kStg * 32 * 32);
-        uint64_t* const bars = c0bar + (warp - 2) * C::kStg;
-        const int32_t z = (int32_t)(sg.b0 + b);
+      if (inplace) {
         const bool obf = a.has_bf16 != 0;
-        const uint32_t box_bytes = obf ? 2048u : 4096u;
         const float alpha = a.has_dalpha ? a.dalpha[sg.dbase + b] : a.alpha;
-        // chunks of this warp inside the output
-        int nch = 0;
-        for (int c = 0; c < kCh; ++c)
-          if (row_base < sg.M && tj * BN + half * (BN / 2) + c * 32 < sg.N) nch = c + 1;
-        auto c0_load = [&](int c) {
-          const uint32_t sb = nstores & (C::kStg - 1);  // buffer of this chunk's store
-          float* dst = stg_base + sb * (32 * 32);
-          if (lane == 0) {
-            // the buffer's previous store has finished reading it
-            if (C::kStg == 2) ptx::bulk_wait_read1();
-            else ptx::bulk_wait_read0();
-            ptx::mbar_arrive_expect_tx(&bars[sb], box_bytes);
-            ptx::tma_load_3d(dst, &sg.tmC, &bars[sb],
-                             (int32_t)(tj * BN + half * (BN / 2) + c * 32), (int32_t)row_base, z);
-          }
-        };
         bool ok_c0 = true;
-        if (nch > 0) c0_load(0);
 #pragma unroll 1
         for (int c = 0; c < nch; ++c) {
-          const uint32_t sb = nstores & (C::kStg - 1);
-          const uint32_t ph = (nc0[sb] & 1u);
-          float* stg = stg_base + sb * (32 * 32);
+          const uint32_t sb = (ip_base + (uint32_t)c) & (C::kStg - 1);
+          const uint32_t ph = (c0ph >> sb) & 1u;
+          float* stg = ip_stg + sb * (32 * 32);
           uint16_t* stg16 = reinterpret_cast<uint16_t*>(stg);
-          const int64_t gj0 = tj * BN + half * (BN / 2) + c * 32;
+          const int64_t gj0 = tj * BN + ip_half * (BN / 2) + c * 32;
           float v[32];
-          ptx::tmem_ld32(tmem_base + ((q * 32u) << 16) + buf * BN + half * (BN / 2) + c * 32, v);
+          ptx::tmem_ld32(tmem_base + ((q * 32u) << 16) + buf * BN + ip_half * (BN / 2) + c * 32, v);
           // C0 of this chunk has landed
           int okw = 1;
-          if (lane == 0) okw = ptx::mbar_wait(&bars[sb], ph, abort_flag) ? 1 : 0;
+          if (lane == 0) okw = ptx::mbar_wait(&ip_bars[sb], ph, abort_flag) ? 1 : 0;
           okw = __shfl_sync(0xffffffffu, okw, 0);
-          ++nc0[sb];
           if (!okw) {
             if (lane == 0) {
               *abort_flag = 1;
@@ -668,6 +635,8 @@ umma_gemm_kernel(const __grid_constant__ UmmaArgs a) {
             ok_c0 = false;
             break;
           }
+          c0ph ^= 1u << sb;
+          c0pend &= ~(1u << sb);
           if (!obf) {
 #pragma unroll
             for (int j = 0; j < 32; j += 4) {
@@ -695,17 +664,20 @@ umma_gemm_kernel(const __grid_constant__ UmmaArgs a) {
           ptx::fence_async_shared();
           __syncwarp();
           if (lane == 0) {
-            ptx::tma_store_3d(&sg.tmC, stg, (int32_t)gj0, (int32_t)row_base, z);
+            ptx::tma_store_3d(&sg.tmC, stg, (int32_t)gj0, (int32_t)ip_row, ip_z);
             ptx::bulk_commit();
+            // the next load reuses the buffer of chunk c + kAhead - kStg,
+            // whose store must have finished reading it
+            if (c + kAhead < nch) {
+              if (C::kStg == 1) ptx::bulk_wait_read0();
+              else ptx::bulk_wait_read1();
+              c0_issue(c + kAhead);
+            }
           }
           ++nstores;
-          if (c + 1 < nch) c0_load(c + 1);
         }
         if (!ok_c0) {
-          // loads still in flight land before the CTA's shared memory goes
-          if (lane == 0)
-            for (int i = 0; i < C::kStg; ++i)
-              ptx::mbar_wait_timed(&bars[i], nc0[i] & 1u, 100000000ull);
+          c0_drain();
           break;
         }
         ptx::tc_fence_before();
@@ -846,83 +818,7 @@ umma_gemm_kernel(const __grid_constant__ UmmaArgs a) {
         }
         continue;
       }
-      if (!a.tri) {
-        // Non-symmetric direct (or dual) outputs.  This warp owns tile rows
-        // q*32 .. q*32+31 (TMEM lanes) and one half of the columns, in
-        // 32 x 32 chunks: finished with row = lane, staged in shared
-        // memory, and stored 16 bytes per lane, 8 lanes per 128-byte row,
-        // 4 rows per instruction, with the prefetched C0 added on the way.
-        const float alpha = (a.has_dalpha && sg.direct) ? a.dalpha[sg.dbase + b] : a.alpha;
-        float* stg = epi_smem + (warp - 2) * (C::kStg * 32 * 32);
-#pragma unroll 1
-        for (int c = 0; c < kCh; ++c) {
-          const int64_t gj0 = tj * BN + pf_half * (BN / 2) + c * 32;
-          const bool next_full = pf && c + 1 < kCh && pf_full(c + 1);
-          if (pf_row >= sg.M || gj0 >= sg.N) continue;  // outside the output
-          const bool full_chunk = pf_row + 32 <= sg.M && gj0 + 32 <= sg.N;
-#pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {  // two 16-column TMEM loads
-            float v[16];
-            ptx::tmem_ld16(tmem_base + ((q * 32u) << 16) + buf * BN +
-                               (uint32_t)(pf_half * (BN / 2) + c * 32 + hh * 16), v);
-#pragma unroll
-            for (int j = 0; j < 16; j += 4)
-              *reinterpret_cast<float4*>(stg + stg_idx(lane, hh * 16 + j)) =
-                  make_float4(alpha * v[j], alpha * v[j + 1], alpha * v[j + 2], alpha * v[j + 3]);
-          }
-          __syncwarp();
-#pragma unroll
-          for (int it = 0; it < 8; ++it) {
-            const int rr = it * 4 + pf_sr;
-            const int64_t gr = pf_row + rr, gc = gj0 + pf_sc;
-            float4 w = *reinterpret_cast<const float4*>(stg + stg_idx(rr, pf_sc));
-            uint32_t mask = 0xFu;
-            if (!full_chunk) {
-              mask = 0;
-#pragma unroll
-              for (int t = 0; t < 4; ++t)
-                if (gr < sg.M && gc + t < sg.N) mask |= 1u << t;
-            }
-            if (pf) {
-              float4 e = pfe[it];
-              if (next_full) pfe[it] = pf_load(c + 1, it);
-              if (!full_chunk) {
-                float x[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                for (int t = 0; t < 4; ++t)
-                  if (mask & (1u << t))
-                    x[t] = a.c0_out ? load_out1(a, pf_to, gr, gc + t)
-                                    : load_c0(sg, b, gr, gc + t, a.c0_bf16);
-                e = make_float4(x[0], x[1], x[2], x[3]);
-              }
-              w.x += a.beta * e.x;
-              w.y += a.beta * e.y;
-              w.z += a.beta * e.z;
-              w.w += a.beta * e.w;
-            }
-            if (a.gamma != 0.f && gr >= gc && gr < gc + 4) {
-              if (gr == gc) w.x += a.gamma;
-              if (gr == gc + 1) w.y += a.gamma;
-              if (gr == gc + 2) w.z += a.gamma;
-              if (gr == gc + 3) w.w += a.gamma;
-            }
-            if (mask) store4t(a, pf_to, gr, gc, w, mask);
-          }
-          __syncwarp();
-        }
-        // The accumulator is free once this warp's TMEM reads have
-        // completed (tcgen05.wait::ld): the arrival is relaxed, so that it
-        // does not wait for the warp's global stores to be performed (a
-        // release arrival would, once per tile).
-        ptx::tc_fence_before();
-        __syncwarp();
-        if (lane == 0) {
-          if (CG == 2) ptx::mbar_arrive_cluster_relaxed(tempty_lead + buf * 8u);
-          else ptx::mbar_arrive_relaxed(&tempty[buf]);
-        }
-        continue;
-      }
-      // Symmetric direct (or dual) outputs.
+      // Direct (or dual) outputs, symmetric or not.
       // This warp owns tile rows q*32 .. q*32+31 (TMEM lanes) and one half
       // of the columns; each chunk is 32 rows x 32 columns.  Values are
       // finished with row = lane (where the symmetric C0 read (j, i) is
@@ -1050,9 +946,9 @@ umma_gemm_kernel(const __grid_constant__ UmmaArgs a) {
       }
       ptx::tc_fence_before();
       __syncwarp();
-      if (lane == 0) {  // relaxed, as in the non-symmetric direct path
-        if (CG == 2) ptx::mbar_arrive_cluster_relaxed(tempty_lead + buf * 8u);
-        else ptx::mbar_arrive_relaxed(&tempty[buf]);
+      if (lane == 0) {
+        if (CG == 2) ptx::mbar_arrive_cluster(tempty_lead + buf * 8u);
+        else ptx::mbar_arrive(&tempty[buf]);
       }
     }
     // bulk stores complete before the CTA (and its shared memory) goes away
@@ -1203,13 +1099,13 @@ cudaLaunchConfig_t launch_cfg(unsigned grid, size_t smem, cudaStream_t stream,
   return cfg;
 }
 
-template <int BN, int FMT, int B_MN, int CG>
+template <int BN, int FMT, int B_MN, int CG, int UPD = 0>
 int launch(const std::vector<GemmDesc>& gs, cudaStream_t stream, int* status) {
-  using C = Cfg<BN, CG>;
+  using C = Cfg<BN, CG, UPD>;
   constexpr int TR = (int)C::kTileRows;
   constexpr uint32_t es = FMT == 1 ? 2 : 4;
   constexpr uint32_t bk = kRowBytes / es;
-  auto kern = umma_gemm_kernel<BN, FMT, B_MN, CG>;
+  auto kern = umma_gemm_kernel<BN, FMT, B_MN, CG, UPD>;
   // per device: shared-memory opt-in done, and how many CTAs (pairs: CTA
   // pairs) of this kernel can be resident at once -- a persistent grid
   // larger than that would run its last CTAs after the others finish
@@ -1305,7 +1201,7 @@ int launch(const std::vector<GemmDesc>& gs, cudaStream_t stream, int* status) {
           const Segment& sg = a.seg[sgi];
           const double per = a.tri ? (double)sg.M * (double)(sg.M + 1) * (double)sg.K
                                    : 2.0 * (double)sg.M * (double)sg.N * (double)sg.K;
-          rec.flops += per * (double)sg.nb;
+          rec.flops += per * (double)sg.nb * (double)sg.npass;
         }
         std::lock_guard<std::mutex> lock(g_tmu);
         g_recs.push_back(rec);
@@ -1328,10 +1224,25 @@ int launch(const std::vector<GemmDesc>& gs, cudaStream_t stream, int* status) {
     const char* env4 = getenv("OUO_TMA_4D");
     const bool b4d = B_MN && CG == 1 && g.N % (kRowBytes / es) == 0 &&
                      !(env4 && env4[0] == '0');
-    if (!B_MN) OUO_TRY(make_map(&proto.tmB, g.B, bk, C::kBRows));
-    else if (b4d) OUO_TRY(make_map4(&proto.tmB, g.B, kRowBytes / es, bk,
-                                    C::kBRows / (kRowBytes / es), mn_swz));
-    else OUO_TRY(make_map(&proto.tmB, g.B, kRowBytes / es, bk, mn_swz));
+    auto make_b = [&](CUtensorMap* m, const Buf& b) -> int {
+      if (!B_MN) return make_map(m, b, bk, C::kBRows);
+      if (b4d) return make_map4(m, b, kRowBytes / es, bk, C::kBRows / (kRowBytes / es), mn_swz);
+      return make_map(m, b, kRowBytes / es, bk, mn_swz);
+    };
+    OUO_TRY(make_b(&proto.tmB, g.B));
+    CUtensorMap lo_a, lo_b;
+    memset(&lo_a, 0, sizeof(lo_a));
+    memset(&lo_b, 0, sizeof(lo_b));
+    proto.npass = g.npass < 1 ? 1 : g.npass;
+    if (proto.npass > 1) {
+      if (FMT != 2 || proto.npass > 3 || g.a_sym || g.b_sym)
+        return set_error(OUO_ERR_INVALID_ARG, "split-tf32 passes: tf32, 2 or 3 passes, "
+                                              "no upper-stored operands");
+      proto.a_lo = g.a_lo & ((1 << proto.npass) - 1);
+      proto.b_lo = g.b_lo & ((1 << proto.npass) - 1);
+      if (proto.a_lo) OUO_TRY(make_map(&lo_a, g.A2, bk, kTileM));
+      if (proto.b_lo) OUO_TRY(make_b(&lo_b, g.B2));
+    }
     proto.M = g.M; proto.N = g.N; proto.K = g.K;
     proto.b4d = b4d ? 1 : 0;
     if (g.a_sym || g.b_sym) {
@@ -1350,7 +1261,7 @@ int launch(const std::vector<GemmDesc>& gs, cudaStream_t stream, int* status) {
     proto.tiles_n = ceil_div(g.N, BN);
     proto.tiles_2d = tiles_per_matrix(g, BN, TR);
     {
-      const int64_t nk = ceil_div(g.K, (int64_t)bk);
+      const int64_t nk = ceil_div(g.K, (int64_t)bk) * proto.npass;
       int64_t ksp = g.ksplit < 1 ? 1 : g.ksplit;
       if (ksp > nk) ksp = nk;
       proto.kbc = ceil_div(nk, ksp);
@@ -1375,6 +1286,8 @@ int launch(const std::vector<GemmDesc>& gs, cudaStream_t stream, int* status) {
       if (a.nseg == kMaxSeg || (tabled && ndirect == kChunk)) OUO_TRY(flush());
       int64_t nb = g.nb - b0;
       if (tabled && nb > kChunk - ndirect) nb = kChunk - ndirect;
+      a.lo_map[a.nseg][0] = lo_a;
+      a.lo_map[a.nseg][1] = lo_b;
       Segment& sg = a.seg[a.nseg++];
       sg = proto;
       sg.b0 = b0;
@@ -1432,9 +1345,9 @@ int gemm_timing_read(int kind, int* launches, double* total_ms, double* flops) {
   return OUO_OK;
 }
 
-int gemm_ksplit_used(int64_t K, int ksplit, int dtype) {
+int gemm_ksplit_used(int64_t K, int ksplit, int dtype, int npass) {
   const int64_t bk = kRowBytes / (dtype == OUO_BF16 ? 2 : 4);
-  const int64_t nk = ceil_div(K, bk);
+  const int64_t nk = ceil_div(K, bk) * (npass < 1 ? 1 : npass);
   int64_t ksp = ksplit < 1 ? 1 : ksplit;
   if (ksp > nk) ksp = nk;
   const int64_t kbc = ceil_div(nk, ksp);
@@ -1452,8 +1365,11 @@ bool cta_pairs_enabled() { return cta_pair_mode() > 0; }
 int launch_kind(const std::vector<GemmDesc>& gs, bool pair, bool wide, cudaStream_t stream,
                 int* status) {
   const GemmDesc& g0 = gs[0];
+  // in-place updates through the TMA (one output matrix, C0 = itself)
+  const bool upd = g0.c0_from_out && g0.direct.empty() && g0.has_f32 != g0.has_bf16;
   if (g0.A.dtype == OUO_BF16) {
     if (g0.b_mn) {
+      if (pair && upd) return launch<256, 1, 1, 2, 1>(gs, stream, status);
       if (pair) return launch<256, 1, 1, 2>(gs, stream, status);
       return wide ? launch<256, 1, 1, 1>(gs, stream, status) : launch<128, 1, 1, 1>(gs, stream, status);
     }
@@ -1461,6 +1377,7 @@ int launch_kind(const std::vector<GemmDesc>& gs, bool pair, bool wide, cudaStrea
     return wide ? launch<256, 1, 0, 1>(gs, stream, status) : launch<128, 1, 0, 1>(gs, stream, status);
   }
   if (g0.b_mn) {
+    if (pair && upd) return launch<256, 2, 1, 2, 1>(gs, stream, status);
     if (pair) return launch<256, 2, 1, 2>(gs, stream, status);
     return wide ? launch<256, 2, 1, 1>(gs, stream, status) : launch<128, 2, 1, 1>(gs, stream, status);
   }

@@ -113,11 +113,23 @@ struct GemmDesc {
   // only K-major B takes them).  Pairs halve the operand bytes per output
   // element, which is what a short-K GEMM with an in-place C0 runs out of.
   bool pair_mn = false;
+  // Split-tf32 passes (tf32 operands, no symmetric operands): the K range is
+  // run `npass` times (1 to 3) into one accumulator; in pass q the A
+  // operand is A2 instead of A when bit q of a_lo is set, and likewise B2
+  // for b_lo.  With A2 / B2 holding the residuals x - tf32(x) of A / B, the
+  // passes (A, B), (A, B2), (A2, B) give the product to about fp32 accuracy
+  // (the tensor core reads A and B truncated to tf32; the residual-residual
+  // term, 2^-20 relative, is left out).  A2 / B2 have the shapes, leading
+  // dimensions and batch strides of A / B.
+  int npass = 1;
+  Buf A2, B2;
+  int a_lo = 0, b_lo = 0;
 };
 
 // Number of K ranges a split-K GEMM of depth K over `dtype` operands
-// actually uses for a requested `ksplit` (every range non-empty).
-int gemm_ksplit_used(int64_t K, int ksplit, int dtype);
+// (run `npass` times) actually uses for a requested `ksplit` (every range
+// non-empty).
+int gemm_ksplit_used(int64_t K, int ksplit, int dtype, int npass = 1);
 
 // Whether K-major tensor-core GEMMs with more than 128 output rows and
 // columns run on CTA-pair tiles (OUO_CTA_PAIR, default on); upper-stored
@@ -167,9 +179,9 @@ struct CholQrJob {
   int64_t ldx = 0;
   int r = 0;
   int64_t L = 0;
-  int64_t gchunk = 0;        // Gram: columns per split (multiple of 32)
-  float* gpart = nullptr;    // Gram partials [ceil(L / gchunk)][r][r]
-  float* S = nullptr;        // summed Gram, r x r, upper storage (j >= i valid)
+  float* Xlo = nullptr;      // Gram: residual operand, r x L, row pitch ldx
+  float* gpart = nullptr;    // Gram partials, cholqr_gram_part_floats(r, L)
+  float* S = nullptr;        // summed Gram, r x r, full symmetric storage
   float* Lb = nullptr;       // R x R (R = r rounded up to 32), ld R: the
                              // strictly lower 32 x 32 blocks of L
   const float* Dd = nullptr; // R x R, ld R: D_i = L_ii^-1 on the diagonal
@@ -183,11 +195,16 @@ struct CholQrJob {
   uint16_t* Ytb = nullptr;   // optional bf16 copy of the transpose, L x r
   int64_t ldytb = 0;
 };
-// Gram splits for an r x L block (columns per split = ceil(L / splits),
-// rounded up to 32).
-int cholqr_gram_splits(int r, int64_t L);
-// Gram partials and their float64 sum S, for every job (2 launches).
-int cholqr_gram(const std::vector<CholQrJob>& jobs, cudaStream_t s);
+// Split-K ranges of the tensor-core Gram of an r x L block, and the floats
+// of its partials ([ranges][r][pitch4(r)]).  A run of jobs whose X, Xlo and
+// gpart are evenly strided (X and Xlo by the same step, gpart by
+// cholqr_gram_part_floats) is computed by one GEMM descriptor.
+int cholqr_gram_ksplit(int r, int64_t L);
+int64_t cholqr_gram_part_floats(int r, int64_t L);
+// Residuals, split-tf32 Gram partials on the tensor cores and their
+// float64 sum S (full symmetric), for every job.  X rows and Xlo on 16-byte
+// boundaries.
+int cholqr_gram(const std::vector<CholQrJob>& jobs, int* status, cudaStream_t s);
 // Whether the one-CTA Cholesky takes rank r (1 <= r <= 256).
 bool cholqr_small_rank(int r);
 // S -> Lb (strictly lower blocks of L and D_i on the diagonal blocks), one
