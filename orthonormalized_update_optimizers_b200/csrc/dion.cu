@@ -387,6 +387,7 @@ int stage_rproject(const std::vector<DGroup>& gs, const ouo_mat* M, Dst dst, int
     d.has_f32 = true;
     d.ksplit = g.ks2;
     d.per_desc_tiles = true;
+    d.pair_mn = true;  // the two CTAs of a pair share each B (momentum) tile
     if (g.ks2 > 1) {
       add_descs(ds, d, g, nullptr, M, g.Pt, Buf(), g.kp2);
       for (int64_t i = 0; i < (int64_t)g.members.size(); ++i) {
