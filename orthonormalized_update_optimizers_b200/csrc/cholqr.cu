@@ -23,9 +23,11 @@
 //            pivot restarts once with the shift of shifted CholeskyQR,
 //            11 (L r + r (r + 1)) u tr(S); a second failure reports
 //            OUO_STATUS_BREAKDOWN and writes the identity.
-//   trsm     Y = L^-1 X by block forward substitution, one CTA per 32-column
-//            strip of X: Y_i = D_i (X_i - sum_{k<i} L_ik Y_k).  Optional
-//            second copy and transposed copy of Y.
+//   trinv    Z = L^-1 from the blocks of L and the D_i, one CTA per block
+//            column, written as Z, Z / 2 and Z - tf32(Z).
+//   solve    Y = Z X on the tensor cores in three split-tf32 passes (one
+//            tcgen05 GEMM over the batch), then optional copies of Y, its
+//            transpose and the transpose's bf16 rounding.
 //   rows     out = sum_s part[s] (split-K partial products) row by row, with
 //            optional row norms (float64, fixed order) and normalized rows
 //            (Dion's column normalization of R, stored transposed).
@@ -113,6 +115,7 @@ __global__ void __launch_bounds__(256) sum_kernel(const __grid_constant__ SumBat
   const float* p = sb.part[j];
   double u[4] = {0.0, 0.0, 0.0, 0.0}, v[4] = {0.0, 0.0, 0.0, 0.0};
   const int cu = bj * 32 + tx, cv = bi * 32 + tx;
+#pragma unroll 4
   for (int q = 0; q < sb.splits[j]; ++q) {
     const float* pq = p + q * sp;
 #pragma unroll
@@ -418,178 +421,315 @@ __global__ void __launch_bounds__(kCT, 1) chol_kernel(const __grid_constant__ Ch
   }
 }
 
-// ------------------------------------------------------------------- trsm
-constexpr int kSP = 36;  // row pitch of the strip and block buffers (floats)
 
-struct TrsmBatch {
-  CholQrJob job[kChunk];
-  int64_t start[kChunk + 1];  // first strip of every job
+// ------------------------------------------------------------------ trinv
+// Z = L^-1 (lower triangular) from the strictly lower blocks L_ij of Lb and
+// the inverted diagonal blocks D_i (in Dd), block column by block column:
+//   Z_jj = D_j,   Z_ij = -D_i sum_{k=j}^{i-1} L_ik Z_kj   (i > j).
+// One CTA per (job, block column j), 256 threads; thread (ty, tx) owns
+// rows ty + 8u (u < 4), column tx of a 32 x 32 block.  Entries outside the
+// r x r matrix, and above the diagonal of a D_i, are read as zero.  The
+// column is written as three planes (R x R, ld R, R = 32 ceil(r / 32)):
+// Z, Z / 2 and Z - tf32(Z), the A operands of the split-tf32 product
+// Y = Z X; blocks above the diagonal are zero.
+constexpr int kZP = 33;  // pitch of a 32 x 32 block in shared memory
+
+struct TrinvBatch {
+  const float* Lb[kChunk];
+  const float* Dd[kChunk];
+  float* Z[kChunk];
+  int r[kChunk];
+  int64_t start[kChunk + 1];  // prefix sums of the jobs' block columns
   int njob;
 };
 
-__device__ __forceinline__ void cp_async16(float* dst, const float* src) {
-  const unsigned d = (unsigned)__cvta_generic_to_shared(dst);
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(d), "l"(src) : "memory");
+// Ranks above 256 (streaming): the L_ik of a block row are fetched in
+// groups of 8 while the column is built; shared memory holds the column,
+// 8 L blocks, D_i and T.
+size_t trinv_smem_bytes(int nb) { return (size_t)(nb + 8 + 2) * 32 * kZP * sizeof(float); }
+
+__device__ __forceinline__ float tf32_trunc(float x) {
+  return __uint_as_float(__float_as_uint(x) & 0xffffe000u);
 }
 
-// Y = L^-1 X on one 32-column strip, block row by block row:
-//   Y_i = D_i X_i;  X_j -= L_ji Y_i for the blocks j > i below.
-// The products run in rounds: a round is D_i X_i, or up to four updates
-// L_ji Y_i, one per group of 64 threads (a thread owns rows ro, ro+8,
-// ro+16, ro+24 and four columns of a 32 x 32 block).  The blocks of L a
-// round needs are copied into shared memory (cp.async) one round ahead.
-__global__ void __launch_bounds__(256) trsm_kernel(const __grid_constant__ TrsmBatch tb) {
-  extern __shared__ __align__(16) float sm[];
-  const int job = find_job(tb.start, tb.njob, blockIdx.x);
-  const CholQrJob& jb = tb.job[job];
-  const int64_t c0g = (blockIdx.x - tb.start[job]) * kB;  // first column of the strip
-  const int r = jb.r, nb = (r + kB - 1) / kB, R = nb * kB;
-  float* xs = sm;                                   // R x kSP
-  float* blk = sm + (size_t)R * kSP;                // [2][4][32][kSP]
-  const int tid = threadIdx.x, grp = tid >> 6, t64 = tid & 63;
-  const int ro = t64 >> 3, cc = 4 * (t64 & 7);
-  const int64_t ncol = jb.L - c0g < kB ? jb.L - c0g : kB;
-  const float* Lb = jb.Lb;
-  const float* Dd = jb.Dd ? jb.Dd : jb.Lb;
-  // rounds: for every block row i, one D round, then ceil((nb-1-i)/4)
-  // update rounds
-  auto round_of = [&](int t, int* i, int* j0) {
-    for (int b = 0; b < nb; ++b) {
-      const int nu = (nb - 1 - b + 3) / 4;
-      if (t == 0) { *i = b; *j0 = -1; return; }
-      if (t <= nu) { *i = b; *j0 = b + 1 + 4 * (t - 1); return; }
-      t -= 1 + nu;
-    }
-    *i = -1;
-    *j0 = -1;
-  };
-  int nrounds = 0;
-  for (int b = 0; b < nb; ++b) nrounds += 1 + (nb - 1 - b + 3) / 4;
-  auto prefetch = [&](int t) {
-    if (t >= nrounds) return;
-    int i, j0;
-    round_of(t, &i, &j0);
-    float* dst = blk + (size_t)(t & 1) * 4 * kB * kSP;
-    // thread: row tid >> 3, 16-byte column group tid & 7 of each block
-    const int br = tid >> 3, bc = 4 * (tid & 7);
-    if (j0 < 0) {
-      cp_async16(dst + br * kSP + bc, Dd + (size_t)(i * kB + br) * R + i * kB + bc);
-    } else {
-      for (int g = 0; g < 4 && j0 + g < nb; ++g)
-        cp_async16(dst + (size_t)g * kB * kSP + br * kSP + bc,
-                   Lb + (size_t)((j0 + g) * kB + br) * R + i * kB + bc);
-    }
-  };
-  prefetch(0);
-  asm volatile("cp.async.commit_group;\n" ::: "memory");
-  // strip in: xs[i][c] = X[i][c0g + c], zero past r or L
-  {
-    const bool vec = (jb.ldx & 3) == 0 && ((uintptr_t)jb.X & 15) == 0 && ncol == kB;
-    for (int e = tid; e < R * 8; e += 256) {
-      const int i = e >> 3, c = (e & 7) * 4;
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (i < r) {
-        const float* src = jb.X + (int64_t)i * jb.ldx + c0g + c;
-        if (vec) {
-          v = *reinterpret_cast<const float4*>(src);
-        } else {
-          float t4[4] = {0.f, 0.f, 0.f, 0.f};
-          for (int q = 0; q < 4; ++q)
-            if (c + q < ncol) t4[q] = src[q];
-          v = make_float4(t4[0], t4[1], t4[2], t4[3]);
-        }
-      }
-      *reinterpret_cast<float4*>(xs + i * kSP + c) = v;
+__device__ __forceinline__ void trinv_store(const TrinvBatch& tb, int job, int j, int nb,
+                                            const float* zc, int zpitch, int bstride) {
+  float* Z0 = tb.Z[job];
+  const int R = nb * kB;
+  const size_t plane = (size_t)R * R;
+  for (int bi = 0; bi < nb; ++bi) {
+    for (int e = threadIdx.x; e < 1024; e += blockDim.x) {
+      const int a = e >> 5, c = e & 31;
+      const float v = bi >= j ? zc[(size_t)bi * bstride + a * zpitch + c] : 0.f;
+      const size_t off = (size_t)(bi * kB + a) * R + j * kB + c;
+      Z0[off] = v;
+      Z0[plane + off] = 0.5f * v;
+      Z0[2 * plane + off] = v - tf32_trunc(v);
     }
   }
-  for (int t = 0; t < nrounds; ++t) {
-    prefetch(t + 1);
-    asm volatile("cp.async.commit_group;\n" ::: "memory");
-    asm volatile("cp.async.wait_group 1;\n" ::: "memory");
-    __syncthreads();
-    int i, j0;
-    round_of(t, &i, &j0);
-    const float* bb = blk + (size_t)(t & 1) * 4 * kB * kSP + (size_t)grp * kB * kSP;
-    const bool active = j0 < 0 ? grp == 0 : j0 + grp < nb;
-    float acc[4][4];
+}
+
+__global__ void __launch_bounds__(256) trinv_kernel(const __grid_constant__ TrinvBatch tb) {
+  extern __shared__ float zs[];
+  const int job = find_job(tb.start, tb.njob, blockIdx.x);
+  const int j = (int)(blockIdx.x - tb.start[job]);
+  const int r = tb.r[job], nb = (r + kB - 1) / kB, R = nb * kB;
+  const float* Lb = tb.Lb[job];
+  const float* Dd = tb.Dd[job];
+  constexpr int kBF = 32 * kZP;  // floats of one block in shared memory
+  float* zc = zs;                       // Z_kj, k = 0 .. nb-1
+  float* lblk = zc + (size_t)nb * kBF;  // up to 8 L_ik
+  float* dblk = lblk + 8 * kBF;         // D_i
+  float* tblk = dblk + kBF;             // T
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+  auto fetch = [&](float* dst, const float* src, int bi, int bj, bool lower, int e) {
+    const int a = e >> 5, c = e & 31;
+    const int gi = bi * kB + a, gc = bj * kB + c;
+    float v = 0.f;
+    if (gi < r && gc < r && (!lower || c <= a)) v = src[(size_t)gi * R + gc];
+    dst[a * kZP + c] = v;
+  };
+  for (int e = threadIdx.x; e < 1024; e += 256) fetch(zc + (size_t)j * kBF, Dd, j, j, true, e);
+  __syncthreads();
+  for (int i = j + 1; i < nb; ++i) {
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int k0 = j; k0 < i; k0 += 8) {
+      const int kn = i - k0 < 8 ? i - k0 : 8;
+      // 4 loads per thread and block, all issued before any is stored
+      for (int q0 = 0; q0 < kn; q0 += 4) {
+        float v[16];
 #pragma unroll
-    for (int u = 0; u < 4; ++u)
-#pragma unroll
-      for (int v = 0; v < 4; ++v) acc[u][v] = 0.f;
-    if (active) {
-      const float* yi = xs + (size_t)(i * kB) * kSP + cc;
-#pragma unroll 2
-      for (int k = 0; k < kB; k += 4) {
-        float a[4][4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const float4 w = *reinterpret_cast<const float4*>(bb + (ro + 8 * u) * kSP + k);
-          a[u][0] = w.x; a[u][1] = w.y; a[u][2] = w.z; a[u][3] = w.w;
+        for (int t = 0; t < 16; ++t) {
+          const int q = q0 + (t >> 2), w = threadIdx.x + 256 * (t & 3);
+          const int gi = i * kB + (w >> 5), gc = (k0 + q) * kB + (w & 31);
+          v[t] = q < kn && gi < r && gc < r ? Lb[(size_t)gi * R + gc] : 0.f;
         }
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float4 y = *reinterpret_cast<const float4*>(yi + (k + q) * kSP);
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            acc[u][0] = fmaf(a[u][q], y.x, acc[u][0]);
-            acc[u][1] = fmaf(a[u][q], y.y, acc[u][1]);
-            acc[u][2] = fmaf(a[u][q], y.z, acc[u][2]);
-            acc[u][3] = fmaf(a[u][q], y.w, acc[u][3]);
-          }
+        for (int t = 0; t < 16; ++t) {
+          const int q = q0 + (t >> 2), w = threadIdx.x + 256 * (t & 3);
+          if (q < kn) lblk[(size_t)q * kBF + (w >> 5) * kZP + (w & 31)] = v[t];
         }
       }
+      __syncthreads();
+      for (int q = 0; q < kn; ++q) {
+        const float* lq = lblk + (size_t)q * kBF;
+        const float* zq = zc + (size_t)(k0 + q) * kBF;
+#pragma unroll 8
+        for (int c = 0; c < 32; ++c) {
+          const float zv = zq[c * kZP + tx];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) acc[u] = fmaf(lq[(ty + 8 * u) * kZP + c], zv, acc[u]);
+        }
+      }
+      __syncthreads();
     }
-    if (j0 < 0) {
-      __syncthreads();  // every read of X_i is done before Y_i replaces it
-      if (active) {
 #pragma unroll
-        for (int u = 0; u < 4; ++u)
-          *reinterpret_cast<float4*>(xs + (size_t)(i * kB + ro + 8 * u) * kSP + cc) =
-              make_float4(acc[u][0], acc[u][1], acc[u][2], acc[u][3]);
+    for (int u = 0; u < 4; ++u) tblk[(ty + 8 * u) * kZP + tx] = acc[u];
+    for (int e = threadIdx.x; e < 1024; e += 256) fetch(dblk, Dd, i, i, true, e);
+    __syncthreads();
+    float z[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 8
+    for (int c = 0; c < 32; ++c) {
+      const float tv = tblk[c * kZP + tx];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) z[u] = fmaf(dblk[(ty + 8 * u) * kZP + c], tv, z[u]);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) zc[(size_t)i * kBF + (ty + 8 * u) * kZP + tx] = -z[u];
+    __syncthreads();
+  }
+  trinv_store(tb, job, j, nb, zc, kZP, kBF);
+}
+
+// Ranks up to 256 (nb <= 8), right-looking: once Z_kj is known, every
+// T_i (i > k) takes its term L_ik Z_kj, and Z_{k+1,j} = -D_{k+1} T_{k+1}.
+// 512 threads: the T_i updates of a step run in parallel on eight groups of
+// 64 threads (T_i belongs to group i - j - 1 and stays in its registers),
+// each thread a 4 x 4 tile from float4 reads (L and D stored transposed, Z
+// and T by rows); the D product is spread over all threads.  All L_ik
+// (k >= j) and D_i (i >= j) of the column are loaded once.
+constexpr int kP4 = 36;  // pitch of a 32 x 32 block read as float4 rows
+constexpr int kB4 = 32 * kP4;
+size_t trinv8_smem_bytes(int nb) {
+  const int m = nb;  // the column j = 0 needs the most
+  return (size_t)(nb + m * (m - 1) / 2 + m + 1) * kB4 * sizeof(float);
+}
+
+constexpr int kT8 = 512;  // threads of the right-looking inverse
+__global__ void __launch_bounds__(kT8) trinv8_kernel(const __grid_constant__ TrinvBatch tb) {
+  extern __shared__ __align__(16) float z8[];
+  const int job = find_job(tb.start, tb.njob, blockIdx.x);
+  const int j = (int)(blockIdx.x - tb.start[job]);
+  const int r = tb.r[job], nb = (r + kB - 1) / kB, R = nb * kB;
+  const float* Lb = tb.Lb[job];
+  const float* Dd = tb.Dd[job];
+  const int m = nb - j;
+  float* zc = z8;                              // Z_kj by rows, k = 0 .. nb-1
+  float* lt = zc + (size_t)nb * kB4;           // L_ik^T, j <= k < i
+  float* dt = lt + (size_t)(m * (m - 1) / 2) * kB4;  // D_i^T, i >= j
+  float* tb4 = dt + (size_t)m * kB4;           // T_{k+1} by rows
+  auto lidx = [&](int i, int k) {
+    const int a = i - j;
+    return (size_t)((a * (a - 1)) / 2 + (k - j)) * kB4;
+  };
+  // loads: transposed copies of L_ik and D_i, Z_jj = D_j by rows; entries
+  // outside the r x r matrix, and above a D_i's diagonal, are zero.  Each
+  // thread issues 16 independent loads before it stores any of them.
+  {
+    const int nl = m * (m - 1) / 2;
+    const int total = (nl + m + 1) * 1024;
+    for (int base = threadIdx.x; base < total; base += kT8 * 16) {
+      float v[16];
+      float* dst[16];
+#pragma unroll
+      for (int q = 0; q < 16; ++q) {
+        const int e = base + q * kT8;
+        v[q] = 0.f;
+        dst[q] = nullptr;
+        if (e >= total) continue;
+        const int blk = e >> 10, w = e & 1023, a = w >> 5, c = w & 31;
+        int bi, bj;
+        bool lower;
+        if (blk < nl) {
+          int aa = 1, qq = blk;
+          while (qq >= aa) { qq -= aa; ++aa; }
+          bi = j + aa;
+          bj = j + qq;
+          dst[q] = lt + (size_t)blk * kB4 + c * kP4 + a;
+          lower = false;
+        } else if (blk < nl + m) {
+          bi = bj = j + (blk - nl);
+          dst[q] = dt + (size_t)(blk - nl) * kB4 + c * kP4 + a;
+          lower = true;
+        } else {
+          bi = bj = j;
+          dst[q] = zc + (size_t)j * kB4 + a * kP4 + c;
+          lower = true;
+        }
+        const int gi = bi * kB + a, gc = bj * kB + c;
+        if (gi < r && gc < r && (!lower || c <= a)) v[q] = (lower ? Dd : Lb)[(size_t)gi * R + gc];
       }
-    } else if (active) {
-      const int jb2 = j0 + grp;
+#pragma unroll
+      for (int q = 0; q < 16; ++q)
+        if (dst[q]) *dst[q] = v[q];
+    }
+  }
+  __syncthreads();
+  const int g = threadIdx.x >> 6, gt = threadIdx.x & 63;
+  const int rr = (gt >> 3) * 4, cc = (gt & 7) * 4;
+  float acc[16];
+#pragma unroll
+  for (int e = 0; e < 16; ++e) acc[e] = 0.f;
+  // acc += A B on a 4 x 4 tile, A given transposed (At[c][row]), B by rows
+  auto mac = [&](const float* At, const float* B) {
+#pragma unroll 8
+    for (int c = 0; c < 32; ++c) {
+      const float4 a4 = *reinterpret_cast<const float4*>(At + c * kP4 + rr);
+      const float4 b4 = *reinterpret_cast<const float4*>(B + c * kP4 + cc);
+      const float av[4] = {a4.x, a4.y, a4.z, a4.w};
+      const float bv[4] = {b4.x, b4.y, b4.z, b4.w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int v = 0; v < 4; ++v) acc[4 * u + v] = fmaf(av[u], bv[v], acc[4 * u + v]);
+    }
+  };
+  for (int k = j; k < nb - 1; ++k) {
+    const float* zk = zc + (size_t)k * kB4;
+    // T_i += L_ik Z_kj for the row i = j + 1 + g this group owns
+    const int i = j + 1 + g;
+    if (i > k && i < nb) mac(lt + lidx(i, k), zk);
+    // T_{k+1} to shared memory by its owner
+    const int i1 = k + 1;
+    if (g == i1 - j - 1) {
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        *reinterpret_cast<float4*>(tb4 + (rr + u) * kP4 + cc) =
+            make_float4(acc[4 * u], acc[4 * u + 1], acc[4 * u + 2], acc[4 * u + 3]);
+    }
+    __syncthreads();
+    // Z_{k+1,j} = -D_{k+1} T_{k+1}: thread: row tid >> 4, two columns
+    {
+      const int row = threadIdx.x >> 4, col = 2 * (threadIdx.x & 15);
+      const float* di = dt + (size_t)(i1 - j) * kB4;
+      float z0 = 0.f, z1 = 0.f;
+#pragma unroll 8
+      for (int c = 0; c < 32; ++c) {
+        const float d = di[c * kP4 + row];
+        const float2 t2 = *reinterpret_cast<const float2*>(tb4 + c * kP4 + col);
+        z0 = fmaf(d, t2.x, z0);
+        z1 = fmaf(d, t2.y, z1);
+      }
+      *reinterpret_cast<float2*>(zc + (size_t)i1 * kB4 + row * kP4 + col) = make_float2(-z0, -z1);
+    }
+    __syncthreads();
+  }
+  trinv_store(tb, job, j, nb, zc, kP4, kB4);
+}
+
+// ------------------------------------------------------------------- post
+// Copies of the solve's result Y (r x L): Y2 = Y, Yt = Y^T (L x r) and its
+// bf16 rounding Ytb, for the jobs that ask.  One CTA per 32 x 32 tile of Y;
+// the transposes go through shared memory so that both sides are read and
+// written along rows.
+struct PostBatch {
+  const float* Y[kChunk];
+  int64_t ldy[kChunk];
+  float* Y2[kChunk];
+  int64_t ldy2[kChunk];
+  float* Yt[kChunk];
+  int64_t ldyt[kChunk];
+  uint16_t* Ytb[kChunk];
+  int64_t ldytb[kChunk];
+  int r[kChunk];
+  int64_t L[kChunk];
+  int64_t start[kChunk + 1];  // prefix sums of the jobs' tiles
+  int njob;
+};
+
+__global__ void __launch_bounds__(256) post_kernel(const __grid_constant__ PostBatch pb) {
+  __shared__ float t[32][33];
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+  const int64_t total = pb.start[pb.njob];
+  for (int64_t g = blockIdx.x; g < total; g += gridDim.x) {
+    const int job = find_job(pb.start, pb.njob, g);
+    const int r = pb.r[job];
+    const int64_t L = pb.L[job];
+    const int64_t ntj = (L + 31) / 32;
+    const int64_t tile = g - pb.start[job];
+    const int ti = (int)(tile / ntj);
+    const int64_t tj = tile - (int64_t)ti * ntj;
+    const float* Y = pb.Y[job];
+    float* Y2 = pb.Y2[job];
+    float* Yt = pb.Yt[job];
+    uint16_t* Ytb = pb.Ytb[job];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i = ti * 32 + ty + 8 * u;
+      const int64_t c = tj * 32 + tx;
+      float v = 0.f;
+      if (i < r && c < L) {
+        v = Y[(int64_t)i * pb.ldy[job] + c];
+        if (Y2) Y2[(int64_t)i * pb.ldy2[job] + c] = v;
+      }
+      t[ty + 8 * u][tx] = v;
+    }
+    __syncthreads();
+    if (Yt || Ytb) {
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
-        float* xp = xs + (size_t)(jb2 * kB + ro + 8 * u) * kSP + cc;
-        float4 x = *reinterpret_cast<float4*>(xp);
-        x.x -= acc[u][0]; x.y -= acc[u][1]; x.z -= acc[u][2]; x.w -= acc[u][3];
-        *reinterpret_cast<float4*>(xp) = x;
+        const int64_t c = tj * 32 + ty + 8 * u;  // row of Y^T
+        const int i = ti * 32 + tx;              // column of Y^T
+        if (c < L && i < r) {
+          const float v = t[tx][ty + 8 * u];
+          if (Yt) Yt[c * pb.ldyt[job] + i] = v;
+          if (Ytb) Ytb[c * pb.ldytb[job] + i] = f32_to_bf16(v);
+        }
       }
     }
     __syncthreads();
   }
-  asm volatile("cp.async.wait_group 0;\n" ::: "memory");
-  // out: Y (and its copy) row-major, Y^T (L x r)
-  for (int e = tid; e < r * 8; e += 256) {
-    const int i = e >> 3, c = (e & 7) * 4;
-    const float4 v = *reinterpret_cast<const float4*>(xs + i * kSP + c);
-    const float vv[4] = {v.x, v.y, v.z, v.w};
-    float* outs[2] = {jb.Y, jb.Y2};
-    const int64_t lds[2] = {jb.ldy, jb.ldy2};
-#pragma unroll
-    for (int o = 0; o < 2; ++o) {
-      if (!outs[o]) continue;
-      float* dst = outs[o] + (int64_t)i * lds[o] + c0g + c;
-      if (ncol == kB && (lds[o] & 3) == 0 && ((uintptr_t)outs[o] & 15) == 0) {
-        *reinterpret_cast<float4*>(dst) = v;
-      } else {
-        for (int q = 0; q < 4; ++q)
-          if (c + q < ncol) dst[q] = vv[q];
-      }
-    }
-  }
-  if (jb.Yt || jb.Ytb) {
-    for (int c = 0; c < ncol; ++c)
-      for (int i = tid; i < r; i += 256) {
-        const float v = xs[i * kSP + c];
-        if (jb.Yt) jb.Yt[(c0g + c) * jb.ldyt + i] = v;
-        if (jb.Ytb) jb.Ytb[(c0g + c) * jb.ldytb + i] = f32_to_bf16(v);
-      }
-  }
 }
-
-size_t trsm_smem_bytes(int R) { return ((size_t)R * kSP + 2 * 4 * kB * kSP) * sizeof(float); }
 
 // ------------------------------------------------------------------- rows
 struct RowsBatch {
@@ -677,11 +817,11 @@ int set_smem_attr(const void* fn, size_t bytes) {
   int dev = 0;
   OUO_CHECK_CUDA(cudaGetDevice(&dev));
   if (dev < 0 || dev >= 64) return set_error(OUO_ERR_UNSUPPORTED, "device ordinal %d", dev);
-  const int slot = fn == (const void*)chol_kernel ? 0 : 1;
+  const int slot = fn == (const void*)chol_kernel ? 0 : fn == (const void*)trinv_kernel ? 1 : 2;
   if (!done[dev][slot]) {
-    OUO_CHECK_CUDA(cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        slot == 0 ? (int)chol_smem_bytes(kMaxNb)
-                                                  : (int)trsm_smem_bytes(1024)));
+    const size_t b = slot == 0 ? chol_smem_bytes(kMaxNb)
+                   : slot == 1 ? trinv_smem_bytes(1024 / kB) : trinv8_smem_bytes(8);
+    OUO_CHECK_CUDA(cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)b));
     done[dev][slot] = 1;
   }
   (void)bytes;
@@ -832,23 +972,150 @@ int cholqr_factor(const std::vector<CholQrJob>& jobs, int* status, cudaStream_t 
   return OUO_OK;
 }
 
-int cholqr_apply(const std::vector<CholQrJob>& jobs, cudaStream_t s) {
-  OUO_TRY(set_smem_attr((const void*)trsm_kernel, 0));
-  for (size_t c0 = 0; c0 < jobs.size(); c0 += kChunk) {
-    const int cn = (int)(jobs.size() - c0 < (size_t)kChunk ? jobs.size() - c0 : kChunk);
-    TrsmBatch tb;
-    tb.njob = cn;
-    tb.start[0] = 0;
-    int Rmax = kB;
-    for (int i = 0; i < cn; ++i) {
-      const CholQrJob& jb = jobs[c0 + i];
-      const int R = (int)(ceil_div(jb.r, kB) * kB);
-      if (R > 1024) return set_error(OUO_ERR_UNSUPPORTED, "triangular solve takes r <= 1024");
-      if (R > Rmax) Rmax = R;
-      tb.job[i] = jb;
-      tb.start[i + 1] = tb.start[i] + ceil_div(jb.L, kB);
+size_t cholqr_z_floats(int r) {
+  const size_t R = (size_t)ceil_div(r, kB) * kB;
+  return 3 * R * R;
+}
+
+int cholqr_apply(const std::vector<CholQrJob>& jobs, int* status, cudaStream_t s) {
+  if (jobs.empty()) return OUO_OK;
+  OUO_TRY(set_smem_attr((const void*)trinv_kernel, 0));
+  OUO_TRY(set_smem_attr((const void*)trinv8_kernel, 0));
+  // Z = L^-1 in three planes: ranks up to 256 on the right-looking kernel,
+  // larger ones on the streaming kernel
+  for (int big = 0; big < 2; ++big) {
+    std::vector<const CholQrJob*> sel;
+    for (const CholQrJob& jb : jobs) {
+      const int nb = (int)ceil_div(jb.r, kB);
+      if (nb * kB > 1024) return set_error(OUO_ERR_UNSUPPORTED, "triangular solve takes r <= 1024");
+      if (!jb.Z || jb.Y == jb.X)
+        return set_error(OUO_ERR_INVALID_ARG, "solve needs Z and an output apart from X");
+      if ((nb > 8) == (big == 1)) sel.push_back(&jb);
     }
-    trsm_kernel<<<(unsigned)tb.start[cn], 256, trsm_smem_bytes(Rmax), s>>>(tb);
+    for (size_t c0 = 0; c0 < sel.size(); c0 += kChunk) {
+      const int cn = (int)(sel.size() - c0 < (size_t)kChunk ? sel.size() - c0 : kChunk);
+      TrinvBatch tb;
+      tb.njob = cn;
+      tb.start[0] = 0;
+      int nbmax = 1;
+      for (int i = 0; i < cn; ++i) {
+        const CholQrJob& jb = *sel[c0 + i];
+        const int nb = (int)ceil_div(jb.r, kB);
+        if (nb > nbmax) nbmax = nb;
+        tb.Lb[i] = jb.Lb;
+        tb.Dd[i] = jb.Dd ? jb.Dd : jb.Lb;
+        tb.Z[i] = jb.Z;
+        tb.r[i] = jb.r;
+        tb.start[i + 1] = tb.start[i] + nb;
+      }
+      if (big) trinv_kernel<<<(unsigned)tb.start[cn], 256, trinv_smem_bytes(nbmax), s>>>(tb);
+      else trinv8_kernel<<<(unsigned)tb.start[cn], kT8, trinv8_smem_bytes(nbmax), s>>>(tb);
+      OUO_CHECK_LAUNCH();
+    }
+  }
+  // Y = Z X in three split-tf32 passes, (Z, X), (Z / 2, 2 lo), (Z - tf32(Z), X):
+  // tf32(Z) tf32(X) + tf32(Z) lo + (Z - tf32(Z)) tf32(X).  One descriptor per
+  // run of jobs laid out evenly (the members of a group).
+  std::vector<GemmDesc> ds;
+  size_t k = 0;
+  while (k < jobs.size()) {
+    const CholQrJob& j0 = jobs[k];
+    const int64_t zf = (int64_t)cholqr_z_floats(j0.r);
+    size_t e = k + 1;
+    int64_t xs = 0, ys = 0, ls = 0, zs = 0;
+    if (e < jobs.size()) {
+      xs = jobs[e].X - j0.X;
+      ys = jobs[e].Y - j0.Y;
+      ls = jobs[e].Xlo - j0.Xlo;
+      zs = jobs[e].Z - j0.Z;
+    }
+    while (e < jobs.size()) {
+      const CholQrJob& je = jobs[e];
+      const int64_t d = (int64_t)(e - k);
+      if (je.r != j0.r || je.L != j0.L || je.ldx != j0.ldx || je.ldy != j0.ldy ||
+          xs < j0.r * j0.ldx || ys < j0.r * j0.ldy || xs != ls || zs != zf ||
+          je.X != j0.X + d * xs || je.Xlo != j0.Xlo + d * ls || je.Y != j0.Y + d * ys ||
+          je.Z != j0.Z + d * zs)
+        break;
+      ++e;
+    }
+    const int64_t cnt = (int64_t)(e - k);
+    if (cnt == 1) {
+      xs = j0.r * j0.ldx;
+      ys = j0.r * j0.ldy;
+    }
+    const int64_t R = ceil_div(j0.r, kB) * kB;
+    GemmDesc d;
+    d.M = j0.r; d.N = j0.L; d.K = j0.r; d.nb = cnt;
+    Buf z;
+    z.p = reinterpret_cast<char*>(j0.Z);
+    z.dtype = OUO_F32;
+    z.rows = j0.r;
+    z.cols = j0.r;
+    z.ld = R;
+    z.stride = zf;
+    z.nb = cnt;
+    d.A = z;
+    d.A2 = z;
+    d.A2.p = reinterpret_cast<char*>(j0.Z + R * R);
+    d.A3 = z;
+    d.A3.p = reinterpret_cast<char*>(j0.Z + 2 * R * R);
+    Buf x;
+    x.p = reinterpret_cast<char*>(const_cast<float*>(j0.X));
+    x.dtype = OUO_F32;
+    x.rows = j0.r;
+    x.cols = j0.L;
+    x.ld = j0.ldx;
+    x.stride = xs;
+    x.nb = cnt;
+    d.B = x;
+    d.B2 = x;
+    d.B2.p = reinterpret_cast<char*>(j0.Xlo);
+    d.b_mn = 1;
+    d.npass = 3;
+    d.a_lo = 2;   // pass 1: Z / 2 against the residuals (stored doubled)
+    d.b_lo = 2;
+    d.a_lo2 = 4;  // pass 2: Z - tf32(Z) against X
+    d.has_f32 = true;
+    Buf o;
+    o.p = reinterpret_cast<char*>(j0.Y);
+    o.dtype = OUO_F32;
+    o.rows = j0.r;
+    o.cols = j0.L;
+    o.ld = j0.ldy;
+    o.stride = ys;
+    o.nb = cnt;
+    d.out_f32 = o;
+    d.per_desc_tiles = true;
+    d.pair_mn = true;
+    ds.push_back(d);
+    k = e;
+  }
+  OUO_TRY(gemm_umma_grouped(ds, s, status));
+  // copies and transposes of Y
+  std::vector<const CholQrJob*> post;
+  for (const CholQrJob& jb : jobs)
+    if (jb.Y2 || jb.Yt || jb.Ytb) post.push_back(&jb);
+  for (size_t c0 = 0; c0 < post.size(); c0 += kChunk) {
+    const int cn = (int)(post.size() - c0 < (size_t)kChunk ? post.size() - c0 : kChunk);
+    PostBatch pb;
+    pb.njob = cn;
+    pb.start[0] = 0;
+    for (int i = 0; i < cn; ++i) {
+      const CholQrJob& jb = *post[c0 + i];
+      pb.Y[i] = jb.Y;
+      pb.ldy[i] = jb.ldy;
+      pb.Y2[i] = jb.Y2;
+      pb.ldy2[i] = jb.ldy2;
+      pb.Yt[i] = jb.Yt;
+      pb.ldyt[i] = jb.ldyt;
+      pb.Ytb[i] = jb.Ytb;
+      pb.ldytb[i] = jb.ldytb;
+      pb.r[i] = jb.r;
+      pb.L[i] = jb.L;
+      pb.start[i + 1] = pb.start[i] + ceil_div(jb.r, 32) * ceil_div(jb.L, 32);
+    }
+    post_kernel<<<grid_cap(pb.start[cn], 1), 256, 0, s>>>(pb);
     OUO_CHECK_LAUNCH();
   }
   return OUO_OK;

@@ -100,9 +100,11 @@ struct DGroup {
   int ks1 = 1, ks2 = 1;      // K splits of Pt = Qt B^T and Rt = Pt B
   Buf Pt, P, Rt, Qn;         // r x m, m x r, r x n, r x n per member
   Buf Pb, Rtb;               // bf16 copies of P and Rt (the M update's operands)
+  Buf T;                     // r x max(m, n): the first CholeskyQR pass's output
   Buf kp1, kp2;              // split-K partials (the same memory)
   float* lo = nullptr;       // Gram residual operands (the same memory again)
   Buf S, Lb, Ld;             // r x r summed Gram; R x R factors
+  float* Z = nullptr;        // L^-1 planes, cholqr_z_floats(r) per member
   float* gpart = nullptr;    // Gram partials, gstride floats per member
   int64_t gstride = 0;
   char* ctl = nullptr;       // cooperative Cholesky control (r > 256)
@@ -151,6 +153,7 @@ std::vector<DGroup> plan(const ouo_mat* M, int nmat, const int* ranks, Arena& ar
     g.Qn = ar.take(OUO_F32, nb, r, n);
     g.Pb = ar.take(OUO_BF16, nb, m, r);
     g.Rtb = ar.take(OUO_BF16, nb, r, n);
+    g.T = ar.take(OUO_F32, nb, r, m > n ? m : n);
     {
       // the two partial sets and the Gram residuals are used one after the
       // other: one region (residuals of member i at i times the stride of
@@ -158,7 +161,8 @@ std::vector<DGroup> plan(const ouo_mat* M, int nmat, const int* ranks, Arena& ar
       const int64_t f1 = g.ks1 > 1 ? g.ks1 * (int64_t)r * pitch4(m) : 0;
       const int64_t f2 = g.ks2 > 1 ? g.ks2 * (int64_t)r * pitch4(n) : 0;
       int64_t f = f1 > f2 ? f1 : f2;
-      const int64_t xs[4] = {g.Pt.stride, g.Rt.stride, g.Qn.stride, (int64_t)r * pitch4(n)};
+      const int64_t xs[5] = {g.Pt.stride, g.Rt.stride, g.Qn.stride, g.T.stride,
+                             (int64_t)r * pitch4(n)};
       for (int64_t x : xs) f = x > f ? x : f;
       Buf region = take_bytes(ar, (size_t)nb * (size_t)f * 4 + 256);
       g.lo = reinterpret_cast<float*>(region.p);
@@ -181,6 +185,7 @@ std::vector<DGroup> plan(const ouo_mat* M, int nmat, const int* ranks, Arena& ar
     g.gpart = reinterpret_cast<float*>(take_bytes(ar, (size_t)nb * g.gstride * 4).p);
     g.S = ar.take(OUO_F32, nb, r, r);
     g.Lb = ar.take(OUO_F32, nb, R, R);
+    g.Z = reinterpret_cast<float*>(take_bytes(ar, (size_t)nb * cholqr_z_floats(r) * 4).p);
     if (!cholqr_small_rank(r)) {
       g.Ld = ar.take(OUO_F32, nb, R, R);
       g.ctl_stride = align_up(chol_blocked_ctl_bytes(r), 256);
@@ -289,7 +294,7 @@ int orth_pass(std::vector<CholQrJob>& jobs, const std::vector<const DGroup*>& ow
   if (jobs.empty()) return OUO_OK;
   if (!gram_done) OUO_TRY(cholqr_gram(jobs, status, s));
   OUO_TRY(orth_factor(jobs, owner, mem, status, s));
-  return cholqr_apply(jobs, s);
+  return cholqr_apply(jobs, status, s);
 }
 
 // A CholeskyQR job on member i of group g (rows X, length L; the members'
@@ -305,6 +310,7 @@ CholQrJob orth_job(const DGroup& g, int64_t i, const float* X, int64_t ldx, int6
   j.L = L;
   j.Xlo = g.lo + i * xstride;
   j.gpart = g.gpart + i * cholqr_gram_part_floats(g.r, L);
+  j.Z = g.Z + i * (int64_t)cholqr_z_floats(g.r);
   j.S = reinterpret_cast<float*>(view(g.S, i, 1).p);
   j.Lb = reinterpret_cast<float*>(view(g.Lb, i, 1).p);
   j.Dd = g.Ld.p ? reinterpret_cast<const float*>(view(g.Ld, i, 1).p) : nullptr;
@@ -344,8 +350,9 @@ int stage_project(const std::vector<DGroup>& gs, const ouo_mat* M, const ouo_mat
   return rows_reduce(red, 0.f, s);
 }
 
-// Stage: passes pass_from .. pass_to - 1 of CholeskyQR2 on every Pt, in
-// place; the second solve also writes P = Pt^T.
+// Stage: passes pass_from .. pass_to - 1 of CholeskyQR2 on every Pt: the
+// first pass solves Pt into T, the second T back into Pt and also writes
+// P = Pt^T and its bf16 copy.
 int stage_orth_p(const std::vector<DGroup>& gs, int* status, cudaStream_t s, int pass_from,
                  int pass_to) {
   for (int pass = pass_from; pass < pass_to; ++pass) {
@@ -354,9 +361,10 @@ int stage_orth_p(const std::vector<DGroup>& gs, int* status, cudaStream_t s, int
     std::vector<int64_t> mem;
     for (const DGroup& g : gs) {
       for (int64_t i = 0; i < (int64_t)g.members.size(); ++i) {
-        CholQrJob j = orth_job(g, i, fp(g.Pt, i), g.Pt.ld, g.m, g.Pt.stride);
-        j.Y = fp(g.Pt, i);
-        j.ldy = g.Pt.ld;
+        CholQrJob j = pass == 0 ? orth_job(g, i, fp(g.Pt, i), g.Pt.ld, g.m, g.Pt.stride)
+                                : orth_job(g, i, fp(g.T, i), g.T.ld, g.m, g.T.stride);
+        j.Y = pass == 0 ? fp(g.T, i) : fp(g.Pt, i);
+        j.ldy = pass == 0 ? g.T.ld : g.Pt.ld;
         if (pass == 1) {
           j.Yt = fp(g.P, i);
           j.ldyt = g.P.ld;
@@ -489,13 +497,13 @@ int stage_qnew(const std::vector<DGroup>& gs, Rtp rt, const ouo_mat* Q_state,
             if (d >= xst && d <= g.Rt.stride) xst = d;
           }
         } else {
-          x = fp(g.Qn, i);
-          ld = g.Qn.ld;
-          xst = g.Qn.stride;
+          x = fp(g.T, i);
+          ld = g.T.ld;
+          xst = g.T.stride;
         }
         CholQrJob j = orth_job(g, i, x, ld, g.n, xst);
-        j.Y = fp(g.Qn, i);
-        j.ldy = g.Qn.ld;
+        j.Y = pass == 0 ? fp(g.T, i) : fp(g.Qn, i);
+        j.ldy = pass == 0 ? g.T.ld : g.Qn.ld;
         if (pass == 1) {
           const int bi = g.members[i];
           j.Y2 = reinterpret_cast<float*>(Q_state[bi].ptr);
@@ -795,13 +803,16 @@ std::vector<int64_t> red_offsets(const ouo_mat* M, const std::vector<int>& ranks
   return off;
 }
 
-// The Gram matrices of every Pt, summed into S = the matrix's block of red.
-int gram_into_red(const std::vector<DGroup>& gs, float* red, const std::vector<int64_t>& off,
-                  int64_t (*rows_of)(const DGroup&), int* status, cudaStream_t s) {
+// The Gram matrices of every member's rows in `which` (Pt, or T after the
+// first solve), summed into S = the matrix's block of red.
+int gram_into_red(const std::vector<DGroup>& gs, Buf DGroup::*which, float* red,
+                  const std::vector<int64_t>& off, int64_t (*rows_of)(const DGroup&),
+                  int* status, cudaStream_t s) {
   std::vector<CholQrJob> jobs;
   for (const DGroup& g : gs) {
+    const Buf& x = g.*which;
     for (int64_t i = 0; i < (int64_t)g.members.size(); ++i) {
-      CholQrJob j = orth_job(g, i, fp(g.Pt, i), g.Pt.ld, rows_of(g), g.Pt.stride);
+      CholQrJob j = orth_job(g, i, fp(x, i), x.ld, rows_of(g), x.stride);
       j.S = red + off[g.members[i]];
       jobs.push_back(j);
     }
@@ -812,8 +823,9 @@ int gram_into_red(const std::vector<DGroup>& gs, float* red, const std::vector<i
 int64_t local_rows(const DGroup& g) { return g.m; }
 
 // orth1 (second = false) and orth2 (second = true): Cholesky of the summed
-// Gram matrices in red, the solve on the local rows of Pt, then red = the
-// next pass's Gram matrices (orth1) or P^T B (orth2).
+// Gram matrices in red, the solve on the local rows (Pt into T, then T
+// back into Pt, as in the unsharded step), then red = the next pass's Gram
+// matrices (orth1) or P^T B (orth2).
 int shard_orth(const ouo_mat* M, const ouo_mat* Q_state, int nmat,
                const ouo_dion_params* p, const int64_t* rows_total, void* ws,
                size_t ws_bytes, float* red, int* dev_status, void* stream, bool second) {
@@ -838,10 +850,12 @@ int shard_orth(const ouo_mat* M, const ouo_mat* Q_state, int nmat,
     for (int64_t i = 0; i < (int64_t)g.members.size(); ++i) {
       const int bi = g.members[i];
       // the shift of a retry takes the global row count
-      CholQrJob j = orth_job(g, i, fp(g.Pt, i), g.Pt.ld, rows_total[bi], g.Pt.stride);
+      const Buf& x = second ? g.T : g.Pt;
+      const Buf& y = second ? g.Pt : g.T;
+      CholQrJob j = orth_job(g, i, fp(x, i), x.ld, rows_total[bi], x.stride);
       j.S = red + off[bi];
-      j.Y = fp(g.Pt, i);
-      j.ldy = g.Pt.ld;
+      j.Y = fp(y, i);
+      j.ldy = y.ld;
       if (second) {
         j.Yt = fp(g.P, i);
         j.ldyt = g.P.ld;
@@ -861,8 +875,8 @@ int shard_orth(const ouo_mat* M, const ouo_mat* Q_state, int nmat,
     for (const DGroup& g : gs)
       for (int64_t i = 0; i < (int64_t)g.members.size(); ++i) jobs[k++].L = g.m;
   }
-  OUO_TRY(cholqr_apply(jobs, s));
-  if (!second) return gram_into_red(gs, red, off, local_rows, dev_status, s);
+  OUO_TRY(cholqr_apply(jobs, dev_status, s));
+  if (!second) return gram_into_red(gs, &DGroup::T, red, off, local_rows, dev_status, s);
   auto dst = [&](const DGroup& g, int64_t i, int64_t* ld) {
     *ld = pitch4(g.n);
     return red + off[g.members[i]];
@@ -915,7 +929,7 @@ extern "C" int dion_shard_project(const ouo_mat* M, const ouo_mat* G, int g_dtyp
   Arena ar{reinterpret_cast<char*>(ws), ws_bytes, 0, false};
   const std::vector<DGroup> gs = plan(M, nmat, ranks.data(), ar);
   OUO_TRY(stage_project(gs, M, Q_state, dev_status, s));
-  return gram_into_red(gs, red, red_offsets(M, ranks), local_rows, dev_status, s);
+  return gram_into_red(gs, &DGroup::Pt, red, red_offsets(M, ranks), local_rows, dev_status, s);
 }
 
 extern "C" int dion_shard_orth1(const ouo_mat* M, const ouo_mat* Q_state, int nmat,

@@ -93,9 +93,9 @@ struct Segment {
   int64_t kbc;
   int64_t tiles_2d;  // output tiles of one matrix (tiles_per_mat / ksplit)
   // split-tf32 passes: the K blocks are walked `npass` times; pass q reads
-  // A from UmmaArgs::lo_map[segment][0] when bit q of a_lo is set (B from
-  // lo_map[segment][1] for b_lo)
-  int npass, a_lo, b_lo;
+  // A from UmmaArgs::lo_map[segment][0] when bit q of a_lo is set (from
+  // lo_map[segment][2] for a_lo2), B from lo_map[segment][1] for b_lo
+  int npass, a_lo, b_lo, a_lo2;
 };
 
 constexpr int kMaxSeg = 6;
@@ -116,9 +116,9 @@ struct UmmaArgs {
   // per-matrix alpha of direct outputs (has_dalpha), else `alpha` for all
   float dalpha[kChunk];
   int has_dalpha;
-  // residual operands of the split-tf32 passes, per segment (A, B); kept
-  // out of Segment so that the fields every tile reads stay compact
-  CUtensorMap lo_map[kMaxSeg][2];
+  // residual operands of the split-tf32 passes, per segment (A2, B2, A3);
+  // kept out of Segment so that the fields every tile reads stay compact
+  CUtensorMap lo_map[kMaxSeg][3];
 };
 static_assert(sizeof(UmmaArgs) <= 32764, "kernel parameters above the 32 KB limit");
 
@@ -398,7 +398,8 @@ umma_gemm_kernel(const __grid_constant__ UmmaArgs a) {
           ok = false;
           break;
         }
-        const CUtensorMap* mA = ((sg.a_lo >> pass) & 1) ? &a.lo_map[g][0] : &sg.tmA;
+        const CUtensorMap* mA = ((sg.a_lo2 >> pass) & 1) ? &a.lo_map[g][2]
+                                : ((sg.a_lo >> pass) & 1) ? &a.lo_map[g][0] : &sg.tmA;
         const CUtensorMap* mB = ((sg.b_lo >> pass) & 1) ? &a.lo_map[g][1] : &sg.tmB;
         // Upper-stored symmetric operands: a K stage left of the tile's block
         // diagonal (256-wide blocks, pair tiles) comes from the transposed
@@ -1230,17 +1231,20 @@ int launch(const std::vector<GemmDesc>& gs, cudaStream_t stream, int* status) {
       return make_map(m, b, kRowBytes / es, bk, mn_swz);
     };
     OUO_TRY(make_b(&proto.tmB, g.B));
-    CUtensorMap lo_a, lo_b;
+    CUtensorMap lo_a, lo_b, lo_a3;
     memset(&lo_a, 0, sizeof(lo_a));
     memset(&lo_b, 0, sizeof(lo_b));
+    memset(&lo_a3, 0, sizeof(lo_a3));
     proto.npass = g.npass < 1 ? 1 : g.npass;
     if (proto.npass > 1) {
       if (FMT != 2 || proto.npass > 3 || g.a_sym || g.b_sym)
         return set_error(OUO_ERR_INVALID_ARG, "split-tf32 passes: tf32, 2 or 3 passes, "
                                               "no upper-stored operands");
       proto.a_lo = g.a_lo & ((1 << proto.npass) - 1);
+      proto.a_lo2 = g.a_lo2 & ((1 << proto.npass) - 1) & ~proto.a_lo;
       proto.b_lo = g.b_lo & ((1 << proto.npass) - 1);
       if (proto.a_lo) OUO_TRY(make_map(&lo_a, g.A2, bk, kTileM));
+      if (proto.a_lo2) OUO_TRY(make_map(&lo_a3, g.A3, bk, kTileM));
       if (proto.b_lo) OUO_TRY(make_b(&lo_b, g.B2));
     }
     proto.M = g.M; proto.N = g.N; proto.K = g.K;
@@ -1288,6 +1292,7 @@ int launch(const std::vector<GemmDesc>& gs, cudaStream_t stream, int* status) {
       if (tabled && nb > kChunk - ndirect) nb = kChunk - ndirect;
       a.lo_map[a.nseg][0] = lo_a;
       a.lo_map[a.nseg][1] = lo_b;
+      a.lo_map[a.nseg][2] = lo_a3;
       Segment& sg = a.seg[a.nseg++];
       sg = proto;
       sg.b0 = b0;

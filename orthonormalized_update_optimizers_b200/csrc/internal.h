@@ -115,15 +115,16 @@ struct GemmDesc {
   bool pair_mn = false;
   // Split-tf32 passes (tf32 operands, no symmetric operands): the K range is
   // run `npass` times (1 to 3) into one accumulator; in pass q the A
-  // operand is A2 instead of A when bit q of a_lo is set, and likewise B2
-  // for b_lo.  With A2 / B2 holding the residuals x - tf32(x) of A / B, the
-  // passes (A, B), (A, B2), (A2, B) give the product to about fp32 accuracy
-  // (the tensor core reads A and B truncated to tf32; the residual-residual
-  // term, 2^-20 relative, is left out).  A2 / B2 have the shapes, leading
-  // dimensions and batch strides of A / B.
+  // operand is A2 instead of A when bit q of a_lo is set (A3 for a_lo2),
+  // and B2 instead of B for b_lo.  With A2 / B2 holding the residuals
+  // x - tf32(x) of A / B, the passes (A, B), (A, B2), (A2, B) give the
+  // product to about fp32 accuracy (the tensor core reads A and B truncated
+  // to tf32; the residual-residual term, 2^-20 relative, is left out).
+  // A2, A3 / B2 have the shapes, leading dimensions and batch strides of
+  // A / B.
   int npass = 1;
-  Buf A2, B2;
-  int a_lo = 0, b_lo = 0;
+  Buf A2, B2, A3;
+  int a_lo = 0, b_lo = 0, a_lo2 = 0;
 };
 
 // Number of K ranges a split-K GEMM of depth K over `dtype` operands
@@ -179,14 +180,16 @@ struct CholQrJob {
   int64_t ldx = 0;
   int r = 0;
   int64_t L = 0;
-  float* Xlo = nullptr;      // Gram: residual operand, r x L, row pitch ldx
+  float* Xlo = nullptr;      // 2 (X - tf32(X)), r x L, row pitch ldx: written
+                             // by the Gram, read again by the solve
   float* gpart = nullptr;    // Gram partials, cholqr_gram_part_floats(r, L)
   float* S = nullptr;        // summed Gram, r x r, full symmetric storage
   float* Lb = nullptr;       // R x R (R = r rounded up to 32), ld R: the
                              // strictly lower 32 x 32 blocks of L
   const float* Dd = nullptr; // R x R, ld R: D_i = L_ii^-1 on the diagonal
                              // blocks (nullptr: they are in Lb)
-  float* Y = nullptr;        // L^-1 X, r x L (may be X itself)
+  float* Z = nullptr;        // cholqr_z_floats(r): L^-1 in three planes
+  float* Y = nullptr;        // L^-1 X, r x L (apart from X)
   int64_t ldy = 0;
   float* Y2 = nullptr;       // optional copy of Y
   int64_t ldy2 = 0;
@@ -211,8 +214,14 @@ bool cholqr_small_rank(int r);
 // CTA per job, r <= 256; breakdown after the shifted retry sets
 // OUO_STATUS_BREAKDOWN and writes the identity.
 int cholqr_factor(const std::vector<CholQrJob>& jobs, int* status, cudaStream_t s);
-// Y = L^-1 X (and Y2, Yt) for every job, r <= 1024.
-int cholqr_apply(const std::vector<CholQrJob>& jobs, cudaStream_t s);
+// Floats of a job's Z (three R x R planes, R = r rounded up to 32).
+size_t cholqr_z_floats(int r);
+// Y = L^-1 X (and Y2, Yt, Ytb) for every job, r <= 1024: Z = L^-1, then
+// the product on the tensor cores in split-tf32 passes, reading the
+// residuals the job's Gram left in Xlo.  A run of jobs whose X, Xlo, Y and
+// Z are evenly strided (X and Xlo by the same step, Z by cholqr_z_floats)
+// is one GEMM descriptor.
+int cholqr_apply(const std::vector<CholQrJob>& jobs, int* status, cudaStream_t s);
 
 // Rows of the sum of `ks` partial matrices (sp floats apart, row pitch
 // ldp), with optional row norms (float64, fixed order) and normalized rows
