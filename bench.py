@@ -167,9 +167,14 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
+    t_warm = time.perf_counter()
     for _ in range(args.warmup):
         _oracle_sample(args, n_matrices=1, first=1)  # k projection, 1024 x 4096
-    per_step = [cpu_baseline(args)["value"] for _ in range(args.steps)]
+    t_warm = time.perf_counter() - t_warm
+    per_step, measured = [], []
+    for _ in range(args.steps):
+        per_step.append(cpu_baseline(args)["value"])
+        measured.append(cpu_baseline.last_seconds)
     ms = statistics.median(per_step)
     line = cpu_baseline.last
     line = dict(line, value=round(ms, 3))
@@ -183,6 +188,14 @@ def run_reference(args):
         "cpu_baseline": line,
         "e2e": {"value": round(ms, 3), "unit": "ms", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
+        # what actually ran: each "step" is one sample of 7 * cpu_sample_layers
+        # matrices, timed and scaled to the whole parameter set
+        "samples_run": {"count": args.steps, "matrices_each": 7 * args.cpu_sample_layers,
+                        "scale_each": len(_workload_shapes(args.layers)) /
+                                      (7 * args.cpu_sample_layers),
+                        "measured_s": [round(x, 3) for x in measured],
+                        "measured_s_total": round(sum(measured), 3),
+                        "warmup_s": round(t_warm, 3)},
     }
     print(json.dumps(out), flush=True)
 
@@ -228,6 +241,7 @@ def cpu_baseline(args):
                       f"extrapolated x{scale:g} to all {len(shapes)} matrices",
             "extrapolated": scale != 1.0}
     cpu_baseline.last = line
+    cpu_baseline.last_seconds = t_total
     return line
 
 

@@ -144,6 +144,24 @@ def test_orth_dion_rank_1024():
         assert e_m <= TOL_BF16 and e_q <= TOL_BF16 and e_w <= TOL_BF16, errs
 
 
+@pytest.mark.parametrize("r", [64, 256])
+def test_cholesky_qr2_reaches_fp32_orthonormality(r):
+    # The CholeskyQR2 of the right factor runs its Gram matrices and solves
+    # as split-tf32 tensor-core products; plain tf32 would leave
+    # ||Q Q^T - I|| near 1e-3, fp32-level products near 1e-6.
+    m, n = 1024, 2048
+    G = synth.lowrank_plus_noise(m, n, 32, 0.02, 91 + r, torch.bfloat16, DEV)
+    M = torch.zeros(m, n, dtype=torch.float32, device=DEV)
+    W = torch.zeros(m, n, dtype=torch.float32, device=DEV)
+    Qt = torch.tensor(_q0(n, r).T.copy(), device=DEV)
+    p = ouo.dion_params(rank=r, lr=1.0, norm_mode="qr")
+    for _ in range(2):
+        ouo.dion_lowrank_step([M], [G], [Qt], [W], p)
+    torch.cuda.synchronize()
+    q = to64(Qt)
+    assert np.max(np.abs(q @ q.T - np.eye(r))) <= 1e-5
+
+
 def test_dion_orthonormal_factors_and_isometry():
     # Orth-Dion's update is a partial isometry: singular values of the
     # applied update P Q^T all equal one (nu_t = 1).
