@@ -298,6 +298,42 @@ __device__ __forceinline__ void sub_rowdot8(float* Tt, const float* A, const flo
       make_float4(s1.x - acc[4], s1.y - acc[5], s1.z - acc[6], s1.w - acc[7]);
 }
 
+// C -= A B^T for whole 32 x 32 blocks (pitch kP), one warp: lane (lr, lc)
+// = (lane / 8, lane % 8) owns rows lr + 4u (u < 8) and columns lc + 8v
+// (v < 4), so that its operands come as float4 runs along k: per four k,
+// 8 reads of A and 4 of B (bank-conflict free: the rows a read instruction
+// touches are four consecutive rows, the columns eight consecutive ones)
+// for 128 FMAs.
+__device__ __forceinline__ void sub_blk32(float* C, const float* A, const float* B) {
+  const int lane = threadIdx.x & 31, lr = lane >> 3, lc = lane & 7;
+  float acc[8][4];
+#pragma unroll
+  for (int u = 0; u < 8; ++u)
+#pragma unroll
+    for (int v = 0; v < 4; ++v) acc[u][v] = 0.f;
+#pragma unroll 2
+  for (int k = 0; k < kB; k += 4) {
+    float4 b4[4];
+#pragma unroll
+    for (int v = 0; v < 4; ++v) b4[v] = *reinterpret_cast<const float4*>(B + (lc + 8 * v) * kP + k);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const float4 a4 = *reinterpret_cast<const float4*>(A + (lr + 4 * u) * kP + k);
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        acc[u][v] = fmaf(a4.x, b4[v].x, acc[u][v]);
+        acc[u][v] = fmaf(a4.y, b4[v].y, acc[u][v]);
+        acc[u][v] = fmaf(a4.z, b4[v].z, acc[u][v]);
+        acc[u][v] = fmaf(a4.w, b4[v].w, acc[u][v]);
+      }
+    }
+  }
+#pragma unroll
+  for (int u = 0; u < 8; ++u)
+#pragma unroll
+    for (int v = 0; v < 4; ++v) C[(lr + 4 * u) * kP + lc + 8 * v] -= acc[u][v];
+}
+
 __global__ void __launch_bounds__(kCT, 1) chol_kernel(const __grid_constant__ CholBatch cb) {
   extern __shared__ __align__(16) float sm[];
   __shared__ int s_bad;
@@ -396,13 +432,13 @@ __global__ void __launch_bounds__(kCT, 1) chol_kernel(const __grid_constant__ Ch
           s_bad = 1;
       }
       if (warp > 0) {
-        // trailing: S(p+1+bi, p+1+bj) -= pan[bi] pan[bj]^T, bj <= bi, except (0, 0)
+        // trailing: S(p+1+bi, p+1+bj) -= pan[bi] pan[bj]^T, bj <= bi, except
+        // (0, 0): whole blocks per warp
         const int tasks = m * (m + 1) / 2 - 1;
-        for (int it = warp - 1; it < 4 * tasks; it += kCW - 1) {
-          const int tt = (it >> 2) + 1, c0 = (it & 3) * 8;
+        for (int it = warp - 1; it < tasks; it += kCW - 1) {
+          const int tt = it + 1;
           const int bi = tri_row_of(tt), bj = tt - bi * (bi + 1) / 2;
-          sub_rowdot8(tile(p + 1 + bi, p + 1 + bj), pan + (size_t)bi * kTF,
-                      pan + (size_t)bj * kTF, c0);
+          sub_blk32(tile(p + 1 + bi, p + 1 + bj), pan + (size_t)bi * kTF, pan + (size_t)bj * kTF);
         }
       }
       __syncthreads();
