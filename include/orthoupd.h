@@ -295,7 +295,9 @@ int apply_update(const ouo_mat* W, int w_dtype, const ouo_mat* O, int o_dtype,
  *   B = M + G;  P = orth(B Q_prev);  R = B^T P;
  *   Q_new = ColNorm(R) or orth(R);   M <- beta B - (beta - mu) P R^T;
  *   W <- (1 - lr wd) W - lr scale P Q_new^T;  Q_state <- Q_new
- * orth() is the QR factor with positive R diagonal (CholeskyQR2 in fp32).
+ * orth() is the QR factor with positive R diagonal (CholeskyQR2 at fp32
+ * accuracy: Gram matrices and solves as split-tf32 tensor-core products,
+ * the Cholesky factor and its inverse in fp32).
  * ColNorm(R)_j = R_j / (||R_j|| + eps).
  * M[i]: fp32 m x n buffer (in/out).  G[i]: m x n, dtype g_dtype.
  * Q_state[i]: fp32, stored TRANSPOSED as r x n (row c = column c of Q),
