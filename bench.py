@@ -930,7 +930,17 @@ def run_micro(args):
         Ms = ouo.batch_empty(shapes, torch.float32, dev)
         Gs = ouo.batch_empty(shapes, torch.bfloat16, dev)
         Ws = ouo.batch_empty(shapes, torch.bfloat16, dev)
-        Qs = ouo.batch_empty([(r, b) for _, b in shapes], torch.float32, dev)
+        # right factors in one block per weight shape (as the bench line's
+        # grouped measurement lays them out), so that every group's Q_state
+        # is evenly strided
+        qblk = {}
+        for i, (a, b) in enumerate(shapes):
+            qblk.setdefault((a, b), []).append(i)
+        Qs = [None] * len(shapes)
+        for (a, b), members in qblk.items():
+            blk = torch.empty((len(members), r, b), dtype=torch.float32, device=dev)
+            for k, i in enumerate(members):
+                Qs[i] = blk[k]
         q0 = {}
         for i, (a, b) in enumerate(shapes):
             Gs[i].copy_(synth.lowrank_plus_noise(a, b, 64, 0.02, synth.seed_for(4, 100 + i),
