@@ -493,6 +493,24 @@ __device__ __forceinline__ void trinv_store(const TrinvBatch& tb, int job, int j
   float* Z0 = tb.Z[job];
   const int R = nb * kB;
   const size_t plane = (size_t)R * R;
+  if ((zpitch & 3) == 0) {
+    // 16-byte groups: four consecutive columns of a row per thread
+    for (int bi = 0; bi < nb; ++bi) {
+      for (int e = threadIdx.x; e < 256; e += blockDim.x) {
+        const int a = e >> 3, c = (e & 7) * 4;
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (bi >= j) v = *reinterpret_cast<const float4*>(zc + (size_t)bi * bstride + a * zpitch + c);
+        const size_t off = (size_t)(bi * kB + a) * R + j * kB + c;
+        *reinterpret_cast<float4*>(Z0 + off) = v;
+        *reinterpret_cast<float4*>(Z0 + plane + off) =
+            make_float4(0.5f * v.x, 0.5f * v.y, 0.5f * v.z, 0.5f * v.w);
+        *reinterpret_cast<float4*>(Z0 + 2 * plane + off) =
+            make_float4(v.x - tf32_trunc(v.x), v.y - tf32_trunc(v.y), v.z - tf32_trunc(v.z),
+                        v.w - tf32_trunc(v.w));
+      }
+    }
+    return;
+  }
   for (int bi = 0; bi < nb; ++bi) {
     for (int e = threadIdx.x; e < 1024; e += blockDim.x) {
       const int a = e >> 5, c = e & 31;
@@ -592,7 +610,7 @@ size_t trinv8_smem_bytes(int nb) {
 }
 
 constexpr int kT8 = 512;  // threads of the right-looking inverse
-__global__ void __launch_bounds__(kT8) trinv8_kernel(const __grid_constant__ TrinvBatch tb) {
+__global__ void __launch_bounds__(kT8, 1) trinv8_kernel(const __grid_constant__ TrinvBatch tb) {
   extern __shared__ __align__(16) float z8[];
   const int job = find_job(tb.start, tb.njob, blockIdx.x);
   const int j = (int)(blockIdx.x - tb.start[job]);
@@ -609,45 +627,51 @@ __global__ void __launch_bounds__(kT8) trinv8_kernel(const __grid_constant__ Tri
     return (size_t)((a * (a - 1)) / 2 + (k - j)) * kB4;
   };
   // loads: transposed copies of L_ik and D_i, Z_jj = D_j by rows; entries
-  // outside the r x r matrix, and above a D_i's diagonal, are zero.  Each
-  // thread issues 16 independent loads before it stores any of them.
+  // outside the r x r matrix, and above a D_i's diagonal, are zero.  Blocks
+  // go in groups of 8 (block indices decoded once per block, the same in
+  // every thread); each thread issues its 16 loads of a group before it
+  // stores any of them.
   {
     const int nl = m * (m - 1) / 2;
-    const int total = (nl + m + 1) * 1024;
-    for (int base = threadIdx.x; base < total; base += kT8 * 16) {
+    const int nblk = nl + m + 1;
+    const int w0 = threadIdx.x;  // elements w0 and w0 + 512 of every block
+    int bl_a = 1, bl_q = 0;      // (a, q) of L block index `blk`, walked in order
+    for (int b0 = 0; b0 < nblk; b0 += 8) {
       float v[16];
       float* dst[16];
 #pragma unroll
-      for (int q = 0; q < 16; ++q) {
-        const int e = base + q * kT8;
-        v[q] = 0.f;
-        dst[q] = nullptr;
-        if (e >= total) continue;
-        const int blk = e >> 10, w = e & 1023, a = w >> 5, c = w & 31;
-        int bi, bj;
-        bool lower;
-        if (blk < nl) {
-          int aa = 1, qq = blk;
-          while (qq >= aa) { qq -= aa; ++aa; }
-          bi = j + aa;
-          bj = j + qq;
-          dst[q] = lt + (size_t)blk * kB4 + c * kP4 + a;
-          lower = false;
-        } else if (blk < nl + m) {
+      for (int t = 0; t < 8; ++t) {
+        const int blk = b0 + t;
+        int bi = 0, bj = 0;
+        bool lower = false, trans = true, valid = blk < nblk;
+        float* base = nullptr;
+        if (valid && blk < nl) {
+          bi = j + bl_a;
+          bj = j + bl_q;
+          base = lt + (size_t)blk * kB4;
+          if (++bl_q == bl_a) { bl_q = 0; ++bl_a; }
+        } else if (valid && blk < nl + m) {
           bi = bj = j + (blk - nl);
-          dst[q] = dt + (size_t)(blk - nl) * kB4 + c * kP4 + a;
+          base = dt + (size_t)(blk - nl) * kB4;
           lower = true;
-        } else {
+        } else if (valid) {
           bi = bj = j;
-          dst[q] = zc + (size_t)j * kB4 + a * kP4 + c;
+          base = zc + (size_t)j * kB4;
           lower = true;
+          trans = false;
         }
-        const int gi = bi * kB + a, gc = bj * kB + c;
-        if (gi < r && gc < r && (!lower || c <= a)) v[q] = (lower ? Dd : Lb)[(size_t)gi * R + gc];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int w = w0 + 512 * h, a = w >> 5, c = w & 31;
+          const int gi = bi * kB + a, gc = bj * kB + c;
+          v[2 * t + h] = valid && gi < r && gc < r && (!lower || c <= a)
+                             ? (lower ? Dd : Lb)[(size_t)gi * R + gc] : 0.f;
+          dst[2 * t + h] = valid ? base + (trans ? c * kP4 + a : a * kP4 + c) : nullptr;
+        }
       }
 #pragma unroll
-      for (int q = 0; q < 16; ++q)
-        if (dst[q]) *dst[q] = v[q];
+      for (int t = 0; t < 16; ++t)
+        if (dst[t]) *dst[t] = v[t];
     }
   }
   __syncthreads();
