@@ -890,6 +890,18 @@ int set_smem_attr(const void* fn, size_t bytes) {
 
 }  // namespace
 
+namespace {
+// Distance in floats from a to b (addresses compared as integers: the two
+// may lie in different allocations), and whether b sits d * step floats
+// after a.
+int64_t fdist(const void* a, const void* b) {
+  return ((int64_t)(uintptr_t)b - (int64_t)(uintptr_t)a) / (int64_t)sizeof(float);
+}
+bool at_step(const void* a, const void* b, int64_t d, int64_t step) {
+  return (int64_t)(uintptr_t)b - (int64_t)(uintptr_t)a == d * step * (int64_t)sizeof(float);
+}
+}  // namespace
+
 int cholqr_gram_ksplit(int r, int64_t L) {
   (void)r;
   // K ranges of at least 32 tf32 K blocks (the two passes counted), at
@@ -939,15 +951,15 @@ int cholqr_gram(const std::vector<CholQrJob>& jobs, int* status, cudaStream_t s)
     size_t e = k + 1;
     int64_t xs = 0, ls = 0;
     if (e < jobs.size()) {
-      xs = jobs[e].X - j0.X;
-      ls = jobs[e].Xlo - j0.Xlo;
+      xs = fdist(j0.X, jobs[e].X);
+      ls = fdist(j0.Xlo, jobs[e].Xlo);
     }
     while (e < jobs.size()) {
       const CholQrJob& je = jobs[e];
       const int64_t d = (int64_t)(e - k);
       if (je.r != j0.r || je.L != j0.L || je.ldx != j0.ldx || xs < j0.r * j0.ldx ||
-          xs != ls || je.X != j0.X + d * xs || je.Xlo != j0.Xlo + d * ls ||
-          je.gpart != j0.gpart + d * pf)
+          xs != ls || !at_step(j0.X, je.X, d, xs) || !at_step(j0.Xlo, je.Xlo, d, ls) ||
+          !at_step(j0.gpart, je.gpart, d, pf))
         break;
       ++e;
     }
@@ -1084,18 +1096,18 @@ int cholqr_apply(const std::vector<CholQrJob>& jobs, int* status, cudaStream_t s
     size_t e = k + 1;
     int64_t xs = 0, ys = 0, ls = 0, zs = 0;
     if (e < jobs.size()) {
-      xs = jobs[e].X - j0.X;
-      ys = jobs[e].Y - j0.Y;
-      ls = jobs[e].Xlo - j0.Xlo;
-      zs = jobs[e].Z - j0.Z;
+      xs = fdist(j0.X, jobs[e].X);
+      ys = fdist(j0.Y, jobs[e].Y);
+      ls = fdist(j0.Xlo, jobs[e].Xlo);
+      zs = fdist(j0.Z, jobs[e].Z);
     }
     while (e < jobs.size()) {
       const CholQrJob& je = jobs[e];
       const int64_t d = (int64_t)(e - k);
       if (je.r != j0.r || je.L != j0.L || je.ldx != j0.ldx || je.ldy != j0.ldy ||
           xs < j0.r * j0.ldx || ys < j0.r * j0.ldy || xs != ls || zs != zf ||
-          je.X != j0.X + d * xs || je.Xlo != j0.Xlo + d * ls || je.Y != j0.Y + d * ys ||
-          je.Z != j0.Z + d * zs)
+          !at_step(j0.X, je.X, d, xs) || !at_step(j0.Xlo, je.Xlo, d, ls) ||
+          !at_step(j0.Y, je.Y, d, ys) || !at_step(j0.Z, je.Z, d, zs))
         break;
       ++e;
     }
