@@ -303,7 +303,15 @@ int apply_update(const ouo_mat* W, int w_dtype, const ouo_mat* O, int o_dtype,
  * Q_state[i]: fp32, stored TRANSPOSED as r x n (row c = column c of Q),
  * in/out; the caller initializes it with orthonormal rows.
  * W[i]: m x n, dtype w_dtype (in/out).  scale: host float[nmat] or NULL.
- * ws / ws_bytes: at least dion_workspace_bytes(...) bytes.
+ * ws / ws_bytes: at least dion_workspace_bytes(...) bytes, 256-byte aligned
+ * (about 4 to 5 r (m + n) floats per matrix: the projections and their
+ * bf16 copies, the CholeskyQR buffers, Gram and split-K partials; 12.9 GB
+ * for the 224-matrix Llama-3-8B-shaped set at r = 256).  The workspace holds no
+ * state between calls, except in the row-sharded step below.
+ * Matrices of the same (rows, cols, rank) run as one group; when their M,
+ * G, Q_state and W each sit evenly strided in memory, every stage of the
+ * group is one descriptor of a grouped launch, and a matrix gives the same
+ * bits alone as in any batch.
  */
 size_t dion_workspace_bytes(const ouo_mat* M, int nmat,
                             const ouo_dion_params* p);
