@@ -23,13 +23,13 @@ def _q0(n, r, seed=1):
 
 
 def _run(m, n, r, mode, steps, seed, w_dtype=torch.float32, beta=1.0,
-         mu=0.95, lr=0.01, scale=1.0, g_same=True):
+         mu=0.95, lr=0.01, scale=1.0, g_same=True, wd=0.0):
     G = synth.lowrank_plus_noise(m, n, min(64, m, n), 0.02, seed, torch.bfloat16, DEV)
     M = torch.zeros(m, n, dtype=torch.float32, device=DEV)
     W = synth.gaussian((m, n), seed + 7, 0.02, w_dtype, DEV)
     q0 = _q0(n, r)
     Qt = torch.tensor(q0.T.copy(), device=DEV)  # state is r x n (Q transposed)
-    p = ouo.dion_params(rank=r, mu=mu, beta=beta, lr=lr,
+    p = ouo.dion_params(rank=r, mu=mu, beta=beta, lr=lr, wd=wd,
                         norm_mode="qr" if mode == odion.QR else "colnorm")
     status = torch.zeros(1, dtype=torch.int32, device=DEV)
     Mr = np.zeros((m, n), dtype=np.float32)
@@ -43,7 +43,7 @@ def _run(m, n, r, mode, steps, seed, w_dtype=torch.float32, beta=1.0,
         ouo.dion_lowrank_step([M], [Gs], [Qt], [W], p, scale=[scale], status=status)
         torch.cuda.synchronize()
         assert status.item() == 0
-        ref = odion.dion_step(Mr, to64(Gs), Qr, Wr, mu, lr, scale, mode, beta=beta)
+        ref = odion.dion_step(Mr, to64(Gs), Qr, Wr, mu, lr, scale, mode, beta=beta, wd=wd)
         e_m = rel_fro(to64(M), ref["M"])
         e_q = rel_fro(to64(Qt).T, ref["Q"])
         W_after = to64(W)
@@ -80,6 +80,15 @@ def test_dion_small(mode, shape, r):
 def test_dion_bf16_weights_and_beta():
     errs = _run(384, 640, 48, odion.QR, steps=2, seed=5, w_dtype=torch.bfloat16,
                 beta=0.5, lr=0.05, scale=2.0)
+    for e_m, e_q, e_w in errs:
+        assert e_m <= TOL_BF16 and e_q <= TOL_BF16 and e_w <= TOL_BF16, errs
+
+
+@pytest.mark.parametrize("mode", [odion.COLNORM, odion.QR])
+def test_dion_weight_decay(mode):
+    # W <- (1 - lr wd) W - lr s P Q_new^T: the decoupled decay rides in the
+    # in-place update's C0 coefficient
+    errs = _run(512, 768, 64, mode, steps=2, seed=31, lr=0.05, wd=0.1, scale=1.5)
     for e_m, e_q, e_w in errs:
         assert e_m <= TOL_BF16 and e_q <= TOL_BF16 and e_w <= TOL_BF16, errs
 
