@@ -23,8 +23,8 @@ def _q0(n, r, seed=1):
 
 
 def _run(m, n, r, mode, steps, seed, w_dtype=torch.float32, beta=1.0,
-         mu=0.95, lr=0.01, scale=1.0, g_same=True, wd=0.0):
-    G = synth.lowrank_plus_noise(m, n, min(64, m, n), 0.02, seed, torch.bfloat16, DEV)
+         mu=0.95, lr=0.01, scale=1.0, g_same=True, wd=0.0, g_dtype=torch.bfloat16):
+    G = synth.lowrank_plus_noise(m, n, min(64, m, n), 0.02, seed, g_dtype, DEV)
     M = torch.zeros(m, n, dtype=torch.float32, device=DEV)
     W = synth.gaussian((m, n), seed + 7, 0.02, w_dtype, DEV)
     q0 = _q0(n, r)
@@ -38,7 +38,7 @@ def _run(m, n, r, mode, steps, seed, w_dtype=torch.float32, beta=1.0,
     errs = []
     for step in range(steps):
         Gs = G if g_same else synth.lowrank_plus_noise(m, n, 64, 0.02, seed + 100 + step,
-                                                       torch.bfloat16, DEV)
+                                                       g_dtype, DEV)
         W_before = to64(W)
         ouo.dion_lowrank_step([M], [Gs], [Qt], [W], p, scale=[scale], status=status)
         torch.cuda.synchronize()
@@ -89,6 +89,14 @@ def test_dion_weight_decay(mode):
     # W <- (1 - lr wd) W - lr s P Q_new^T: the decoupled decay rides in the
     # in-place update's C0 coefficient
     errs = _run(512, 768, 64, mode, steps=2, seed=31, lr=0.05, wd=0.1, scale=1.5)
+    for e_m, e_q, e_w in errs:
+        assert e_m <= TOL_BF16 and e_q <= TOL_BF16 and e_w <= TOL_BF16, errs
+
+
+def test_dion_fp32_gradient():
+    # fp32 gradients take the momentum kernel's fp32 path; the rest of the
+    # step is the same
+    errs = _run(384, 512, 32, odion.QR, steps=2, seed=41, g_dtype=torch.float32)
     for e_m, e_q, e_w in errs:
         assert e_m <= TOL_BF16 and e_q <= TOL_BF16 and e_w <= TOL_BF16, errs
 
