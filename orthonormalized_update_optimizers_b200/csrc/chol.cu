@@ -1,6 +1,6 @@
-// Blocked Cholesky factorization (and optionally the triangular inverse) for
-// CholeskyQR on ranks above 256: one cooperative multi-CTA launch
-// (chol_blocked).  Ranks up to 256 take the one-CTA kernel of cholqr.cu.
+// Blocked Cholesky factorization for CholeskyQR on ranks above 256: one
+// cooperative multi-CTA launch (chol_blocked).  Ranks up to 256 take the
+// one-CTA kernel of cholqr.cu.
 //
 // Source: "Orth-Dion: Eliminating Geometric Mismatch in Distributed Low-Rank
 // Spectral Optimization", Orth-Dion (the right factor, and in Dion the left
@@ -10,25 +10,23 @@
 // diagonal (the unique QR).
 //
 // S arrives as `splits` partial Gram matrices in upper storage (entry (i, j)
-// valid for j >= i), summed here in float64 in a fixed order.  The r x r problem is padded to R = 32 * ceil(r / 32) with an
-// identity block and processed in 32 x 32 blocks:
+// valid for j >= i), summed here in float64 in a fixed order.  The r x r
+// problem is padded to R = 32 * ceil(r / 32) with an identity block and
+// processed in 32 x 32 blocks:
 //   for each block column p:
 //     the diagonal block S_pp = L_pp L_pp^T is factored and inverted
 //       (D_p = L_pp^-1) by one warp, in registers, in every CTA that needs
 //       it (identical bits), and published by CTA 0;
 //     the blocks below it become L_ip = S_ip D_p^T;
-//     the trailing lower blocks are updated S_ij -= L_ip L_jp^T;
-//   then (with `inverse`) L^-1 by recursive doubling over neighbouring
-//   diagonal super-blocks [[A, 0], [B, C]]^-1 = [[A^-1, 0], [-C^-1 B A^-1, C^-1]];
-//   without it the strictly lower blocks L_ij stay in S and the inverted
-//   diagonal blocks D_p in the diagonal blocks of Linv (the form the
-//   batched triangular solve of cholqr.cu reads).
-// In the cooperative kernel phases are separated by a grid barrier whose
-// wait is bounded in time (a barrier that runs out sets OUO_STATUS_TIMEOUT
-// and every later barrier passes at once).  In both kernels a non-positive
-// pivot restarts the factorization once with the shift of shifted
-// CholeskyQR, 11 (L r + r (r + 1)) u tr(S); a second failure sets
-// OUO_STATUS_BREAKDOWN and returns L^-1 = I.
+//     the trailing lower blocks are updated S_ij -= L_ip L_jp^T.
+// The strictly lower blocks L_ij stay in S and the inverted diagonal blocks
+// D_p go to the diagonal blocks of Linv: the form the block inverse of
+// cholqr.cu reads.  Phases are separated by a grid barrier whose wait is
+// bounded in time (a barrier that runs out sets OUO_STATUS_TIMEOUT and
+// every later barrier passes at once).  A non-positive pivot restarts the
+// factorization once with the shift of shifted CholeskyQR,
+// 11 (L r + r (r + 1)) u tr(S); a second failure sets OUO_STATUS_BREAKDOWN
+// and returns L = I.
 #include <atomic>
 #include <cmath>
 
@@ -51,7 +49,6 @@ struct CholBArgs {
   int* flags;         // [0] pivot failed, [1] barrier timed out
   double* diag;       // unshifted diagonal of S (r values)
   int* status;
-  int inverse;        // form L^-1 (else leave L in S and D_p in Linv)
 };
 
 // Grid-wide barrier over all CTAs of the cooperative launch; the wait is
@@ -237,74 +234,6 @@ __device__ void trailing(const CholBArgs& a, int p) {
 }
 
 // Transposed 32 x 32 block into shared memory: t[c][r] = g[r][c].
-__device__ __forceinline__ void load_blk_t(float (*t)[kNb + 1], const float* g, int R) {
-  for (int e = threadIdx.x; e < kNb * kNb; e += blockDim.x) {
-    const int r = e >> 5, c = e & 31;
-    t[c][r] = g[(size_t)r * R + c];
-  }
-}
-
-// L^-1 by recursive doubling over block sizes s = 32, 64, ...: for each
-// pair of neighbouring diagonal super-blocks [[A, 0], [B, C]] with A^-1, C^-1
-// known, the lower-left block of the inverse is -C^-1 (B A^-1).
-//   step 1: T = B A^-1, kept transposed in the unused upper triangle of S
-//           (T[i][j] at S[j][i]);
-//   step 2: Linv_BA = -C^-1 T.
-// Step 1 of super-block size s (in 32-blocks: h = s / 32), pair q.
-__device__ void inv_step1(const CholBArgs& a, int h) {
-  __shared__ float sb[kNb][kNb + 1];
-  __shared__ float sv[kNb][kNb + 1];
-  const int i = threadIdx.x >> 3, j0 = (threadIdx.x & 7) * 4;
-  const int pairs = (a.nblk + 2 * h - 1) / (2 * h);
-  // task = (pair, bi in B's block rows, bj in A's block columns)
-  const int per_pair = h * h;
-  for (int t = blockIdx.x; t < pairs * per_pair; t += gridDim.x) {
-    const int q = t / per_pair, w = t - q * per_pair;
-    const int bi = w / h, bj = w - (w / h) * h;
-    const int a0 = 2 * h * q, c0 = a0 + h;  // first 32-blocks of A and C
-    if (c0 + bi >= a.nblk) continue;        // B row outside the matrix
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int k = bj; k < h; ++k) {           // A^-1 is lower triangular
-      load_blk(sb, blk(a.S, a.R, c0 + bi, a0 + k), a.R);
-      load_blk_t(sv, blk(a.Linv, a.R, a0 + k, a0 + bj), a.R);
-      __syncthreads();
-      mma_bt(sb, sv, acc);
-      __syncthreads();
-    }
-    // T[bi][bj] stored transposed at S block (a0 + bj, c0 + bi)
-    float* g = blk(a.S, a.R, a0 + bj, c0 + bi);
-#pragma unroll
-    for (int u = 0; u < 4; ++u) g[(size_t)(j0 + u) * a.R + i] = acc[u];
-  }
-}
-
-__device__ void inv_step2(const CholBArgs& a, int h) {
-  __shared__ float sc[kNb][kNb + 1];
-  __shared__ float sv[kNb][kNb + 1];
-  const int i = threadIdx.x >> 3, j0 = (threadIdx.x & 7) * 4;
-  const int pairs = (a.nblk + 2 * h - 1) / (2 * h);
-  const int per_pair = h * h;
-  for (int t = blockIdx.x; t < pairs * per_pair; t += gridDim.x) {
-    const int q = t / per_pair, w = t - q * per_pair;
-    const int bi = w / h, bj = w - (w / h) * h;
-    const int a0 = 2 * h * q, c0 = a0 + h;
-    if (c0 + bi >= a.nblk) continue;
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int k = 0; k <= bi; ++k) {          // C^-1 is lower triangular
-      if (c0 + k >= a.nblk) break;
-      load_blk(sc, blk(a.Linv, a.R, c0 + bi, c0 + k), a.R);
-      // T[k][bj] is S block (a0 + bj, c0 + k) transposed, which is the B^T
-      // form mma_bt wants as is
-      load_blk(sv, blk(a.S, a.R, a0 + bj, c0 + k), a.R);
-      __syncthreads();
-      mma_bt(sc, sv, acc);
-      __syncthreads();
-    }
-    float* g = blk(a.Linv, a.R, c0 + bi, a0 + bj);
-#pragma unroll
-    for (int u = 0; u < 4; ++u) g[(size_t)i * a.R + j0 + u] = -acc[u];
-  }
-}
 
 // tr(S) from the diagonal kept by assemble(); every CTA forms the same sum
 // in the same (fixed) order.
@@ -367,14 +296,7 @@ __global__ void __launch_bounds__(kCholThreads) chol_blocked_kernel(const CholBA
          e += (size_t)gridDim.x * blockDim.x) {
       const int i = (int)(e / a.R), j = (int)(e - (e / a.R) * a.R);
       a.Linv[e] = i == j ? 1.f : 0.f;
-      if (!a.inverse && j / kNb < i / kNb) a.S[e] = 0.f;  // L = I
-    }
-  } else if (a.inverse) {
-    for (int h = 1; h < a.nblk; h *= 2) {
-      inv_step1(a, h);
-      grid_barrier(a);
-      inv_step2(a, h);
-      grid_barrier(a);
+      if (j / kNb < i / kNb) a.S[e] = 0.f;  // L = I
     }
   }
   if (blockIdx.x == 0 && threadIdx.x == 0 &&
@@ -387,8 +309,7 @@ __global__ void __launch_bounds__(kCholThreads) chol_blocked_kernel(const CholBA
 size_t chol_blocked_ctl_bytes(int r) { return 64 + (size_t)r * sizeof(double); }
 
 int chol_blocked(const float* part, int splits, int r, int64_t L, float* S,
-                 float* Linv, void* ctl, int* status, cudaStream_t stream,
-                 bool inverse) {
+                 float* Linv, void* ctl, int* status, cudaStream_t stream) {
   CholBArgs a;
   a.part = part;
   a.splits = splits;
@@ -402,7 +323,6 @@ int chol_blocked(const float* part, int splits, int r, int64_t L, float* S,
   a.flags = reinterpret_cast<int*>(reinterpret_cast<char*>(ctl) + 16);
   a.diag = reinterpret_cast<double*>(reinterpret_cast<char*>(ctl) + 64);
   a.status = status;
-  a.inverse = inverse ? 1 : 0;
   OUO_CHECK_CUDA(cudaMemsetAsync(ctl, 0, 64, stream));
   // every CTA must be resident at once: at most one per SM times the
   // occupancy, and no more than the widest phase needs

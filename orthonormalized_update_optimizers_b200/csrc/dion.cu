@@ -282,7 +282,7 @@ int orth_factor(std::vector<CholQrJob>& jobs, const std::vector<const DGroup*>& 
     const int64_t i = mem[k];
     OUO_TRY(chol_blocked(jobs[k].S, 1, jobs[k].r, jobs[k].L, jobs[k].Lb,
                          const_cast<float*>(jobs[k].Dd), g.ctl + (size_t)i * g.ctl_stride,
-                         status, s, false));
+                         status, s));
   }
   return cholqr_factor(small, status, s);
 }

@@ -244,15 +244,13 @@ struct RowsJob {
 int rows_reduce(const std::vector<RowsJob>& jobs, float eps, cudaStream_t s);
 
 // Cooperative blocked Cholesky for ranks above 256 (chol.cu): S = sum of
-// `splits` partial r x r Gram matrices in upper storage.  With `inverse`,
-// writes L^-1 into Linv (R x R, ld R, R = r rounded up to 32); without it,
-// leaves the strictly lower blocks of L in S (R x R, ld R) and the inverted
-// diagonal blocks in the diagonal blocks of Linv.  ctl is
+// `splits` partial r x r Gram matrices in upper storage.  Leaves the
+// strictly lower blocks of L in S (R x R, ld R, R = r rounded up to 32) and
+// the inverted diagonal blocks in the diagonal blocks of Linv.  ctl is
 // chol_blocked_ctl_bytes(r) bytes of 8-byte aligned scratch.
 size_t chol_blocked_ctl_bytes(int r);
 int chol_blocked(const float* part, int splits, int r, int64_t L, float* S,
-                 float* Linv, void* ctl, int* status, cudaStream_t stream,
-                 bool inverse);
+                 float* Linv, void* ctl, int* status, cudaStream_t stream);
 int convert_buf(const Buf& src, const Buf& dst, cudaStream_t stream);
 
 }  // namespace ouo
